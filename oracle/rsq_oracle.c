@@ -1,0 +1,382 @@
+/*
+ * rsq_oracle.c -- plain, slow, float64 CPU oracle of the online activation path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * execute this file or the library built from it; only the tests, the smoke
+ * check and the bench's CPU-baseline leg do.  It shares no code, header, table
+ * or constant with the CUDA path.
+ *
+ * Every step is written as its definition, one scalar loop per formula, with
+ * no blocking, fusion or reordering beyond what the definition states.  All
+ * arithmetic is IEEE double (build with -ffp-contract=off so that no fused
+ * multiply-add changes a rounding).  Inputs are the exact float32/bf16 values
+ * of the arrays the GPU reads, widened to double by the caller.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [RSQ]  "ReSpinQuant: Efficient Layer-Wise LLM Quantization via Subspace
+ *          Residual Rotation Approximation" (paper notes), key design 2
+ *          (T_hat = I + Q (R_sub - I_r) Q^T) and key design 3 (the three-step
+ *          online path y = Q^T x, z = M y, x_out = x + Q z, M = R_sub - I_r).
+ *   [QS]   "QuaRot and SpinQuant" (scholia log), section 1.3 (normalised 4x4
+ *          Hadamard worked example, absmax/7 step) and section 2.2 (fast
+ *          Walsh-Hadamard transform, O(d log d), d a power of two).
+ *   [IQ2]  "Infra Quant II", QuaRot / Background (normalised Hadamard entries
+ *          +-1/sqrt(d); H_d = H_{2^n} (x) H_m for d = 2^n m; randomised
+ *          H diag(s)), QuaRot / Method (per-token symmetric activation
+ *          quantisation, row absmax / 7, scale-free RMSNorm in FP32), and
+ *          SpinQuant / Motivation (symmetric quantiser
+ *          alpha = max|X| / (2^(N-1) - 1), X_Q = alpha * round(X / alpha)).
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *   - rounding is to nearest, ties to even (rint in the default mode);
+ *   - codes are clamped to the symmetric range [-qmax, qmax];
+ *   - an all-zero row gets scale 0 and all codes 0;
+ *   - the randomised transform is v = H (s .* x) / sqrt(d): signs first;
+ *   - Kronecker index map i = a*m + b (a < 2^n, b < m):
+ *       w[a m + b] = sum_{a',b'} H_{2^n}[a,a'] H_m[b,b'] u[a' m + b'];
+ *   - the order-12 matrix is Paley type I at q = 11;
+ *   - RMSNorm is n = x / sqrt(mean(x^2) + eps), with no weight;
+ *   - INT4 packing: element 2i in the low nibble of byte i, 2i+1 in the high
+ *     nibble, two's complement; INT3 packing: 8 codes per 3 bytes, code k of a
+ *     group in bits [3k, 3k+3) of the little-endian 24-bit word.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* threads                                                                  */
+/* ------------------------------------------------------------------------ */
+
+int ora_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Hadamard matrices                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Sylvester Hadamard matrix of order n = 2^k, entries +-1 (unnormalised),
+ * built by the doubling rule H_{2l} = [[H_l, H_l], [H_l, -H_l]] starting from
+ * H_1 = [1].  Row-major n x n.  [QS] 1.3 prints the normalised n = 4 case. */
+int ora_sylvester(int n, double *H)
+{
+    if (n < 1 || (n & (n - 1))) return -1;
+    H[0] = 1.0;
+    for (int l = 1; l < n; l *= 2) {
+        for (int i = 0; i < l; ++i) {
+            for (int j = 0; j < l; ++j) {
+                double h = H[(int64_t)i * n + j];
+                H[(int64_t)i * n + (j + l)] = h;
+                H[(int64_t)(i + l) * n + j] = h;
+                H[(int64_t)(i + l) * n + (j + l)] = -h;
+            }
+        }
+    }
+    return 0;
+}
+
+static int is_prime(int q)
+{
+    if (q < 2) return 0;
+    for (int p = 2; p * p <= q; ++p)
+        if (q % p == 0) return 0;
+    return 1;
+}
+
+/* Paley type-I Hadamard matrix of order q + 1 for a prime q = 3 (mod 4),
+ * entries +-1.  chi is the quadratic character mod q, the Jacobsthal matrix
+ * is J[i][j] = chi(j - i), S = [[0, 1^T], [-1, J]] and H = I + S.
+ * [IQ2] Background: "m is the order of some known Hadamard matrix". */
+int ora_paley1(int q, double *H)
+{
+    if (!is_prime(q) || q % 4 != 3) return -1;
+    int n = q + 1;
+    int *chi = (int *)calloc((size_t)q, sizeof(int));
+    if (!chi) return -2;
+    for (int a = 1; a < q; ++a) chi[(int)(((int64_t)a * a) % q)] = 1;
+    for (int a = 1; a < q; ++a)
+        if (!chi[a]) chi[a] = -1;
+    chi[0] = 0;
+    for (int i = 0; i < n; ++i)
+        for (int j = 0; j < n; ++j) {
+            double s;
+            if (i == 0 && j == 0) s = 0.0;
+            else if (i == 0) s = 1.0;
+            else if (j == 0) s = -1.0;
+            else s = (double)chi[((j - 1) - (i - 1) + q) % q];
+            H[(int64_t)i * n + j] = (i == j ? 1.0 : 0.0) + s;
+        }
+    free(chi);
+    return 0;
+}
+
+/* In-place fast Walsh-Hadamard transform of the n = 2^k values
+ * v[0], v[stride], ..., v[(n-1) stride]: v <- H_n v with the Sylvester H_n,
+ * unnormalised.  [QS] 2.2: O(n log n) butterflies, n a power of two. */
+void ora_fwht(int n, int64_t stride, double *v)
+{
+    for (int h = 1; h < n; h *= 2)
+        for (int i = 0; i < n; i += 2 * h)
+            for (int j = i; j < i + h; ++j) {
+                double a = v[(int64_t)j * stride];
+                double b = v[(int64_t)(j + h) * stride];
+                v[(int64_t)j * stride] = a + b;
+                v[(int64_t)(j + h) * stride] = a - b;
+            }
+}
+
+/* ------------------------------------------------------------------------ */
+/* per-row steps                                                            */
+/* ------------------------------------------------------------------------ */
+
+/* [RSQ] key design 3: y = Q^T x (D -> r), z = M y, x_out = x + Q z.
+ * Q is D x r row-major (Q[i r + k]); M is r x r row-major, z_j = sum_k M[j r + k] y_k. */
+static void align_row(int D, int r, const double *x, const double *Q, const double *M,
+                      double *y, double *z, double *xo)
+{
+    for (int k = 0; k < r; ++k) {
+        double s = 0.0;
+        for (int i = 0; i < D; ++i) s += Q[(int64_t)i * r + k] * x[i];
+        y[k] = s;
+    }
+    for (int j = 0; j < r; ++j) {
+        double s = 0.0;
+        for (int k = 0; k < r; ++k) s += M[(int64_t)j * r + k] * y[k];
+        z[j] = s;
+    }
+    for (int i = 0; i < D; ++i) {
+        double s = 0.0;
+        for (int j = 0; j < r; ++j) s += Q[(int64_t)i * r + j] * z[j];
+        xo[i] = x[i] + s;
+    }
+}
+
+/* [IQ2] Method / Background: RMSNorm whose scale has been folded into the next
+ * weights, n = x / sqrt(mean(x^2) + eps). */
+static void rmsnorm_row(int D, double eps, const double *x, double *n)
+{
+    double ss = 0.0;
+    for (int i = 0; i < D; ++i) ss += x[i] * x[i];
+    double rs = 1.0 / sqrt(ss / (double)D + eps);
+    for (int i = 0; i < D; ++i) n[i] = x[i] * rs;
+}
+
+/* [IQ2] SpinQuant / Motivation, symmetric case: alpha = max|v| / (2^(N-1) - 1),
+ * q = round(v / alpha) (beta = 0); [IQ2] QuaRot / Method: per token, row
+ * absmax / 7 for INT4.  Codes are clamped to [-qmax, qmax]; pre receives v/alpha. */
+static double quant_row(int n, int bits, const double *v, int8_t *q, double *pre)
+{
+    int qmax = (1 << (bits - 1)) - 1;
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i) {
+        double a = fabs(v[i]);
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0) {
+        for (int i = 0; i < n; ++i) {
+            q[i] = 0;
+            if (pre) pre[i] = 0.0;
+        }
+        return 0.0;
+    }
+    double alpha = amax / (double)qmax;
+    for (int i = 0; i < n; ++i) {
+        double p = v[i] / alpha;
+        double c = rint(p);
+        if (c > qmax) c = qmax;
+        if (c < -qmax) c = -qmax;
+        q[i] = (int8_t)c;
+        if (pre) pre[i] = p;
+    }
+    return alpha;
+}
+
+/* [IQ2] Background: randomised Hadamard v = H_d diag(s) x / sqrt(d), with
+ * H_d = H_{2^n} (x) H_m when d = 2^n m.  The 2^n-point transform runs along
+ * stride m, then the dense m x m matrix acts on each contiguous group of m. */
+static void rht_row(int d, int m, const double *Hm, const double *x, const int8_t *s,
+                    double *u, double *w)
+{
+    int n2 = d / m;
+    for (int i = 0; i < d; ++i) u[i] = (double)s[i] * x[i];
+    for (int b = 0; b < m; ++b) ora_fwht(n2, m, u + b);
+    for (int a = 0; a < n2; ++a)
+        for (int b = 0; b < m; ++b) {
+            double acc = 0.0;
+            for (int bp = 0; bp < m; ++bp) acc += Hm[b * m + bp] * u[(int64_t)a * m + bp];
+            w[(int64_t)a * m + b] = acc;
+        }
+    double c = 1.0 / sqrt((double)d);
+    for (int i = 0; i < d; ++i) w[i] = w[i] * c;
+}
+
+static void pack_int4_row(int n, const int8_t *q, uint8_t *out)
+{
+    for (int i = 0; i < n / 2; ++i)
+        out[i] = (uint8_t)(((unsigned)q[2 * i] & 0xFu) | (((unsigned)q[2 * i + 1] & 0xFu) << 4));
+}
+
+static void pack_int3_row(int n, const int8_t *q, uint8_t *out)
+{
+    for (int g = 0; g < n / 8; ++g) {
+        uint32_t word = 0;
+        for (int k = 0; k < 8; ++k) word |= ((uint32_t)q[8 * g + k] & 7u) << (3 * k);
+        out[3 * g + 0] = (uint8_t)(word & 0xFFu);
+        out[3 * g + 1] = (uint8_t)((word >> 8) & 0xFFu);
+        out[3 * g + 2] = (uint8_t)((word >> 16) & 0xFFu);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* exported batched entry points (OpenMP over independent token rows)       */
+/* ------------------------------------------------------------------------ */
+
+int ora_residual_align(int64_t T, int D, int r, const double *x, const double *Q,
+                       const double *M, double *xo)
+{
+    int err = 0;
+#pragma omp parallel
+    {
+        double *y = (double *)malloc(sizeof(double) * (size_t)r);
+        double *z = (double *)malloc(sizeof(double) * (size_t)r);
+        if (!y || !z) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t)
+                align_row(D, r, x + t * D, Q, M, y, z, xo + t * D);
+        }
+        free(y);
+        free(z);
+    }
+    return err;
+}
+
+int ora_rmsnorm(int64_t T, int D, double eps, const double *x, double *n)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) rmsnorm_row(D, eps, x + t * D, n + t * D);
+    return 0;
+}
+
+int ora_quant_sym(int64_t T, int n, int bits, const double *v, int8_t *q, double *alpha, double *pre)
+{
+    if (bits < 2 || bits > 8) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        alpha[t] = quant_row(n, bits, v + t * n, q + t * n, pre ? pre + t * n : NULL);
+    return 0;
+}
+
+int ora_rht(int64_t T, int d, int m, const double *Hm, const double *x, const int8_t *s, double *v)
+{
+    if (m < 1 || d % m) return -1;
+    int n2 = d / m;
+    if (n2 & (n2 - 1)) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *u = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!u) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) rht_row(d, m, Hm, x + t * d, s, u, v + t * d);
+        }
+        free(u);
+    }
+    return err;
+}
+
+int ora_pack(int64_t T, int n, int bits, const int8_t *q, uint8_t *out)
+{
+    if (bits == 4 && n % 2 == 0) {
+        for (int64_t t = 0; t < T; ++t) pack_int4_row(n, q + t * n, out + t * (n / 2));
+        return 0;
+    }
+    if (bits == 3 && n % 8 == 0) {
+        for (int64_t t = 0; t < T; ++t) pack_int3_row(n, q + t * n, out + t * (3 * n / 8));
+        return 0;
+    }
+    return -1;
+}
+
+/* Full align -> RMSNorm -> quantise -> pack pipeline, one row at a time.
+ * xo (T x D), q (T x D), codes (T x D bits / 8), scales (T) are outputs; pre may be NULL. */
+int ora_align_norm_quant(int64_t T, int D, int r, int bits, double eps, const double *x,
+                         const double *Q, const double *M, double *xo, int8_t *q,
+                         uint8_t *codes, double *scales, double *pre)
+{
+    if ((bits != 3 && bits != 4) || (D * bits) % 8 || (bits == 3 && D % 8)) return -1;
+    int err = 0;
+    int row_bytes = D * bits / 8;
+#pragma omp parallel
+    {
+        double *y = (double *)malloc(sizeof(double) * (size_t)r);
+        double *z = (double *)malloc(sizeof(double) * (size_t)r);
+        double *nrm = (double *)malloc(sizeof(double) * (size_t)D);
+        if (!y || !z || !nrm) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                align_row(D, r, x + t * D, Q, M, y, z, xo + t * D);
+                rmsnorm_row(D, eps, xo + t * D, nrm);
+                scales[t] = quant_row(D, bits, nrm, q + t * D, pre ? pre + t * D : NULL);
+                if (bits == 4) pack_int4_row(D, q + t * D, codes + t * row_bytes);
+                else pack_int3_row(D, q + t * D, codes + t * row_bytes);
+            }
+        }
+        free(y);
+        free(z);
+        free(nrm);
+    }
+    return err;
+}
+
+/* Randomised Hadamard -> quantise -> pack (no normalisation). */
+int ora_rht_quant(int64_t T, int d, int m, int bits, const double *Hm, const double *x,
+                  const int8_t *s, int8_t *q, uint8_t *codes, double *scales, double *pre)
+{
+    if ((bits != 3 && bits != 4) || (d * bits) % 8 || (bits == 3 && d % 8)) return -1;
+    if (m < 1 || d % m) return -1;
+    int n2 = d / m;
+    if (n2 & (n2 - 1)) return -1;
+    int err = 0;
+    int row_bytes = d * bits / 8;
+#pragma omp parallel
+    {
+        double *u = (double *)malloc(sizeof(double) * (size_t)d);
+        double *v = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!u || !v) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                rht_row(d, m, Hm, x + t * d, s, u, v);
+                scales[t] = quant_row(d, bits, v, q + t * d, pre ? pre + t * d : NULL);
+                if (bits == 4) pack_int4_row(d, q + t * d, codes + t * row_bytes);
+                else pack_int3_row(d, q + t * d, codes + t * row_bytes);
+            }
+        }
+        free(u);
+        free(v);
+    }
+    return err;
+}

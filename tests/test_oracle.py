@@ -1,0 +1,316 @@
+"""Pins of the float64 oracle against facts fixed by the pages and by mathematics.
+
+None of these tests needs a GPU.  Each pin is chosen so that a plausible slip in
+the oracle (a dropped term, a wrong sign or index, a transposed operand, a wrong
+row order, a wrong rounding or packing rule) makes at least one of them fail.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle
+from w3a3_quantization_online_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# Hadamard: worked example, order, orthogonality, FWHT == dense
+# --------------------------------------------------------------------------
+
+def test_worked_example_matrix_and_transform():
+    g = _golden("hadamard4_worked_example.json")
+    Hn = np.array(g["H_normalised"])
+    np.testing.assert_array_equal(oracle.sylvester(4) / 2.0, Hn)  # row order of the printed H
+    x = np.array([g["x"]])
+    ones = np.ones(4, dtype=np.int8)
+    np.testing.assert_array_equal(Hn.T @ x[0], g["HT_x"])  # the page's own arithmetic
+    np.testing.assert_array_equal(oracle.rht(x, ones, 1)[0], g["HT_x"])
+    np.testing.assert_array_equal(oracle.rht(np.array([g["x_back"]]), ones, 1)[0], g["H_x_back"])
+
+
+def test_worked_example_quantisation():
+    g = _golden("hadamard4_worked_example.json")
+    ones = np.ones(4, dtype=np.int8)
+    before = oracle.rht_quant(np.array([g["H_x_back"]]), ones, 1, 4)   # rht([20,0,0,0]) = [10]*4
+    after = oracle.rht_quant(np.array([g["x_back"]]), ones, 1, 4)      # rht([10]*4) = [20,0,0,0]
+    # rht maps [20,0,0,0] to [10,10,10,10] (step 10/7) and back (step 20/7)
+    assert round(after["scales"][0], g["printed_decimals"]) == g["step_before_printed"]
+    assert round(before["scales"][0], g["printed_decimals"]) == g["step_after_printed"]
+    np.testing.assert_array_equal(after["q"][0], g["codes_before"])
+    np.testing.assert_array_equal(before["q"][0], g["codes_after"])
+    for res, v in ((before, [10.0] * 4), (after, [20.0, 0, 0, 0])):
+        deq = res["scales"][0] * res["q"][0].astype(np.float64)
+        assert np.max(np.abs(deq - np.array(v))) <= 1e-12 + g["dequant_error"]
+    # the qmax of INT4 is the page's divisor 7
+    assert g["qmax_int4"] == 2 ** (4 - 1) - 1
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 16, 64, 256, 1024])
+def test_sylvester_matches_library_and_is_orthogonal(n):
+    H = oracle.sylvester(n)
+    np.testing.assert_array_equal(H, scipy.linalg.hadamard(n))  # textbook Sylvester construction
+    np.testing.assert_array_equal(H.T @ H, n * np.eye(n))      # H^T H = I after 1/sqrt(n)
+
+
+@pytest.mark.parametrize("n", [2, 4, 8, 16, 32, 64])
+def test_fwht_equals_dense_bruteforce(n):
+    rng = np.random.default_rng(n)
+    v = rng.standard_normal((5, n))
+    dense = v @ scipy.linalg.hadamard(n).T
+    np.testing.assert_allclose(oracle.fwht(v), dense, rtol=0, atol=1e-12 * n)
+
+
+@pytest.mark.parametrize("d", [4, 16, 64, 256])
+def test_randomised_hadamard_equals_dense(d):
+    rng = np.random.default_rng(d)
+    x = rng.standard_normal((3, d))
+    s = np.where(rng.integers(0, 2, d) == 1, 1, -1).astype(np.int8)
+    Hs = scipy.linalg.hadamard(d) @ np.diag(s.astype(np.float64)) / math.sqrt(d)
+    np.testing.assert_allclose(Hs @ Hs.T, np.eye(d), atol=1e-12)    # H diag(s) is orthogonal
+    np.testing.assert_allclose(oracle.rht(x, s, 1), x @ Hs.T, atol=1e-12)
+    # all-ones signs reduce to the plain normalised H
+    np.testing.assert_allclose(oracle.rht(x, np.ones(d, np.int8), 1),
+                               x @ scipy.linalg.hadamard(d).T / math.sqrt(d), atol=1e-12)
+
+
+@pytest.mark.parametrize("d", [4096, 8192])
+def test_randomised_hadamard_preserves_norm(d):
+    case = inputs.rht_case(4, d, 1, 7, dtype="f32", n_outliers=4, outlier_scale=100.0)
+    v = oracle.rht(case.x, case.signs, 1)
+    np.testing.assert_allclose(np.linalg.norm(v, axis=1),
+                               np.linalg.norm(case.x.astype(np.float64), axis=1), rtol=1e-13)
+    # the outlier energy is spread: the largest coordinate shrinks for these inputs
+    assert np.all(np.abs(v).max(axis=1) < np.abs(case.x).max(axis=1))
+
+
+# --------------------------------------------------------------------------
+# Paley order-12 matrix and the Kronecker transform
+# --------------------------------------------------------------------------
+
+def _quadratic_character(a, q):
+    a %= q
+    if a == 0:
+        return 0
+    return 1 if pow(a, (q - 1) // 2, q) == 1 else -1  # Euler's criterion
+
+
+def test_paley12_is_hadamard_and_follows_the_textbook_construction():
+    q = 11
+    H = oracle.paley1(q)
+    np.testing.assert_array_equal(H @ H.T, 12 * np.eye(12))
+    S = H - np.eye(12)
+    np.testing.assert_array_equal(S, -S.T)                  # Paley I: H - I is skew
+    np.testing.assert_array_equal(H[0], np.ones(12))
+    np.testing.assert_array_equal(H[1:, 0], -np.ones(11))
+    for i in range(1, 12):
+        for j in range(1, 12):
+            if i != j:
+                assert H[i, j] == _quadratic_character(j - i, q)
+
+
+def test_paley_rejects_bad_orders():
+    with pytest.raises(ValueError):
+        oracle.paley1(13)   # 13 = 1 mod 4
+    with pytest.raises(ValueError):
+        oracle.paley1(15)   # not prime
+
+
+@pytest.mark.parametrize("k", [0, 1, 2, 3])
+def test_kronecker_transform_equals_dense_bruteforce(k):
+    n2 = 2 ** k
+    d = 12 * n2
+    rng = np.random.default_rng(100 + k)
+    x = rng.standard_normal((3, d))
+    s = np.where(rng.integers(0, 2, d) == 1, 1, -1).astype(np.int8)
+    Hd = np.kron(scipy.linalg.hadamard(n2), oracle.paley1(11)) / math.sqrt(d)
+    np.testing.assert_allclose(Hd @ Hd.T, np.eye(d), atol=1e-12)
+    want = x @ (Hd @ np.diag(s.astype(np.float64))).T
+    np.testing.assert_allclose(oracle.rht(x, s, 12), want, atol=1e-12)
+
+
+def test_kronecker_12288_preserves_norm():
+    case = inputs.down_proj_case(T=3)
+    v = oracle.rht(case.x, case.signs, 12)
+    np.testing.assert_allclose(np.linalg.norm(v, axis=1),
+                               np.linalg.norm(case.x.astype(np.float64), axis=1), rtol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Residual subspace alignment
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("D,r", [(64, 1), (128, 8), (256, 8), (256, 32)])
+def test_low_rank_path_equals_dense_T_hat(D, r):
+    case = inputs.align_case(9, D, r, 11, dtype="f32", n_outliers=2, outlier_scale=30.0)
+    Q, R = case.Q64, case.R64
+    T_hat = np.eye(D) + Q @ (R - np.eye(r)) @ Q.T
+    np.testing.assert_allclose(T_hat.T @ T_hat, np.eye(D), atol=1e-10)   # T_hat orthogonal
+    assert abs(np.linalg.det(T_hat) - 1.0) < 1e-9                       # ... and in SO(D)
+    assert abs(np.linalg.det(R) - 1.0) < 1e-12                           # Cayley map is in SO(r)
+    x = case.x.astype(np.float64)
+    xo = oracle.residual_align(x, Q, R - np.eye(r))
+    np.testing.assert_allclose(xo, x @ T_hat.T, atol=1e-11 * np.abs(x).max())
+    np.testing.assert_allclose(np.linalg.norm(xo, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+
+
+def test_zero_M_is_identity():
+    case = inputs.align_case(5, 256, 8, 3, dtype="f32")
+    xo = oracle.residual_align(case.x, case.Q64, np.zeros((8, 8)))
+    np.testing.assert_array_equal(xo, case.x.astype(np.float64))
+
+
+def test_full_rank_subspace_reproduces_the_rotation():
+    # r = D: Q is a full orthogonal basis and T_hat = Q R Q^T exactly
+    D = 16
+    case = inputs.align_case(4, D, D, 5, dtype="f32")
+    Q, R = case.Q64, case.R64
+    xo = oracle.residual_align(case.x, Q, R - np.eye(D))
+    np.testing.assert_allclose(xo, case.x.astype(np.float64) @ (Q @ R @ Q.T).T, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# RMSNorm and the quantiser
+# --------------------------------------------------------------------------
+
+def test_rmsnorm_mean_square_and_rotation_commute():
+    case = inputs.align_case(6, 128, 8, 4, dtype="f32", n_outliers=3, outlier_scale=20.0)
+    eps = 1e-5
+    x = case.x.astype(np.float64)
+    n = oracle.rmsnorm(x, eps)
+    ms = np.mean(x * x, axis=1)
+    rs2 = 1.0 / (ms + eps)
+    np.testing.assert_allclose(np.mean(n * n, axis=1), 1.0 - eps * rs2, rtol=0, atol=1e-14)
+    T_hat = np.eye(128) + case.Q64 @ (case.R64 - np.eye(8)) @ case.Q64.T
+    np.testing.assert_allclose(oracle.rmsnorm(x @ T_hat.T, eps), n @ T_hat.T, atol=1e-12)
+    # eps = 0: invariant to a positive row factor
+    np.testing.assert_allclose(oracle.rmsnorm(3.0 * x, 0.0), oracle.rmsnorm(x, 0.0), atol=1e-14)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_quantiser_error_bound_range_and_absmax(bits):
+    rng = np.random.default_rng(bits)
+    v = rng.standard_t(3, size=(50, 96)) * rng.uniform(0.01, 100, size=(50, 1))
+    q, a, pre = oracle.quant_sym(v, bits)
+    qmax = 2 ** (bits - 1) - 1
+    assert q.min() >= -qmax and q.max() <= qmax
+    # dequantisation error at most half a step
+    assert np.all(np.abs(a[:, None] * q - v) <= a[:, None] / 2 * (1 + 1e-12))
+    # the absmax element lands on +-qmax
+    am = np.argmax(np.abs(v), axis=1)
+    assert np.all(np.abs(q[np.arange(50), am]) == qmax)
+    np.testing.assert_allclose(a, np.abs(v).max(axis=1) / qmax, rtol=1e-15)
+    # odd symmetry and invariance to power-of-two row factors (exact in binary)
+    q2, _, _ = oracle.quant_sym(-v, bits)
+    np.testing.assert_array_equal(q2, -q)
+    for c in (0.25, 4.0):
+        q3, a3, _ = oracle.quant_sym(c * v, bits)
+        np.testing.assert_array_equal(q3, q)
+        np.testing.assert_allclose(a3, c * a, rtol=1e-15)
+
+
+def test_quantiser_rounds_half_to_even_and_handles_zero_rows():
+    # qmax = 7: alpha = 1 exactly when the absmax is 7; ties at 0.5, 1.5, 2.5
+    v = np.array([[7.0, 0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 0.0],
+                  [0.0] * 8])
+    q, a, pre = oracle.quant_sym(v, 4)
+    np.testing.assert_array_equal(q[0], [7, 0, 2, 2, 0, -2, -2, 0])
+    assert a[1] == 0.0 and np.all(q[1] == 0) and np.all(pre[1] == 0)
+
+
+# --------------------------------------------------------------------------
+# Packing
+# --------------------------------------------------------------------------
+
+def _unpack_int4(b, n):
+    lo = (b & 0xF).astype(np.int16)
+    hi = (b >> 4).astype(np.int16)
+    out = np.empty(b.shape[:-1] + (n,), dtype=np.int16)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return np.where(out >= 8, out - 16, out).astype(np.int8)
+
+
+def _unpack_int3(b, n):
+    b = b.astype(np.uint32).reshape(b.shape[:-1] + (n // 8, 3))
+    word = b[..., 0] | (b[..., 1] << 8) | (b[..., 2] << 16)
+    k = np.arange(8, dtype=np.uint32)
+    c = ((word[..., None] >> (3 * k)) & 7).astype(np.int16)
+    c = np.where(c >= 4, c - 8, c)
+    return c.reshape(b.shape[:-2] + (n,)).astype(np.int8)
+
+
+def test_pack_int4_layout_and_exhaustive_round_trip():
+    np.testing.assert_array_equal(oracle.pack(np.array([[1, -1, 7, -7]]), 4)[0], [0xF1, 0x97])
+    vals = np.arange(-7, 8)
+    pairs = np.array([[a, b] for a in vals for b in vals], dtype=np.int8)
+    packed = oracle.pack(pairs, 4)
+    np.testing.assert_array_equal(_unpack_int4(packed, 2), pairs)
+
+
+def test_pack_int3_layout_and_exhaustive_round_trip():
+    np.testing.assert_array_equal(oracle.pack(np.array([[1, 0, 0, 0, 0, 0, 0, 0]]), 3)[0], [1, 0, 0])
+    np.testing.assert_array_equal(oracle.pack(np.array([[-1] * 8]), 3)[0], [0xFF, 0xFF, 0xFF])
+    np.testing.assert_array_equal(oracle.pack(np.array([[0, 0, 0, 3, 0, 0, 0, -3]]), 3)[0],
+                                  [0x00, 0x06, 0xA0])
+    # every group of 8 codes in [-3, 3]: 7^8 = 5,764,801 groups
+    idx = np.arange(7 ** 8, dtype=np.int64)
+    groups = np.stack([(idx // 7 ** k) % 7 - 3 for k in range(8)], axis=1).astype(np.int8)
+    packed = oracle.pack(groups, 3)
+    np.testing.assert_array_equal(_unpack_int3(packed, 8), groups)
+
+
+# --------------------------------------------------------------------------
+# Pipelines and counts
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_align_norm_quant_is_the_composition_of_its_steps(bits):
+    case = inputs.align_case(7, 256, 8, 21, dtype="bf16", bits=bits, n_outliers=4, outlier_scale=50.0)
+    res = oracle.align_norm_quant(case.x, case.Q, case.M, bits, case.eps)
+    xo = oracle.residual_align(case.x, case.Q, case.M)
+    n = oracle.rmsnorm(xo, case.eps)
+    q, a, pre = oracle.quant_sym(n, bits)
+    np.testing.assert_array_equal(res["x_out"], xo)
+    np.testing.assert_array_equal(res["q"], q)
+    np.testing.assert_array_equal(res["scales"], a)
+    np.testing.assert_array_equal(res["codes"], oracle.pack(q, bits))
+    # scale invariance of the codes: RMSNorm output times a positive factor
+    # (exact power of two) gives the same codes
+    q4, _, _ = oracle.quant_sym(4.0 * n, bits)
+    np.testing.assert_array_equal(q4, q)
+
+
+def test_rht_quant_is_the_composition_of_its_steps():
+    case = inputs.rht_case(5, 768, 12, 9, dtype="bf16", bits=4)
+    res = oracle.rht_quant(case.x, case.signs, 12, 4)
+    q, a, pre = oracle.quant_sym(oracle.rht(case.x, case.signs, 12), 4)
+    np.testing.assert_array_equal(res["q"], q)
+    np.testing.assert_array_equal(res["scales"], a)
+    np.testing.assert_array_equal(res["codes"], oracle.pack(q, 4))
+
+
+def test_online_parameter_count():
+    g = _golden("online_param_count.json")
+    case = inputs.align_case(1, g["D"], g["r"], 0, dtype="f32")
+    per_module = case.Q.size + case.M.size
+    total = g["modules_per_layer"] * g["layers"] * per_module
+    assert math.floor(total / 1e5) / 10 == g["printed_millions"]
+
+
+def test_inputs_are_deterministic_and_on_the_bf16_grid():
+    a1, _ = inputs.llama7b_case(T=8)
+    a2, _ = inputs.llama7b_case(T=8)
+    np.testing.assert_array_equal(a1.x, a2.x)
+    u = a1.x.view(np.uint32)
+    assert np.all(u & 0xFFFF == 0)
+    np.testing.assert_allclose(a1.Q64.T @ a1.Q64, np.eye(32), atol=1e-13)

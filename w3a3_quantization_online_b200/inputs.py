@@ -1,0 +1,232 @@
+"""Seeded synthetic inputs for the online activation path.
+
+This module only draws random numbers and shapes them into the arrays that the
+GPU path and the float64 oracle both read; it holds none of the method's
+arithmetic (no projection, no Hadamard transform, no normalisation, no
+quantisation).  Both sides receive exactly the same bits.
+
+Recipe (numpy ``Generator(PCG64)``, one independent stream per array, keyed by
+``SeedSequence([seed, stream])``):
+
+* activations ``x``: float64 draws of the stated distribution, outlier channels
+  (chosen once per seed, identical for every token) multiplied by a factor, then
+  cast once to float32 and, for bf16 I/O, rounded to bf16 (round to nearest
+  even).  ``x`` is always returned as a float32 array holding the exact I/O
+  values;
+* ``Q``: the orthonormal factor of the QR decomposition of a D x r standard
+  Gaussian matrix, columns sign-fixed so that diag(R) > 0 (ReSpinQuant page,
+  "key design 2": an orthonormal basis Q of the subspace);
+* ``M = R_sub - I_r`` with ``R_sub = (I - A)^-1 (I + A)``, the Cayley map of a
+  skew-symmetric A whose upper triangle is drawn N(0, 0.05^2); this stands in
+  for the polar-decomposed rotation that calibration would produce
+  (ReSpinQuant page, "key design 2" and "key design 3");
+* ``signs``: int8 +-1 drawn uniformly (Infra Quant II page, QuaRot background:
+  the randomised Hadamard H diag(s) with s drawn from {+1, -1}).
+
+Q and M are handed to the kernels as float32; the float64 originals are kept
+for the pins that need exact orthogonality.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+# stream ids of SeedSequence([seed, stream])
+_S_X, _S_OUTLIER, _S_Q, _S_A, _S_SIGNS, _S_GATE = 0, 1, 2, 3, 4, 5
+
+_CHUNK_ROWS = 2048
+
+
+def _rng(seed: int, stream: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(np.random.SeedSequence([int(seed), int(stream)])))
+
+
+def round_to_bf16(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bf16 (ties to even); returns float32."""
+    a32 = np.ascontiguousarray(a, dtype=np.float32)
+    u = a32.view(np.uint32).astype(np.uint64)
+    u = (u + (((u >> 16) & 1) + 0x7FFF)) >> 16 << 16
+    return u.astype(np.uint32).view(np.float32)
+
+
+def _cast_io(a64: np.ndarray, dtype: str) -> np.ndarray:
+    a32 = a64.astype(np.float32)
+    if dtype == "bf16":
+        return round_to_bf16(a32)
+    if dtype == "f32":
+        return a32
+    raise ValueError(f"unknown I/O dtype {dtype!r}")
+
+
+def activations(T: int, D: int, seed: int, dist: str = "normal", n_outliers: int = 0,
+                outlier_scale: float = 1.0, dtype: str = "bf16") -> np.ndarray:
+    """T x D activations: ``dist`` in {"normal", "student_t3", "silu_gate"}.
+
+    ``silu_gate`` is the FFN down_proj input SiLU(a) * b with a, b ~ N(0, 1),
+    computed in float64 here (it is input preparation, not part of the path).
+    """
+    rx = _rng(seed, _S_X)
+    rg = _rng(seed, _S_GATE)
+    out = np.empty((T, D), dtype=np.float32)
+    ch = None
+    if n_outliers:
+        ch = _rng(seed, _S_OUTLIER).choice(D, size=n_outliers, replace=False)
+    for r0 in range(0, T, _CHUNK_ROWS):
+        n = min(_CHUNK_ROWS, T - r0)
+        if dist == "normal":
+            blk = rx.standard_normal((n, D))
+        elif dist == "student_t3":
+            blk = rx.standard_t(3.0, size=(n, D))
+        elif dist == "silu_gate":
+            a = rx.standard_normal((n, D))
+            b = rg.standard_normal((n, D))
+            blk = a / (1.0 + np.exp(-a)) * b
+        else:
+            raise ValueError(dist)
+        if ch is not None:
+            blk[:, ch] *= outlier_scale
+        out[r0:r0 + n] = _cast_io(blk, dtype)
+    return out
+
+
+def outlier_channels(D: int, seed: int, n_outliers: int) -> np.ndarray:
+    return np.sort(_rng(seed, _S_OUTLIER).choice(D, size=n_outliers, replace=False))
+
+
+def subspace_basis(D: int, r: int, seed: int) -> np.ndarray:
+    """D x r orthonormal Q (float64) from the QR of a seeded Gaussian matrix."""
+    g = _rng(seed, _S_Q).standard_normal((D, r))
+    q, rr = np.linalg.qr(g)
+    sgn = np.sign(np.diag(rr))
+    sgn[sgn == 0] = 1.0
+    return q * sgn[None, :]
+
+
+def cayley_rotation(r: int, seed: int, sigma: float = 0.05) -> np.ndarray:
+    """r x r rotation (I - A)^-1 (I + A) of a seeded skew-symmetric A (float64)."""
+    u = np.triu(_rng(seed, _S_A).normal(0.0, sigma, size=(r, r)), k=1)
+    a = u - u.T
+    eye = np.eye(r)
+    return np.linalg.solve(eye - a, eye + a)
+
+
+def random_signs(d: int, seed: int) -> np.ndarray:
+    return np.where(_rng(seed, _S_SIGNS).integers(0, 2, size=d) == 1, 1, -1).astype(np.int8)
+
+
+@dataclasses.dataclass
+class AlignCase:
+    """Inputs of one residual-alignment problem (float32 arrays as handed to the kernels)."""
+    name: str
+    x: np.ndarray          # T x D float32 holding the exact I/O values
+    Q: np.ndarray          # D x r float32
+    M: np.ndarray          # r x r float32, z_j = sum_k M[j,k] y_k
+    Q64: np.ndarray        # float64 originals
+    R64: np.ndarray        # r x r rotation, M64 = R64 - I
+    dtype: str             # "f32" | "bf16"
+    bits: int
+    eps: float = 1e-5
+
+    @property
+    def T(self) -> int:
+        return self.x.shape[0]
+
+    @property
+    def D(self) -> int:
+        return self.x.shape[1]
+
+    @property
+    def r(self) -> int:
+        return self.Q.shape[1]
+
+
+@dataclasses.dataclass
+class RhtCase:
+    """Inputs of one randomised-Hadamard problem."""
+    name: str
+    x: np.ndarray          # T x d float32 holding the exact I/O values
+    signs: np.ndarray      # d int8 +-1
+    m: int                 # 1 (pure Sylvester) or 12 (Kronecker with the order-12 Paley matrix)
+    dtype: str
+    bits: int
+
+    @property
+    def T(self) -> int:
+        return self.x.shape[0]
+
+    @property
+    def d(self) -> int:
+        return self.x.shape[1]
+
+
+def align_case(T: int, D: int, r: int, seed: int, *, dtype: str = "bf16", bits: int = 4,
+               dist: str = "normal", n_outliers: int = 0, outlier_scale: float = 1.0,
+               qm_seed: Optional[int] = None, eps: float = 1e-5, name: str = "") -> AlignCase:
+    qs = seed if qm_seed is None else qm_seed
+    q64 = subspace_basis(D, r, qs)
+    r64 = cayley_rotation(r, qs)
+    x = activations(T, D, seed, dist, n_outliers, outlier_scale, dtype)
+    return AlignCase(name or f"align_T{T}_D{D}_r{r}", x, q64.astype(np.float32),
+                     (r64 - np.eye(r)).astype(np.float32), q64, r64, dtype, bits, eps)
+
+
+def rht_case(T: int, d: int, m: int, seed: int, *, dtype: str = "bf16", bits: int = 4,
+             dist: str = "normal", n_outliers: int = 0, outlier_scale: float = 1.0,
+             name: str = "") -> RhtCase:
+    x = activations(T, d, seed, dist, n_outliers, outlier_scale, dtype)
+    return RhtCase(name or f"rht_T{T}_d{d}_m{m}", x, random_signs(d, seed), m, dtype, bits)
+
+
+# ---------------------------------------------------------------------------
+# The five workloads.  ``T`` may be overridden (the parity tests shrink it; the
+# bench uses the full sizes).
+# ---------------------------------------------------------------------------
+
+def tiny_case(T: int = 64):
+    """T=64, D=256, r=8, fp32 I/O, 4 outlier channels x50, INT4, order-256 RHT."""
+    a = align_case(T, 256, 8, 0, dtype="f32", bits=4, n_outliers=4, outlier_scale=50.0, name="tiny")
+    h = rht_case(T, 256, 1, 0, dtype="f32", bits=4, n_outliers=4, outlier_scale=50.0, name="tiny_rht")
+    return a, h
+
+
+def llama7b_case(T: int = 2048):
+    """Llama-7B-like hidden stream: D=4096, r=32, bf16, 8 outlier channels x100, INT4; FWHT 2^12."""
+    a = align_case(T, 4096, 32, 1, dtype="bf16", bits=4, n_outliers=8, outlier_scale=100.0,
+                   name=f"hidden_T{T}_D4096")
+    h = rht_case(T, 4096, 1, 1, dtype="bf16", bits=4, n_outliers=8, outlier_scale=100.0,
+                 name=f"rht_T{T}_d4096")
+    return a, h
+
+
+def down_proj_case(T: int = 4096):
+    """FFN down_proj input SiLU(a)*b, d=12288=1024*12, bf16, H_1024 (x) H_12, INT4."""
+    return rht_case(T, 12288, 12, 2, dtype="bf16", bits=4, dist="silu_gate", name=f"downproj_T{T}_d12288")
+
+
+def w3a3_case(T: int = 8192):
+    """W3A3 large hidden: D=8192, r=32, bf16, Student-t(3) + 16 outlier channels x200, INT3; FWHT 2^13."""
+    a = align_case(T, 8192, 32, 3, dtype="bf16", bits=3, dist="student_t3", n_outliers=16,
+                   outlier_scale=200.0, name=f"w3a3_T{T}_D8192")
+    h = rht_case(T, 8192, 1, 3, dtype="bf16", bits=3, dist="student_t3", n_outliers=16,
+                 outlier_scale=200.0, name=f"w3a3_rht_T{T}_d8192")
+    return a, h
+
+
+CHAIN_LAYERS = 32
+
+
+def chain_case(T: int = 16, layers: int = CHAIN_LAYERS):
+    """32 independent (Q_i, M_i) pairs (seeds 1000+i) over one bf16 residual stream, D=4096, r=32."""
+    x = activations(T, 4096, 4, "normal", 8, 100.0, "bf16")
+    qs, ms, q64s, r64s = [], [], [], []
+    for i in range(layers):
+        q64 = subspace_basis(4096, 32, 1000 + i)
+        r64 = cayley_rotation(32, 1000 + i)
+        q64s.append(q64)
+        r64s.append(r64)
+        qs.append(q64.astype(np.float32))
+        ms.append((r64 - np.eye(32)).astype(np.float32))
+    return x, qs, ms, q64s, r64s
+

@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the online activation path on B200.
+
+One step = one pass of the whole hot path over one batch resident in HBM:
+residual alignment -> RMSNorm -> INT4 (rsq_align_norm_quant) and the
+randomised Hadamard 2^12 -> INT4 (rht_quant), both on the same T x D bf16
+batch (T = 16384 tokens per GPU, D = 4096, r = 32).  Token rows are
+independent, so N GPUs process N independent shards with no collective on the
+data path ("weak" scaling); the only collectives are the timing barrier and the
+max-over-ranks of the elapsed time.
+
+Prints ONE JSON line on rank 0.  `--impl reference` times the float64 CPU
+oracle instead (rank 0 only, bounded samples).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s & HBM GB/s (frac of B200 peak), fused align+FWHT+INT4 quant, D=4096"
+T_TOK, D, R, BITS, EPS = 16384, 4096, 32, 4, 1e-5
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 10 ** 6
+
+
+def algorithmic_bytes(T: int) -> dict:
+    """Bytes each kernel must move per launch (the roofline numerators).
+
+    align+norm+quant: read x (2 B/elem), write x_out (2 B/elem), write codes
+    (D/2 B), write one fp32 scale per token; Q (D r fp32) and M (r^2 fp32)
+    once per launch.  rht+quant: read x, write codes and scale; signs once."""
+    per_tok_align = 2 * D * 2 + D * BITS // 8 + 4
+    per_tok_rht = D * 2 + D * BITS // 8 + 4
+    return {
+        "align_norm_quant": T * per_tok_align + D * R * 4 + R * R * 4,
+        "rht_quant": T * per_tok_rht + D,
+        "per_token_align": per_tok_align,
+        "per_token_rht": per_tok_rht,
+    }
+
+
+def workload_config(T: int, n: int) -> dict:
+    b = algorithmic_bytes(T)
+    ws = b["align_norm_quant"] + b["rht_quant"]
+    return {
+        "workload": f"hidden stream T={T}/GPU, D={D}, r={R}, bf16 I/O: residual align -> RMSNorm -> INT4, "
+                    f"and randomised Hadamard 2^12 -> INT4",
+        "T_per_gpu": T, "D": D, "r": R, "bits": BITS, "io_dtype": "bf16", "eps": EPS,
+        "global_tokens": T * n, "parallelism": f"token-sharded replicas x{n}, no data-path collective",
+        "l2": f"no flush: the bf16 input batch alone ({T * D * 2 / 1e6:.0f} MB) exceeds the {L2_BYTES / 1e6:.0f} MB L2; per-step traffic {ws / 1e6:.0f} MB",
+    }
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def kernel_source_sha(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """dram bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    if rec.get("source_sha") != kernel_source_sha(rec.get("sources", [])):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [s.strip() for s in line.split(",")]))
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        inside = [s for ts, s in self.samples if t0 <= ts <= t1]
+        note = None
+        if not inside:  # timed region shorter than the sampling period: nearest samples
+            inside = [s for ts, s in sorted(self.samples, key=lambda p: min(abs(p[0] - t0), abs(p[0] - t1)))[:2]]
+            note = "timed region shorter than the sampling period; nearest samples"
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for s in inside:
+            try:
+                sm.append(float(s[1]))
+                smax.append(float(s[2]))
+                power.append(float(s[3]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, s[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": max(smax) if smax else None,
+               "reasons": sorted(reasons), "samples": len(sm),
+               "power_w_max": max(power) if power else None}
+        if note:
+            out["note"] = note
+        return out
+
+
+def smi_id(dev) -> str:
+    """nvidia-smi -i selector of a torch device (PCI bus id, robust to CUDA_VISIBLE_DEVICES)."""
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    try:
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except AttributeError:
+        return str(dev.index)
+
+
+def oracle_sample_rate(T_sample: int, threads: int) -> dict:
+    """Time the float64 oracle (as it stands) on T_sample tokens of the workload."""
+    import oracle
+    from w3a3_quantization_online_b200 import inputs
+    a, h = inputs.llama7b_case(T=T_sample)
+    used = oracle.set_threads(threads)
+    t0 = time.perf_counter()
+    oracle.align_norm_quant(a.x, a.Q, a.M, BITS, EPS, want_pre=False)
+    oracle.rht_quant(h.x, h.signs, 1, BITS, want_pre=False)
+    dt = time.perf_counter() - t0
+    return {"seconds": dt, "tokens": T_sample, "cores": used}
+
+
+def cpu_baseline(target_s: float = 15.0) -> dict:
+    cores = os.cpu_count() or 1
+    probe = oracle_sample_rate(max(8, cores), cores)
+    per_tok = probe["seconds"] / probe["tokens"]
+    T_s = int(max(cores, min(T_TOK, target_s / max(per_tok, 1e-9))))
+    r = oracle_sample_rate(T_s, cores)
+    return {"value": r["tokens"] / r["seconds"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
+            "sample": f"{T_s} tokens of the same workload (both pipelines, float64 C oracle, OpenMP over "
+                      f"tokens), {r['seconds']:.1f} s"}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    cores = os.cpu_count() or 1
+    probe = oracle_sample_rate(max(8, cores), cores)
+    per_tok = probe["seconds"] / probe["tokens"]
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    tps = int(max(1, min(T_TOK, budget / max(per_tok, 1e-9))))
+    import oracle
+    from w3a3_quantization_online_b200 import inputs
+    a, h = inputs.llama7b_case(T=tps)
+    oracle.set_threads(cores)
+    for _ in range(args.warmup):
+        oracle.align_norm_quant(a.x, a.Q, a.M, BITS, EPS, want_pre=False)
+        oracle.rht_quant(h.x, h.signs, 1, BITS, want_pre=False)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.align_norm_quant(a.x, a.Q, a.M, BITS, EPS, want_pre=False)
+        oracle.rht_quant(h.x, h.signs, 1, BITS, want_pre=False)
+    dt = time.perf_counter() - t0
+    value = tps * args.steps / dt
+    sample = f"{tps} tokens per step of the same workload (float64 C oracle, OpenMP over tokens)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(T_TOK, n),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_gpu(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    rank = int(os.environ.get("RANK", "0"))
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={n}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if n > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    from w3a3_quantization_online_b200 import inputs, rsq
+
+    T = args.tokens
+    a = inputs.align_case(T, D, R, 1 + 1000 * rank, dtype="bf16", bits=BITS, n_outliers=8,
+                          outlier_scale=100.0, qm_seed=1)
+    signs_np = inputs.random_signs(D, 1)
+    x_host = torch.from_numpy(a.x).to(torch.bfloat16).pin_memory()
+    x = x_host.to(dev)
+    Q = torch.from_numpy(a.Q).to(dev)
+    M = torch.from_numpy(a.M).to(dev)
+    signs = torch.from_numpy(signs_np).to(dev)
+    x_out = torch.empty_like(x)
+    codes_a = torch.empty((T, D * BITS // 8), dtype=torch.uint8, device=dev)
+    scales_a = torch.empty((T,), dtype=torch.float32, device=dev)
+    codes_h = torch.empty_like(codes_a)
+    scales_h = torch.empty_like(scales_a)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        rsq.rsq_align_norm_quant(x, Q, M, x_out, codes_a, scales_a, bits=BITS, eps=EPS, stream=stream)
+        rsq.rht_quant(x, signs, 1, codes_h, scales_h, bits=BITS, stream=stream)
+
+    def barrier():
+        if n > 1:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(dev)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(smi_id(dev))
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = rsq.launch_count()
+    t_wall0 = time.time()
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            ev[k][0].record(stream)
+            rsq.rsq_align_norm_quant(x, Q, M, x_out, codes_a, scales_a, bits=BITS, eps=EPS, stream=stream)
+            ev[k][1].record(stream)
+            rsq.rht_quant(x, signs, 1, codes_h, scales_h, bits=BITS, stream=stream)
+            ev[k][2].record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier()
+    launches = rsq.launch_count() - launches0
+    time.sleep(0.2)
+    clocks = sampler.stop(t_wall0, t_wall1)
+
+    total_ms = ev[0][0].elapsed_time(ev[-1][2])
+    align_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    rht_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if n > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = T * n * args.steps / (total_ms / 1e3)
+
+    # end to end through the C ABI with host buffers: pinned H2D of the batch,
+    # both kernels, D2H of every output, all inside the timed region
+    x_out_h = torch.empty_like(x_out, device="cpu").pin_memory()
+    ca_h = torch.empty_like(codes_a, device="cpu").pin_memory()
+    sa_h = torch.empty_like(scales_a, device="cpu").pin_memory()
+    ch_h = torch.empty_like(codes_h, device="cpu").pin_memory()
+    sh_h = torch.empty_like(scales_h, device="cpu").pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        step()
+        x_out_h.copy_(x_out, non_blocking=True)
+        ca_h.copy_(codes_a, non_blocking=True)
+        sa_h.copy_(scales_a, non_blocking=True)
+        ch_h.copy_(codes_h, non_blocking=True)
+        sh_h.copy_(scales_h, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if n > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = T * n * e2e_steps / (float(te.item()) / 1e3)
+    h2d = x_host.numel() * 2
+    d2h = x_out.numel() * 2 + codes_a.numel() + codes_h.numel() + 4 * (scales_a.numel() + scales_h.numel())
+
+    if rank != 0:
+        if n > 1:
+            dist.destroy_process_group()
+        return
+
+    pk = peaks()
+    ab = algorithmic_bytes(T)
+    kern = {}
+    for name, ms in (("align_norm_quant", align_ms), ("rht_quant", rht_ms)):
+        avg = statistics.mean(ms)
+        gbs = ab[name] / (avg / 1e3) / 1e9
+        kern[name] = {"avg_us": avg * 1e3, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"],
+                      "tokens_per_s": T / (avg / 1e3)}
+    dom = max(kern, key=lambda k: kern[k]["avg_us"])
+    roof = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["achieved_gbs"], "peak": pk["hbm_gbs"],
+            "unit": "GB/s", "frac": kern[dom]["frac"], "traffic": recorded_traffic(dom),
+            "algorithmic_bytes_per_launch": ab[dom],
+            "peak_source": f"{pk['source']} (STREAM-style copy, burst)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; see DESIGN.md input recipe)",
+        "config": workload_config(T, n),
+        "roofline": roof,
+        "kernels": kern,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    if n > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["rsq", "reference"], default="rsq")
+    ap.add_argument("--tokens", type=int, default=T_TOK, help="tokens per GPU (default 16384)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,125 @@
+/*
+ * rsq.h -- C ABI of the B200 (sm_100a) online activation path of rotation-based
+ * low-bit LLM quantisation.
+ *
+ * Two online transforms, each fused with per-token symmetric absmax
+ * quantisation into packed INT4 / INT3 codes and float32 scales:
+ *
+ *   1. residual subspace alignment (ReSpinQuant):
+ *        y = Q^T x (D -> r),  z = M y,  x_out = x + Q z,   M = R_sub - I_r,
+ *      i.e. x_out = T_hat x with T_hat = I + Q (R_sub - I_r) Q^T, never formed;
+ *      followed by a weight-free RMSNorm and the quantiser;
+ *   2. randomised Hadamard transform (QuaRot): v = H_d diag(s) x / sqrt(d) with
+ *      H_d the Sylvester matrix of order d = 2^n, or H_{2^n} (x) H_12 (Paley
+ *      type I, q = 11) for d = 2^n * 12; followed by the quantiser.
+ *
+ * Sources, by page title and section:
+ *   "ReSpinQuant: Efficient Layer-Wise LLM Quantization via Subspace Residual
+ *    Rotation Approximation" (paper notes): key design 2 (T_hat) and key
+ *    design 3 (three-step online path).
+ *   "Infra Quant II": QuaRot / Background (normalised Hadamard, Kronecker
+ *    construction, randomised H diag(s)), QuaRot / Method (per-token
+ *    symmetric activation quantisation, row absmax / 7; scale-free RMSNorm in
+ *    FP32), SpinQuant / Motivation (alpha = max|X| / (2^(N-1) - 1)).
+ *   "QuaRot and SpinQuant" (scholia log): 1.3 (4x4 worked example), 2.2 (FWHT).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Ownership   The caller owns every buffer.  Device pointers are CUDA global
+ *             memory on the current device; the library keeps no pointer after
+ *             the call returns and allocates no device memory.
+ * Layouts     Row-major.  x, x_out: T x D elements of `dtype` (RSQ_F32 or
+ *             RSQ_BF16).  Q: D x r float32, Q[i*r + k].  M: r x r float32,
+ *             z_j = sum_k M[j*r + k] y_k.  signs: d int8 values, each +1 or -1.
+ *             scales: T float32.  codes: T rows of D*bits/8 bytes:
+ *               INT4: element 2i in the low nibble of byte i, 2i+1 in the high
+ *                     nibble, 4-bit two's complement, values in [-7, 7];
+ *               INT3: each group of 8 elements is one little-endian 24-bit word
+ *                     (3 bytes), element k of the group in bits [3k, 3k+3),
+ *                     3-bit two's complement, values in [-3, 3].
+ * Quantiser   alpha_t = max_i |v_ti| / qmax (qmax = 2^(bits-1) - 1) is written
+ *             to scales[t]; code = clamp(round_half_even(v / alpha), +-qmax);
+ *             an all-zero row gets alpha = 0 and all codes 0.  The alignment
+ *             path quantises the float32 (unrounded) x_out after RMSNorm; the
+ *             Hadamard path quantises v directly (no normalisation).
+ * Streams     `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *             work is enqueued on it and the call returns without
+ *             synchronising.
+ * Errors      Arguments are validated on the host before anything is
+ *             launched; a rejected call returns a nonzero rsq_status and
+ *             touches no memory.  A launch failure returns RSQ_ERR_CUDA and
+ *             rsq_last_cuda_error() gives the cudaError_t.  No entry point
+ *             traps, aborts or prints.  T == 0 returns RSQ_OK without
+ *             launching (pointers may then be NULL).
+ * Alignment   Every pointer must be 16-byte aligned (RSQ_ERR_ALIGN).
+ * Aliasing    x_out == x (in-place update of the residual stream) is allowed.
+ *             Any other overlap between distinct buffers is RSQ_ERR_ALIAS.
+ * Determinism No atomics in any reduction: outputs are bitwise reproducible
+ *             run to run for the same inputs and launch configuration.
+ */
+#ifndef RSQ_H_
+#define RSQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RSQ_OK = 0,
+    RSQ_ERR_NULL = 1,        /* a required pointer is NULL                       */
+    RSQ_ERR_SHAPE = 2,       /* T < 0, or D / d / r / m outside the supported set */
+    RSQ_ERR_DTYPE = 3,       /* dtype is not RSQ_F32 or RSQ_BF16                  */
+    RSQ_ERR_BITS = 4,        /* bits is not 3 or 4                                */
+    RSQ_ERR_ALIGN = 5,       /* a pointer is not 16-byte aligned                  */
+    RSQ_ERR_ALIAS = 6,       /* buffers overlap other than x_out == x             */
+    RSQ_ERR_UNSUPPORTED = 7, /* valid in principle but not built (e.g. m != 1, 12)*/
+    RSQ_ERR_CUDA = 8,        /* a CUDA call failed; see rsq_last_cuda_error()     */
+    RSQ_ERR_VALUE = 9        /* eps negative or not finite                        */
+} rsq_status;
+
+typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
+
+/* Supported shapes (RSQ_ERR_SHAPE otherwise):
+ *   alignment:  D % 16 == 0, 16 <= D <= 32768, 1 <= r <= 64;
+ *   quantised outputs additionally need D * bits % 8 == 0 (always true here);
+ *   Hadamard:   m in {1, 12} (else RSQ_ERR_UNSUPPORTED), d % m == 0,
+ *               n = d / m a power of two with 16 <= n <= 16384, d <= 32768,
+ *               d % 16 == 0. */
+
+/* Residual subspace alignment only: x_out = x + Q (M (Q^T x)) per token row.
+ * ReSpinQuant paper notes, key design 3.  x_out may equal x. */
+int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_out,
+                       int64_t T, int D, int r, int dtype, void *stream);
+
+/* Alignment -> weight-free RMSNorm n = x_out / sqrt(mean(x_out^2) + eps) ->
+ * per-token symmetric absmax quantisation of n -> packed codes.
+ * ReSpinQuant key design 3; Infra Quant II, QuaRot / Method and SpinQuant /
+ * Motivation.  Writes x_out (rounded to dtype), codes and scales
+ * (scales[t] = max_i |n_ti| / qmax).  x_out may equal x. */
+int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_out,
+                         uint8_t *codes, float *scales, int64_t T, int D, int r,
+                         int bits, float eps, int dtype, void *stream);
+
+/* Randomised Hadamard v = H_d diag(signs) x / sqrt(d) -> per-token symmetric
+ * absmax quantisation -> packed codes.  Infra Quant II, QuaRot / Background
+ * and QuaRot / Method.  m = 1: H_d Sylvester of order d; m = 12:
+ * H_d = H_{d/12} (x) H_12 with index i = a*12 + b.  scales[t] = max_i |v_ti| / qmax. */
+int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *scales,
+              int64_t T, int d, int bits, int dtype, void *stream);
+
+/* Human-readable name of an rsq_status value (static storage; never NULL). */
+const char *rsq_status_string(int status);
+
+/* cudaError_t of the most recent RSQ_ERR_CUDA returned on this host thread (0 if none). */
+int rsq_last_cuda_error(void);
+
+/* Number of kernels this library has launched in this process (all threads). */
+uint64_t rsq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSQ_H_ */

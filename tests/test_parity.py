@@ -1,0 +1,263 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small cases are compared element by element over whole outputs; full-size
+workloads are run in the bench's launch configuration and compared on sampled
+rows (token rows are independent, so the oracle recomputes just those rows).
+Tolerances are the ones in tests/helpers.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import helpers as H
+from w3a3_quantization_online_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _rsq():
+    from w3a3_quantization_online_b200 import rsq
+    return rsq
+
+
+def _to_dev(x: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(x)).to(DEV)
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def _host(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy() if t.dtype == torch.bfloat16 else t.cpu().numpy()
+
+
+def run_align(case, x_dev=None, in_place=False):
+    rsq = _rsq()
+    x = _to_dev(case.x, case.dtype) if x_dev is None else x_dev
+    Q = torch.from_numpy(case.Q).to(DEV)
+    M = torch.from_numpy(case.M).to(DEV)
+    xo = x if in_place else None
+    xo, codes, scales = rsq.rsq_align_norm_quant(x, Q, M, x_out=xo, bits=case.bits, eps=case.eps)
+    torch.cuda.synchronize()
+    return _host(xo), codes.cpu().numpy(), scales.cpu().numpy()
+
+
+def run_rht(case):
+    rsq = _rsq()
+    x = _to_dev(case.x, case.dtype)
+    s = torch.from_numpy(case.signs).to(DEV)
+    codes, scales = rsq.rht_quant(x, s, case.m, bits=case.bits)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy()
+
+
+def check_align(case, rows=None, label=""):
+    xo, codes, scales = run_align(case)
+    sel = slice(None) if rows is None else rows
+    ref = oracle.align_norm_quant(case.x[sel], case.Q, case.M, case.bits, case.eps)
+    H.check_aligned(xo[sel], ref["x_out"], case.x[sel], case.dtype, label)
+    H.check_scales(scales[sel], ref["scales"], label)
+    return H.check_codes(codes[sel], ref["q"], ref["pre"], case.bits, label)
+
+
+def check_rht(case, rows=None, label=""):
+    codes, scales = run_rht(case)
+    sel = slice(None) if rows is None else rows
+    ref = oracle.rht_quant(case.x[sel], case.signs, case.m, case.bits)
+    H.check_scales(scales[sel], ref["scales"], label)
+    return H.check_codes(codes[sel], ref["q"], ref["pre"], case.bits, label)
+
+
+# --------------------------------------------------------------------------
+# the five workloads at oracle-friendly sizes (several tiles plus a ragged tail)
+# --------------------------------------------------------------------------
+
+def test_tiny_config_full():
+    a, h = inputs.tiny_case(T=64)
+    check_align(a, label="tiny align")
+    check_rht(h, label="tiny rht")
+
+
+@pytest.mark.parametrize("T", [1, 131, 512])
+def test_hidden_4096_align_int4(T):
+    a, _ = inputs.llama7b_case(T=T)
+    check_align(a, label=f"hidden T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 131, 512])
+def test_hidden_4096_rht_int4(T):
+    _, h = inputs.llama7b_case(T=T)
+    check_rht(h, label=f"rht4096 T={T}")
+
+
+@pytest.mark.parametrize("T", [3, 200])
+def test_down_proj_kronecker_12288(T):
+    check_rht(inputs.down_proj_case(T=T), label=f"kron T={T}")
+
+
+@pytest.mark.parametrize("T", [2, 131])
+def test_w3a3_8192_int3(T):
+    a, h = inputs.w3a3_case(T=T)
+    check_align(a, label=f"w3a3 align T={T}")
+    check_rht(h, label=f"w3a3 rht T={T}")
+
+
+@pytest.mark.parametrize("T", [16, 300])
+def test_chain_32_layers_teacher_forced(T):
+    """Each layer runs in place on the residual stream; the oracle layer i takes
+    the GPU's bf16 stream before layer i as its input."""
+    rsq = _rsq()
+    x0, qs, ms, _, _ = inputs.chain_case(T=T)
+    x = _to_dev(x0, "bf16")
+    for i in range(len(qs)):
+        x_in = _host(x).copy()
+        Q = torch.from_numpy(qs[i]).to(DEV)
+        M = torch.from_numpy(ms[i]).to(DEV)
+        _, codes, scales = rsq.rsq_align_norm_quant(x, Q, M, x_out=x, bits=4)
+        torch.cuda.synchronize()
+        ref = oracle.align_norm_quant(x_in, qs[i], ms[i], 4, 1e-5)
+        H.check_aligned(_host(x), ref["x_out"], x_in, "bf16", f"layer {i}")
+        H.check_scales(scales.cpu().numpy(), ref["scales"], f"layer {i}")
+        H.check_codes(codes.cpu().numpy(), ref["q"], ref["pre"], 4, f"layer {i}")
+    # the stream keeps its norm through 32 orthogonal maps (up to bf16 rounding)
+    n0 = np.linalg.norm(x0.astype(np.float64), axis=1)
+    n1 = np.linalg.norm(_host(x).astype(np.float64), axis=1)
+    np.testing.assert_allclose(n1, n0, rtol=2e-2)
+
+
+# --------------------------------------------------------------------------
+# full sizes, sampled rows
+# --------------------------------------------------------------------------
+
+def _sample(T, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = np.unique(np.concatenate([[0, T - 1], rng.choice(T, n, replace=False)]))
+    return rows
+
+
+def test_full_hidden_16384_sampled():
+    a, h = inputs.llama7b_case(T=16384)
+    rows = _sample(16384)
+    check_align(a, rows, "hidden T=16384")
+    check_rht(h, rows, "rht4096 T=16384")
+
+
+def test_full_down_proj_sampled():
+    h = inputs.down_proj_case(T=4096)
+    check_rht(h, _sample(4096, 24), "kron T=4096")
+
+
+def test_full_w3a3_sampled():
+    a, h = inputs.w3a3_case(T=8192)
+    rows = _sample(8192, 24)
+    check_align(a, rows, "w3a3 T=8192")
+    check_rht(h, rows, "w3a3 rht T=8192")
+
+
+# --------------------------------------------------------------------------
+# edge cases
+# --------------------------------------------------------------------------
+
+def test_empty_batch_launches_nothing():
+    rsq = _rsq()
+    before = rsq.launch_count()
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device=DEV)
+    Q = torch.zeros((256, 8), device=DEV)
+    M = torch.zeros((8, 8), device=DEV)
+    xo, codes, scales = rsq.rsq_align_norm_quant(x, Q, M)
+    codes2, scales2 = rsq.rht_quant(x, torch.ones(256, dtype=torch.int8, device=DEV))
+    assert xo.shape == (0, 256) and codes.shape == (0, 128) and codes2.shape == (0, 128)
+    assert rsq.launch_count() == before
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_zero_rows_give_zero_scale_and_codes(dtype):
+    a = inputs.align_case(9, 256, 8, 5, dtype=dtype)
+    a.x[[0, 4, 8]] = 0.0
+    xo, codes, scales = run_align(a)
+    assert np.all(scales[[0, 4, 8]] == 0) and np.all(codes[[0, 4, 8]] == 0)
+    assert np.all(xo[[0, 4, 8]] == 0)
+    check_align(a, label="zero rows")
+    h = inputs.rht_case(9, 256, 1, 5, dtype=dtype)
+    h.x[[1, 7]] = 0.0
+    codes, scales = run_rht(h)
+    assert np.all(scales[[1, 7]] == 0) and np.all(codes[[1, 7]] == 0)
+    check_rht(h, label="zero rows rht")
+
+
+def test_in_place_update_equals_out_of_place():
+    a, _ = inputs.llama7b_case(T=77)
+    xo1, c1, s1 = run_align(a)
+    x = _to_dev(a.x, "bf16")
+    xo2, c2, s2 = run_align(a, x_dev=x, in_place=True)
+    np.testing.assert_array_equal(xo1, xo2)
+    np.testing.assert_array_equal(c1, c2)
+    np.testing.assert_array_equal(s1, s2)
+    np.testing.assert_array_equal(_host(x), xo2)
+
+
+@pytest.mark.parametrize("D,r", [(16, 1), (48, 3), (64, 64), (272, 17), (1024, 32), (12288, 32)])
+@pytest.mark.parametrize("dtype,bits", [("f32", 4), ("bf16", 3)])
+def test_odd_shapes(D, r, dtype, bits):
+    a = inputs.align_case(37, D, r, D + r, dtype=dtype, bits=bits, n_outliers=2, outlier_scale=20.0)
+    check_align(a, label=f"D={D} r={r}")
+
+
+@pytest.mark.parametrize("d,m", [(16, 1), (64, 1), (2048, 1), (16384, 1),
+                                 (192, 12), (24576, 12)])
+@pytest.mark.parametrize("dtype,bits", [("f32", 4), ("bf16", 3)])
+def test_rht_shapes(d, m, dtype, bits):
+    h = inputs.rht_case(19, d, m, d + m, dtype=dtype, bits=bits, n_outliers=3, outlier_scale=40.0)
+    check_rht(h, label=f"d={d} m={m}")
+
+
+def test_residual_align_only_matches_oracle():
+    rsq = _rsq()
+    for dtype in ("f32", "bf16"):
+        a = inputs.align_case(50, 4096, 32, 8, dtype=dtype, n_outliers=8, outlier_scale=100.0)
+        x = _to_dev(a.x, dtype)
+        xo = rsq.rsq_residual_align(x, torch.from_numpy(a.Q).to(DEV), torch.from_numpy(a.M).to(DEV))
+        torch.cuda.synchronize()
+        H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, dtype, f"align {dtype}")
+
+
+def test_exact_ties_round_half_to_even():
+    """w = H x with small integers chosen so that v/alpha hits exact ties; both
+    sides must round them to even with no exemption."""
+    d = 16
+    w = np.zeros((1, d))
+    w[0, :7] = [14, 1, 3, 5, -1, -3, -5]
+    Hd = oracle.sylvester(d)
+    x = (w @ Hd) / d                       # H symmetric, H H = d I: H x = w exactly
+    h = inputs.RhtCase("ties", x.astype(np.float32), np.ones(d, np.int8), 1, "f32", 4)
+    codes, scales = run_rht(h)
+    ref = oracle.rht_quant(h.x, h.signs, 1, 4)
+    np.testing.assert_array_equal(H.unpack(codes, d, 4), ref["q"])
+    np.testing.assert_array_equal(ref["q"][0, :7], [7, 0, 2, 2, 0, -2, -2])
+
+
+def test_worked_example_on_gpu():
+    """The 4x4 worked example, embedded in d = 16 (H_16 = H_4 (x) H_4 on a spike)."""
+    d = 16
+    x = np.zeros((2, d), np.float32)
+    x[0, 0] = 20.0
+    x[1, :] = 20.0 / 4.0        # H_16 maps a constant row to a spike
+    h = inputs.RhtCase("worked", x, np.ones(d, np.int8), 1, "f32", 4)
+    codes, scales = run_rht(h)
+    q = H.unpack(codes, d, 4)
+    np.testing.assert_array_equal(q[0], np.full(d, 7))
+    np.testing.assert_array_equal(q[1], [7] + [0] * (d - 1))
+    np.testing.assert_allclose(scales, [20.0 / 4.0 / 7.0, 20.0 / 7.0], rtol=1e-7)
+
+
+def test_deterministic_repeat():
+    a, h = inputs.llama7b_case(T=300)
+    r1 = run_align(a)
+    r2 = run_align(a)
+    for u, v in zip(r1, r2):
+        np.testing.assert_array_equal(u, v)
+    c1 = run_rht(h)
+    c2 = run_rht(h)
+    for u, v in zip(c1, c2):
+        np.testing.assert_array_equal(u, v)

@@ -1,0 +1,147 @@
+// common.cuh -- device helpers shared by the rsq kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rsq {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------
+// I/O element types
+// ---------------------------------------------------------------------------
+
+struct F32 {
+    using T = float;
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+
+struct BF16 {
+    using T = __nv_bfloat16;
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+// Load 8 consecutive elements (16 B for bf16, 32 B for fp32) as float.
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p);
+    const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8]) {
+    uint4 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    u.z = pack_bf16x2(v[4], v[5]);
+    u.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4 *>(p) = u;
+}
+
+// ---------------------------------------------------------------------------
+// Quantiser: code = clamp(round_half_even(v * inv), -qmax, qmax).
+// fmaf(v, inv, 1.5 * 2^23) rounds the exact product v*inv to the nearest
+// integer (ties to even) because the float grid has unit spacing there; the
+// integer is read back from the low mantissa bits.  Valid for |v*inv| < 2^22.
+// ---------------------------------------------------------------------------
+
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;
+
+__device__ __forceinline__ int quant_code(float v, float inv, int qmax) {
+    const int c = __float_as_int(fmaf(v, inv, kRoundMagic)) - kRoundMagicBits;
+    return max(-qmax, min(qmax, c));
+}
+
+// Pack 8 codes (each in [-qmax, qmax]).
+__device__ __forceinline__ uint32_t pack8_int4(const int (&c)[8]) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w |= (uint32_t(c[k]) & 0xFu) << (4 * k);
+    return w;
+}
+
+__device__ __forceinline__ uint32_t pack8_int3(const int (&c)[8]) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) w |= (uint32_t(c[k]) & 0x7u) << (3 * k);
+    return w;  // 24 significant bits
+}
+
+// Store the packed 8-code group g of a row (INT4: 4 bytes at 4g, INT3: 3 bytes at 3g).
+__device__ __forceinline__ void store_group(uint8_t *row, int g, int bits, const int (&c)[8]) {
+    if (bits == 4) {
+        *reinterpret_cast<uint32_t *>(row + 4 * g) = pack8_int4(c);
+    } else {
+        const uint32_t w = pack8_int3(c);
+        uint8_t *p = row + 3 * g;
+        p[0] = uint8_t(w);
+        p[1] = uint8_t(w >> 8);
+        p[2] = uint8_t(w >> 16);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Block reductions (deterministic: fixed tree, no atomics).  `red` must hold
+// blockDim.x / 32 entries; all threads must call.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float block_max(float v, float *red) {
+    v = warp_max(v);
+    const int w = threadIdx.x / kWarp, l = threadIdx.x % kWarp;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float r = red[0];
+    for (int i = 1; i < int(blockDim.x / kWarp); ++i) r = fmaxf(r, red[i]);
+    return r;
+}
+
+__device__ __forceinline__ double block_sum(double v, double *red) {
+    v = warp_sum(v);
+    const int w = threadIdx.x / kWarp, l = threadIdx.x % kWarp;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = red[0];
+    for (int i = 1; i < int(blockDim.x / kWarp); ++i) r += red[i];
+    return r;
+}
+
+}  // namespace rsq

@@ -1,0 +1,27 @@
+// kernels.h -- internal launchers behind the C ABI (not part of the public interface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rsq {
+
+// Device properties of the current device (cached per device ordinal).
+int num_sms();
+int max_smem_optin();
+
+// Bump the process-wide launch counter (read by rsq_launch_count()).
+void count_launch(int n = 1);
+
+// Generic CUDA-core path: any supported D, r, dtype.  quant=false computes
+// x_out only (codes / scales ignored).
+cudaError_t launch_align_generic(const void *x, const float *Q, const float *M, void *x_out,
+                                 uint8_t *codes, float *scales, int64_t T, int D, int r,
+                                 int bits, float eps, int dtype, bool quant, cudaStream_t s);
+
+// Generic randomised Hadamard + quantiser: m in {1, 12}, any supported d.
+cudaError_t launch_rht_generic(const void *x, const int8_t *signs, int m, uint8_t *codes,
+                               float *scales, int64_t T, int d, int bits, int dtype,
+                               cudaStream_t s);
+
+}  // namespace rsq

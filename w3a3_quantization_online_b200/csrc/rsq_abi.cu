@@ -1,0 +1,173 @@
+// rsq_abi.cu -- the extern "C" entry points declared in include/rsq.h.
+//
+// Every argument is checked on the host before anything is enqueued; a
+// rejected call returns a status and touches no memory.  The entry points then
+// pick a kernel by shape and dtype and enqueue it on the caller's stream.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kernels.h"
+#include "rsq.h"
+
+namespace rsq {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+thread_local int g_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];
+int g_smem[kMaxDevices];
+
+int cur_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    return dev;
+}
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+
+int num_sms() {
+    const int dev = cur_device();
+    if (g_sms[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        g_sms[dev] = v;
+    }
+    return g_sms[dev];
+}
+
+int max_smem_optin() {
+    const int dev = cur_device();
+    if (g_smem[dev] == 0) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || v <= 0)
+            v = 227 * 1024;
+        g_smem[dev] = v;
+    }
+    return g_smem[dev];
+}
+
+}  // namespace rsq
+
+namespace {
+
+using rsq::g_last_cuda_error;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Span {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+
+Span span(const void *p, uint64_t bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Span{a, a + uintptr_t(bytes)};
+}
+
+bool overlap(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi; }
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int finish(cudaError_t e) {
+    if (e != cudaSuccess) {
+        g_last_cuda_error = int(e);
+        return RSQ_ERR_CUDA;
+    }
+    return RSQ_OK;
+}
+
+int elem_bytes(int dtype) { return dtype == RSQ_F32 ? 4 : 2; }
+
+// Shared checks of the alignment entry points.
+int check_align_args(const void *x, const float *Q, const float *M, const void *x_out, int64_t T,
+                     int D, int r, int dtype) {
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (T < 0 || D < 16 || D > 32768 || D % 16 != 0 || r < 1 || r > 64) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!x || !Q || !M || !x_out) return RSQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(Q) || !aligned16(M) || !aligned16(x_out)) return RSQ_ERR_ALIGN;
+    const uint64_t act = uint64_t(T) * uint64_t(D) * uint64_t(elem_bytes(dtype));
+    const Span sx = span(x, act), so = span(x_out, act);
+    const Span sq = span(Q, uint64_t(D) * r * 4), sm = span(M, uint64_t(r) * r * 4);
+    if (x != x_out && overlap(sx, so)) return RSQ_ERR_ALIAS;
+    if (overlap(so, sq) || overlap(so, sm)) return RSQ_ERR_ALIAS;
+    return RSQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_out, int64_t T,
+                       int D, int r, int dtype, void *stream) {
+    int st = check_align_args(x, Q, M, x_out, T, D, r, dtype);
+    if (st != RSQ_OK || T == 0) return st;
+    return finish(rsq::launch_align_generic(x, Q, M, x_out, nullptr, nullptr, T, D, r, 4, 0.f, dtype,
+                                            false, static_cast<cudaStream_t>(stream)));
+}
+
+int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_out,
+                         uint8_t *codes, float *scales, int64_t T, int D, int r, int bits,
+                         float eps, int dtype, void *stream) {
+    if (bits != 3 && bits != 4) return RSQ_ERR_BITS;
+    int st = check_align_args(x, Q, M, x_out, T, D, r, dtype);
+    if (st != RSQ_OK) return st;
+    if (!std::isfinite(eps) || eps < 0.f) return RSQ_ERR_VALUE;
+    if (T == 0) return RSQ_OK;
+    if (!codes || !scales) return RSQ_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales)) return RSQ_ERR_ALIGN;
+    const uint64_t act = uint64_t(T) * uint64_t(D) * uint64_t(elem_bytes(dtype));
+    const Span sx = span(x, act), so = span(x_out, act);
+    const Span sc = span(codes, uint64_t(T) * uint64_t(D) * bits / 8), ss = span(scales, uint64_t(T) * 4);
+    if (overlap(sc, sx) || overlap(sc, so) || overlap(ss, sx) || overlap(ss, so) || overlap(sc, ss) ||
+        overlap(sc, span(Q, uint64_t(D) * r * 4)) || overlap(ss, span(Q, uint64_t(D) * r * 4)) ||
+        overlap(sc, span(M, uint64_t(r) * r * 4)) || overlap(ss, span(M, uint64_t(r) * r * 4)))
+        return RSQ_ERR_ALIAS;
+    return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
+                                            true, static_cast<cudaStream_t>(stream)));
+}
+
+int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *scales, int64_t T,
+              int d, int bits, int dtype, void *stream) {
+    if (bits != 3 && bits != 4) return RSQ_ERR_BITS;
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (m != 1 && m != 12) return RSQ_ERR_UNSUPPORTED;
+    if (T < 0 || d < 16 || d > 32768 || d % 16 != 0 || d % m != 0) return RSQ_ERR_SHAPE;
+    const int n2 = d / m;
+    if (!is_pow2(n2) || n2 < 16 || n2 > 16384) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!x || !signs || !codes || !scales) return RSQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(signs) || !aligned16(codes) || !aligned16(scales)) return RSQ_ERR_ALIGN;
+    const Span sx = span(x, uint64_t(T) * d * elem_bytes(dtype)), sg = span(signs, uint64_t(d));
+    const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * 4);
+    if (overlap(sc, sx) || overlap(sc, sg) || overlap(sc, ss) || overlap(ss, sx) || overlap(ss, sg))
+        return RSQ_ERR_ALIAS;
+    return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+const char *rsq_status_string(int status) {
+    switch (status) {
+        case RSQ_OK: return "RSQ_OK";
+        case RSQ_ERR_NULL: return "RSQ_ERR_NULL: a required pointer is NULL";
+        case RSQ_ERR_SHAPE: return "RSQ_ERR_SHAPE: unsupported or invalid shape";
+        case RSQ_ERR_DTYPE: return "RSQ_ERR_DTYPE: dtype must be RSQ_F32 or RSQ_BF16";
+        case RSQ_ERR_BITS: return "RSQ_ERR_BITS: bits must be 3 or 4";
+        case RSQ_ERR_ALIGN: return "RSQ_ERR_ALIGN: pointers must be 16-byte aligned";
+        case RSQ_ERR_ALIAS: return "RSQ_ERR_ALIAS: buffers overlap (only x_out == x is allowed)";
+        case RSQ_ERR_UNSUPPORTED: return "RSQ_ERR_UNSUPPORTED: configuration not built";
+        case RSQ_ERR_CUDA: return "RSQ_ERR_CUDA: a CUDA call failed (see rsq_last_cuda_error)";
+        case RSQ_ERR_VALUE: return "RSQ_ERR_VALUE: eps must be finite and >= 0";
+        default: return "unknown rsq status";
+    }
+}
+
+int rsq_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t rsq_launch_count(void) { return rsq::g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

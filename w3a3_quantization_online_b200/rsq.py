@@ -1,0 +1,148 @@
+"""Thin Python binding of librsq.so (include/rsq.h): argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels.  PyTorch supplies
+device memory and the current CUDA stream.  There is no CPU fallback: if the
+library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librsq.so")
+
+RSQ_F32, RSQ_BF16 = 0, 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'` "
+        "or `python w3a3_quantization_online_b200/build.py` (the CUDA path has no fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i64, _i32, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+_lib.rsq_residual_align.argtypes = [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.rsq_residual_align.restype = _i32
+_lib.rsq_align_norm_quant.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _i32, _vp]
+_lib.rsq_align_norm_quant.restype = _i32
+_lib.rht_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.rht_quant.restype = _i32
+_lib.rsq_status_string.argtypes = [_i32]
+_lib.rsq_status_string.restype = ctypes.c_char_p
+_lib.rsq_last_cuda_error.argtypes = []
+_lib.rsq_last_cuda_error.restype = _i32
+_lib.rsq_launch_count.argtypes = []
+_lib.rsq_launch_count.restype = ctypes.c_uint64
+
+EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_status_string",
+            "rsq_last_cuda_error", "rsq_launch_count")
+
+
+class RsqError(RuntimeError):
+    def __init__(self, status: int):
+        msg = _lib.rsq_status_string(status).decode()
+        if status == 8:
+            msg += f" (cudaError {int(_lib.rsq_last_cuda_error())})"
+        super().__init__(msg)
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def launch_count() -> int:
+    return int(_lib.rsq_launch_count())
+
+
+def status_string(status: int) -> str:
+    return _lib.rsq_status_string(status).decode()
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise RsqError(status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RSQ_F32
+    if t.dtype == torch.bfloat16:
+        return RSQ_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def rsq_residual_align(x: torch.Tensor, Q: torch.Tensor, M: torch.Tensor,
+                       x_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x_out = x + Q (M (Q^T x)) per row of the T x D activations x (in place if x_out is x)."""
+    _need(x, "x"); _need(Q, "Q", torch.float32); _need(M, "M", torch.float32)
+    T, D = x.shape
+    r = Q.shape[1]
+    if x_out is None:
+        x_out = torch.empty_like(x)
+    _need(x_out, "x_out", x.dtype)
+    _check(_lib.rsq_residual_align(_ptr(x), _ptr(Q), _ptr(M), _ptr(x_out), T, D, r,
+                                   _dtype_code(x), _stream(stream)))
+    return x_out
+
+
+def rsq_align_norm_quant(x: torch.Tensor, Q: torch.Tensor, M: torch.Tensor,
+                         x_out: Optional[torch.Tensor] = None, codes: Optional[torch.Tensor] = None,
+                         scales: Optional[torch.Tensor] = None, bits: int = 4, eps: float = 1e-5,
+                         stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Alignment -> weight-free RMSNorm -> per-token symmetric INT{bits} codes.
+
+    Returns (x_out, codes uint8 T x D*bits/8, scales float32 T)."""
+    _need(x, "x"); _need(Q, "Q", torch.float32); _need(M, "M", torch.float32)
+    T, D = x.shape
+    r = Q.shape[1]
+    if x_out is None:
+        x_out = torch.empty_like(x)
+    if codes is None:
+        codes = torch.empty((T, D * bits // 8), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _need(x_out, "x_out", x.dtype); _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
+    _check(_lib.rsq_align_norm_quant(_ptr(x), _ptr(Q), _ptr(M), _ptr(x_out), _ptr(codes), _ptr(scales),
+                                     T, D, r, bits, float(eps), _dtype_code(x), _stream(stream)))
+    return x_out, codes, scales
+
+
+def rht_quant(x: torch.Tensor, signs: torch.Tensor, m: int = 1, codes: Optional[torch.Tensor] = None,
+              scales: Optional[torch.Tensor] = None, bits: int = 4,
+              stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Randomised Hadamard H_d diag(signs) x / sqrt(d) -> per-token symmetric INT{bits} codes.
+
+    Returns (codes uint8 T x d*bits/8, scales float32 T)."""
+    _need(x, "x"); _need(signs, "signs", torch.int8)
+    T, d = x.shape
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
+    _check(_lib.rht_quant(_ptr(x), _ptr(signs), m, _ptr(codes), _ptr(scales), T, d, bits,
+                          _dtype_code(x), _stream(stream)))
+    return codes, scales

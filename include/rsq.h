@@ -118,6 +118,20 @@ int rsq_last_cuda_error(void);
 /* Number of kernels this library has launched in this process (all threads). */
 uint64_t rsq_launch_count(void);
 
+/* Kernel used by rsq_align_norm_quant: 0 = automatic (tensor-core cluster
+ * kernel for bf16, D in {4096, 8192}, r <= 32; CUDA-core kernel otherwise),
+ * 1 = always the CUDA-core kernel, 2 = only the tensor-core kernel (calls it
+ * cannot serve return RSQ_ERR_UNSUPPORTED).  Process-wide; returns the previous
+ * setting, or -1 for an invalid value.  Both kernels compute the same
+ * function; this exists for testing and measurement. */
+int rsq_select_align_kernel(int which);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device into *status: 0 if no kernel reported a problem, otherwise the
+ * OR of error bits (1 = a bounded wait inside a kernel timed out; that call's
+ * outputs are invalid).  Returns an rsq_status. */
+int rsq_device_status(void *stream, int *status);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,555 @@
+// align_tc.cu -- tensor-core (tcgen05) residual subspace alignment fused with
+// the weight-free RMSNorm and the per-token symmetric quantiser, bf16 I/O.
+//
+// ReSpinQuant paper notes, key design 3: y = Q^T x (D -> r), z = M y,
+// x_out = x + Q z.  Infra Quant II, QuaRot / Method: scale-free RMSNorm in FP32
+// and per-token symmetric absmax quantisation (SpinQuant / Motivation gives
+// alpha = max|X| / (2^(N-1) - 1)).
+//
+// Design (B200, sm_100a):
+//  * A cluster of CS CTAs splits the hidden dimension: CTA c owns columns
+//    [512 c, 512 c + 512) and keeps its 512 x 32 slice of Q resident in shared
+//    memory for the whole persistent kernel.  Every token tile (up to 128 rows)
+//    is read from HBM exactly once by TMA and stays in shared memory until its
+//    x_out and codes are written.
+//  * Both rank-32 contractions run on the 5th-generation tensor cores with fp32
+//    accumulators in TMEM.  x is exact in bf16; Q and z are split into bf16
+//    high and low parts (Q = Q_hi + Q_lo), which keeps the products accurate to
+//    about 2^-16 relative:
+//        y   = x [Q_hi | Q_lo]              (M=128, N=64, K=512 per CTA)
+//        c   = z_hi Q_hi^T + z_hi Q_lo^T + z_lo Q_hi^T   (M=128, N=2x256, K=96)
+//    The same shared-memory Q buffer serves as the MN-major B operand of the
+//    first product and the K-major B operand of the second.
+//  * The partial projections of the CS CTAs are reduced through distributed
+//    shared memory: the CTA that owns 128/CS token rows sums their partials,
+//    applies the r x r matrix M and writes z (split hi/lo) into every CTA's A
+//    operand buffer.  The RMS and absmax statistics are exchanged the same way.
+//  * x_out = x + c is formed in fp32, rounded to bf16 in place in the tile
+//    buffer and written back by TMA; the fp32 value goes back to TMEM, from
+//    which the codes are computed once the row statistics are known.
+// Every mbarrier wait is bounded; a timeout sets a bit in the device status
+// word and the kernel keeps its barrier sequence so that no CTA is left
+// waiting.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rsq {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kTileM = 128;                  // token rows per tile (MMA M)
+constexpr int kCols = 512;                   // hidden columns owned by one CTA
+constexpr int kSlabCols = 64;                // bf16 columns per 128-byte swizzle row
+constexpr int kSlabs = kCols / kSlabCols;    // 8
+constexpr int kSlabBytes = kTileM * 128;     // 16 KB
+constexpr int kXBytes = kSlabs * kSlabBytes; // 128 KB
+constexpr int kQBytes = kCols * 128;         // 64 KB: 512 rows x [Q_hi(32) | Q_lo(32)] bf16
+constexpr int kZBytes = kTileM * 128;        // 16 KB: partial y (fp32) / z hi|lo (bf16), per row
+constexpr int kThreads = 128;
+constexpr int kTmemCols = 512;
+
+struct AlignTcArgs {
+    const float *Q;
+    const float *M;
+    uint8_t *codes;
+    float *scales;
+    int *status;
+    long long T;
+    int D;
+    int r;
+    int rows_per_tile;
+    int tiles_per_cluster;
+    float eps;
+};
+
+template <int CS>
+struct Layout {
+    static constexpr int kTokPerOwner = kTileM / CS;
+    static constexpr int kOffX = 0;
+    static constexpr int kOffQ = kOffX + kXBytes;
+    static constexpr int kOffZ = kOffQ + kQBytes;
+    static constexpr int kOffYred = kOffZ + kZBytes;
+    static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;
+    static constexpr int kOffBar = kOffStat + kTileM * 16;
+    static constexpr int kOffTmem = kOffBar + 16;
+    static constexpr int kBytes = kOffTmem + 16;
+    static constexpr int kSmem = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {  // SWIZZLE_128B chunk position
+    return uint32_t(((chunk ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    return *reinterpret_cast<const uint16_t *>(&h);
+}
+
+__device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+
+template <int CS, int BITS>
+__global__ void __launch_bounds__(kThreads, 1)
+k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xo,
+           const AlignTcArgs p) {
+    using L = Layout<CS>;
+    constexpr int TPO = L::kTokPerOwner;  // token rows reduced by each CTA
+    constexpr int KPT = 32 / CS;          // projection entries per thread in the reduction
+    static_assert(CS * kCols <= 16384 && 32 % CS == 0, "cluster shape");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sx = base + L::kOffX;
+    uint8_t *sq = base + L::kOffQ;
+    uint8_t *sz = base + L::kOffZ;
+    float *syred = reinterpret_cast<float *>(base + L::kOffYred);
+    uint8_t *sstat = base + L::kOffStat;
+    const uint32_t bar_load = smem_u32(base + L::kOffBar);
+    const uint32_t bar_mma = bar_load + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L::kOffTmem);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t crank = cluster_ctarank();
+    const uint32_t cid = cluster_id_x(), ncl = ncluster_x();
+    const int col0 = int(crank) * kCols;
+    const int r = p.r;
+    const int qmax = (1 << (BITS - 1)) - 1;
+    const long long row_bytes = (long long)p.D * BITS / 8;
+    int err = 0;
+
+    if (tid == 0) {
+        mbar_init(bar_load, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_xo);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+
+    // Q slice -> shared memory as [Q_hi | Q_lo] bf16 rows, SWIZZLE_128B.
+    for (int idx = tid; idx < kCols * 8; idx += kThreads) {
+        const int d = idx >> 3, ch = idx & 7;
+        const int j0 = (ch & 3) * 8;
+        const bool lo = ch >= 4;
+        const float *qrow = p.Q + (size_t)(col0 + d) * r;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint16_t h2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int j = j0 + 2 * e + u;
+                const float q = j < r ? __ldg(qrow + j) : 0.f;
+                const uint16_t hi = bf16_bits(q);
+                h2[u] = lo ? bf16_bits(q - bf16_val(hi)) : hi;
+            }
+            w[e] = uint32_t(h2[0]) | (uint32_t(h2[1]) << 16);
+        }
+        *reinterpret_cast<uint4 *>(sq + d * 128 + swz(d, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    cluster_sync();
+
+    const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
+    const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
+    uint32_t ph_load = 0, ph_mma = 0;
+    const int R = p.rows_per_tile;
+
+    auto issue_load = [&](long long t0) {
+        mbar_expect_tx(bar_load, uint32_t(kSlabs * R * 128));
+#pragma unroll
+        for (int s = 0; s < kSlabs; ++s)
+            tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(t0), bar_load);
+    };
+
+    for (int it = 0; it < p.tiles_per_cluster; ++it) {
+        const long long t0 = ((long long)cid + (long long)it * ncl) * R;
+        if (t0 >= p.T) break;  // uniform over the cluster
+        const int nrows = int(p.T - t0 < R ? p.T - t0 : R);
+        if (tid == 0 && it == 0) issue_load(t0);
+
+        // ---- y = x [Q_hi | Q_lo] over this CTA's 512 columns
+        if (!mbar_wait(bar_load, ph_load)) err |= kErrMbarTimeout;
+        ph_load ^= 1;
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < kSlabs; ++s)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint64_t ad = smem_desc_sw128(smem_u32(sx + s * kSlabBytes) + k * 32, 1024);
+                    const uint64_t bd = smem_desc_sw128(smem_u32(sq) + (s * 4 + k) * 2048, 1024);
+                    umma_f16(tmem, ad, bd, idesc_y, (s | k) != 0);
+                }
+            umma_commit(bar_mma);
+        }
+        if (!mbar_wait(bar_mma, ph_mma)) err |= kErrMbarTimeout;
+        ph_mma ^= 1;
+        tc_fence_after();
+        {
+            uint32_t a[32], b[32];
+            tmem_ld32(tmem + lane_base + 0, a);
+            tmem_ld32(tmem + lane_base + 32, b);
+            tmem_wait_ld();
+            uint8_t *prow = sz + tid * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                float4 v;
+                v.x = __uint_as_float(a[4 * c + 0]) + __uint_as_float(b[4 * c + 0]);
+                v.y = __uint_as_float(a[4 * c + 1]) + __uint_as_float(b[4 * c + 1]);
+                v.z = __uint_as_float(a[4 * c + 2]) + __uint_as_float(b[4 * c + 2]);
+                v.w = __uint_as_float(a[4 * c + 3]) + __uint_as_float(b[4 * c + 3]);
+                *reinterpret_cast<float4 *>(prow + swz(tid, c)) = v;
+            }
+        }
+        tc_fence_before();
+        cluster_sync();  // partial projections of all CTAs are visible
+
+        // ---- owner CTA: sum partials of its TPO rows, z = M y, scatter z hi|lo
+        {
+            const int mloc = tid / CS, kq = tid % CS;
+            const int m = int(crank) * TPO + mloc;
+            const uint32_t row_addr = smem_u32(sz + m * 128);
+            float ys[KPT];
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) ys[e] = 0.f;
+            for (int c = 0; c < CS; ++c) {
+                const uint32_t ra = mapa(row_addr, uint32_t(c));
+                if constexpr (KPT == 4) {
+                    const float4 v = ld_dsmem_f4(ra + swz(m, kq));
+                    ys[0] += v.x; ys[1] += v.y; ys[2] += v.z; ys[3] += v.w;
+                } else {
+                    const float2 v = ld_dsmem_f2(ra + swz(m, kq >> 1) + 8 * (kq & 1));
+                    ys[0] += v.x; ys[1] += v.y;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) syred[mloc * 32 + kq * KPT + e] = ys[e];
+            __syncwarp();
+            uint16_t hi[KPT], lo[KPT];
+#pragma unroll
+            for (int e = 0; e < KPT; ++e) {
+                const int j = kq * KPT + e;
+                float acc = 0.f;
+                if (j < r) {
+                    const float *mrow = p.M + (size_t)j * r;
+                    for (int k = 0; k < r; ++k) acc = fmaf(__ldg(mrow + k), syred[mloc * 32 + k], acc);
+                }
+                hi[e] = bf16_bits(acc);
+                lo[e] = bf16_bits(acc - bf16_val(hi[e]));
+            }
+            __syncwarp();
+            for (int c = 0; c < CS; ++c) {
+                const uint32_t ra = mapa(row_addr, uint32_t(c));
+                if constexpr (KPT == 4) {
+                    const uint32_t h01 = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
+                    const uint32_t h23 = uint32_t(hi[2]) | (uint32_t(hi[3]) << 16);
+                    const uint32_t l01 = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
+                    const uint32_t l23 = uint32_t(lo[2]) | (uint32_t(lo[3]) << 16);
+                    st_dsmem_u32x2(ra + swz(m, kq >> 1) + 8 * (kq & 1), h01, h23);
+                    st_dsmem_u32x2(ra + swz(m, 4 + (kq >> 1)) + 8 * (kq & 1), l01, l23);
+                } else {
+                    const uint32_t h01 = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
+                    const uint32_t l01 = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
+                    st_dsmem_u32(ra + swz(m, kq >> 2) + 4 * (kq & 3), h01);
+                    st_dsmem_u32(ra + swz(m, 4 + (kq >> 2)) + 4 * (kq & 3), l01);
+                }
+            }
+        }
+        fence_proxy_async();
+        cluster_sync();  // z of all rows is in every CTA's operand buffer
+
+        // ---- c = z Q^T (hi/lo split) into TMEM columns [0, 512)
+        if (tid == 0) {
+            tc_fence_after();
+            fence_proxy_async();
+            constexpr int kPairs[6][2] = {{0, 0}, {1, 1}, {0, 2}, {1, 3}, {2, 0}, {3, 1}};
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int s = 0; s < 6; ++s) {
+                    const uint64_t ad = smem_desc_sw128(smem_u32(sz) + kPairs[s][0] * 32, 1024);
+                    const uint64_t bd = smem_desc_sw128(smem_u32(sq) + h * 32768 + kPairs[s][1] * 32, 1024);
+                    umma_f16(tmem + h * 256, ad, bd, idesc_c, s != 0);
+                }
+            umma_commit(bar_mma);
+        }
+        if (!mbar_wait(bar_mma, ph_mma)) err |= kErrMbarTimeout;
+        ph_mma ^= 1;
+        tc_fence_after();
+
+        // ---- pass 1: x_out = x + c (fp32 back to TMEM, bf16 in place), statistics
+        double ss = 0.0;
+        float amax = 0.f;
+        {
+            const int m = tid;
+            for (int cb = 0; cb < kCols / 32; ++cb) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + cb * 32, v);
+                tmem_wait_ld();
+                uint8_t *rowp = sx + (cb >> 1) * kSlabBytes + m * 128;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint8_t *cp = rowp + swz(m, (cb & 1) * 4 + q);
+                    const uint4 u = *reinterpret_cast<const uint4 *>(cp);
+                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t o[4];
+                    float s8 = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = __uint_as_float(w[e] << 16);
+                        const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
+                        const float y0 = x0 + __uint_as_float(v[q * 8 + 2 * e]);
+                        const float y1 = x1 + __uint_as_float(v[q * 8 + 2 * e + 1]);
+                        v[q * 8 + 2 * e] = __float_as_uint(y0);
+                        v[q * 8 + 2 * e + 1] = __float_as_uint(y1);
+                        s8 = fmaf(y0, y0, s8);
+                        s8 = fmaf(y1, y1, s8);
+                        amax = fmaxf(amax, fmaxf(fabsf(y0), fabsf(y1)));
+                        o[e] = pack_bf16x2(y0, y1);
+                    }
+                    ss += double(s8);
+                    *reinterpret_cast<uint4 *>(cp) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                tmem_st32(tmem + lane_base + cb * 32, v);
+            }
+            tmem_wait_st();
+            double *st = reinterpret_cast<double *>(sstat + m * 16);
+            st[0] = ss;
+            reinterpret_cast<float *>(sstat + m * 16)[2] = amax;
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        cluster_sync();  // statistics visible; x_out tile complete in shared memory
+
+        if (tid == 0) {
+#pragma unroll
+            for (int s = 0; s < kSlabs; ++s)
+                tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
+            bulk_commit();
+        }
+        // row totals over the cluster (fixed order: deterministic)
+        double ss_t = 0.0;
+        float am_t = 0.f;
+        {
+            const uint32_t sa = smem_u32(sstat + tid * 16);
+            for (int c = 0; c < CS; ++c) {
+                const float4 v = ld_dsmem_f4(mapa(sa, uint32_t(c)));
+                ss_t += __hiloint2double(__float_as_int(v.y), __float_as_int(v.x));
+                am_t = fmaxf(am_t, v.z);
+            }
+        }
+        const float ms = float(ss_t / double(p.D));
+        const float rs = 1.0f / sqrtf(ms + p.eps);
+        const float inv = am_t > 0.f ? float(qmax) / am_t : 0.f;
+        const bool valid = tid < nrows;
+        if (crank == 0 && valid) p.scales[t0 + tid] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+
+        // the tile buffer is free once TMA has read x_out: fetch the next tile
+        if (tid == 0) {
+            bulk_wait_read0();
+            const long long tn = ((long long)cid + (long long)(it + 1) * ncl) * R;
+            if (it + 1 < p.tiles_per_cluster && tn < p.T) issue_load(tn);
+        }
+
+        // ---- pass 2: codes from the fp32 x_out in TMEM
+        {
+            uint8_t *crow = p.codes + (t0 + tid) * row_bytes + (long long)col0 * BITS / 8;
+#pragma unroll 1
+            for (int cb4 = 0; cb4 < kCols / 128; ++cb4) {
+                uint32_t words[BITS * 4];
+#pragma unroll
+                for (int sub = 0; sub < 4; ++sub) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_base + (cb4 * 4 + sub) * 32, v);
+                    tmem_wait_ld();
+                    uint32_t g[4];
+#pragma unroll
+                    for (int gi = 0; gi < 4; ++gi) {
+                        int c[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) c[e] = quant_code(__uint_as_float(v[gi * 8 + e]), inv, qmax);
+                        g[gi] = BITS == 4 ? pack8_int4(c) : pack8_int3(c);
+                    }
+                    if (BITS == 4) {
+#pragma unroll
+                        for (int gi = 0; gi < 4; ++gi) words[sub * 4 + gi] = g[gi];
+                    } else {
+                        words[sub * 3 + 0] = g[0] | (g[1] << 24);
+                        words[sub * 3 + 1] = (g[1] >> 8) | (g[2] << 16);
+                        words[sub * 3 + 2] = (g[2] >> 16) | (g[3] << 8);
+                    }
+                }
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(crow + cb4 * (BITS * 16));
+#pragma unroll
+                    for (int w = 0; w < BITS; ++w)
+                        dst[w] = make_uint4(words[4 * w], words[4 * w + 1], words[4 * w + 2], words[4 * w + 3]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();  // TMEM reads done before the next tile's MMAs
+    }
+
+    if (tid == 0) bulk_wait0();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    if (err && lane == 0) atomicOr(p.status, err);
+    cluster_sync();  // no CTA leaves while a peer may still read its shared memory
+}
+
+// -------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, const void *ptr, long long T, int D, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(T)};
+    const cuuint64_t strides[1] = {cuuint64_t(D) * 2};
+    const cuuint32_t box[2] = {cuuint32_t(kSlabCols), cuuint32_t(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int CS, int BITS>
+struct TcKernel {
+    static int max_clusters[64];
+    static bool configured[64];
+
+    static cudaError_t configure(int dev) {
+        if (configured[dev]) return cudaSuccess;
+        auto kern = k_align_tc<CS, BITS>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Layout<CS>::kSmem);
+        if (e != cudaSuccess) return e;
+        if (CS > 8) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(CS, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = Layout<CS>::kSmem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        max_clusters[dev] = n;
+        configured[dev] = true;
+        return cudaSuccess;
+    }
+
+    static cudaError_t launch(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                              float *scales, long long T, int D, int r, float eps, int *status, cudaStream_t s,
+                              bool *launched) {
+        *launched = false;
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64) return cudaSuccess;
+        e = configure(dev);
+        if (e != cudaSuccess) return e;
+        const int maxcl = max_clusters[dev];
+        if (maxcl < 1) return cudaSuccess;  // cannot co-schedule this cluster shape: caller uses another kernel
+        const long long base_tiles = (T + kTileM - 1) / kTileM;
+        const int ncl = int(base_tiles < maxcl ? base_tiles : maxcl);
+        const int tpc = int((base_tiles + ncl - 1) / ncl);
+        const long long ntiles = (long long)ncl * tpc;
+        const int R = int((T + ntiles - 1) / ntiles);
+        CUtensorMap mx, mxo;
+        if (!make_map(&mx, x, T, D, R) || !make_map(&mxo, x_out, T, D, R)) return cudaErrorInvalidValue;
+        AlignTcArgs a;
+        a.Q = Q;
+        a.M = M;
+        a.codes = codes;
+        a.scales = scales;
+        a.status = status;
+        a.T = T;
+        a.D = D;
+        a.r = r;
+        a.rows_per_tile = R;
+        a.tiles_per_cluster = tpc;
+        a.eps = eps;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(CS * ncl, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = Layout<CS>::kSmem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, k_align_tc<CS, BITS>, mx, mxo, a);
+        if (e == cudaSuccess) {
+            *launched = true;
+            count_launch();
+        }
+        return e;
+    }
+};
+
+template <int CS, int BITS>
+int TcKernel<CS, BITS>::max_clusters[64];
+template <int CS, int BITS>
+bool TcKernel<CS, BITS>::configured[64];
+
+}  // namespace
+
+bool align_tc_supports(int D, int r, int dtype, long long T) {
+    return dtype == 1 && (D == 4096 || D == 8192) && r >= 1 && r <= 32 && T >= 1 && T <= 0x7FFFFFFFLL;
+}
+
+cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                            float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
+                            bool *launched) {
+    int *status = device_status_word();
+    if (!status) return cudaErrorInvalidDevice;
+    if (D == 4096)
+        return bits == 4 ? TcKernel<8, 4>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched)
+                         : TcKernel<8, 3>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched);
+    return bits == 4 ? TcKernel<16, 4>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched)
+                     : TcKernel<16, 3>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched);
+}
+
+}  // namespace rsq

@@ -24,4 +24,16 @@ cudaError_t launch_rht_generic(const void *x, const int8_t *signs, int m, uint8_
                                float *scales, int64_t T, int d, int bits, int dtype,
                                cudaStream_t s);
 
+// Device-side status word of the current device (bits from sm100::kErr*), or
+// nullptr if its address cannot be obtained.
+int *device_status_word();
+
+// Tensor-core alignment + RMSNorm + quantiser (bf16, D in {4096, 8192}, r <= 32).
+bool align_tc_supports(int D, int r, int dtype, long long T);
+// *launched is false (and cudaSuccess returned) when the cluster shape cannot be
+// scheduled on this device; the caller then uses the generic kernel.
+cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                            float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
+                            bool *launched);
+
 }  // namespace rsq

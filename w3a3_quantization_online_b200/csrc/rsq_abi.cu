@@ -13,8 +13,13 @@
 
 namespace rsq {
 
+// Device-side status word: kernels OR error bits into it (bounded waits that
+// timed out); rsq_device_status() reads and clears it.
+__device__ int g_device_status;
+
 namespace {
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 tensor core
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -38,6 +43,17 @@ int num_sms() {
         g_sms[dev] = v;
     }
     return g_sms[dev];
+}
+
+int *device_status_word() {
+    static int *addr[kMaxDevices];
+    const int dev = cur_device();
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
 }
 
 int max_smem_optin() {
@@ -127,6 +143,15 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         overlap(sc, span(Q, uint64_t(D) * r * 4)) || overlap(ss, span(Q, uint64_t(D) * r * 4)) ||
         overlap(sc, span(M, uint64_t(r) * r * 4)) || overlap(ss, span(M, uint64_t(r) * r * 4)))
         return RSQ_ERR_ALIAS;
+    const int which = rsq::g_align_kernel.load(std::memory_order_relaxed);
+    if (which != 1 && rsq::align_tc_supports(D, r, dtype, T)) {
+        bool launched = false;
+        const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, codes, scales, T, D, r, bits, eps,
+                                                   static_cast<cudaStream_t>(stream), &launched);
+        if (e != cudaSuccess) return finish(e);
+        if (launched) return RSQ_OK;
+    }
+    if (which == 2) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
                                             true, static_cast<cudaStream_t>(stream)));
 }
@@ -167,6 +192,22 @@ const char *rsq_status_string(int status) {
 }
 
 int rsq_last_cuda_error(void) { return g_last_cuda_error; }
+
+int rsq_select_align_kernel(int which) {
+    if (which < 0 || which > 2) return -1;
+    return rsq::g_align_kernel.exchange(which);
+}
+
+int rsq_device_status(void *stream, int *status) {
+    if (!status) return RSQ_ERR_NULL;
+    int *word = rsq::device_status_word();
+    if (!word) return finish(cudaErrorInvalidDevice);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) e = cudaMemcpy(status, word, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(word, 0, sizeof(int));
+    return finish(e);
+}
 
 uint64_t rsq_launch_count(void) { return rsq::g_launches.load(std::memory_order_relaxed); }
 

@@ -36,9 +36,15 @@ _lib.rsq_last_cuda_error.argtypes = []
 _lib.rsq_last_cuda_error.restype = _i32
 _lib.rsq_launch_count.argtypes = []
 _lib.rsq_launch_count.restype = ctypes.c_uint64
+_lib.rsq_select_align_kernel.argtypes = [_i32]
+_lib.rsq_select_align_kernel.restype = _i32
+_lib.rsq_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
+_lib.rsq_device_status.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_status_string",
-            "rsq_last_cuda_error", "rsq_launch_count")
+            "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_device_status")
+
+ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE = 0, 1, 2
 
 
 class RsqError(RuntimeError):
@@ -56,6 +62,21 @@ def library() -> ctypes.CDLL:
 
 def launch_count() -> int:
     return int(_lib.rsq_launch_count())
+
+
+def select_align_kernel(which: int) -> int:
+    """0 auto, 1 CUDA-core kernel, 2 tensor-core kernel only; returns the previous setting."""
+    prev = int(_lib.rsq_select_align_kernel(int(which)))
+    if prev < 0:
+        raise ValueError(which)
+    return prev
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word (0 = healthy)."""
+    out = _i32(0)
+    _check(_lib.rsq_device_status(_stream(stream), ctypes.byref(out)))
+    return int(out.value)
 
 
 def status_string(status: int) -> str:

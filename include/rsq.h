@@ -126,6 +126,12 @@ uint64_t rsq_launch_count(void);
  * function; this exists for testing and measurement. */
 int rsq_select_align_kernel(int which);
 
+/* Kernel used by rht_quant: 0 = automatic (warp-per-row kernel for bf16,
+ * d = 4096, m = 1; shared-memory radix-16 kernel otherwise), 1 = always the
+ * radix-16 kernel, 2 = only the specialised kernel (RSQ_ERR_UNSUPPORTED
+ * otherwise).  Process-wide; returns the previous setting, -1 if invalid. */
+int rsq_select_rht_kernel(int which);
+
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device into *status: 0 if no kernel reported a problem, otherwise the
  * OR of error bits (1 = a bounded wait inside a kernel timed out; that call's

@@ -3,7 +3,9 @@
 Tolerances (written here once, used by every parity test):
   * aligned values, float32 I/O: max |gpu - oracle| <= 1e-4 * max|x| per row;
   * aligned values, bf16 I/O:    max |gpu - oracle| <= 4e-3 * max|oracle| per row;
-  * scales: relative error <= 1e-6 (both exactly 0 for an all-zero row);
+  * scales: relative error <= 1e-6 (both exactly 0 for an all-zero row); a
+    scale below the float32 normal range cannot carry that relative precision,
+    so the bound is 1e-6 * scale + 2^-149 (half the float32 subnormal spacing);
   * codes: equal, except +-1 where the oracle's pre-round value v/alpha lies
     within 1e-4 of a rounding tie (|frac(|v/alpha|) - 0.5| < 1e-4); such
     mismatches may number at most 1e-5 of all codes, rounded up to a whole code.
@@ -71,9 +73,11 @@ def check_scales(gpu: np.ndarray, ora: np.ndarray, label: str = "") -> float:
     gpu = np.asarray(gpu, dtype=np.float64)
     zero = ora == 0
     assert np.all(gpu[zero] == 0), f"{label}: nonzero scale on an all-zero row"
-    rel = np.abs(gpu[~zero] - ora[~zero]) / ora[~zero]
+    err = np.abs(gpu[~zero] - ora[~zero])
+    ok = err <= SCALE_REL * ora[~zero] + 2.0 ** -149
+    rel = err / ora[~zero]
     worst = float(rel.max()) if rel.size else 0.0
-    assert worst <= SCALE_REL, f"{label}: scale rel err {worst:.3e} > {SCALE_REL}"
+    assert ok.all(), f"{label}: scale rel err {float(rel[~ok].max()):.3e} > {SCALE_REL}"
     return worst
 
 

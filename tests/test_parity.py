@@ -48,7 +48,7 @@ def run_rht(case):
     x = _to_dev(case.x, case.dtype)
     s = torch.from_numpy(case.signs).to(DEV)
     codes, scales = rsq.rht_quant(x, s, case.m, bits=case.bits)
-    torch.cuda.synchronize()
+    assert rsq.device_status() == 0
     return codes.cpu().numpy(), scales.cpu().numpy()
 
 
@@ -253,6 +253,38 @@ def test_odd_shapes(D, r, dtype, bits):
 def test_rht_shapes(d, m, dtype, bits):
     h = inputs.rht_case(19, d, m, d + m, dtype=dtype, bits=bits, n_outliers=3, outlier_scale=40.0)
     check_rht(h, label=f"d={d} m={m}")
+
+
+def test_rht_kernels_agree_with_the_oracle_at_4096():
+    rsq = _rsq()
+    for which in (rsq.RHT_SPECIALISED, rsq.RHT_GENERIC):
+        prev = rsq.select_rht_kernel(which)
+        try:
+            for T in (1, 7, 600):
+                for bits in (4, 3):
+                    h = inputs.rht_case(T, 4096, 1, 60 + T + bits, dtype="bf16", bits=bits, n_outliers=8,
+                                        outlier_scale=100.0)
+                    check_rht(h, label=f"rht kernel {which} T={T} bits={bits}")
+        finally:
+            rsq.select_rht_kernel(prev)
+
+
+@pytest.mark.parametrize("which", [1, 2])
+def test_tiny_and_zero_rows_rht_4096(which):
+    rsq = _rsq()
+    prev = rsq.select_rht_kernel(which)
+    try:
+        h = inputs.rht_case(6, 4096, 1, 3, dtype="bf16")
+        h.x[1] = 0.0
+        h.x[2] *= np.float32(2.0 ** -120)      # absmax far below 2^-64: rescaled path
+        h.x[3, :] = 0.0
+        h.x[3, 17] = np.float32(2.0 ** -130)   # a single subnormal-range value
+        h.x = inputs.round_to_bf16(h.x)
+        codes, scales = run_rht(h)
+        assert scales[1] == 0 and np.all(codes[1] == 0)
+        check_rht(h, label=f"tiny rows kernel {which}")
+    finally:
+        rsq.select_rht_kernel(prev)
 
 
 def test_residual_align_only_matches_oracle():

@@ -103,12 +103,12 @@ k_align_generic(const typename IO::T *x, const float *__restrict__ Q,
             const double sum = block_sum(double(ss), red_d);
             const float ms = float(sum / double(D));
             const float rs = 1.0f / sqrtf(ms + eps);
-            const float inv = amax > 0.f ? float(qmax) / amax : 0.f;
+            const RowQuant rq = row_quant(amax, qmax);
             uint8_t *crow = codes + t * row_bytes;
             for (int gq = tid; gq < D / 8; gq += blockDim.x) {
                 int c[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) c[k] = quant_code(xr[8 * gq + k], inv, qmax);
+                for (int k = 0; k < 8; ++k) c[k] = quant_code(xr[8 * gq + k], rq, qmax);
                 store_group(crow, gq, bits, c);
             }
             if (tid == 0) scales[t] = amax > 0.f ? (amax * rs) / float(qmax) : 0.f;

@@ -181,7 +181,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         if (tid == 0 && it == 0) issue_load(t0);
 
         // ---- y = x [Q_hi | Q_lo] over this CTA's 512 columns
-        if (!mbar_wait(bar_load, ph_load)) err |= kErrMbarTimeout;
+        if (!mbar_wait(bar_load, ph_load, err != 0)) err |= kErrMbarTimeout;
         ph_load ^= 1;
         if (tid == 0) {
             tc_fence_after();
@@ -195,7 +195,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
             umma_commit(bar_mma);
         }
-        if (!mbar_wait(bar_mma, ph_mma)) err |= kErrMbarTimeout;
+        if (!mbar_wait(bar_mma, ph_mma, err != 0)) err |= kErrMbarTimeout;
         ph_mma ^= 1;
         tc_fence_after();
         {
@@ -286,7 +286,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
             umma_commit(bar_mma);
         }
-        if (!mbar_wait(bar_mma, ph_mma)) err |= kErrMbarTimeout;
+        if (!mbar_wait(bar_mma, ph_mma, err != 0)) err |= kErrMbarTimeout;
         ph_mma ^= 1;
         tc_fence_after();
 
@@ -353,7 +353,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         }
         const float ms = float(ss_t / double(p.D));
         const float rs = 1.0f / sqrtf(ms + p.eps);
-        const float inv = am_t > 0.f ? float(qmax) / am_t : 0.f;
+        const RowQuant rq = row_quant(am_t, qmax);
         const bool valid = tid < nrows;
         if (crank == 0 && valid) p.scales[t0 + tid] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
 
@@ -380,7 +380,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     for (int gi = 0; gi < 4; ++gi) {
                         int c[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) c[e] = quant_code(__uint_as_float(v[gi * 8 + e]), inv, qmax);
+                        for (int e = 0; e < 8; ++e) c[e] = quant_code(__uint_as_float(v[gi * 8 + e]), rq, qmax);
                         g[gi] = BITS == 4 ? pack8_int4(c) : pack8_int3(c);
                     }
                     if (BITS == 4) {

@@ -77,6 +77,25 @@ __device__ __forceinline__ int quant_code(float v, float inv, int qmax) {
     return max(-qmax, min(qmax, c));
 }
 
+// Per-row quantiser constants.  Codes do not depend on a positive row factor,
+// so a row whose absmax is so small that qmax / amax would overflow float32 is
+// quantised after an exact scaling by 2^64 (pre).
+struct RowQuant {
+    float inv;  // qmax / (amax * pre), 0 for an all-zero row
+    float pre;  // 1, or 2^64 for rows with amax < 2^-64
+};
+
+__device__ __forceinline__ RowQuant row_quant(float amax, int qmax) {
+    RowQuant q;
+    q.pre = amax < 0x1p-64f ? 0x1p64f : 1.0f;
+    q.inv = amax > 0.f ? float(qmax) / (amax * q.pre) : 0.f;
+    return q;
+}
+
+__device__ __forceinline__ int quant_code(float v, const RowQuant &q, int qmax) {
+    return quant_code(v * q.pre, q.inv, qmax);
+}
+
 // Pack 8 codes (each in [-qmax, qmax]).
 __device__ __forceinline__ uint32_t pack8_int4(const int (&c)[8]) {
     uint32_t w = 0;

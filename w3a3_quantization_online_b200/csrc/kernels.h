@@ -36,4 +36,9 @@ cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void 
                             float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
                             bool *launched);
 
+// Warp-per-row randomised Hadamard of order 4096 (m = 1, bf16, INT4/INT3).
+bool rht_fast_supports(int d, int m, int dtype, int bits, long long T);
+cudaError_t launch_rht_fast(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
+                            int bits, cudaStream_t s);
+
 }  // namespace rsq

@@ -112,12 +112,12 @@ k_rht_generic(const typename IO::T *__restrict__ x, const int8_t *__restrict__ s
         float mx = 0.f;
         for (int e = tid; e < d; e += blockDim.x) mx = fmaxf(mx, fabsf(v[pidx(e)]));
         const float amax = block_max(mx, red_f);
-        const float inv = amax > 0.f ? float(qmax) / amax : 0.f;
+        const RowQuant rq = row_quant(amax, qmax);
         uint8_t *crow = codes + t * row_bytes;
         for (int g = tid; g < d / 8; g += blockDim.x) {
             int c[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) c[k] = quant_code(v[pidx(8 * g + k)], inv, qmax);
+            for (int k = 0; k < 8; ++k) c[k] = quant_code(v[pidx(8 * g + k)], rq, qmax);
             store_group(crow, g, bits, c);
         }
         if (tid == 0) scales[t] = amax > 0.f ? amax / step_den : 0.f;

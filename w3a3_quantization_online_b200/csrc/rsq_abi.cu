@@ -20,6 +20,7 @@ __device__ int g_device_status;
 namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 tensor core
+std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 specialised
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -171,6 +172,9 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
     const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * 4);
     if (overlap(sc, sx) || overlap(sc, sg) || overlap(sc, ss) || overlap(ss, sx) || overlap(ss, sg))
         return RSQ_ERR_ALIAS;
+    if (rsq::g_rht_kernel.load(std::memory_order_relaxed) != 1 && rsq::rht_fast_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_fast(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
+    if (rsq::g_rht_kernel.load(std::memory_order_relaxed) == 2) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
                                           static_cast<cudaStream_t>(stream)));
 }
@@ -196,6 +200,11 @@ int rsq_last_cuda_error(void) { return g_last_cuda_error; }
 int rsq_select_align_kernel(int which) {
     if (which < 0 || which > 2) return -1;
     return rsq::g_align_kernel.exchange(which);
+}
+
+int rsq_select_rht_kernel(int which) {
+    if (which < 0 || which > 2) return -1;
+    return rsq::g_rht_kernel.exchange(which);
 }
 
 int rsq_device_status(void *stream, int *status) {

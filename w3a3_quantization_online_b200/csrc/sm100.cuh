@@ -13,9 +13,9 @@ namespace sm100 {
 // Error bits a kernel reports through the device-side status word.
 enum : int { kErrMbarTimeout = 1 };
 
-// Upper bound of try_wait polls before a wait is declared failed (each poll can
-// itself suspend the thread for a while, so this bounds the wait to seconds).
-constexpr uint32_t kMaxPolls = 1u << 24;
+// A wait that has not completed after this many nanoseconds of %globaltimer is
+// declared failed.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -46,13 +46,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: returns false (and the caller records an error) if the phase
-// never completes.  The caller keeps executing the same control flow so that
-// cluster barriers stay matched.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false if the phase has not
+// completed within kWaitLimitNs, or at once if `failed` is already set (after a
+// first failure a kernel stops waiting, so it ends quickly).  The caller keeps
+// executing the same control flow so that cluster barriers stay matched, and
+// reports the failure through the device status word.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool failed = false) {
+    if (failed) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
 }
 
 // ---------------------------------------------------------------- proxies
@@ -66,6 +79,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
 }
 

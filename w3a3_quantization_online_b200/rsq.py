@@ -38,13 +38,16 @@ _lib.rsq_launch_count.argtypes = []
 _lib.rsq_launch_count.restype = ctypes.c_uint64
 _lib.rsq_select_align_kernel.argtypes = [_i32]
 _lib.rsq_select_align_kernel.restype = _i32
+_lib.rsq_select_rht_kernel.argtypes = [_i32]
+_lib.rsq_select_rht_kernel.restype = _i32
 _lib.rsq_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.rsq_device_status.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_status_string",
-            "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_device_status")
+            "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status")
 
 ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE = 0, 1, 2
+RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED = 0, 1, 2
 
 
 class RsqError(RuntimeError):
@@ -67,6 +70,14 @@ def launch_count() -> int:
 def select_align_kernel(which: int) -> int:
     """0 auto, 1 CUDA-core kernel, 2 tensor-core kernel only; returns the previous setting."""
     prev = int(_lib.rsq_select_align_kernel(int(which)))
+    if prev < 0:
+        raise ValueError(which)
+    return prev
+
+
+def select_rht_kernel(which: int) -> int:
+    """0 auto, 1 radix-16 shared-memory kernel, 2 specialised kernel only; returns the previous setting."""
+    prev = int(_lib.rsq_select_rht_kernel(int(which)))
     if prev < 0:
         raise ValueError(which)
     return prev

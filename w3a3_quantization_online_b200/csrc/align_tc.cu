@@ -50,8 +50,11 @@ constexpr int kSlabBytes = kTileM * 128;     // 16 KB
 constexpr int kXBytes = kSlabs * kSlabBytes; // 128 KB
 constexpr int kQBytes = kCols * 128;         // 64 KB: 512 rows x [Q_hi(32) | Q_lo(32)] bf16
 constexpr int kZBytes = kTileM * 128;        // 16 KB: partial y (fp32) / z hi|lo (bf16), per row
-constexpr int kThreads = 128;
+constexpr int kConsumerWarps = 8;             // two warps per TMEM lane quadrant
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kThreads = kConsumers;
 constexpr int kTmemCols = 512;
+constexpr int kHalfCols = kCols / 2;           // columns per consumer warp group
 
 struct AlignTcArgs {
     const float *Q;
@@ -73,10 +76,12 @@ struct Layout {
     static constexpr int kOffX = 0;
     static constexpr int kOffQ = kOffX + kXBytes;
     static constexpr int kOffZ = kOffQ + kQBytes;
-    static constexpr int kOffYred = kOffZ + kZBytes;
-    static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;
-    static constexpr int kOffBar = kOffStat + kTileM * 16;
-    static constexpr int kOffTmem = kOffBar + 16;
+    static constexpr int kOffM = kOffZ + kZBytes;                       // M^T, 32 x 32 fp32, zero padded
+    static constexpr int kOffYred = kOffM + 32 * 32 * 4;
+    static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;  // [2 halves][128 rows] x 16 B
+    static constexpr int kOffBar = kOffStat + 2 * kTileM * 16;
+    static constexpr int kNumBars = 5;  // load, y, c0, c1, x_out ready
+    static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffTmem + 16;
     static constexpr int kSmem = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -92,24 +97,74 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
+// x_out = x + c for one 32-column block of row m: updates the fp32 values in
+// v (TMEM copy), writes bf16 x_out in place over x, accumulates the sum of
+// squares (pairs, fp32) and the absmax (four independent partial maxima).
+__device__ __forceinline__ void xout_block(uint32_t (&v)[32], uint8_t *rowp, int m, int chunk0, float2 &s2,
+                                           float (&am)[4]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint8_t *cp = rowp + swz(m, chunk0 + q);
+        const uint4 u = *reinterpret_cast<const uint4 *>(cp);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 xv = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xFFFF0000u));
+            const float2 cv = make_float2(__uint_as_float(v[q * 8 + 2 * e]), __uint_as_float(v[q * 8 + 2 * e + 1]));
+            const float2 y = add2(xv, cv);
+            v[q * 8 + 2 * e] = __float_as_uint(y.x);
+            v[q * 8 + 2 * e + 1] = __float_as_uint(y.y);
+            s2 = fma2(y, y, s2);
+            am[e] = fmaxf(am[e], fmaxf(fabsf(y.x), fabsf(y.y)));
+            o[e] = pack_bf16x2(y.x, y.y);
+        }
+        *reinterpret_cast<uint4 *>(cp) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// Codes of one 32-column block (INT4: 4 words, INT3: 3 words).
+template <int BITS>
+__device__ __forceinline__ void code_block(const uint32_t (&v)[32], const RowQuant &rq, bool scaled,
+                                           uint32_t *words) {
+    uint32_t g[4];
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[gi * 8 + e]);
+        g[gi] = pack8_fast<BITS>(f, rq.inv, rq.pre, scaled);
+    }
+    if (BITS == 4) {
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) words[gi] = g[gi];
+    } else {
+        words[0] = g[0] | (g[1] << 24);
+        words[1] = (g[1] >> 8) | (g[2] << 16);
+        words[2] = (g[2] >> 16) | (g[3] << 8);
+    }
+}
+
 template <int CS, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
 k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xo,
            const AlignTcArgs p) {
     using L = Layout<CS>;
-    constexpr int TPO = L::kTokPerOwner;  // token rows reduced by each CTA
-    constexpr int KPT = 32 / CS;          // projection entries per thread in the reduction
-    static_assert(CS * kCols <= 16384 && 32 % CS == 0, "cluster shape");
+    constexpr int TPO = L::kTokPerOwner;    // token rows reduced by each CTA
+    constexpr int KPT = 32 * TPO / kConsumers;  // projection entries per thread in the reduction
+    constexpr int TPT = 32 / KPT;           // threads per token row in the reduction
+    static_assert(CS * kCols <= 16384 && (KPT == 1 || KPT == 2) && TPT <= 32, "cluster shape");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sx = base + L::kOffX;
     uint8_t *sq = base + L::kOffQ;
     uint8_t *sz = base + L::kOffZ;
+    float *sm = reinterpret_cast<float *>(base + L::kOffM);
     float *syred = reinterpret_cast<float *>(base + L::kOffYred);
     uint8_t *sstat = base + L::kOffStat;
     const uint32_t bar_load = smem_u32(base + L::kOffBar);
-    const uint32_t bar_mma = bar_load + 8;
+    const uint32_t bar_y = bar_load + 8, bar_c0 = bar_load + 16, bar_c1 = bar_load + 24, bar_xo = bar_load + 32;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L::kOffTmem);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -119,21 +174,27 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     const int r = p.r;
     const int qmax = (1 << (BITS - 1)) - 1;
     const long long row_bytes = (long long)p.D * BITS / 8;
+    const int R = p.rows_per_tile;
     int err = 0;
 
     if (tid == 0) {
         mbar_init(bar_load, 1);
-        mbar_init(bar_mma, 1);
+        mbar_init(bar_y, 1);
+        mbar_init(bar_c0, 1);
+        mbar_init(bar_c1, 1);
+        mbar_init(bar_xo, kConsumers);
         fence_mbar_init();
-        prefetch_tmap(&tm_x);
-        prefetch_tmap(&tm_xo);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
+    if (tid == 32) {
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_xo);
+    }
 
-    // Q slice -> shared memory as [Q_hi | Q_lo] bf16 rows, SWIZZLE_128B.
+    // Q slice -> shared memory as [Q_hi | Q_lo] bf16 rows, SWIZZLE_128B; M -> 32x32 fp32.
     for (int idx = tid; idx < kCols * 8; idx += kThreads) {
         const int d = idx >> 3, ch = idx & 7;
         const int j0 = (ch & 3) * 8;
@@ -154,257 +215,275 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         }
         *reinterpret_cast<uint4 *>(sq + d * 128 + swz(d, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    fence_proxy_async();
+    for (int idx = tid; idx < 32 * 32; idx += kThreads) {  // sm[k][j] = M[j][k]
+        const int k = idx >> 5, j = idx & 31;
+        sm[idx] = (j < r && k < r) ? __ldg(p.M + j * r + k) : 0.f;
+    }
+    fence_proxy_async_cta();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
     cluster_sync();
 
-    const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
-    const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
-    uint32_t ph_load = 0, ph_mma = 0;
-    const int R = p.rows_per_tile;
+    auto tile_t0 = [&](int it) { return ((long long)cid + (long long)it * ncl) * R; };
 
-    auto issue_load = [&](long long t0) {
-        mbar_expect_tx(bar_load, uint32_t(kSlabs * R * 128));
-#pragma unroll
-        for (int s = 0; s < kSlabs; ++s)
-            tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(t0), bar_load);
-    };
-
-    for (int it = 0; it < p.tiles_per_cluster; ++it) {
-        const long long t0 = ((long long)cid + (long long)it * ncl) * R;
-        if (t0 >= p.T) break;  // uniform over the cluster
-        const int nrows = int(p.T - t0 < R ? p.T - t0 : R);
-        if (tid == 0 && it == 0) issue_load(t0);
-
-        // ---- y = x [Q_hi | Q_lo] over this CTA's 512 columns
-        if (!mbar_wait(bar_load, ph_load, err != 0)) err |= kErrMbarTimeout;
-        ph_load ^= 1;
-        if (tid == 0) {
-            tc_fence_after();
+    {
+        auto issue_load = [&](long long t0) {  // thread 0 only
+            mbar_expect_tx(bar_load, uint32_t(kSlabs * R * 128));
 #pragma unroll
             for (int s = 0; s < kSlabs; ++s)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t ad = smem_desc_sw128(smem_u32(sx + s * kSlabBytes) + k * 32, 1024);
-                    const uint64_t bd = smem_desc_sw128(smem_u32(sq) + (s * 4 + k) * 2048, 1024);
-                    umma_f16(tmem, ad, bd, idesc_y, (s | k) != 0);
-                }
-            umma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, ph_mma, err != 0)) err |= kErrMbarTimeout;
-        ph_mma ^= 1;
-        tc_fence_after();
-        {
-            uint32_t a[32], b[32];
-            tmem_ld32(tmem + lane_base + 0, a);
-            tmem_ld32(tmem + lane_base + 32, b);
-            tmem_wait_ld();
-            uint8_t *prow = sz + tid * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                float4 v;
-                v.x = __uint_as_float(a[4 * c + 0]) + __uint_as_float(b[4 * c + 0]);
-                v.y = __uint_as_float(a[4 * c + 1]) + __uint_as_float(b[4 * c + 1]);
-                v.z = __uint_as_float(a[4 * c + 2]) + __uint_as_float(b[4 * c + 2]);
-                v.w = __uint_as_float(a[4 * c + 3]) + __uint_as_float(b[4 * c + 3]);
-                *reinterpret_cast<float4 *>(prow + swz(tid, c)) = v;
-            }
-        }
-        tc_fence_before();
-        cluster_sync();  // partial projections of all CTAs are visible
+                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(t0), bar_load);
+        };
+        uint32_t ph_xo = 0;
+        // ------------------------------------------------ consumer warps
+        const int quad = warp & 3, half = warp >> 2;
+        const int m = quad * 32 + lane;  // tile row == TMEM lane
+        const uint32_t lane_base = uint32_t(quad * 32) << 16;
+        const uint32_t tcol = uint32_t(half * kHalfCols);
+        const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
+        const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
+        uint32_t ph = 0;  // every consumer barrier completes once per tile
 
-        // ---- owner CTA: sum partials of its TPO rows, z = M y, scatter z hi|lo
-        {
-            const int mloc = tid / CS, kq = tid % CS;
-            const int m = int(crank) * TPO + mloc;
-            const uint32_t row_addr = smem_u32(sz + m * 128);
-            float ys[KPT];
-#pragma unroll
-            for (int e = 0; e < KPT; ++e) ys[e] = 0.f;
-            for (int c = 0; c < CS; ++c) {
-                const uint32_t ra = mapa(row_addr, uint32_t(c));
-                if constexpr (KPT == 4) {
-                    const float4 v = ld_dsmem_f4(ra + swz(m, kq));
-                    ys[0] += v.x; ys[1] += v.y; ys[2] += v.z; ys[3] += v.w;
-                } else {
-                    const float2 v = ld_dsmem_f2(ra + swz(m, kq >> 1) + 8 * (kq & 1));
-                    ys[0] += v.x; ys[1] += v.y;
-                }
-            }
-#pragma unroll
-            for (int e = 0; e < KPT; ++e) syred[mloc * 32 + kq * KPT + e] = ys[e];
-            __syncwarp();
-            uint16_t hi[KPT], lo[KPT];
-#pragma unroll
-            for (int e = 0; e < KPT; ++e) {
-                const int j = kq * KPT + e;
-                float acc = 0.f;
-                if (j < r) {
-                    const float *mrow = p.M + (size_t)j * r;
-                    for (int k = 0; k < r; ++k) acc = fmaf(__ldg(mrow + k), syred[mloc * 32 + k], acc);
-                }
-                hi[e] = bf16_bits(acc);
-                lo[e] = bf16_bits(acc - bf16_val(hi[e]));
-            }
-            __syncwarp();
-            for (int c = 0; c < CS; ++c) {
-                const uint32_t ra = mapa(row_addr, uint32_t(c));
-                if constexpr (KPT == 4) {
-                    const uint32_t h01 = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
-                    const uint32_t h23 = uint32_t(hi[2]) | (uint32_t(hi[3]) << 16);
-                    const uint32_t l01 = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
-                    const uint32_t l23 = uint32_t(lo[2]) | (uint32_t(lo[3]) << 16);
-                    st_dsmem_u32x2(ra + swz(m, kq >> 1) + 8 * (kq & 1), h01, h23);
-                    st_dsmem_u32x2(ra + swz(m, 4 + (kq >> 1)) + 8 * (kq & 1), l01, l23);
-                } else {
-                    const uint32_t h01 = uint32_t(hi[0]) | (uint32_t(hi[1]) << 16);
-                    const uint32_t l01 = uint32_t(lo[0]) | (uint32_t(lo[1]) << 16);
-                    st_dsmem_u32(ra + swz(m, kq >> 2) + 4 * (kq & 3), h01);
-                    st_dsmem_u32(ra + swz(m, 4 + (kq >> 2)) + 4 * (kq & 3), l01);
-                }
-            }
-        }
-        fence_proxy_async();
-        cluster_sync();  // z of all rows is in every CTA's operand buffer
+        for (int it = 0; it < p.tiles_per_cluster; ++it) {
+            const long long t0 = tile_t0(it);
+            if (t0 >= p.T) break;
+            const int nrows = int(p.T - t0 < R ? p.T - t0 : R);
+            if (tid == 0 && it == 0) issue_load(t0);
 
-        // ---- c = z Q^T (hi/lo split) into TMEM columns [0, 512)
-        if (tid == 0) {
-            tc_fence_after();
-            fence_proxy_async();
-            constexpr int kPairs[6][2] = {{0, 0}, {1, 1}, {0, 2}, {1, 3}, {2, 0}, {3, 1}};
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                for (int s = 0; s < 6; ++s) {
-                    const uint64_t ad = smem_desc_sw128(smem_u32(sz) + kPairs[s][0] * 32, 1024);
-                    const uint64_t bd = smem_desc_sw128(smem_u32(sq) + h * 32768 + kPairs[s][1] * 32, 1024);
-                    umma_f16(tmem + h * 256, ad, bd, idesc_c, s != 0);
-                }
-            umma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, ph_mma, err != 0)) err |= kErrMbarTimeout;
-        ph_mma ^= 1;
-        tc_fence_after();
-
-        // ---- pass 1: x_out = x + c (fp32 back to TMEM, bf16 in place), statistics
-        double ss = 0.0;
-        float amax = 0.f;
-        {
-            const int m = tid;
-            for (int cb = 0; cb < kCols / 32; ++cb) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_base + cb * 32, v);
-                tmem_wait_ld();
-                uint8_t *rowp = sx + (cb >> 1) * kSlabBytes + m * 128;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint8_t *cp = rowp + swz(m, (cb & 1) * 4 + q);
-                    const uint4 u = *reinterpret_cast<const uint4 *>(cp);
-                    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-                    uint32_t o[4];
-                    float s8 = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = __uint_as_float(w[e] << 16);
-                        const float x1 = __uint_as_float(w[e] & 0xFFFF0000u);
-                        const float y0 = x0 + __uint_as_float(v[q * 8 + 2 * e]);
-                        const float y1 = x1 + __uint_as_float(v[q * 8 + 2 * e + 1]);
-                        v[q * 8 + 2 * e] = __float_as_uint(y0);
-                        v[q * 8 + 2 * e + 1] = __float_as_uint(y1);
-                        s8 = fmaf(y0, y0, s8);
-                        s8 = fmaf(y1, y1, s8);
-                        amax = fmaxf(amax, fmaxf(fabsf(y0), fabsf(y1)));
-                        o[e] = pack_bf16x2(y0, y1);
-                    }
-                    ss += double(s8);
-                    *reinterpret_cast<uint4 *>(cp) = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-                tmem_st32(tmem + lane_base + cb * 32, v);
-            }
-            tmem_wait_st();
-            double *st = reinterpret_cast<double *>(sstat + m * 16);
-            st[0] = ss;
-            reinterpret_cast<float *>(sstat + m * 16)[2] = amax;
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        cluster_sync();  // statistics visible; x_out tile complete in shared memory
-
-        if (tid == 0) {
-#pragma unroll
-            for (int s = 0; s < kSlabs; ++s)
-                tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
-            bulk_commit();
-        }
-        // row totals over the cluster (fixed order: deterministic)
-        double ss_t = 0.0;
-        float am_t = 0.f;
-        {
-            const uint32_t sa = smem_u32(sstat + tid * 16);
-            for (int c = 0; c < CS; ++c) {
-                const float4 v = ld_dsmem_f4(mapa(sa, uint32_t(c)));
-                ss_t += __hiloint2double(__float_as_int(v.y), __float_as_int(v.x));
-                am_t = fmaxf(am_t, v.z);
-            }
-        }
-        const float ms = float(ss_t / double(p.D));
-        const float rs = 1.0f / sqrtf(ms + p.eps);
-        const RowQuant rq = row_quant(am_t, qmax);
-        const bool valid = tid < nrows;
-        if (crank == 0 && valid) p.scales[t0 + tid] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
-
-        // the tile buffer is free once TMA has read x_out: fetch the next tile
-        if (tid == 0) {
-            bulk_wait_read0();
-            const long long tn = ((long long)cid + (long long)(it + 1) * ncl) * R;
-            if (it + 1 < p.tiles_per_cluster && tn < p.T) issue_load(tn);
-        }
-
-        // ---- pass 2: codes from the fp32 x_out in TMEM
-        {
-            uint8_t *crow = p.codes + (t0 + tid) * row_bytes + (long long)col0 * BITS / 8;
+            // ---- y = x [Q_hi | Q_lo] over this CTA's 512 columns
+            if (!mbar_wait(bar_load, ph, err != 0)) err |= kErrMbarTimeout;
+            if (tid == 0) {
+                tc_fence_after();
+                // descriptors advance by 16-byte units in their start-address field
+                const uint64_t ad0 = smem_desc_sw128(smem_u32(sx), 1024);
+                const uint64_t bd0 = smem_desc_sw128(smem_u32(sq), 1024);
 #pragma unroll 1
-            for (int cb4 = 0; cb4 < kCols / 128; ++cb4) {
-                uint32_t words[BITS * 4];
-#pragma unroll
-                for (int sub = 0; sub < 4; ++sub) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_base + (cb4 * 4 + sub) * 32, v);
-                    tmem_wait_ld();
-                    uint32_t g[4];
-#pragma unroll
-                    for (int gi = 0; gi < 4; ++gi) {
-                        int c[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) c[e] = quant_code(__uint_as_float(v[gi * 8 + e]), rq, qmax);
-                        g[gi] = BITS == 4 ? pack8_int4(c) : pack8_int3(c);
-                    }
-                    if (BITS == 4) {
-#pragma unroll
-                        for (int gi = 0; gi < 4; ++gi) words[sub * 4 + gi] = g[gi];
-                    } else {
-                        words[sub * 3 + 0] = g[0] | (g[1] << 24);
-                        words[sub * 3 + 1] = (g[1] >> 8) | (g[2] << 16);
-                        words[sub * 3 + 2] = (g[2] >> 16) | (g[3] << 8);
-                    }
+                for (int i = 0; i < kSlabs * 4; ++i) {  // K = 512 in steps of 16
+                    const uint32_t aoff = uint32_t((i >> 2) * kSlabBytes + (i & 3) * 32) >> 4;
+                    const uint32_t boff = uint32_t(i * 2048) >> 4;
+                    umma_f16(tmem, ad0 + aoff, bd0 + boff, idesc_y, i != 0);
                 }
-                if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(crow + cb4 * (BITS * 16));
+                umma_commit(bar_y);
+            }
+            if (!mbar_wait(bar_y, ph, err != 0)) err |= kErrMbarTimeout;
+            tc_fence_after();
+            if (half == 0) {
+                uint32_t a[32], b[32];
+                tmem_ld32(tmem + lane_base + 0, a);
+                tmem_ld32(tmem + lane_base + 32, b);
+                tmem_wait_ld();
+                uint8_t *prow = sz + m * 128;
 #pragma unroll
-                    for (int w = 0; w < BITS; ++w)
-                        dst[w] = make_uint4(words[4 * w], words[4 * w + 1], words[4 * w + 2], words[4 * w + 3]);
+                for (int c = 0; c < 8; ++c) {
+                    float4 v;
+                    v.x = __uint_as_float(a[4 * c + 0]) + __uint_as_float(b[4 * c + 0]);
+                    v.y = __uint_as_float(a[4 * c + 1]) + __uint_as_float(b[4 * c + 1]);
+                    v.z = __uint_as_float(a[4 * c + 2]) + __uint_as_float(b[4 * c + 2]);
+                    v.w = __uint_as_float(a[4 * c + 3]) + __uint_as_float(b[4 * c + 3]);
+                    *reinterpret_cast<float4 *>(prow + swz(m, c)) = v;
                 }
             }
+            tc_fence_before();
+            cluster_sync();  // #1 partial projections of all CTAs are visible
+
+            // ---- owner CTA: sum partials of its TPO rows, z = M y, scatter z hi|lo
+            {
+                const int mloc = tid / TPT, kq = tid % TPT;
+                const int mo = int(crank) * TPO + mloc;
+                const uint32_t row_addr = smem_u32(sz + mo * 128);
+                float ys[KPT];
+                if constexpr (KPT == 2) {
+                    float2 pv[CS];
+#pragma unroll
+                    for (int c = 0; c < CS; ++c)
+                        pv[c] = ld_dsmem_f2(mapa(row_addr, uint32_t(c)) + swz(mo, kq >> 1) + 8 * (kq & 1));
+                    ys[0] = 0.f;
+                    ys[1] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < CS; ++c) {
+                        ys[0] += pv[c].x;
+                        ys[1] += pv[c].y;
+                    }
+                } else {
+                    float pv[CS];
+#pragma unroll
+                    for (int c = 0; c < CS; ++c)
+                        pv[c] = ld_dsmem_f32(mapa(row_addr, uint32_t(c)) + swz(mo, kq >> 2) + 4 * (kq & 3));
+                    ys[0] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < CS; ++c) ys[0] += pv[c];
+                }
+#pragma unroll
+                for (int e = 0; e < KPT; ++e) syred[mloc * 32 + kq * KPT + e] = ys[e];
+                __syncwarp();
+                uint16_t hi[KPT], lo[KPT];
+#pragma unroll
+                for (int e = 0; e < KPT; ++e) {
+                    const int j = kq * KPT + e;
+                    const float *yv = syred + mloc * 32;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) acc = fmaf(sm[k * 32 + j], yv[k], acc);
+                    hi[e] = bf16_bits(acc);
+                    lo[e] = bf16_bits(acc - bf16_val(hi[e]));
+                }
+                __syncwarp();
+#pragma unroll
+                for (int c = 0; c < CS; ++c) {
+                    const uint32_t ra = mapa(row_addr, uint32_t(c));
+                    if constexpr (KPT == 2) {
+                        st_dsmem_u32(ra + swz(mo, kq >> 2) + 4 * (kq & 3), uint32_t(hi[0]) | (uint32_t(hi[1]) << 16));
+                        st_dsmem_u32(ra + swz(mo, 4 + (kq >> 2)) + 4 * (kq & 3),
+                                     uint32_t(lo[0]) | (uint32_t(lo[1]) << 16));
+                    } else {
+                        st_dsmem_u16(ra + swz(mo, kq >> 3) + 2 * (kq & 7), hi[0]);
+                        st_dsmem_u16(ra + swz(mo, 4 + (kq >> 3)) + 2 * (kq & 7), lo[0]);
+                    }
+                }
+            }
+            fence_proxy_async();
+            cluster_sync();  // #2 z of all rows is in every CTA's operand buffer
+
+            // ---- c = z Q^T (hi/lo split): half h into TMEM columns [256 h, 256 h + 256)
+            if (tid == 0) {
+                tc_fence_after();
+                fence_proxy_async();
+                // (A K-step, B K-step) pairs: z_hi Q_hi^T, z_hi Q_lo^T, z_lo Q_hi^T; K-steps of 16
+                // columns are 32 bytes apart inside the 128-byte swizzled rows
+                const uint64_t ad0 = smem_desc_sw128(smem_u32(sz), 1024);
+                const uint64_t bd0 = smem_desc_sw128(smem_u32(sq), 1024);
+                const uint64_t pairs = 0x130231201100ull;  // byte s = (b << 4) | a: (0,0) (1,1) (0,2) (1,3) (2,0) (3,1)
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll 1
+                    for (int s = 0; s < 6; ++s) {
+                        const uint32_t ka = uint32_t(pairs >> (8 * s)) & 0xF, kb = uint32_t(pairs >> (8 * s + 4)) & 0xF;
+                        umma_f16(tmem + h * kHalfCols, ad0 + ((ka * 32) >> 4),
+                                 bd0 + ((uint32_t(h) * 32768 + kb * 32) >> 4), idesc_c, s != 0);
+                    }
+                    umma_commit(h == 0 ? bar_c0 : bar_c1);
+                }
+            }
+            if (!mbar_wait(half == 0 ? bar_c0 : bar_c1, ph, err != 0)) err |= kErrMbarTimeout;
+            tc_fence_after();
+
+            // ---- pass 1: x_out = x + c over this warp's 256 columns (TMEM loads pipelined:
+            // the load of the next 32-column block overlaps the arithmetic of the current one)
+            double ss = 0.0;
+            float amax = 0.f;
+            {
+                float2 s2 = make_float2(0.f, 0.f);
+                float am[4] = {0.f, 0.f, 0.f, 0.f};
+                constexpr int kBlocks = kHalfCols / 32;
+                uint32_t va[32], vb[32];
+                const uint32_t taddr = tmem + lane_base + tcol;
+                uint8_t *xbase = sx + m * 128;
+                tmem_ld32(taddr, va);
+                tmem_wait_ld();
+#pragma unroll 1
+                for (int b = 0; b < kBlocks; b += 2) {
+                    const int cb = half * kBlocks + b;  // 32-column block within the CTA slice
+                    tmem_wait_st();
+                    tmem_ld32(taddr + (b + 1) * 32, vb);
+                    xout_block(va, xbase + (cb >> 1) * kSlabBytes, m, (cb & 1) * 4, s2, am);
+                    tmem_st32(taddr + b * 32, va);
+                    tmem_wait_ld();
+                    tmem_wait_st();
+                    if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
+                    xout_block(vb, xbase + ((cb + 1) >> 1) * kSlabBytes, m, ((cb + 1) & 1) * 4, s2, am);
+                    tmem_st32(taddr + (b + 1) * 32, vb);
+                    tmem_wait_ld();
+                    // fold the fp32 pair sums of these 64 columns into float64
+                    ss += double(s2.x) + double(s2.y);
+                    s2 = make_float2(0.f, 0.f);
+                }
+                tmem_wait_st();
+                amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
+            }
+            fence_proxy_async_cta();
+            mbar_arrive(bar_xo);  // this thread's part of x_out is in the tile buffer
+            if (tid == 0) {       // write x_out back as soon as the whole tile is in place
+                if (!mbar_wait(bar_xo, ph_xo, err != 0)) err |= kErrMbarTimeout;
+#pragma unroll
+                for (int s = 0; s < kSlabs; ++s)
+                    tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
+                bulk_commit();
+            }
+            ph_xo ^= 1;
+            {
+                uint8_t *st = sstat + (half * kTileM + m) * 16;
+                reinterpret_cast<double *>(st)[0] = ss;
+                reinterpret_cast<float *>(st)[2] = amax;
+            }
+            tc_fence_before();
+            cluster_sync();  // #3 statistics visible
+
+            // row totals over the cluster and both halves (fixed order: deterministic)
+            double ss_t = 0.0;
+            float am_t = 0.f;
+            {
+                float4 sv[2 * CS];
+#pragma unroll
+                for (int c = 0; c < CS; ++c)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        sv[2 * c + h] = ld_dsmem_f4(mapa(smem_u32(sstat + (h * kTileM + m) * 16), uint32_t(c)));
+#pragma unroll
+                for (int i = 0; i < 2 * CS; ++i) {
+                    ss_t += __hiloint2double(__float_as_int(sv[i].y), __float_as_int(sv[i].x));
+                    am_t = fmaxf(am_t, sv[i].z);
+                }
+            }
+            const float ms = float(ss_t / double(p.D));
+            const float rs = 1.0f / sqrtf(ms + p.eps);
+            const RowQuant rq = row_quant(am_t, qmax);
+            const bool scaled = rq.pre != 1.0f;
+            const bool valid = m < nrows;
+            if (crank == 0 && half == 0 && valid) p.scales[t0 + m] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+            if (tid == 0) {  // the tile buffer is free once TMA has read x_out: fetch the next tile
+                bulk_wait_read0();
+                const long long tn = tile_t0(it + 1);
+                if (it + 1 < p.tiles_per_cluster && tn < p.T) issue_load(tn);
+            }
+
+            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined)
+            {
+                constexpr int kBlocks = kHalfCols / 32;
+                uint8_t *crow = p.codes + (t0 + m) * row_bytes + (long long)(col0 + half * kHalfCols) * BITS / 8;
+                const uint32_t taddr = tmem + lane_base + tcol;
+                uint32_t va[32], vb[32];
+                tmem_ld32(taddr, va);
+                tmem_wait_ld();
+#pragma unroll 1
+                for (int b = 0; b < kBlocks; b += 2) {
+                    uint32_t words[2 * BITS];
+                    tmem_ld32(taddr + (b + 1) * 32, vb);
+                    code_block<BITS>(va, rq, scaled, words);
+                    tmem_wait_ld();
+                    if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
+                    code_block<BITS>(vb, rq, scaled, words + BITS);
+                    if (valid) {  // 64 codes = BITS * 8 bytes
+                        uint8_t *dst = crow + (b / 2) * (BITS * 8);
+                        if (BITS == 4) {
+                            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(words[4], words[5], words[6], words[7]);
+                        } else {
+                            reinterpret_cast<uint2 *>(dst)[0] = make_uint2(words[0], words[1]);
+                            reinterpret_cast<uint2 *>(dst)[1] = make_uint2(words[2], words[3]);
+                            reinterpret_cast<uint2 *>(dst)[2] = make_uint2(words[4], words[5]);
+                        }
+                    }
+                    tmem_wait_ld();
+                }
+            }
+            tc_fence_before();
+            named_sync(1, kConsumers);  // TMEM reads done before the next tile's MMAs
+            ph ^= 1;
         }
-        tc_fence_before();
-        __syncthreads();  // TMEM reads done before the next tile's MMAs
+        if (tid == 0) bulk_wait0();
     }
 
-    if (tid == 0) bulk_wait0();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -96,6 +96,53 @@ __device__ __forceinline__ int quant_code(float v, const RowQuant &q, int qmax) 
     return quant_code(v * q.pre, q.inv, qmax);
 }
 
+// ---------------------------------------------------------------------------
+// Packed two-wide fp32 arithmetic (sm_100): one instruction per pair.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// Codes of 8 consecutive values packed into one INT4 word (or 24 bits of INT3).
+// round(v * inv) uses the 1.5*2^23 trick; because |v| <= amax and
+// inv = qmax / amax, |v * inv| <= qmax up to one rounding of inv, so no clamp
+// is needed and the low bits of the result hold the code in two's complement.
+// `pre` (1, or 2^64 for rows with a tiny absmax) is applied first when `scaled`.
+template <int BITS>
+__device__ __forceinline__ uint32_t pack8_fast(const float (&v)[8], float inv, float pre, bool scaled) {
+    constexpr uint32_t mask = (1u << BITS) - 1u;
+    const float2 inv2 = make_float2(inv, inv);
+    const float2 mag2 = make_float2(kRoundMagic, kRoundMagic);
+    uint32_t w = 0;
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+        float2 t = make_float2(v[e], v[e + 1]);
+        if (scaled) t = make_float2(t.x * pre, t.y * pre);
+        const float2 r = fma2(t, inv2, mag2);
+        w |= (__float_as_uint(r.x) & mask) << (BITS * e);
+        w |= (__float_as_uint(r.y) & mask) << (BITS * (e + 1));
+    }
+    return w;
+}
+
 // Pack 8 codes (each in [-qmax, qmax]).
 __device__ __forceinline__ uint32_t pack8_int4(const int (&c)[8]) {
     uint32_t w = 0;

@@ -43,29 +43,6 @@ constexpr int kOffBar = kOffMask + 64 * 128;                 // kWarps x kStages
 constexpr int kBytes = kOffBar + kWarps * kStages * 8;
 constexpr int kSmem = kBytes + 1024;
 
-// ---- packed two-wide fp32 arithmetic (sm_100)
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-    float2 d;
-    asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-    float2 d;
-    asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-
 // In-place 64-point Sylvester transform of the 64 pairs v[0..63] (each pair is
 // two independent transforms, one per component).
 __device__ __forceinline__ void fwht64x2(float2 (&v)[64]) {
@@ -234,10 +211,14 @@ k_rht4096(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ s
         __syncwarp();
         fwht64x2(u);  // along b for rows 2l, 2l+1
 
-        float m = 0.f;
+        float mx[8];  // independent partial maxima (short dependency chains)
 #pragma unroll
-        for (int b = 0; b < 64; ++b) m = fmaxf(m, fmaxf(fabsf(u[b].x), fabsf(u[b].y)));
-        const float amax = warp_max(m);
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(fabsf(u[k].x), fabsf(u[k].y));
+#pragma unroll
+        for (int b = 8; b < 64; ++b) mx[b & 7] = fmaxf(mx[b & 7], fmaxf(fabsf(u[b].x), fabsf(u[b].y)));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], mx[k + 4]);
+        const float amax = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
         quant_store<BITS>(u, amax, codes + t * row_bytes + lane * (BITS * 16));
         if (lane == 0) {
             constexpr int qmax = (1 << (BITS - 1)) - 1;

@@ -78,8 +78,9 @@ struct Layout {
     static constexpr int kOffZ = kOffQ + kQBytes;
     static constexpr int kOffM = kOffZ + kZBytes;                       // M^T, 32 x 32 fp32, zero padded
     static constexpr int kOffYred = kOffM + 32 * 32 * 4;
-    static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;  // [2 halves][128 rows] x 16 B
-    static constexpr int kOffBar = kOffStat + 2 * kTileM * 16;
+    static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;  // per row: CTA partial (ss, amax), 16 B
+    static constexpr int kOffLoc = kOffStat + kTileM * 16;              // per row: half-1 partial, then row quantiser
+    static constexpr int kOffBar = kOffLoc + kTileM * 16;
     static constexpr int kNumBars = 5;  // load, y, c0, c1, x_out ready
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffTmem + 16;
@@ -88,6 +89,13 @@ struct Layout {
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {  // SWIZZLE_128B chunk position
     return uint32_t(((chunk ^ (row & 7)) << 4));
+}
+
+// Opaque copy: keeps the compiler from hoisting descriptor arithmetic out of the
+// tile loop (which would pin dozens of 64-bit descriptors in registers).
+__device__ __forceinline__ uint64_t opaque(uint64_t v) {
+    asm volatile("mov.b64 %0, %0;" : "+l"(v));
+    return v;
 }
 
 __device__ __forceinline__ uint16_t bf16_bits(float v) {
@@ -163,6 +171,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     float *sm = reinterpret_cast<float *>(base + L::kOffM);
     float *syred = reinterpret_cast<float *>(base + L::kOffYred);
     uint8_t *sstat = base + L::kOffStat;
+    uint8_t *sloc = base + L::kOffLoc;
     const uint32_t bar_load = smem_u32(base + L::kOffBar);
     const uint32_t bar_y = bar_load + 8, bar_c0 = bar_load + 16, bar_c1 = bar_load + 24, bar_xo = bar_load + 32;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L::kOffTmem);
@@ -256,9 +265,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (tid == 0) {
                 tc_fence_after();
                 // descriptors advance by 16-byte units in their start-address field
-                const uint64_t ad0 = smem_desc_sw128(smem_u32(sx), 1024);
-                const uint64_t bd0 = smem_desc_sw128(smem_u32(sq), 1024);
-#pragma unroll 1
+                const uint64_t ad0 = opaque(smem_desc_sw128(smem_u32(sx), 1024));
+                const uint64_t bd0 = opaque(smem_desc_sw128(smem_u32(sq), 1024));
+#pragma unroll
                 for (int i = 0; i < kSlabs * 4; ++i) {  // K = 512 in steps of 16
                     const uint32_t aoff = uint32_t((i >> 2) * kSlabBytes + (i & 3) * 32) >> 4;
                     const uint32_t boff = uint32_t(i * 2048) >> 4;
@@ -351,17 +360,15 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 fence_proxy_async();
                 // (A K-step, B K-step) pairs: z_hi Q_hi^T, z_hi Q_lo^T, z_lo Q_hi^T; K-steps of 16
                 // columns are 32 bytes apart inside the 128-byte swizzled rows
-                const uint64_t ad0 = smem_desc_sw128(smem_u32(sz), 1024);
-                const uint64_t bd0 = smem_desc_sw128(smem_u32(sq), 1024);
-                const uint64_t pairs = 0x130231201100ull;  // byte s = (b << 4) | a: (0,0) (1,1) (0,2) (1,3) (2,0) (3,1)
-#pragma unroll 1
+                const uint64_t ad0 = opaque(smem_desc_sw128(smem_u32(sz), 1024));
+                const uint64_t bd0 = opaque(smem_desc_sw128(smem_u32(sq), 1024));
+                constexpr uint32_t kA[6] = {0, 1, 0, 1, 2, 3}, kB[6] = {0, 1, 2, 3, 0, 1};
+#pragma unroll
                 for (int h = 0; h < 2; ++h) {
-#pragma unroll 1
-                    for (int s = 0; s < 6; ++s) {
-                        const uint32_t ka = uint32_t(pairs >> (8 * s)) & 0xF, kb = uint32_t(pairs >> (8 * s + 4)) & 0xF;
-                        umma_f16(tmem + h * kHalfCols, ad0 + ((ka * 32) >> 4),
-                                 bd0 + ((uint32_t(h) * 32768 + kb * 32) >> 4), idesc_c, s != 0);
-                    }
+#pragma unroll
+                    for (int s = 0; s < 6; ++s)
+                        umma_f16(tmem + h * kHalfCols, ad0 + ((kA[s] * 32) >> 4),
+                                 bd0 + ((uint32_t(h) * 32768 + kB[s] * 32) >> 4), idesc_c, s != 0);
                     umma_commit(h == 0 ? bar_c0 : bar_c1);
                 }
             }
@@ -411,41 +418,52 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 bulk_commit();
             }
             ph_xo ^= 1;
-            {
-                uint8_t *st = sstat + (half * kTileM + m) * 16;
-                reinterpret_cast<double *>(st)[0] = ss;
-                reinterpret_cast<float *>(st)[2] = amax;
+            // statistics: fold the two column halves of each row, publish one entry per row
+            if (half == 1) {
+                reinterpret_cast<double *>(sloc + m * 16)[0] = ss;
+                reinterpret_cast<float *>(sloc + m * 16)[2] = amax;
+            }
+            named_sync(1, kConsumers);
+            if (half == 0) {
+                ss += reinterpret_cast<const double *>(sloc + m * 16)[0];
+                amax = fmaxf(amax, reinterpret_cast<const float *>(sloc + m * 16)[2]);
+                reinterpret_cast<double *>(sstat + m * 16)[0] = ss;
+                reinterpret_cast<float *>(sstat + m * 16)[2] = amax;
             }
             tc_fence_before();
             cluster_sync();  // #3 statistics visible
 
-            // row totals over the cluster and both halves (fixed order: deterministic)
-            double ss_t = 0.0;
-            float am_t = 0.f;
-            {
-                float4 sv[2 * CS];
+            // row totals over the cluster (fixed order: deterministic), computed by
+            // the half-0 thread of each row and handed to its half-1 partner
+            if (half == 0) {
+                float4 sv[CS];
 #pragma unroll
-                for (int c = 0; c < CS; ++c)
+                for (int c = 0; c < CS; ++c) sv[c] = ld_dsmem_f4(mapa(smem_u32(sstat + m * 16), uint32_t(c)));
+                double ss_t = 0.0;
+                float am_t = 0.f;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        sv[2 * c + h] = ld_dsmem_f4(mapa(smem_u32(sstat + (h * kTileM + m) * 16), uint32_t(c)));
-#pragma unroll
-                for (int i = 0; i < 2 * CS; ++i) {
-                    ss_t += __hiloint2double(__float_as_int(sv[i].y), __float_as_int(sv[i].x));
-                    am_t = fmaxf(am_t, sv[i].z);
+                for (int c = 0; c < CS; ++c) {
+                    ss_t += __hiloint2double(__float_as_int(sv[c].y), __float_as_int(sv[c].x));
+                    am_t = fmaxf(am_t, sv[c].z);
                 }
+                const float ms = float(ss_t / double(p.D));
+                const float rs = 1.0f / sqrtf(ms + p.eps);
+                const RowQuant q = row_quant(am_t, qmax);
+                if (crank == 0 && m < nrows) p.scales[t0 + m] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+                reinterpret_cast<float *>(sloc + m * 16)[0] = q.inv;
+                reinterpret_cast<float *>(sloc + m * 16)[1] = q.pre;
             }
-            const float ms = float(ss_t / double(p.D));
-            const float rs = 1.0f / sqrtf(ms + p.eps);
-            const RowQuant rq = row_quant(am_t, qmax);
-            const bool scaled = rq.pre != 1.0f;
-            const bool valid = m < nrows;
-            if (crank == 0 && half == 0 && valid) p.scales[t0 + m] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
             if (tid == 0) {  // the tile buffer is free once TMA has read x_out: fetch the next tile
                 bulk_wait_read0();
                 const long long tn = tile_t0(it + 1);
                 if (it + 1 < p.tiles_per_cluster && tn < p.T) issue_load(tn);
             }
+            named_sync(1, kConsumers);
+            RowQuant rq;
+            rq.inv = reinterpret_cast<const float *>(sloc + m * 16)[0];
+            rq.pre = reinterpret_cast<const float *>(sloc + m * 16)[1];
+            const bool scaled = rq.pre != 1.0f;
+            const bool valid = m < nrows;
 
             // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined)
             {

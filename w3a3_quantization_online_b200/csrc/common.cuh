@@ -126,21 +126,43 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 // inv = qmax / amax, |v * inv| <= qmax up to one rounding of inv, so no clamp
 // is needed and the low bits of the result hold the code in two's complement.
 // `pre` (1, or 2^64 for rows with a tiny absmax) is applied first when `scaled`.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Codes of 8 consecutive values packed into one INT4 word (or 24 bits of INT3).
+// round(v * inv) uses the 1.5*2^23 trick; because |v| <= amax and
+// inv = qmax / amax, |v * inv| <= qmax up to one rounding of inv, so no clamp
+// is needed and the low bits of the result hold the code in two's complement.
+// `pre` (1, or 2^64 for rows with a tiny absmax) is applied first when `scaled`.
 template <int BITS>
 __device__ __forceinline__ uint32_t pack8_fast(const float (&v)[8], float inv, float pre, bool scaled) {
-    constexpr uint32_t mask = (1u << BITS) - 1u;
     const float2 inv2 = make_float2(inv, inv);
     const float2 mag2 = make_float2(kRoundMagic, kRoundMagic);
-    uint32_t w = 0;
+    uint32_t r[8];
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
         float2 t = make_float2(v[e], v[e + 1]);
         if (scaled) t = make_float2(t.x * pre, t.y * pre);
-        const float2 r = fma2(t, inv2, mag2);
-        w |= (__float_as_uint(r.x) & mask) << (BITS * e);
-        w |= (__float_as_uint(r.y) & mask) << (BITS * (e + 1));
+        const float2 q = fma2(t, inv2, mag2);
+        r[e] = __float_as_uint(q.x);
+        r[e + 1] = __float_as_uint(q.y);
     }
-    return w;
+    if (BITS == 4) {
+        // byte k = low nibble of r[2k] | low nibble of r[2k+1] << 4 (bits above
+        // the byte are don't-care), then gather the four low bytes
+        uint32_t b[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) b[k] = (r[2 * k] & 0x0Fu) | ((r[2 * k + 1] << 4) & 0xF0u);
+        return prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+    } else {
+        uint32_t w = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w |= (r[e] & 0x7u) << (3 * e);
+        return w;
+    }
 }
 
 // Pack 8 codes (each in [-qmax, qmax]).

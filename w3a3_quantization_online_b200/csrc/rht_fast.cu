@@ -15,10 +15,12 @@
 // owns the 128 contiguous outputs [128 l, 128 l + 128): the absmax is a warp
 // reduction and the packed codes go out as coalesced 16-byte stores.
 //
-// Each warp streams its own rows through a two-stage TMA pipeline (one 8 KB
-// row per stage, SWIZZLE_128B so the column-pair reads are conflict-free) and
-// transposes between the phases through its own 16 KB fp32 buffer.  The
-// 1/sqrt(4096) = 1/64 factor is applied to the scale only.
+// Each warp streams its own rows through a one-row TMA buffer (8 KB,
+// SWIZZLE_128B so the column-pair reads are conflict-free): the next row is
+// requested as soon as the current one is in registers, so its load overlaps
+// the whole transform.  The phases are joined by a transpose through the
+// warp's own 16 KB fp32 buffer.  The 1/sqrt(4096) = 1/64 factor is applied to
+// the scale only.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -31,14 +33,14 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kWarps = 6;                   // warps (rows in flight) per CTA
+constexpr int kWarps = 8;                   // warps (rows in flight) per CTA
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 2;
+constexpr int kStages = 1;
 constexpr int kRowIn = 64 * 64 * 2;         // 8 KB bf16 row
 constexpr int kRowS = 64 * 64 * 4;          // 16 KB fp32 transpose buffer
 constexpr int kOffIn = 0;                                    // kWarps x kStages x 8 KB
 constexpr int kOffS = kOffIn + kWarps * kStages * kRowIn;    // kWarps x 16 KB
-constexpr int kOffMask = kOffS + kWarps * kRowS;             // 8 KB sign masks
+constexpr int kOffMask = kOffS + kWarps * kRowS;             // 8 KB sign masks, [lane][row]
 constexpr int kOffBar = kOffMask + 64 * 128;                 // kWarps x kStages mbarriers
 constexpr int kBytes = kOffBar + kWarps * kStages * 8;
 constexpr int kSmem = kBytes + 1024;
@@ -62,6 +64,9 @@ __device__ __forceinline__ void fwht64x2(float2 (&v)[64]) {
 __device__ __forceinline__ uint32_t in_off(int a, int l) {  // (a, 2l..2l+1) in a SWIZZLE_128B 64x64 bf16 tile
     return uint32_t(a * 128 + (((l >> 2) ^ (a & 7)) << 4) + (l & 3) * 4);
 }
+__device__ __forceinline__ uint32_t mask_off(int l, int c) {  // rows 4c..4c+3 of lane l
+    return uint32_t(l * 256 + ((c ^ (l & 15)) << 4));
+}
 __device__ __forceinline__ uint32_t s_off(int a, int chunk) {  // 16-byte chunk of row a of the 64x64 fp32 buffer
     return uint32_t(a * 256 + ((chunk ^ (a & 15)) << 4));
 }
@@ -71,32 +76,31 @@ __device__ __forceinline__ void quant_store(const float2 (&u)[64], float amax, u
     constexpr int qmax = (1 << (BITS - 1)) - 1;
     // Codes do not depend on a positive row factor: rows whose absmax is so
     // small that qmax / amax would overflow are first scaled by 2^64 (exact).
-    const bool tiny = amax < 0x1p-64f;
-    const float ps = tiny ? 0x1p64f : 1.0f;
-    const float inv = amax > 0.f ? float(qmax) / (amax * ps) : 0.f;
-    const float2 inv2 = make_float2(inv, inv);
-    const float2 ps2 = make_float2(ps, ps);
+    const RowQuant rq = row_quant(amax, qmax);
+    const bool tiny = rq.pre != 1.0f;
+    const float2 inv2 = make_float2(rq.inv, rq.inv);
     const float2 mag2 = make_float2(kRoundMagic, kRoundMagic);
     // round(v * inv) via the 1.5*2^23 trick; |v| * qmax / amax <= qmax (+1 ulp),
     // so no clamp is needed and the low bits hold the code in two's complement.
     auto code_bits = [&](float2 v) {
-        if (tiny) v = make_float2(v.x * ps2.x, v.y * ps2.y);
+        if (tiny) v = make_float2(v.x * rq.pre, v.y * rq.pre);
         const float2 t = fma2(v, inv2, mag2);
         return make_uint2(__float_as_uint(t.x), __float_as_uint(t.y));
     };
     uint32_t w[BITS * 4];
     if (BITS == 4) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            uint32_t a0 = 0, a1 = 0;
+        for (int k = 0; k < 8; ++k) {  // 8 columns -> one word per row
+            uint32_t b0[4], b1[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint2 c = code_bits(u[8 * k + e]);
-                a0 |= (c.x & 0xFu) << (4 * e);
-                a1 |= (c.y & 0xFu) << (4 * e);
+            for (int e = 0; e < 4; ++e) {
+                const uint2 c0 = code_bits(u[8 * k + 2 * e]);
+                const uint2 c1 = code_bits(u[8 * k + 2 * e + 1]);
+                b0[e] = (c0.x & 0x0Fu) | ((c1.x << 4) & 0xF0u);
+                b1[e] = (c0.y & 0x0Fu) | ((c1.y << 4) & 0xF0u);
             }
-            w[k] = a0;
-            w[8 + k] = a1;
+            w[k] = prmt(prmt(b0[0], b0[1], 0x0040u), prmt(b0[2], b0[3], 0x0040u), 0x5410u);
+            w[8 + k] = prmt(prmt(b1[0], b1[1], 0x0040u), prmt(b1[2], b1[3], 0x0040u), 0x5410u);
         }
     } else {
 #pragma unroll
@@ -140,13 +144,13 @@ k_rht4096(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ s
     const uint32_t bar0 = smem_u32(base + kOffBar + warp * kStages * 8);
     int err = 0;
 
-    // sign masks: bit 15 / bit 31 of word (a, l) flip the signs of elements
-    // 64a + 2l and 64a + 2l + 1 (bf16 pairs), laid out like the input tile
+    // sign masks: bit 15 / bit 31 of word (l, a) flip the signs of elements
+    // 64a + 2l and 64a + 2l + 1 (bf16 pairs); lane l reads rows 4c..4c+3 at once
     for (int idx = threadIdx.x; idx < 64 * 32; idx += kThreads) {
         const int a = idx >> 5, l = idx & 31;
         const int i = 64 * a + 2 * l;
         const uint32_t m = (signs[i] < 0 ? 0x8000u : 0u) | (signs[i + 1] < 0 ? 0x80000000u : 0u);
-        *reinterpret_cast<uint32_t *>(smask + in_off(a, l)) = m;
+        reinterpret_cast<uint32_t *>(smask + mask_off(l, a >> 2))[a & 3] = m;
     }
     if (lane == 0) {
         for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
@@ -170,21 +174,25 @@ k_rht4096(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ s
 
     int it = 0;
     for (long long t = gw; t < T; t += nw, ++it) {
-        const int s = it & 1;
-        if (!mbar_wait(bar0 + 8 * s, uint32_t((it >> 1) & 1), err != 0)) err |= kErrMbarTimeout;
+        const int s = 0;
+        if (!mbar_wait(bar0, uint32_t(it & 1), err != 0)) err |= kErrMbarTimeout;
 
         // phase 1: columns (2l, 2l+1), all rows a; signs applied on the bf16 pairs
         float2 v[64];
         const uint8_t *xin = sin + s * kRowIn;
 #pragma unroll
-        for (int a = 0; a < 64; ++a) {
-            const uint32_t o = in_off(a, lane);
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(xin + o) ^
-                               *reinterpret_cast<const uint32_t *>(smask + o);
-            v[a] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+        for (int c = 0; c < 16; ++c) {
+            const uint4 mk = *reinterpret_cast<const uint4 *>(smask + mask_off(lane, c));
+            const uint32_t m4[4] = {mk.x, mk.y, mk.z, mk.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int a = 4 * c + e;
+                const uint32_t w = *reinterpret_cast<const uint32_t *>(xin + in_off(a, lane)) ^ m4[e];
+                v[a] = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+            }
         }
         __syncwarp();
-        if (lane == 0) {  // stage s is free: prefetch the row two iterations ahead
+        if (lane == 0) {  // the row buffer is free: request the next row now
             const long long tn = t + kStages * nw;
             if (tn < T) {
                 mbar_expect_tx(bar0 + 8 * s, kRowIn);

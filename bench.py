@@ -378,6 +378,101 @@ def run_gpu(args) -> None:
         dist.destroy_process_group()
 
 
+def run_secondary(args) -> None:
+    """Secondary workloads (one JSON line each, rank 0 only, 1 GPU): the 32-layer
+    chain at decode (T=16) and prefill (T=16384) sizes, timed as one CUDA graph
+    per pass, and the W3A3 / down_proj parity workloads."""
+    import torch
+    from w3a3_quantization_online_b200 import inputs, rsq
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    stream = torch.cuda.Stream(device=dev)
+    out = {"workload": args.workload, "steps": args.steps, "warmup": args.warmup, "data": "synthetic"}
+    if args.workload.startswith("chain"):
+        T = 16 if args.workload == "chain16" else 16384
+        x0, qs, ms, _, _ = inputs.chain_case(T=T)
+        x = torch.from_numpy(x0).to(dev).to(torch.bfloat16)
+        Qd = [torch.from_numpy(q).to(dev) for q in qs]
+        Md = [torch.from_numpy(m).to(dev) for m in ms]
+        codes = torch.empty((T, 2048), dtype=torch.uint8, device=dev)
+        scales = torch.empty((T,), dtype=torch.float32, device=dev)
+        L = len(qs)
+
+        def chain():
+            for i in range(L):
+                rsq.rsq_align_norm_quant(x, Qd[i], Md[i], x, codes, scales, bits=4, stream=stream)
+
+        with torch.cuda.stream(stream):
+            chain()  # configure kernels outside capture
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            chain()
+        for _ in range(args.warmup):
+            g.replay()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_pass = e0.elapsed_time(e1) / args.steps
+        per_layer_us = ms_pass * 1e3 / L
+        bytes_layer = T * (2 * 4096 * 2 + 2048 + 4) + 4096 * 32 * 4 + 32 * 32 * 4
+        gbs = bytes_layer / (per_layer_us * 1e-6) / 1e9
+        out.update({"metric": "per-layer latency and HBM GB/s, 32-layer align+norm+INT4 chain, D=4096",
+                    "T": T, "layers": L, "us_per_layer": per_layer_us, "achieved_gbs": gbs,
+                    "frac": gbs / pk["hbm_gbs"], "tokens_per_s_per_layer": T / (per_layer_us * 1e-6),
+                    "timing": "CUDA graph of the 32 in-place layer calls, CUDA events over the replays"})
+        del g
+    else:
+        if args.workload == "w3a3":
+            a, h = inputs.w3a3_case(T=8192)
+        elif args.workload == "downproj":
+            a, h = None, inputs.down_proj_case(T=4096)
+        else:
+            raise SystemExit(f"unknown workload {args.workload}")
+        res = {}
+        if a is not None:
+            x = torch.from_numpy(a.x).to(dev).to(torch.bfloat16)
+            Q, M = torch.from_numpy(a.Q).to(dev), torch.from_numpy(a.M).to(dev)
+            xo = torch.empty_like(x)
+            c = torch.empty((a.T, a.D * a.bits // 8), dtype=torch.uint8, device=dev)
+            sc = torch.empty((a.T,), dtype=torch.float32, device=dev)
+            f = lambda: rsq.rsq_align_norm_quant(x, Q, M, xo, c, sc, bits=a.bits, stream=stream)
+            byts = a.T * (2 * a.D * 2 + a.D * a.bits // 8 + 4) + a.D * a.r * 4
+            res["align_norm_quant"] = (f, byts, a.T)
+        xh = torch.from_numpy(h.x).to(dev).to(torch.bfloat16)
+        sg = torch.from_numpy(h.signs).to(dev)
+        ch = torch.empty((h.T, h.d * h.bits // 8), dtype=torch.uint8, device=dev)
+        sh = torch.empty((h.T,), dtype=torch.float32, device=dev)
+        fr = lambda: rsq.rht_quant(xh, sg, h.m, ch, sh, bits=h.bits, stream=stream)
+        res["rht_quant"] = (fr, h.T * (h.d * 2 + h.d * h.bits // 8 + 4) + h.d, h.T)
+        kern = {}
+        for name, (f, byts, T) in res.items():
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    f()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(args.steps):
+                    f()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            us = e0.elapsed_time(e1) * 1e3 / args.steps
+            kern[name] = {"avg_us": us, "achieved_gbs": byts / (us * 1e-6) / 1e9,
+                          "frac": byts / (us * 1e-6) / 1e9 / pk["hbm_gbs"], "tokens_per_s": T / (us * 1e-6)}
+        out.update({"metric": "tokens/s and HBM GB/s per kernel", "kernels": kern})
+    out["peak_gbs"] = pk["hbm_gbs"]
+    print(json.dumps(out), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -386,11 +481,17 @@ def main():
     ap.add_argument("--impl", choices=["rsq", "reference"], default="rsq")
     ap.add_argument("--tokens", type=int, default=T_TOK, help="tokens per GPU (default 16384)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="hidden",
+                    choices=["hidden", "chain16", "chain16384", "w3a3", "downproj"],
+                    help="hidden = the headline step (default); the others print a secondary line")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != "hidden":
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_secondary(args)
     else:
         run_gpu(args)
 

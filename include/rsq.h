@@ -118,18 +118,22 @@ int rsq_last_cuda_error(void);
 /* Number of kernels this library has launched in this process (all threads). */
 uint64_t rsq_launch_count(void);
 
-/* Kernel used by rsq_align_norm_quant: 0 = automatic (tensor-core cluster
- * kernel for bf16, D in {4096, 8192}, r <= 32; CUDA-core kernel otherwise),
- * 1 = always the CUDA-core kernel, 2 = only the tensor-core kernel (calls it
- * cannot serve return RSQ_ERR_UNSUPPORTED).  Process-wide; returns the previous
- * setting, or -1 for an invalid value.  Both kernels compute the same
- * function; this exists for testing and measurement. */
+/* Kernel used by rsq_align_norm_quant: 0 = automatic (for bf16, D in
+ * {4096, 8192} and r <= 32 the single-tile tensor-core cluster kernel; the
+ * CUDA-core kernel otherwise),
+ * 1 = always the CUDA-core kernel, 2 = only the single-tile tensor-core
+ * kernel, 3 = only the double-buffered one (2 and 3 return RSQ_ERR_UNSUPPORTED
+ * for calls they cannot serve).  Process-wide; returns the previous setting, or
+ * -1 for an invalid value.  All compute the same function; this exists for
+ * testing and measurement. */
 int rsq_select_align_kernel(int which);
 
-/* Kernel used by rht_quant: 0 = automatic (warp-per-row kernel for bf16,
+/* Kernel used by rht_quant: 0 = automatic (tensor-core kernel for bf16,
  * d = 4096, m = 1; shared-memory radix-16 kernel otherwise), 1 = always the
- * radix-16 kernel, 2 = only the specialised kernel (RSQ_ERR_UNSUPPORTED
- * otherwise).  Process-wide; returns the previous setting, -1 if invalid. */
+ * radix-16 kernel, 2 = only the warp-per-row CUDA-core kernel, 3 = only the
+ * tensor-core kernel (2 and 3 return RSQ_ERR_UNSUPPORTED for other shapes).
+ * Process-wide; returns the previous setting, -1 if invalid.  All compute the
+ * same function; this exists for testing and measurement. */
 int rsq_select_rht_kernel(int which);
 
 /* Synchronise `stream`, then read and clear the device status word of the

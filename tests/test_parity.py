@@ -208,23 +208,40 @@ def test_generic_kernel_at_the_tensor_core_shapes(generic_align, T):
     check_align(a, label=f"generic w3a3 T={T}")
 
 
-def test_tensor_core_kernel_serves_the_hot_shapes():
+@pytest.mark.parametrize("which", [2, 3])
+def test_tensor_core_kernel_serves_the_hot_shapes(which):
     rsq = _rsq()
-    prev = rsq.select_align_kernel(rsq.ALIGN_TENSOR_CORE)
+    prev = rsq.select_align_kernel(which)
     try:
         for T in (1, 128, 129, 1000):
             a, _ = inputs.llama7b_case(T=T)
             check_align(a, label=f"tc hidden T={T}")
-        a, _ = inputs.w3a3_case(T=257)
-        check_align(a, label="tc w3a3 T=257")
+        if which == 2:
+            a, _ = inputs.w3a3_case(T=257)
+            check_align(a, label="tc w3a3 T=257")
         for r in (1, 7, 32):
             a = inputs.align_case(300, 4096, r, 40 + r, dtype="bf16", n_outliers=8, outlier_scale=100.0)
             check_align(a, label=f"tc r={r}")
+        for T in (3000,):  # several tiles per cluster, ragged last tile
+            a, _ = inputs.llama7b_case(T=T)
+            check_align(a, rows=np.arange(0, T, 7), label=f"tc hidden T={T}")
         a = inputs.align_case(96, 4096, 32, 77, dtype="bf16", dist="student_t3")
         a.x[[0, 50, 95]] = 0.0
         xo, codes, scales = run_align(a)
         assert np.all(scales[[0, 50, 95]] == 0) and np.all(codes[[0, 50, 95]] == 0)
         check_align(a, label="tc zero rows")
+        # codes buffer only 16-byte aligned: the kernel must not use 32-byte stores
+        a, _ = inputs.llama7b_case(T=40)
+        x = _to_dev(a.x, "bf16")
+        Q = torch.from_numpy(a.Q).to(DEV)
+        M = torch.from_numpy(a.M).to(DEV)
+        big = torch.zeros(40 * 2048 + 16, dtype=torch.uint8, device=DEV)
+        codes16 = big[16:].view(40, 2048)
+        _, _, sc = rsq.rsq_align_norm_quant(x, Q, M, codes=codes16, bits=4)
+        assert rsq.device_status() == 0
+        ref = oracle.align_norm_quant(a.x, a.Q, a.M, 4, a.eps)
+        H.check_codes(codes16.cpu().numpy(), ref["q"], ref["pre"], 4, "tc 16B-aligned codes")
+        H.check_scales(sc.cpu().numpy(), ref["scales"], "tc 16B-aligned codes")
     finally:
         rsq.select_align_kernel(prev)
 
@@ -257,7 +274,7 @@ def test_rht_shapes(d, m, dtype, bits):
 
 def test_rht_kernels_agree_with_the_oracle_at_4096():
     rsq = _rsq()
-    for which in (rsq.RHT_SPECIALISED, rsq.RHT_GENERIC):
+    for which in (rsq.RHT_TENSOR_CORE, rsq.RHT_SPECIALISED, rsq.RHT_GENERIC):
         prev = rsq.select_rht_kernel(which)
         try:
             for T in (1, 7, 600):
@@ -269,7 +286,7 @@ def test_rht_kernels_agree_with_the_oracle_at_4096():
             rsq.select_rht_kernel(prev)
 
 
-@pytest.mark.parametrize("which", [1, 2])
+@pytest.mark.parametrize("which", [1, 2, 3])
 def test_tiny_and_zero_rows_rht_4096(which):
     rsq = _rsq()
     prev = rsq.select_rht_kernel(which)

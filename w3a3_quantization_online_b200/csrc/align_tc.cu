@@ -173,7 +173,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     uint8_t *sstat = base + L::kOffStat;
     uint8_t *sloc = base + L::kOffLoc;
     const uint32_t bar_load = smem_u32(base + L::kOffBar);
-    const uint32_t bar_y = bar_load + 8, bar_c0 = bar_load + 16, bar_c1 = bar_load + 24, bar_xo = bar_load + 32;
+    const uint32_t bar_y = bar_load + 8, bar_c0 = bar_load + 16, bar_c1 = bar_load + 24;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L::kOffTmem);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -191,7 +191,6 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         mbar_init(bar_y, 1);
         mbar_init(bar_c0, 1);
         mbar_init(bar_c1, 1);
-        mbar_init(bar_xo, kConsumers);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -244,7 +243,6 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             for (int s = 0; s < kSlabs; ++s)
                 tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(t0), bar_load);
         };
-        uint32_t ph_xo = 0;
         // ------------------------------------------------ consumer warps
         const int quad = warp & 3, half = warp >> 2;
         const int m = quad * 32 + lane;  // tile row == TMEM lane
@@ -253,6 +251,30 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
         const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
         uint32_t ph = 0;  // every consumer barrier completes once per tile
+        // codes and scale of the previous tile, waiting to be stored
+        uint32_t pend[BITS * (kHalfCols / 32)];
+        uint8_t *pend_at = nullptr;
+        float pend_scale = 0.f;
+        float *pend_scale_at = nullptr;
+        auto flush = [&]() {
+            if (pend_at) {
+                if (BITS == 4) {
+#pragma unroll
+                    for (int w = 0; w < BITS * (kHalfCols / 32) / 4; ++w)
+                        reinterpret_cast<uint4 *>(pend_at)[w] =
+                            make_uint4(pend[4 * w], pend[4 * w + 1], pend[4 * w + 2], pend[4 * w + 3]);
+                } else {  // INT3 rows are 8-byte aligned here
+#pragma unroll
+                    for (int w = 0; w < BITS * (kHalfCols / 32) / 2; ++w)
+                        reinterpret_cast<uint2 *>(pend_at)[w] = make_uint2(pend[2 * w], pend[2 * w + 1]);
+                }
+                pend_at = nullptr;
+            }
+            if (pend_scale_at) {
+                *pend_scale_at = pend_scale;
+                pend_scale_at = nullptr;
+            }
+        };
 
         for (int it = 0; it < p.tiles_per_cluster; ++it) {
             const long long t0 = tile_t0(it);
@@ -353,6 +375,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             fence_proxy_async();
             cluster_sync();  // #2 z of all rows is in every CTA's operand buffer
+            flush();         // previous tile's codes and scales
 
             // ---- c = z Q^T (hi/lo split): half h into TMEM columns [256 h, 256 h + 256)
             if (tid == 0) {
@@ -408,16 +431,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tmem_wait_st();
                 amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
             }
-            fence_proxy_async_cta();
-            mbar_arrive(bar_xo);  // this thread's part of x_out is in the tile buffer
-            if (tid == 0) {       // write x_out back as soon as the whole tile is in place
-                if (!mbar_wait(bar_xo, ph_xo, err != 0)) err |= kErrMbarTimeout;
-#pragma unroll
-                for (int s = 0; s < kSlabs; ++s)
-                    tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
-                bulk_commit();
-            }
-            ph_xo ^= 1;
+            fence_proxy_async_cta();  // x_out (generic writes) -> TMA store (async proxy)
             // statistics: fold the two column halves of each row, publish one entry per row
             if (half == 1) {
                 reinterpret_cast<double *>(sloc + m * 16)[0] = ss;
@@ -431,7 +445,14 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 reinterpret_cast<float *>(sstat + m * 16)[2] = amax;
             }
             tc_fence_before();
-            cluster_sync();  // #3 statistics visible
+            cluster_sync();  // #3 statistics visible; every thread's x_out is in the tile buffer
+            if (tid == 0) {  // x_out back to HBM (issued after the barrier, whose release
+                             // semantics would otherwise wait for this bulk store)
+#pragma unroll
+                for (int s = 0; s < kSlabs; ++s)
+                    tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
+                bulk_commit();
+            }
 
             // row totals over the cluster (fixed order: deterministic), computed by
             // the half-0 thread of each row and handed to its half-1 partner
@@ -449,7 +470,10 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const float ms = float(ss_t / double(p.D));
                 const float rs = 1.0f / sqrtf(ms + p.eps);
                 const RowQuant q = row_quant(am_t, qmax);
-                if (crank == 0 && m < nrows) p.scales[t0 + m] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+                if (crank == 0 && m < nrows) {  // stored after the next tile's second barrier
+                    pend_scale = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+                    pend_scale_at = p.scales + t0 + m;
+                }
                 reinterpret_cast<float *>(sloc + m * 16)[0] = q.inv;
                 reinterpret_cast<float *>(sloc + m * 16)[1] = q.pre;
             }
@@ -465,40 +489,32 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             const bool scaled = rq.pre != 1.0f;
             const bool valid = m < nrows;
 
-            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined)
+            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined); the codes
+            // stay in registers and are stored after the next tile's second cluster
+            // barrier, so that no barrier's release has to wait for these stores
             {
                 constexpr int kBlocks = kHalfCols / 32;
-                uint8_t *crow = p.codes + (t0 + m) * row_bytes + (long long)(col0 + half * kHalfCols) * BITS / 8;
                 const uint32_t taddr = tmem + lane_base + tcol;
                 uint32_t va[32], vb[32];
                 tmem_ld32(taddr, va);
                 tmem_wait_ld();
-#pragma unroll 1
+#pragma unroll
                 for (int b = 0; b < kBlocks; b += 2) {
-                    uint32_t words[2 * BITS];
                     tmem_ld32(taddr + (b + 1) * 32, vb);
-                    code_block<BITS>(va, rq, scaled, words);
+                    code_block<BITS>(va, rq, scaled, pend + b * BITS);
                     tmem_wait_ld();
                     if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
-                    code_block<BITS>(vb, rq, scaled, words + BITS);
-                    if (valid) {  // 64 codes = BITS * 8 bytes
-                        uint8_t *dst = crow + (b / 2) * (BITS * 8);
-                        if (BITS == 4) {
-                            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(words[4], words[5], words[6], words[7]);
-                        } else {
-                            reinterpret_cast<uint2 *>(dst)[0] = make_uint2(words[0], words[1]);
-                            reinterpret_cast<uint2 *>(dst)[1] = make_uint2(words[2], words[3]);
-                            reinterpret_cast<uint2 *>(dst)[2] = make_uint2(words[4], words[5]);
-                        }
-                    }
+                    code_block<BITS>(vb, rq, scaled, pend + (b + 1) * BITS);
                     tmem_wait_ld();
                 }
+                pend_at = valid ? p.codes + (t0 + m) * row_bytes + (long long)(col0 + half * kHalfCols) * BITS / 8
+                                : nullptr;
             }
             tc_fence_before();
             named_sync(1, kConsumers);  // TMEM reads done before the next tile's MMAs
             ph ^= 1;
         }
+        flush();
         if (tid == 0) bulk_wait0();
     }
 

@@ -36,9 +36,20 @@ cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void 
                             float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
                             bool *launched);
 
+// Double-buffered tensor-core alignment kernel for D = 4096 (cluster of 16).
+bool align_tc_db_supports(int D, int r, int dtype, long long T);
+cudaError_t launch_align_tc_db(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                               float *scales, long long T, int r, int bits, float eps, cudaStream_t s,
+                               bool *launched);
+
 // Warp-per-row randomised Hadamard of order 4096 (m = 1, bf16, INT4/INT3).
 bool rht_fast_supports(int d, int m, int dtype, int bits, long long T);
 cudaError_t launch_rht_fast(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
                             int bits, cudaStream_t s);
+
+// Randomised Hadamard of order 4096 with the first 64-point stage on tcgen05
+// (m = 1, bf16, INT4/INT3; same support as rht_fast_supports).
+cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int bits,
+                          cudaStream_t s);
 
 }  // namespace rsq

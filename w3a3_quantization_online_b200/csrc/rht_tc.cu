@@ -1,0 +1,335 @@
+// rht_tc.cu -- randomised Hadamard transform of order 4096 + per-token
+// symmetric quantiser, bf16 input; the first half of the transform runs on the
+// tensor cores.
+//
+// Infra Quant II, QuaRot / Background: v = H diag(s) x / sqrt(d) with the
+// Sylvester H of order d = 2^12; QuaRot / Method: per-token symmetric absmax
+// quantisation.
+//
+// A token row is the 64 x 64 matrix U[a][b] = s_i x_i (i = 64 a + b).  The
+// Sylvester matrix factors as H_4096 = H_64 (x) H_64, so the transform is
+// W = H_64 U H_64:
+//  * Y = H_64 U (along a) for four tokens at once is one tcgen05 product
+//        D[(p, a)][(q, b)] = sum_{(p', a')} diag(H_64, H_64)[(p, a)][(p', a')] B[(p', a')][(q, b)]
+//    with B the four TMA-loaded token tiles (token p + 2 q): M = 128, N = 128,
+//    K = 128.  The products are +-1 x bf16, exact; accumulation is fp32 in TMEM.
+//  * W = Y H_64 (along b): each thread reads one row a of one token (64
+//    columns) from TMEM and finishes it with register butterflies (packed
+//    f32x2), then owns the 64 contiguous outputs [64 a, 64 a + 64).
+// The signs are applied to the tiles in shared memory (XOR of the bf16 sign
+// bits) before the product.  The 1/sqrt(4096) = 1/64 factor goes to the scale.
+//
+// Pipeline: 2 tile stages (4 tokens, 32 KB each) loaded by TMA ahead of use;
+// 2 TMEM slots of 128 columns, so the product of group g overlaps the
+// epilogue of group g - 1.  Two CTAs share each SM (104 KB of shared memory and
+// 256 TMEM columns each), so one CTA's barriers and waits hide behind the
+// other's work.  Waits are bounded (device status word).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rsq {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kTok = 4;                       // tokens per group (one MMA set)
+constexpr int kTileBytes = 64 * 128;          // one token: 64 rows x 128 B (bf16)
+constexpr int kStageBytes = kTok * kTileBytes;  // 32 KB
+constexpr int kStages = 2;
+constexpr int kSlots = 2;                     // TMEM slots of 128 columns
+constexpr int kCtasPerSm = 2;                 // two independent pipelines per SM
+constexpr int kOffA = 0;                      // diag(H_64, H_64), K-major SW128: 2 slabs x 16 KB
+constexpr int kOffMask = kOffA + 2 * 16384;   // 8 KB sign masks, laid out like a token tile
+constexpr int kOffStage = kOffMask + kTileBytes;
+constexpr int kOffRed = kOffStage + kStages * kStageBytes;  // [token 4][half-quadrant 2] absmax partials
+constexpr int kOffBar = kOffRed + kTok * 2 * 4;
+constexpr int kOffTmem = kOffBar + (kStages + kSlots) * 8;
+constexpr int kBytes = kOffTmem + 16;
+constexpr int kSmem = kBytes + 1024;
+
+__device__ __forceinline__ uint32_t tile_off(int a, int chunk) {  // SWIZZLE_128B 64 x 128 B tile
+    return uint32_t(a * 128 + ((chunk ^ (a & 7)) << 4));
+}
+
+// In-place 64-point Sylvester transform of v[0..63]: stages for index bits 0..4
+// act on the pairs (v[k], v[k + 32]) with packed two-wide arithmetic, the stage
+// for bit 5 combines the two halves.
+__device__ __forceinline__ void fwht64(float (&v)[64]) {
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            if ((k & h) == 0) {
+                const float2 u = make_float2(v[k], v[k + 32]);
+                const float2 w = make_float2(v[k + h], v[k + h + 32]);
+                const float2 s = add2(u, w), d = sub2(u, w);
+                v[k] = s.x;
+                v[k + 32] = s.y;
+                v[k + h] = d.x;
+                v[k + h + 32] = d.y;
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float u = v[k], w = v[k + 32];
+        v[k] = u + w;
+        v[k + 32] = u - w;
+    }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ signs,
+             uint8_t *__restrict__ codes, float *__restrict__ scales, long long T, int *status) {
+    constexpr int qmax = (1 << (BITS - 1)) - 1;
+    constexpr int row_bytes = 4096 * BITS / 8;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sa = base + kOffA;
+    uint8_t *smask = base + kOffMask;
+    uint8_t *sstage = base + kOffStage;
+    float *sred = reinterpret_cast<float *>(base + kOffRed);
+    const uint32_t bar_full = smem_u32(base + kOffBar);             // kStages barriers
+    const uint32_t bar_mma = bar_full + 8 * kStages;                // kSlots barriers
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTmem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int err = 0;
+
+    // constants: A = diag(H_64, H_64) with H_64[a][a'] = (-1)^popcount(a & a'),
+    // bf16 +-1 (K-major, SWIZZLE_128B: slab kk holds K columns 64 kk .. 64 kk + 63)
+    for (int idx = tid; idx < 2 * 128 * 8; idx += kThreads) {
+        const int kk = idx >> 10, m = (idx >> 3) & 127, ch = idx & 7;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            uint32_t pair = 0;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int k = 64 * kk + ch * 8 + 2 * e + u;
+                uint32_t hv = 0;  // 0 outside the diagonal blocks
+                if ((m >> 6) == (k >> 6)) hv = (__popc((m & 63) & (k & 63)) & 1) ? 0xBF80u : 0x3F80u;
+                pair |= hv << (16 * u);
+            }
+            w[e] = pair;
+        }
+        *reinterpret_cast<uint4 *>(sa + kk * 16384 + tile_off(m, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    // sign masks: bit 15 / 31 of the word for (a, b-pair) flips elements 64a + 2j, 64a + 2j + 1
+    for (int idx = tid; idx < 64 * 32; idx += kThreads) {
+        const int a = idx >> 5, j = idx & 31;
+        const int i = 64 * a + 2 * j;
+        const uint32_t mk = (signs[i] < 0 ? 0x8000u : 0u) | (signs[i + 1] < 0 ? 0x80000000u : 0u);
+        *reinterpret_cast<uint32_t *>(smask + tile_off(a, j >> 2) + (j & 3) * 4) = mk;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(bar_full + 8 * s, 1);
+        for (int s = 0; s < kSlots; ++s) mbar_init(bar_mma + 8 * s, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_x);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kSlots * 128);
+        tmem_relinquish();
+    }
+    fence_proxy_async_cta();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const long long ngroups = (T + kTok - 1) / kTok;
+    const long long g0 = blockIdx.x, gstep = gridDim.x;
+    const int nmine = g0 < ngroups ? int((ngroups - 1 - g0) / gstep + 1) : 0;
+    auto issue_load = [&](int it) {  // thread 0
+        const int s = it % kStages;
+        mbar_expect_tx(bar_full + 8 * s, kStageBytes);
+        tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok), bar_full + 8 * s);
+    };
+    if (tid == 0)
+        for (int it = 0; it < kStages && it < nmine; ++it) issue_load(it);
+
+    const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+    // epilogue mapping: TMEM lane (p, a) = 64 p + a, column half q
+    const int quad = warp & 3, q = warp >> 2;
+    const int lrow = quad * 32 + lane;
+    const int p = lrow >> 6, a = lrow & 63;
+    const int tslot = p + 2 * q;  // token within the group
+
+    auto epilogue = [&](int it) {
+        const int slot = it % kSlots;
+        if (!mbar_wait(bar_mma + 8 * slot, uint32_t((it / kSlots) & 1), err != 0)) err |= kErrMbarTimeout;
+        tc_fence_after();
+        float v[64];
+        {
+            uint32_t r0[32], r1[32];
+            const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + uint32_t(slot * 128 + q * 64);
+            tmem_ld32(taddr, r0);
+            tmem_ld32(taddr + 32, r1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                v[k] = __uint_as_float(r0[k]);
+                v[k + 32] = __uint_as_float(r1[k]);
+            }
+        }
+        fwht64(v);  // along b: row a of token tslot is now final
+        float mx[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mx[k] = fabsf(v[k]);
+#pragma unroll
+        for (int k = 4; k < 64; ++k) mx[k & 3] = fmaxf(mx[k & 3], fabsf(v[k]));
+        const float wm = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+        // the 64 rows of a token live in quadrants 2p, 2p+1 of column half q
+        if (lane == 0) sred[tslot * 2 + (quad & 1)] = wm;
+        named_sync(1, kThreads);
+        const float amax = fmaxf(sred[tslot * 2], sred[tslot * 2 + 1]);
+        const long long t = (g0 + (long long)it * gstep) * kTok + tslot;
+        if (t < T) {
+            const RowQuant rq = row_quant(amax, qmax);
+            const bool scaled = rq.pre != 1.0f;
+            uint32_t w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = v[8 * k + e];
+                w[k] = pack8_fast<BITS>(f, rq.inv, rq.pre, scaled);
+            }
+            uint8_t *dst = codes + t * row_bytes + a * (8 * BITS);
+            if (BITS == 4) {
+                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {  // 8 groups of 24 bits -> 6 words
+                uint32_t o[6];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    o[3 * h + 0] = w[4 * h] | (w[4 * h + 1] << 24);
+                    o[3 * h + 1] = (w[4 * h + 1] >> 8) | (w[4 * h + 2] << 16);
+                    o[3 * h + 2] = (w[4 * h + 2] >> 16) | (w[4 * h + 3] << 8);
+                }
+#pragma unroll
+                for (int h = 0; h < 3; ++h) reinterpret_cast<uint2 *>(dst)[h] = make_uint2(o[2 * h], o[2 * h + 1]);
+            }
+            if (a == 0) scales[t] = amax > 0.f ? amax / float(qmax * 64) : 0.f;
+        }
+        tc_fence_before();
+        named_sync(1, kThreads);  // sred reuse; TMEM slot reads done
+    };
+
+    for (int it = 0; it < nmine; ++it) {
+        const int s = it % kStages, slot = it % kSlots;
+        if (!mbar_wait(bar_full + 8 * s, uint32_t((it / kStages) & 1), err != 0)) err |= kErrMbarTimeout;
+        // apply the random signs to the four tiles (XOR of bf16 sign bits)
+        uint8_t *st = sstage + s * kStageBytes;
+#pragma unroll
+        for (int k = 0; k < (kStageBytes / 16) / kThreads; ++k) {
+            const int c = tid + k * kThreads;           // 16-byte chunk within the stage
+            const int within = c & (kTileBytes / 16 - 1);  // same position in the mask tile
+            uint4 xv = reinterpret_cast<uint4 *>(st)[c];
+            const uint4 mv = reinterpret_cast<const uint4 *>(smask)[within];
+            xv.x ^= mv.x;
+            xv.y ^= mv.y;
+            xv.z ^= mv.z;
+            xv.w ^= mv.w;
+            reinterpret_cast<uint4 *>(st)[c] = xv;
+        }
+        fence_proxy_async_cta();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // A: K-major, K-steps of 16 are 32 bytes apart within a slab, slabs 16 KB apart.
+            // B: MN-major, K rows (p', a') 128 B apart (16 per K-step: 2 KB), the two
+            //    64-column atoms (token pairs q = 0, 1) 16 KB apart.
+            const uint64_t ad0 = smem_desc_sw128(smem_u32(sa), 1024);
+            const uint64_t bd0 = smem_desc_sw128_lbo(smem_u32(st), 16384, 1024);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t aoff = uint32_t((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                const uint32_t boff = uint32_t(k * 2048) >> 4;
+                umma_f16(tmem + uint32_t(slot * 128), ad0 + aoff, bd0 + boff, idesc, k != 0);
+            }
+            umma_commit(bar_mma + 8 * slot);
+        }
+        if (it >= 1) {
+            epilogue(it - 1);
+            // group it-1's product has completed, so its stage can be refilled
+            if (tid == 0 && it - 1 + kStages < nmine) issue_load(it - 1 + kStages);
+        }
+    }
+    if (nmine > 0) epilogue(nmine - 1);
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kSlots * 128);
+    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    if (err && lane == 0) atomicOr(status, err);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int BITS>
+cudaError_t launch_bits(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
+                        cudaStream_t st) {
+    static bool configured[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    auto kern = k_rht4096_tc<BITS>;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    EncodeTiledFn enc = encode_fn();
+    int *status = device_status_word();
+    if (!enc || !status) return cudaErrorInvalidValue;
+    CUtensorMap map;
+    const cuuint64_t dims[3] = {64, 64, cuuint64_t(T)};
+    const cuuint64_t strides[2] = {128, 8192};
+    const cuuint32_t box[3] = {64, 64, kTok};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const long long ngroups = (T + kTok - 1) / kTok;
+    long long grid = (long long)num_sms() * kCtasPerSm;
+    if (grid > ngroups) grid = ngroups;
+    kern<<<int(grid), kThreads, kSmem, st>>>(map, signs, codes, scales, T, status);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch();
+    return e;
+}
+
+}  // namespace
+
+cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int bits,
+                          cudaStream_t s) {
+    return bits == 4 ? launch_bits<4>(x, signs, codes, scales, T, s) : launch_bits<3>(x, signs, codes, scales, T, s);
+}
+
+}  // namespace rsq

@@ -19,8 +19,8 @@ __device__ int g_device_status;
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
-std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 tensor core
-std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 specialised
+std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 double-buffered
+std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 warp-per-row, 3 tensor core
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -145,14 +145,20 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         overlap(sc, span(M, uint64_t(r) * r * 4)) || overlap(ss, span(M, uint64_t(r) * r * 4)))
         return RSQ_ERR_ALIAS;
     const int which = rsq::g_align_kernel.load(std::memory_order_relaxed);
-    if (which != 1 && rsq::align_tc_supports(D, r, dtype, T)) {
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (which == 3 && rsq::align_tc_db_supports(D, r, dtype, T)) {
         bool launched = false;
-        const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, codes, scales, T, D, r, bits, eps,
-                                                   static_cast<cudaStream_t>(stream), &launched);
+        const cudaError_t e = rsq::launch_align_tc_db(x, Q, M, x_out, codes, scales, T, r, bits, eps, cs, &launched);
         if (e != cudaSuccess) return finish(e);
         if (launched) return RSQ_OK;
     }
-    if (which == 2) return RSQ_ERR_UNSUPPORTED;
+    if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
+        bool launched = false;
+        const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, cs, &launched);
+        if (e != cudaSuccess) return finish(e);
+        if (launched) return RSQ_OK;
+    }
+    if (which == 2 || which == 3) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
                                             true, static_cast<cudaStream_t>(stream)));
 }
@@ -172,9 +178,12 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
     const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * 4);
     if (overlap(sc, sx) || overlap(sc, sg) || overlap(sc, ss) || overlap(ss, sx) || overlap(ss, sg))
         return RSQ_ERR_ALIAS;
-    if (rsq::g_rht_kernel.load(std::memory_order_relaxed) != 1 && rsq::rht_fast_supports(d, m, dtype, bits, T))
+    const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
+    if ((which == 0 || which == 3) && rsq::rht_fast_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
+    if (which == 2 && rsq::rht_fast_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_fast(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
-    if (rsq::g_rht_kernel.load(std::memory_order_relaxed) == 2) return RSQ_ERR_UNSUPPORTED;
+    if (which == 2 || which == 3) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
                                           static_cast<cudaStream_t>(stream)));
 }
@@ -198,12 +207,12 @@ const char *rsq_status_string(int status) {
 int rsq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int rsq_select_align_kernel(int which) {
-    if (which < 0 || which > 2) return -1;
+    if (which < 0 || which > 3) return -1;
     return rsq::g_align_kernel.exchange(which);
 }
 
 int rsq_select_rht_kernel(int which) {
-    if (which < 0 || which > 2) return -1;
+    if (which < 0 || which > 3) return -1;
     return rsq::g_rht_kernel.exchange(which);
 }
 

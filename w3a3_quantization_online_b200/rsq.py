@@ -46,8 +46,8 @@ _lib.rsq_device_status.restype = _i32
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status")
 
-ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE = 0, 1, 2
-RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED = 0, 1, 2
+ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DOUBLE_BUFFERED = 0, 1, 2, 3
+RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED, RHT_TENSOR_CORE = 0, 1, 2, 3
 
 
 class RsqError(RuntimeError):
@@ -68,7 +68,7 @@ def launch_count() -> int:
 
 
 def select_align_kernel(which: int) -> int:
-    """0 auto, 1 CUDA-core kernel, 2 tensor-core kernel only; returns the previous setting."""
+    """0 auto, 1 CUDA-core, 2 single-tile tensor-core, 3 double-buffered tensor-core; returns the previous setting."""
     prev = int(_lib.rsq_select_align_kernel(int(which)))
     if prev < 0:
         raise ValueError(which)
@@ -76,7 +76,7 @@ def select_align_kernel(which: int) -> int:
 
 
 def select_rht_kernel(which: int) -> int:
-    """0 auto, 1 radix-16 shared-memory kernel, 2 specialised kernel only; returns the previous setting."""
+    """0 auto, 1 radix-16 SMEM kernel, 2 warp-per-row kernel, 3 tensor-core kernel; returns the previous setting."""
     prev = int(_lib.rsq_select_rht_kernel(int(which)))
     if prev < 0:
         raise ValueError(which)

@@ -67,6 +67,7 @@ struct AlignTcArgs {
     int r;
     int rows_per_tile;
     int tiles_per_cluster;
+    int codes_v8;  // codes pointer is 32-byte aligned: 256-bit stores
     float eps;
 };
 
@@ -243,6 +244,12 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             for (int s = 0; s < kSlabs; ++s)
                 tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(t0), bar_load);
         };
+        // next tile's slabs, each issued once the x_out store has read that slab
+        long long next_t0 = -1;
+        auto refill = [&](int s) {  // thread 0 only
+            if (next_t0 >= 0)
+                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(next_t0), bar_load);
+        };
         // ------------------------------------------------ consumer warps
         const int quad = warp & 3, half = warp >> 2;
         const int m = quad * 32 + lane;  // tile row == TMEM lane
@@ -251,30 +258,6 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
         const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
         uint32_t ph = 0;  // every consumer barrier completes once per tile
-        // codes and scale of the previous tile, waiting to be stored
-        uint32_t pend[BITS * (kHalfCols / 32)];
-        uint8_t *pend_at = nullptr;
-        float pend_scale = 0.f;
-        float *pend_scale_at = nullptr;
-        auto flush = [&]() {
-            if (pend_at) {
-                if (BITS == 4) {
-#pragma unroll
-                    for (int w = 0; w < BITS * (kHalfCols / 32) / 4; ++w)
-                        reinterpret_cast<uint4 *>(pend_at)[w] =
-                            make_uint4(pend[4 * w], pend[4 * w + 1], pend[4 * w + 2], pend[4 * w + 3]);
-                } else {  // INT3 rows are 8-byte aligned here
-#pragma unroll
-                    for (int w = 0; w < BITS * (kHalfCols / 32) / 2; ++w)
-                        reinterpret_cast<uint2 *>(pend_at)[w] = make_uint2(pend[2 * w], pend[2 * w + 1]);
-                }
-                pend_at = nullptr;
-            }
-            if (pend_scale_at) {
-                *pend_scale_at = pend_scale;
-                pend_scale_at = nullptr;
-            }
-        };
 
         for (int it = 0; it < p.tiles_per_cluster; ++it) {
             const long long t0 = tile_t0(it);
@@ -375,7 +358,6 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             fence_proxy_async();
             cluster_sync();  // #2 z of all rows is in every CTA's operand buffer
-            flush();         // previous tile's codes and scales
 
             // ---- c = z Q^T (hi/lo split): half h into TMEM columns [256 h, 256 h + 256)
             if (tid == 0) {
@@ -447,11 +429,16 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             tc_fence_before();
             cluster_sync();  // #3 statistics visible; every thread's x_out is in the tile buffer
             if (tid == 0) {  // x_out back to HBM (issued after the barrier, whose release
-                             // semantics would otherwise wait for this bulk store)
+                             // semantics would otherwise wait for this bulk store); one
+                             // bulk group per slab so the slabs can be refilled one by one
 #pragma unroll
-                for (int s = 0; s < kSlabs; ++s)
+                for (int s = 0; s < kSlabs; ++s) {
                     tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
-                bulk_commit();
+                    bulk_commit();
+                }
+                const long long tn = tile_t0(it + 1);
+                next_t0 = (it + 1 < p.tiles_per_cluster && tn < p.T) ? tn : -1;
+                if (next_t0 >= 0) mbar_expect_tx(bar_load, uint32_t(kSlabs * R * 128));
             }
 
             // row totals over the cluster (fixed order: deterministic), computed by
@@ -470,17 +457,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const float ms = float(ss_t / double(p.D));
                 const float rs = 1.0f / sqrtf(ms + p.eps);
                 const RowQuant q = row_quant(am_t, qmax);
-                if (crank == 0 && m < nrows) {  // stored after the next tile's second barrier
-                    pend_scale = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
-                    pend_scale_at = p.scales + t0 + m;
-                }
+                if (crank == 0 && m < nrows) p.scales[t0 + m] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
                 reinterpret_cast<float *>(sloc + m * 16)[0] = q.inv;
                 reinterpret_cast<float *>(sloc + m * 16)[1] = q.pre;
-            }
-            if (tid == 0) {  // the tile buffer is free once TMA has read x_out: fetch the next tile
-                bulk_wait_read0();
-                const long long tn = tile_t0(it + 1);
-                if (it + 1 < p.tiles_per_cluster && tn < p.T) issue_load(tn);
             }
             named_sync(1, kConsumers);
             RowQuant rq;
@@ -489,32 +468,52 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             const bool scaled = rq.pre != 1.0f;
             const bool valid = m < nrows;
 
-            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined); the codes
-            // stay in registers and are stored after the next tile's second cluster
-            // barrier, so that no barrier's release has to wait for these stores
+            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined); thread 0
+            // also refills the tile buffer slab by slab as the x_out store drains
             {
                 constexpr int kBlocks = kHalfCols / 32;
                 const uint32_t taddr = tmem + lane_base + tcol;
+                uint8_t *crow = p.codes + (t0 + m) * row_bytes + (long long)(col0 + half * kHalfCols) * BITS / 8;
                 uint32_t va[32], vb[32];
                 tmem_ld32(taddr, va);
                 tmem_wait_ld();
 #pragma unroll
                 for (int b = 0; b < kBlocks; b += 2) {
+                    uint32_t words[2 * BITS];  // 64 codes
                     tmem_ld32(taddr + (b + 1) * 32, vb);
-                    code_block<BITS>(va, rq, scaled, pend + b * BITS);
+                    code_block<BITS>(va, rq, scaled, words);
                     tmem_wait_ld();
                     if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
-                    code_block<BITS>(vb, rq, scaled, pend + (b + 1) * BITS);
+                    code_block<BITS>(vb, rq, scaled, words + BITS);
+                    if (valid) {
+                        uint8_t *dst = crow + (b / 2) * (BITS * 8);
+                        if (BITS == 4 && p.codes_v8) {
+                            st_global_v8(dst, words);
+                        } else if (BITS == 4) {
+                            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(words[4], words[5], words[6], words[7]);
+                        } else {
+                            reinterpret_cast<uint2 *>(dst)[0] = make_uint2(words[0], words[1]);
+                            reinterpret_cast<uint2 *>(dst)[1] = make_uint2(words[2], words[3]);
+                            reinterpret_cast<uint2 *>(dst)[2] = make_uint2(words[4], words[5]);
+                        }
+                    }
+                    if (tid == 0) {  // slabs 2j, 2j+1 of x_out have been read: reload them
+                        const int j = b / 2;
+                        if (j == 0) bulk_wait_read<6>();
+                        else if (j == 1) bulk_wait_read<4>();
+                        else if (j == 2) bulk_wait_read<2>();
+                        else bulk_wait_read<0>();
+                        refill(2 * j);
+                        refill(2 * j + 1);
+                    }
                     tmem_wait_ld();
                 }
-                pend_at = valid ? p.codes + (t0 + m) * row_bytes + (long long)(col0 + half * kHalfCols) * BITS / 8
-                                : nullptr;
             }
             tc_fence_before();
             named_sync(1, kConsumers);  // TMEM reads done before the next tile's MMAs
             ph ^= 1;
         }
-        flush();
         if (tid == 0) bulk_wait0();
     }
 
@@ -620,6 +619,7 @@ struct TcKernel {
         a.r = r;
         a.rows_per_tile = R;
         a.tiles_per_cluster = tpc;
+        a.codes_v8 = (reinterpret_cast<uintptr_t>(codes) & 31u) == 0;
         a.eps = eps;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];

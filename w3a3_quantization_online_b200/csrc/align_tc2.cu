@@ -90,12 +90,6 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 
 __device__ __forceinline__ float bf16_val(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
 
-__device__ __forceinline__ void st_global_v8(void *p, const uint32_t *w) {
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
-                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-                 : "memory");
-}
-
 // x_out = x + c for one 32-column block (see align_tc.cu).
 __device__ __forceinline__ void xout_block(uint32_t (&v)[32], uint8_t *rowp, int m, int chunk0, float2 &s2,
                                            float (&am)[4]) {

@@ -19,11 +19,12 @@
 // The signs are applied to the tiles in shared memory (XOR of the bf16 sign
 // bits) before the product.  The 1/sqrt(4096) = 1/64 factor goes to the scale.
 //
-// Pipeline: 2 tile stages (4 tokens, 32 KB each) loaded by TMA ahead of use;
-// 2 TMEM slots of 128 columns, so the product of group g overlaps the
-// epilogue of group g - 1.  Two CTAs share each SM (104 KB of shared memory and
-// 256 TMEM columns each), so one CTA's barriers and waits hide behind the
-// other's work.  Waits are bounded (device status word).
+// Pipeline (one CTA per SM): a producer warp streams 4-token groups into 5
+// tile stages (32 KB each) by TMA; two consumer warp groups (8 warps each) take
+// alternate groups, each with two of the four 128-column TMEM slots, so one
+// group's product overlaps its own previous epilogue and the other warp group's
+// work.  A stage is released by the tcgen05 commit of the product that read
+// it.  Waits are bounded (device status word).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -36,20 +37,21 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int kGroupWarps = 8;                // one consumer warp group
+constexpr int kGroupThreads = kGroupWarps * 32;
+constexpr int kConsumerGroups = 2;
+constexpr int kThreads = kConsumerGroups * kGroupThreads + 32;  // + producer warp
 constexpr int kTok = 4;                       // tokens per group (one MMA set)
 constexpr int kTileBytes = 64 * 128;          // one token: 64 rows x 128 B (bf16)
 constexpr int kStageBytes = kTok * kTileBytes;  // 32 KB
-constexpr int kStages = 2;
-constexpr int kSlots = 2;                     // TMEM slots of 128 columns
-constexpr int kCtasPerSm = 2;                 // two independent pipelines per SM
+constexpr int kStages = 5;
+constexpr int kSlots = 4;                     // TMEM slots of 128 columns (two per warp group)
 constexpr int kOffA = 0;                      // diag(H_64, H_64), K-major SW128: 2 slabs x 16 KB
 constexpr int kOffMask = kOffA + 2 * 16384;   // 8 KB sign masks, laid out like a token tile
 constexpr int kOffStage = kOffMask + kTileBytes;
-constexpr int kOffRed = kOffStage + kStages * kStageBytes;  // [token 4][half-quadrant 2] absmax partials
-constexpr int kOffBar = kOffRed + kTok * 2 * 4;
-constexpr int kOffTmem = kOffBar + (kStages + kSlots) * 8;
+constexpr int kOffRed = kOffStage + kStages * kStageBytes;  // [warp group][token 4][half-quadrant 2]
+constexpr int kOffBar = kOffRed + kConsumerGroups * kTok * 2 * 4;
+constexpr int kOffTmem = kOffBar + (2 * kStages + kSlots) * 8;  // full[], empty[], mma[]
 constexpr int kBytes = kOffTmem + 16;
 constexpr int kSmem = kBytes + 1024;
 
@@ -85,7 +87,7 @@ __device__ __forceinline__ void fwht64(float (&v)[64]) {
 }
 
 template <int BITS>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
 k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ signs,
              uint8_t *__restrict__ codes, float *__restrict__ scales, long long T, int *status) {
     constexpr int qmax = (1 << (BITS - 1)) - 1;
@@ -95,9 +97,9 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
     uint8_t *sa = base + kOffA;
     uint8_t *smask = base + kOffMask;
     uint8_t *sstage = base + kOffStage;
-    float *sred = reinterpret_cast<float *>(base + kOffRed);
-    const uint32_t bar_full = smem_u32(base + kOffBar);             // kStages barriers
-    const uint32_t bar_mma = bar_full + 8 * kStages;                // kSlots barriers
+    const uint32_t bar_full = smem_u32(base + kOffBar);   // kStages: tile landed
+    const uint32_t bar_empty = bar_full + 8 * kStages;    // kStages: tile consumed by its product
+    const uint32_t bar_mma = bar_empty + 8 * kStages;     // kSlots: product done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTmem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int err = 0;
@@ -129,7 +131,10 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
         *reinterpret_cast<uint32_t *>(smask + tile_off(a, j >> 2) + (j & 3) * 4) = mk;
     }
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(bar_full + 8 * s, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
         for (int s = 0; s < kSlots; ++s) mbar_init(bar_mma + 8 * s, 1);
         fence_mbar_init();
         prefetch_tmap(&tm_x);
@@ -147,124 +152,138 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
     const long long ngroups = (T + kTok - 1) / kTok;
     const long long g0 = blockIdx.x, gstep = gridDim.x;
     const int nmine = g0 < ngroups ? int((ngroups - 1 - g0) / gstep + 1) : 0;
-    auto issue_load = [&](int it) {  // thread 0
-        const int s = it % kStages;
-        mbar_expect_tx(bar_full + 8 * s, kStageBytes);
-        tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok), bar_full + 8 * s);
-    };
-    if (tid == 0)
-        for (int it = 0; it < kStages && it < nmine; ++it) issue_load(it);
 
-    const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
-    // epilogue mapping: TMEM lane (p, a) = 64 p + a, column half q
-    const int quad = warp & 3, q = warp >> 2;
-    const int lrow = quad * 32 + lane;
-    const int p = lrow >> 6, a = lrow & 63;
-    const int tslot = p + 2 * q;  // token within the group
-
-    auto epilogue = [&](int it) {
-        const int slot = it % kSlots;
-        if (!mbar_wait(bar_mma + 8 * slot, uint32_t((it / kSlots) & 1), err != 0)) err |= kErrMbarTimeout;
-        tc_fence_after();
-        float v[64];
-        {
-            uint32_t r0[32], r1[32];
-            const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + uint32_t(slot * 128 + q * 64);
-            tmem_ld32(taddr, r0);
-            tmem_ld32(taddr + 32, r1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                v[k] = __uint_as_float(r0[k]);
-                v[k + 32] = __uint_as_float(r1[k]);
+    if (warp == kConsumerGroups * kGroupWarps) {
+        // ------------------------------------------------ producer warp
+        if (lane == 0) {
+            for (int it = 0; it < nmine; ++it) {
+                const int s = it % kStages;
+                if (it >= kStages)  // the product of group it - kStages has read this stage
+                    if (!mbar_wait(bar_empty + 8 * s, uint32_t((it / kStages - 1) & 1), err != 0))
+                        err |= kErrMbarTimeout;
+                mbar_expect_tx(bar_full + 8 * s, kStageBytes);
+                tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok),
+                            bar_full + 8 * s);
             }
         }
-        fwht64(v);  // along b: row a of token tslot is now final
-        float mx[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) mx[k] = fabsf(v[k]);
-#pragma unroll
-        for (int k = 4; k < 64; ++k) mx[k & 3] = fmaxf(mx[k & 3], fabsf(v[k]));
-        const float wm = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
-        // the 64 rows of a token live in quadrants 2p, 2p+1 of column half q
-        if (lane == 0) sred[tslot * 2 + (quad & 1)] = wm;
-        named_sync(1, kThreads);
-        const float amax = fmaxf(sred[tslot * 2], sred[tslot * 2 + 1]);
-        const long long t = (g0 + (long long)it * gstep) * kTok + tslot;
-        if (t < T) {
-            const RowQuant rq = row_quant(amax, qmax);
-            const bool scaled = rq.pre != 1.0f;
-            uint32_t w[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = v[8 * k + e];
-                w[k] = pack8_fast<BITS>(f, rq.inv, rq.pre, scaled);
-            }
-            uint8_t *dst = codes + t * row_bytes + a * (8 * BITS);
-            if (BITS == 4) {
-                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            } else {  // 8 groups of 24 bits -> 6 words
-                uint32_t o[6];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    o[3 * h + 0] = w[4 * h] | (w[4 * h + 1] << 24);
-                    o[3 * h + 1] = (w[4 * h + 1] >> 8) | (w[4 * h + 2] << 16);
-                    o[3 * h + 2] = (w[4 * h + 2] >> 16) | (w[4 * h + 3] << 8);
-                }
-#pragma unroll
-                for (int h = 0; h < 3; ++h) reinterpret_cast<uint2 *>(dst)[h] = make_uint2(o[2 * h], o[2 * h + 1]);
-            }
-            if (a == 0) scales[t] = amax > 0.f ? amax / float(qmax * 64) : 0.f;
-        }
-        tc_fence_before();
-        named_sync(1, kThreads);  // sred reuse; TMEM slot reads done
-    };
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ consumer warp groups
+        const int wg = warp / kGroupWarps;              // takes local groups wg, wg + 2, ...
+        const int gtid = tid - wg * kGroupThreads;      // thread within the warp group
+        const int gw = warp - wg * kGroupWarps;
+        const uint32_t named = 1 + wg;
+        float *sred = reinterpret_cast<float *>(base + kOffRed) + wg * kTok * 2;
+        const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
+        // epilogue mapping: TMEM lane (p, a) = 64 p + a, column half q
+        const int quad = gw & 3, q = gw >> 2;
+        const int lrow = quad * 32 + lane;
+        const int p = lrow >> 6, a = lrow & 63;
+        const int tslot = p + 2 * q;  // token within the group
 
-    for (int it = 0; it < nmine; ++it) {
-        const int s = it % kStages, slot = it % kSlots;
-        if (!mbar_wait(bar_full + 8 * s, uint32_t((it / kStages) & 1), err != 0)) err |= kErrMbarTimeout;
-        // apply the random signs to the four tiles (XOR of bf16 sign bits)
-        uint8_t *st = sstage + s * kStageBytes;
-#pragma unroll
-        for (int k = 0; k < (kStageBytes / 16) / kThreads; ++k) {
-            const int c = tid + k * kThreads;           // 16-byte chunk within the stage
-            const int within = c & (kTileBytes / 16 - 1);  // same position in the mask tile
-            uint4 xv = reinterpret_cast<uint4 *>(st)[c];
-            const uint4 mv = reinterpret_cast<const uint4 *>(smask)[within];
-            xv.x ^= mv.x;
-            xv.y ^= mv.y;
-            xv.z ^= mv.z;
-            xv.w ^= mv.w;
-            reinterpret_cast<uint4 *>(st)[c] = xv;
-        }
-        fence_proxy_async_cta();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+        auto epilogue = [&](int it) {
+            const int slot = it % kSlots;
+            if (!mbar_wait(bar_mma + 8 * slot, uint32_t((it / kSlots) & 1), err != 0)) err |= kErrMbarTimeout;
             tc_fence_after();
-            // A: K-major, K-steps of 16 are 32 bytes apart within a slab, slabs 16 KB apart.
-            // B: MN-major, K rows (p', a') 128 B apart (16 per K-step: 2 KB), the two
-            //    64-column atoms (token pairs q = 0, 1) 16 KB apart.
-            const uint64_t ad0 = smem_desc_sw128(smem_u32(sa), 1024);
-            const uint64_t bd0 = smem_desc_sw128_lbo(smem_u32(st), 16384, 1024);
+            float v[64];
+            {
+                uint32_t r0[32], r1[32];
+                const uint32_t taddr = tmem + (uint32_t(quad * 32) << 16) + uint32_t(slot * 128 + q * 64);
+                tmem_ld32(taddr, r0);
+                tmem_ld32(taddr + 32, r1);
+                tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t aoff = uint32_t((k >> 2) * 16384 + (k & 3) * 32) >> 4;
-                const uint32_t boff = uint32_t(k * 2048) >> 4;
-                umma_f16(tmem + uint32_t(slot * 128), ad0 + aoff, bd0 + boff, idesc, k != 0);
+                for (int k = 0; k < 32; ++k) {
+                    v[k] = __uint_as_float(r0[k]);
+                    v[k + 32] = __uint_as_float(r1[k]);
+                }
             }
-            umma_commit(bar_mma + 8 * slot);
+            fwht64(v);  // along b: row a of token tslot is now final
+            float mx[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx[k] = fabsf(v[k]);
+#pragma unroll
+            for (int k = 4; k < 64; ++k) mx[k & 3] = fmaxf(mx[k & 3], fabsf(v[k]));
+            const float wm = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+            // the 64 rows of a token live in quadrants 2p, 2p+1 of column half q
+            if (lane == 0) sred[tslot * 2 + (quad & 1)] = wm;
+            named_sync(named, kGroupThreads);
+            const float amax = fmaxf(sred[tslot * 2], sred[tslot * 2 + 1]);
+            const long long t = (g0 + (long long)it * gstep) * kTok + tslot;
+            if (t < T) {
+                const RowQuant rq = row_quant(amax, qmax);
+                const bool scaled = rq.pre != 1.0f;
+                uint32_t w[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = v[8 * k + e];
+                    w[k] = pack8_fast<BITS>(f, rq.inv, rq.pre, scaled);
+                }
+                uint8_t *dst = codes + t * row_bytes + a * (8 * BITS);
+                if (BITS == 4) {
+                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                } else {  // 8 groups of 24 bits -> 6 words
+                    uint32_t o[6];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        o[3 * h + 0] = w[4 * h] | (w[4 * h + 1] << 24);
+                        o[3 * h + 1] = (w[4 * h + 1] >> 8) | (w[4 * h + 2] << 16);
+                        o[3 * h + 2] = (w[4 * h + 2] >> 16) | (w[4 * h + 3] << 8);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 3; ++h) reinterpret_cast<uint2 *>(dst)[h] = make_uint2(o[2 * h], o[2 * h + 1]);
+                }
+                if (a == 0) scales[t] = amax > 0.f ? amax / float(qmax * 64) : 0.f;
+            }
+            tc_fence_before();
+            named_sync(named, kGroupThreads);  // sred reuse; TMEM slot reads done
+        };
+
+        int prev = -1;
+        for (int it = wg; it < nmine; it += kConsumerGroups) {
+            const int s = it % kStages, slot = it % kSlots;
+            if (!mbar_wait(bar_full + 8 * s, uint32_t((it / kStages) & 1), err != 0)) err |= kErrMbarTimeout;
+            // apply the random signs to the four tiles (XOR of bf16 sign bits)
+            uint8_t *st = sstage + s * kStageBytes;
+#pragma unroll
+            for (int k = 0; k < (kStageBytes / 16) / kGroupThreads; ++k) {
+                const int c = gtid + k * kGroupThreads;        // 16-byte chunk within the stage
+                const int within = c & (kTileBytes / 16 - 1);  // same position in the mask tile
+                uint4 xv = reinterpret_cast<uint4 *>(st)[c];
+                const uint4 mv = reinterpret_cast<const uint4 *>(smask)[within];
+                xv.x ^= mv.x;
+                xv.y ^= mv.y;
+                xv.z ^= mv.z;
+                xv.w ^= mv.w;
+                reinterpret_cast<uint4 *>(st)[c] = xv;
+            }
+            fence_proxy_async_cta();
+            tc_fence_before();
+            named_sync(named, kGroupThreads);
+            if (gtid == 0) {
+                tc_fence_after();
+                // A: K-major, K-steps of 16 are 32 bytes apart within a slab, slabs 16 KB apart.
+                // B: MN-major, K rows (p', a') 128 B apart (16 per K-step: 2 KB), the two
+                //    64-column atoms (token pairs q = 0, 1) 16 KB apart.
+                const uint64_t ad0 = smem_desc_sw128(smem_u32(sa), 1024);
+                const uint64_t bd0 = smem_desc_sw128_lbo(smem_u32(st), 16384, 1024);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t aoff = uint32_t((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+                    const uint32_t boff = uint32_t(k * 2048) >> 4;
+                    umma_f16(tmem + uint32_t(slot * 128), ad0 + aoff, bd0 + boff, idesc, k != 0);
+                }
+                umma_commit(bar_mma + 8 * slot);
+                umma_commit(bar_empty + 8 * s);  // the stage can be refilled once the product is done
+            }
+            if (prev >= 0) epilogue(prev);
+            prev = it;
         }
-        if (it >= 1) {
-            epilogue(it - 1);
-            // group it-1's product has completed, so its stage can be refilled
-            if (tid == 0 && it - 1 + kStages < nmine) issue_load(it - 1 + kStages);
-        }
+        if (prev >= 0) epilogue(prev);
     }
-    if (nmine > 0) epilogue(nmine - 1);
 
     tc_fence_before();
     __syncthreads();
@@ -317,7 +336,7 @@ cudaError_t launch_bits(const void *x, const int8_t *signs, uint8_t *codes, floa
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const long long ngroups = (T + kTok - 1) / kTok;
-    long long grid = (long long)num_sms() * kCtasPerSm;
+    long long grid = num_sms();
     if (grid > ngroups) grid = ngroups;
     kern<<<int(grid), kThreads, kSmem, st>>>(map, signs, codes, scales, T, status);
     e = cudaGetLastError();

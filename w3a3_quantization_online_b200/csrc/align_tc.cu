@@ -50,11 +50,12 @@ constexpr int kSlabBytes = kTileM * 128;     // 16 KB
 constexpr int kXBytes = kSlabs * kSlabBytes; // 128 KB
 constexpr int kQBytes = kCols * 128;         // 64 KB: 512 rows x [Q_hi(32) | Q_lo(32)] bf16
 constexpr int kZBytes = kTileM * 128;        // 16 KB: partial y (fp32) / z hi|lo (bf16), per row
-constexpr int kConsumerWarps = 8;             // two warps per TMEM lane quadrant
+constexpr int kParts = 4;                      // warps per TMEM lane quadrant (column parts)
+constexpr int kConsumerWarps = 4 * kParts;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers;
 constexpr int kTmemCols = 512;
-constexpr int kHalfCols = kCols / 2;           // columns per consumer warp group
+constexpr int kPartCols = kCols / kParts;      // columns per thread (128)
 
 struct AlignTcArgs {
     const float *Q;
@@ -80,8 +81,8 @@ struct Layout {
     static constexpr int kOffM = kOffZ + kZBytes;                       // M^T, 32 x 32 fp32, zero padded
     static constexpr int kOffYred = kOffM + 32 * 32 * 4;
     static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;  // per row: CTA partial (ss, amax), 16 B
-    static constexpr int kOffLoc = kOffStat + kTileM * 16;              // per row: half-1 partial, then row quantiser
-    static constexpr int kOffBar = kOffLoc + kTileM * 16;
+    static constexpr int kOffLoc = kOffStat + kTileM * 16;  // per row: parts 1.. partials, then row quantiser
+    static constexpr int kOffBar = kOffLoc + (kParts - 1) * kTileM * 16;
     static constexpr int kNumBars = 5;  // load, y, c0, c1, x_out ready
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffTmem + 16;
@@ -125,7 +126,7 @@ __device__ __forceinline__ void xout_block(uint32_t (&v)[32], uint8_t *rowp, int
             v[q * 8 + 2 * e] = __float_as_uint(y.x);
             v[q * 8 + 2 * e + 1] = __float_as_uint(y.y);
             s2 = fma2(y, y, s2);
-            am[e] = fmaxf(am[e], fmaxf(fabsf(y.x), fabsf(y.y)));
+            am[e] = max3(am[e], fabsf(y.x), fabsf(y.y));
             o[e] = pack_bf16x2(y.x, y.y);
         }
         *reinterpret_cast<uint4 *>(cp) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -159,10 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xo,
            const AlignTcArgs p) {
     using L = Layout<CS>;
-    constexpr int TPO = L::kTokPerOwner;    // token rows reduced by each CTA
-    constexpr int KPT = 32 * TPO / kConsumers;  // projection entries per thread in the reduction
-    constexpr int TPT = 32 / KPT;           // threads per token row in the reduction
-    static_assert(CS * kCols <= 16384 && (KPT == 1 || KPT == 2) && TPT <= 32, "cluster shape");
+    constexpr int TPO = L::kTokPerOwner;    // token rows reduced by each CTA: one warp each
+    static_assert(CS * kCols <= 16384 && TPO <= kConsumerWarps, "cluster shape");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -251,10 +250,11 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(next_t0), bar_load);
         };
         // ------------------------------------------------ consumer warps
-        const int quad = warp & 3, half = warp >> 2;
+        const int quad = warp & 3, part = warp >> 2;
+        const int half = part >> 1;      // which MMA2 half (256 columns) this warp reads
         const int m = quad * 32 + lane;  // tile row == TMEM lane
         const uint32_t lane_base = uint32_t(quad * 32) << 16;
-        const uint32_t tcol = uint32_t(half * kHalfCols);
+        const uint32_t tcol = uint32_t(part * kPartCols);
         const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
         const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
         uint32_t ph = 0;  // every consumer barrier completes once per tile
@@ -282,7 +282,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             if (!mbar_wait(bar_y, ph, err != 0)) err |= kErrMbarTimeout;
             tc_fence_after();
-            if (half == 0) {
+            if (part == 0) {
                 uint32_t a[32], b[32];
                 tmem_ld32(tmem + lane_base + 0, a);
                 tmem_ld32(tmem + lane_base + 32, b);
@@ -302,58 +302,30 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             cluster_sync();  // #1 partial projections of all CTAs are visible
 
             // ---- owner CTA: sum partials of its TPO rows, z = M y, scatter z hi|lo
-            {
-                const int mloc = tid / TPT, kq = tid % TPT;
+            // (one warp per row, one projection entry per lane)
+            if (warp < TPO) {
+                const int mloc = warp, kq = lane;
                 const int mo = int(crank) * TPO + mloc;
                 const uint32_t row_addr = smem_u32(sz + mo * 128);
-                float ys[KPT];
-                if constexpr (KPT == 2) {
-                    float2 pv[CS];
+                float pv[CS];
 #pragma unroll
-                    for (int c = 0; c < CS; ++c)
-                        pv[c] = ld_dsmem_f2(mapa(row_addr, uint32_t(c)) + swz(mo, kq >> 1) + 8 * (kq & 1));
-                    ys[0] = 0.f;
-                    ys[1] = 0.f;
+                for (int c = 0; c < CS; ++c)
+                    pv[c] = ld_dsmem_f32(mapa(row_addr, uint32_t(c)) + swz(mo, kq >> 2) + 4 * (kq & 3));
+                float y = 0.f;
 #pragma unroll
-                    for (int c = 0; c < CS; ++c) {
-                        ys[0] += pv[c].x;
-                        ys[1] += pv[c].y;
-                    }
-                } else {
-                    float pv[CS];
-#pragma unroll
-                    for (int c = 0; c < CS; ++c)
-                        pv[c] = ld_dsmem_f32(mapa(row_addr, uint32_t(c)) + swz(mo, kq >> 2) + 4 * (kq & 3));
-                    ys[0] = 0.f;
-#pragma unroll
-                    for (int c = 0; c < CS; ++c) ys[0] += pv[c];
-                }
-#pragma unroll
-                for (int e = 0; e < KPT; ++e) syred[mloc * 32 + kq * KPT + e] = ys[e];
+                for (int c = 0; c < CS; ++c) y += pv[c];
+                syred[mloc * 32 + kq] = y;
                 __syncwarp();
-                uint16_t hi[KPT], lo[KPT];
+                float acc = 0.f;
 #pragma unroll
-                for (int e = 0; e < KPT; ++e) {
-                    const int j = kq * KPT + e;
-                    const float *yv = syred + mloc * 32;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) acc = fmaf(sm[k * 32 + j], yv[k], acc);
-                    hi[e] = bf16_bits(acc);
-                    lo[e] = bf16_bits(acc - bf16_val(hi[e]));
-                }
+                for (int k = 0; k < 32; ++k) acc = fmaf(sm[k * 32 + kq], syred[mloc * 32 + k], acc);
+                const uint16_t hi = bf16_bits(acc), lo = bf16_bits(acc - bf16_val(bf16_bits(acc)));
                 __syncwarp();
 #pragma unroll
                 for (int c = 0; c < CS; ++c) {
                     const uint32_t ra = mapa(row_addr, uint32_t(c));
-                    if constexpr (KPT == 2) {
-                        st_dsmem_u32(ra + swz(mo, kq >> 2) + 4 * (kq & 3), uint32_t(hi[0]) | (uint32_t(hi[1]) << 16));
-                        st_dsmem_u32(ra + swz(mo, 4 + (kq >> 2)) + 4 * (kq & 3),
-                                     uint32_t(lo[0]) | (uint32_t(lo[1]) << 16));
-                    } else {
-                        st_dsmem_u16(ra + swz(mo, kq >> 3) + 2 * (kq & 7), hi[0]);
-                        st_dsmem_u16(ra + swz(mo, 4 + (kq >> 3)) + 2 * (kq & 7), lo[0]);
-                    }
+                    st_dsmem_u16(ra + swz(mo, kq >> 3) + 2 * (kq & 7), hi);
+                    st_dsmem_u16(ra + swz(mo, 4 + (kq >> 3)) + 2 * (kq & 7), lo);
                 }
             }
             fence_proxy_async();
@@ -372,7 +344,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 for (int h = 0; h < 2; ++h) {
 #pragma unroll
                     for (int s = 0; s < 6; ++s)
-                        umma_f16(tmem + h * kHalfCols, ad0 + ((kA[s] * 32) >> 4),
+                        umma_f16(tmem + h * 256, ad0 + ((kA[s] * 32) >> 4),
                                  bd0 + ((uint32_t(h) * 32768 + kB[s] * 32) >> 4), idesc_c, s != 0);
                     umma_commit(h == 0 ? bar_c0 : bar_c1);
                 }
@@ -380,14 +352,14 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             if (!mbar_wait(half == 0 ? bar_c0 : bar_c1, ph, err != 0)) err |= kErrMbarTimeout;
             tc_fence_after();
 
-            // ---- pass 1: x_out = x + c over this warp's 256 columns (TMEM loads pipelined:
+            // ---- pass 1: x_out = x + c over this warp's 128 columns (TMEM loads pipelined:
             // the load of the next 32-column block overlaps the arithmetic of the current one)
             double ss = 0.0;
             float amax = 0.f;
             {
                 float2 s2 = make_float2(0.f, 0.f);
                 float am[4] = {0.f, 0.f, 0.f, 0.f};
-                constexpr int kBlocks = kHalfCols / 32;
+                constexpr int kBlocks = kPartCols / 32;
                 uint32_t va[32], vb[32];
                 const uint32_t taddr = tmem + lane_base + tcol;
                 uint8_t *xbase = sx + m * 128;
@@ -395,7 +367,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tmem_wait_ld();
 #pragma unroll 1
                 for (int b = 0; b < kBlocks; b += 2) {
-                    const int cb = half * kBlocks + b;  // 32-column block within the CTA slice
+                    const int cb = part * kBlocks + b;  // 32-column block within the CTA slice
                     tmem_wait_st();
                     tmem_ld32(taddr + (b + 1) * 32, vb);
                     xout_block(va, xbase + (cb >> 1) * kSlabBytes, m, (cb & 1) * 4, s2, am);
@@ -414,15 +386,18 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
             }
             fence_proxy_async_cta();  // x_out (generic writes) -> TMA store (async proxy)
-            // statistics: fold the two column halves of each row, publish one entry per row
-            if (half == 1) {
-                reinterpret_cast<double *>(sloc + m * 16)[0] = ss;
-                reinterpret_cast<float *>(sloc + m * 16)[2] = amax;
+            // statistics: fold the column parts of each row, publish one entry per row
+            if (part > 0) {
+                reinterpret_cast<double *>(sloc + ((part - 1) * kTileM + m) * 16)[0] = ss;
+                reinterpret_cast<float *>(sloc + ((part - 1) * kTileM + m) * 16)[2] = amax;
             }
             named_sync(1, kConsumers);
-            if (half == 0) {
-                ss += reinterpret_cast<const double *>(sloc + m * 16)[0];
-                amax = fmaxf(amax, reinterpret_cast<const float *>(sloc + m * 16)[2]);
+            if (part == 0) {
+#pragma unroll
+                for (int k = 0; k < kParts - 1; ++k) {
+                    ss += reinterpret_cast<const double *>(sloc + (k * kTileM + m) * 16)[0];
+                    amax = fmaxf(amax, reinterpret_cast<const float *>(sloc + (k * kTileM + m) * 16)[2]);
+                }
                 reinterpret_cast<double *>(sstat + m * 16)[0] = ss;
                 reinterpret_cast<float *>(sstat + m * 16)[2] = amax;
             }
@@ -442,8 +417,8 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
 
             // row totals over the cluster (fixed order: deterministic), computed by
-            // the half-0 thread of each row and handed to its half-1 partner
-            if (half == 0) {
+            // the part-0 thread of each row and handed to the other parts
+            if (part == 0) {
                 float4 sv[CS];
 #pragma unroll
                 for (int c = 0; c < CS; ++c) sv[c] = ld_dsmem_f4(mapa(smem_u32(sstat + m * 16), uint32_t(c)));
@@ -471,9 +446,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined); thread 0
             // also refills the tile buffer slab by slab as the x_out store drains
             {
-                constexpr int kBlocks = kHalfCols / 32;
+                constexpr int kBlocks = kPartCols / 32;
                 const uint32_t taddr = tmem + lane_base + tcol;
-                uint8_t *crow = p.codes + (t0 + m) * row_bytes + (long long)(col0 + half * kHalfCols) * BITS / 8;
+                uint8_t *crow = p.codes + (t0 + m) * row_bytes + (long long)(col0 + part * kPartCols) * BITS / 8;
                 uint32_t va[32], vb[32];
                 tmem_ld32(taddr, va);
                 tmem_wait_ld();
@@ -498,14 +473,12 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                             reinterpret_cast<uint2 *>(dst)[2] = make_uint2(words[4], words[5]);
                         }
                     }
-                    if (tid == 0) {  // slabs 2j, 2j+1 of x_out have been read: reload them
+                    if (tid == 0) {  // slabs 4j .. 4j+3 of x_out have been read: reload them
                         const int j = b / 2;
-                        if (j == 0) bulk_wait_read<6>();
-                        else if (j == 1) bulk_wait_read<4>();
-                        else if (j == 2) bulk_wait_read<2>();
+                        if (j == 0) bulk_wait_read<4>();
                         else bulk_wait_read<0>();
-                        refill(2 * j);
-                        refill(2 * j + 1);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) refill(4 * j + q);
                     }
                     tmem_wait_ld();
                 }

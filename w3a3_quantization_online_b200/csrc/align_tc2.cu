@@ -107,7 +107,7 @@ __device__ __forceinline__ void xout_block(uint32_t (&v)[32], uint8_t *rowp, int
             v[q * 8 + 2 * e] = __float_as_uint(y.x);
             v[q * 8 + 2 * e + 1] = __float_as_uint(y.y);
             s2 = fma2(y, y, s2);
-            am[e] = fmaxf(am[e], fmaxf(fabsf(y.x), fabsf(y.y)));
+            am[e] = max3(am[e], fabsf(y.x), fabsf(y.y));
             o[e] = pack_bf16x2(y.x, y.y);
         }
         *reinterpret_cast<uint4 *>(cp) = make_uint4(o[0], o[1], o[2], o[3]);

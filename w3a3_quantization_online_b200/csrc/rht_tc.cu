@@ -59,30 +59,31 @@ __device__ __forceinline__ uint32_t tile_off(int a, int chunk) {  // SWIZZLE_128
     return uint32_t(a * 128 + ((chunk ^ (a & 7)) << 4));
 }
 
-// In-place 64-point Sylvester transform of v[0..63]: stages for index bits 0..4
-// act on the pairs (v[k], v[k + 32]) with packed two-wide arithmetic, the stage
-// for bit 5 combines the two halves.
+// In-place 64-point Sylvester transform of v[0..63].  Adjacent elements form
+// the packed pairs (v[2j], v[2j+1]) -- the register pairs the TMEM load
+// delivers -- so the stages for index bits 1..5 are packed two-wide
+// butterflies between pairs and the stage for bit 0 works inside each pair.
 __device__ __forceinline__ void fwht64(float (&v)[64]) {
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1) {
+    for (int hv = 1; hv < 32; hv <<= 1) {  // pair stride: element stride 2 hv
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            if ((k & h) == 0) {
-                const float2 u = make_float2(v[k], v[k + 32]);
-                const float2 w = make_float2(v[k + h], v[k + h + 32]);
+        for (int j = 0; j < 32; ++j) {
+            if ((j & hv) == 0) {
+                const float2 u = make_float2(v[2 * j], v[2 * j + 1]);
+                const float2 w = make_float2(v[2 * (j + hv)], v[2 * (j + hv) + 1]);
                 const float2 s = add2(u, w), d = sub2(u, w);
-                v[k] = s.x;
-                v[k + 32] = s.y;
-                v[k + h] = d.x;
-                v[k + h + 32] = d.y;
+                v[2 * j] = s.x;
+                v[2 * j + 1] = s.y;
+                v[2 * (j + hv)] = d.x;
+                v[2 * (j + hv) + 1] = d.y;
             }
         }
     }
 #pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const float u = v[k], w = v[k + 32];
-        v[k] = u + w;
-        v[k + 32] = u - w;
+    for (int j = 0; j < 32; ++j) {
+        const float u = v[2 * j], w = v[2 * j + 1];
+        v[2 * j] = u + w;
+        v[2 * j + 1] = u - w;
     }
 }
 
@@ -199,12 +200,10 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
                 }
             }
             fwht64(v);  // along b: row a of token tslot is now final
-            float mx[4];
+            float mx[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains of three-input maxima
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mx[k] = fabsf(v[k]);
-#pragma unroll
-            for (int k = 4; k < 64; ++k) mx[k & 3] = fmaxf(mx[k & 3], fabsf(v[k]));
-            const float wm = warp_max(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+            for (int k = 0; k < 64; k += 2) mx[(k >> 1) & 3] = max3(mx[(k >> 1) & 3], fabsf(v[k]), fabsf(v[k + 1]));
+            const float wm = warp_max(max3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
             // the 64 rows of a token live in quadrants 2p, 2p+1 of column half q
             if (lane == 0) sred[tslot * 2 + (quad & 1)] = wm;
             named_sync(named, kGroupThreads);

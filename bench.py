@@ -64,6 +64,28 @@ def workload_config(T: int, n: int) -> dict:
     }
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank value over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, n_ranks: int, steps: int, elapsed_ms: float) -> float:
+    """Tokens per second over the whole job: every rank processes its own shard
+    of tokens_per_rank tokens per step; elapsed_ms is the max over ranks."""
+    return tokens_per_rank * n_ranks * steps / (elapsed_ms / 1e3)
+
+
+def shard_seed(rank: int) -> int:
+    """Seed of this rank's token shard (Q, M and signs are shared by all ranks)."""
+    return 1 + 1000 * rank
+
+
 def peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -245,7 +267,7 @@ def run_gpu(args) -> None:
     from w3a3_quantization_online_b200 import inputs, rsq
 
     T = args.tokens
-    a = inputs.align_case(T, D, R, 1 + 1000 * rank, dtype="bf16", bits=BITS, n_outliers=8,
+    a = inputs.align_case(T, D, R, shard_seed(rank), dtype="bf16", bits=BITS, n_outliers=8,
                           outlier_scale=100.0, qm_seed=1)
     signs_np = inputs.random_signs(D, 1)
     x_host = torch.from_numpy(a.x).to(torch.bfloat16).pin_memory()
@@ -298,12 +320,9 @@ def run_gpu(args) -> None:
     total_ms = ev[0][0].elapsed_time(ev[-1][2])
     align_ms = [e[0].elapsed_time(e[1]) for e in ev]
     rht_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if n > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
-    value = T * n * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(T, n, args.steps, total_ms)
 
     # end to end through the C ABI with host buffers: pinned H2D of the batch,
     # both kernels, D2H of every output, all inside the timed region
@@ -334,10 +353,8 @@ def run_gpu(args) -> None:
             e2e_step()
         e1.record(stream)
     torch.cuda.synchronize(dev)
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if n > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = T * n * e2e_steps / (float(te.item()) / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = whole_job_rate(T, n, e2e_steps, e2e_ms)
     h2d = x_host.numel() * 2
     d2h = x_out.numel() * 2 + codes_a.numel() + codes_h.numel() + 4 * (scales_a.numel() + scales_h.numel())
 

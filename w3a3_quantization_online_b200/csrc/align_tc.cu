@@ -11,22 +11,32 @@
 //    [512 c, 512 c + 512) and keeps its 512 x 32 slice of Q resident in shared
 //    memory for the whole persistent kernel.  Every token tile (up to 128 rows)
 //    is read from HBM exactly once by TMA and stays in shared memory until its
-//    x_out and codes are written.
+//    x_out has been written.
 //  * Both rank-32 contractions run on the 5th-generation tensor cores with fp32
 //    accumulators in TMEM.  x is exact in bf16; Q and z are split into bf16
 //    high and low parts (Q = Q_hi + Q_lo), which keeps the products accurate to
 //    about 2^-16 relative:
 //        y   = x [Q_hi | Q_lo]              (M=128, N=64, K=512 per CTA)
-//        c   = z_hi Q_hi^T + z_hi Q_lo^T + z_lo Q_hi^T   (M=128, N=2x256, K=96)
+//        c   = z_hi Q_hi^T + z_hi Q_lo^T + z_lo Q_hi^T   (M=128, N=4x128, K=96)
 //    The same shared-memory Q buffer serves as the MN-major B operand of the
 //    first product and the K-major B operand of the second.
-//  * The partial projections of the CS CTAs are reduced through distributed
-//    shared memory: the CTA that owns 128/CS token rows sums their partials,
-//    applies the r x r matrix M and writes z (split hi/lo) into every CTA's A
-//    operand buffer.  The RMS and absmax statistics are exchanged the same way.
+//  * Sixteen warps, four per TMEM lane quadrant, each on 128 columns of its 32
+//    rows.  Thread 0 also issues the tensor-core products (those of the first
+//    contraction follow the tile's slabs as they land) and the last warp the
+//    x_out stores and the next tile's loads.
+//  * Cross-CTA exchange.  After one cluster barrier the CTA that owns 128/CS
+//    token rows reads their CS partial projections through distributed shared
+//    memory, applies the r x r matrix M and copies z (split hi/lo) into every
+//    CTA's operand buffer by bulk copy, counted on a local mbarrier there.  The
+//    row statistics (sum of squares, absmax) are pushed with st.async to the
+//    row's owner, which forms the row quantiser and pushes it back to all CTAs.
+//    Every exchange needs all CTAs of the cluster, so one buffer per exchange
+//    suffices: no CTA can run a whole tile ahead of another.
 //  * x_out = x + c is formed in fp32, rounded to bf16 in place in the tile
-//    buffer and written back by TMA; the fp32 value goes back to TMEM, from
-//    which the codes are computed once the row statistics are known.
+//    buffer and written back by TMA, slab by slab; each slab takes the next
+//    tile as soon as its store has read it, so the load overlaps the statistics
+//    exchange and the codes.  The fp32 value goes back to TMEM, from which the
+//    codes are computed once the row quantiser arrives.
 // Every mbarrier wait is bounded; a timeout sets a bit in the device status
 // word and the kernel keeps its barrier sequence so that no CTA is left
 // waiting.
@@ -50,12 +60,12 @@ constexpr int kSlabBytes = kTileM * 128;     // 16 KB
 constexpr int kXBytes = kSlabs * kSlabBytes; // 128 KB
 constexpr int kQBytes = kCols * 128;         // 64 KB: 512 rows x [Q_hi(32) | Q_lo(32)] bf16
 constexpr int kZBytes = kTileM * 128;        // 16 KB: partial y (fp32) / z hi|lo (bf16), per row
-constexpr int kParts = 4;                      // warps per TMEM lane quadrant (column parts)
+constexpr int kParts = 4;                    // consumer warps per TMEM lane quadrant (column parts)
 constexpr int kConsumerWarps = 4 * kParts;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers;
 constexpr int kTmemCols = 512;
-constexpr int kPartCols = kCols / kParts;      // columns per thread (128)
+constexpr int kPartCols = kCols / kParts;    // columns per consumer thread (128)
 
 struct AlignTcArgs {
     const float *Q;
@@ -72,18 +82,28 @@ struct AlignTcArgs {
     float eps;
 };
 
+// mbarriers (each completes once per tile)
+enum : int {
+    kBarLd = 0,               // kSlabs: x slab landed (TMA)
+    kBarY = kBarLd + kSlabs,  // partial projection in TMEM (commit)
+    kBarZ,                    // z of all rows in the operand buffer (local owner warps + bulk copies)
+    kBarC,                    // 4: correction columns [128 q, 128 q + 128) in TMEM (commit)
+    kBarSt = kBarC + 4,       // owner: row statistics of all CTAs pushed (st.async)
+    kBarPrm,                  // row quantisers of all rows pushed (st.async)
+    kNumBars
+};
+
 template <int CS>
 struct Layout {
     static constexpr int kTokPerOwner = kTileM / CS;
     static constexpr int kOffX = 0;
     static constexpr int kOffQ = kOffX + kXBytes;
     static constexpr int kOffZ = kOffQ + kQBytes;
-    static constexpr int kOffM = kOffZ + kZBytes;                       // M^T, 32 x 32 fp32, zero padded
-    static constexpr int kOffYred = kOffM + 32 * 32 * 4;
-    static constexpr int kOffStat = kOffYred + kTokPerOwner * 32 * 4;  // per row: CTA partial (ss, amax), 16 B
-    static constexpr int kOffLoc = kOffStat + kTileM * 16;  // per row: parts 1.. partials, then row quantiser
+    static constexpr int kOffM = kOffZ + kZBytes;            // M^T, 32 x 32 fp32, zero padded
+    static constexpr int kOffSt = kOffM + 32 * 32 * 4;       // owner: [source CTA][own row] (ss, amax), 16 B
+    static constexpr int kOffPrm = kOffSt + CS * kTokPerOwner * 16;  // per row: (inv, pre)
+    static constexpr int kOffLoc = kOffPrm + kTileM * 8;     // column-part partial statistics, 16 B
     static constexpr int kOffBar = kOffLoc + (kParts - 1) * kTileM * 16;
-    static constexpr int kNumBars = 5;  // load, y, c0, c1, x_out ready
     static constexpr int kOffTmem = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffTmem + 16;
     static constexpr int kSmem = kBytes + 1024;  // slack for 1024-byte alignment
@@ -133,6 +153,20 @@ __device__ __forceinline__ void xout_block(uint32_t (&v)[32], uint8_t *rowp, int
     }
 }
 
+// Wait until at most n (0..7) of this thread's bulk groups still read shared memory.
+__device__ __forceinline__ void bulk_wait_read_n(int n) {
+    switch (n) {
+        case 0: bulk_wait_read<0>(); break;
+        case 1: bulk_wait_read<1>(); break;
+        case 2: bulk_wait_read<2>(); break;
+        case 3: bulk_wait_read<3>(); break;
+        case 4: bulk_wait_read<4>(); break;
+        case 5: bulk_wait_read<5>(); break;
+        case 6: bulk_wait_read<6>(); break;
+        default: bulk_wait_read<7>(); break;
+    }
+}
+
 // Codes of one 32-column block (INT4: 4 words, INT3: 3 words).
 template <int BITS>
 __device__ __forceinline__ void code_block(const uint32_t (&v)[32], const RowQuant &rq, bool scaled,
@@ -160,8 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xo,
            const AlignTcArgs p) {
     using L = Layout<CS>;
-    constexpr int TPO = L::kTokPerOwner;    // token rows reduced by each CTA: one warp each
-    static_assert(CS * kCols <= 16384 && TPO <= kConsumerWarps, "cluster shape");
+    constexpr int TPO = L::kTokPerOwner;    // token rows owned by each CTA: one consumer warp each
+    static_assert(CS * kCols <= 16384 && TPO <= kConsumerWarps && CS * TPO == kTileM, "cluster shape");
+    static_assert(TPO * CS <= kConsumers, "owner statistics threads");
+    constexpr int kZTx = (CS - 1) * TPO * 128;  // z rows arriving from the other CTAs
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,11 +205,11 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     uint8_t *sq = base + L::kOffQ;
     uint8_t *sz = base + L::kOffZ;
     float *sm = reinterpret_cast<float *>(base + L::kOffM);
-    float *syred = reinterpret_cast<float *>(base + L::kOffYred);
-    uint8_t *sstat = base + L::kOffStat;
+    uint8_t *sst = base + L::kOffSt;
+    uint8_t *sprm = base + L::kOffPrm;
     uint8_t *sloc = base + L::kOffLoc;
-    const uint32_t bar_load = smem_u32(base + L::kOffBar);
-    const uint32_t bar_y = bar_load + 8, bar_c0 = bar_load + 16, bar_c1 = bar_load + 24;
+    const uint32_t bars = smem_u32(base + L::kOffBar);
+    auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L::kOffTmem);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -186,12 +222,19 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     const int R = p.rows_per_tile;
     int err = 0;
 
+    auto tile_t0 = [&](int it) { return ((long long)cid + (long long)it * ncl) * R; };
+    auto has_tile = [&](int it) { return it < p.tiles_per_cluster && tile_t0(it) < p.T; };
+
     if (tid == 0) {
-        mbar_init(bar_load, 1);
-        mbar_init(bar_y, 1);
-        mbar_init(bar_c0, 1);
-        mbar_init(bar_c1, 1);
+        for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), i == kBarZ ? 1 + TPO : 1);
         fence_mbar_init();
+        // the pushed exchanges of the first tile (each barrier is re-armed by its
+        // waiter once the previous phase has completed)
+        if (has_tile(0)) {
+            mbar_expect_tx(bar(kBarZ), uint32_t(kZTx));
+            mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
+            mbar_expect_tx(bar(kBarPrm), uint32_t(kTileM * 8));
+        }
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -232,57 +275,55 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    cluster_sync();
-
-    auto tile_t0 = [&](int it) { return ((long long)cid + (long long)it * ncl) * R; };
+    cluster_sync();  // barriers initialised in every CTA before any push
 
     {
-        auto issue_load = [&](long long t0) {  // thread 0 only
-            mbar_expect_tx(bar_load, uint32_t(kSlabs * R * 128));
-#pragma unroll
-            for (int s = 0; s < kSlabs; ++s)
-                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(t0), bar_load);
-        };
-        // next tile's slabs, each issued once the x_out store has read that slab
-        long long next_t0 = -1;
-        auto refill = [&](int s) {  // thread 0 only
-            if (next_t0 >= 0)
-                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(next_t0), bar_load);
-        };
-        // ------------------------------------------------ consumer warps
         const int quad = warp & 3, part = warp >> 2;
-        const int half = part >> 1;      // which MMA2 half (256 columns) this warp reads
         const int m = quad * 32 + lane;  // tile row == TMEM lane
         const uint32_t lane_base = uint32_t(quad * 32) << 16;
         const uint32_t tcol = uint32_t(part * kPartCols);
         const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
-        const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
-        uint32_t ph = 0;  // every consumer barrier completes once per tile
+        const uint32_t idesc_c = idesc_bf16_f32(128, 128, false, false);
+        const uint32_t slab_tx = uint32_t(R * 128);
+        if (tid == 0 && has_tile(0)) {
+#pragma unroll 1
+            for (int s = 0; s < kSlabs; ++s) {
+                mbar_expect_tx(bar(kBarLd + s), slab_tx);
+                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(0)),
+                            bar(kBarLd + s));
+            }
+        }
 
-        for (int it = 0; it < p.tiles_per_cluster; ++it) {
+        for (int it = 0; has_tile(it); ++it) {
+            const uint32_t ph = uint32_t(it) & 1u;
             const long long t0 = tile_t0(it);
-            if (t0 >= p.T) break;
             const int nrows = int(p.T - t0 < R ? p.T - t0 : R);
-            if (tid == 0 && it == 0) issue_load(t0);
+            const bool next = has_tile(it + 1);
 
-            // ---- y = x [Q_hi | Q_lo] over this CTA's 512 columns
-            if (!mbar_wait(bar_load, ph, err != 0)) err |= kErrMbarTimeout;
+            // ---- y = x [Q_hi | Q_lo] over this CTA's 512 columns, slab by slab as the tile lands
             if (tid == 0) {
-                tc_fence_after();
-                // descriptors advance by 16-byte units in their start-address field
                 const uint64_t ad0 = opaque(smem_desc_sw128(smem_u32(sx), 1024));
                 const uint64_t bd0 = opaque(smem_desc_sw128(smem_u32(sq), 1024));
+#pragma unroll 1
+                for (int s = 0; s < kSlabs; ++s) {
+                    if (!mbar_wait(bar(kBarLd + s), ph, err != 0)) err |= kErrMbarTimeout;
+                    tc_fence_after();
 #pragma unroll
-                for (int i = 0; i < kSlabs * 4; ++i) {  // K = 512 in steps of 16
-                    const uint32_t aoff = uint32_t((i >> 2) * kSlabBytes + (i & 3) * 32) >> 4;
-                    const uint32_t boff = uint32_t(i * 2048) >> 4;
-                    umma_f16(tmem, ad0 + aoff, bd0 + boff, idesc_y, i != 0);
+                    for (int k = 0; k < 4; ++k) {  // K steps of 16 columns, 32 bytes apart
+                        const int i = 4 * s + k;
+                        const uint32_t aoff = uint32_t(s * kSlabBytes + k * 32) >> 4;
+                        const uint32_t boff = uint32_t(i * 2048) >> 4;
+                        umma_f16(tmem, ad0 + aoff, bd0 + boff, idesc_y, i != 0);
+                    }
                 }
-                umma_commit(bar_y);
+                umma_commit(bar(kBarY));
             }
-            if (!mbar_wait(bar_y, ph, err != 0)) err |= kErrMbarTimeout;
-            tc_fence_after();
+            __syncwarp();  // lanes of warp 0 wait here, not in a poll that competes with lane 0
+
+            // ---- partial projection of this CTA's columns -> operand buffer (fp32)
             if (part == 0) {
+                if (!mbar_wait(bar(kBarY), ph, err != 0)) err |= kErrMbarTimeout;
+                tc_fence_after();
                 uint32_t a[32], b[32];
                 tmem_ld32(tmem + lane_base + 0, a);
                 tmem_ld32(tmem + lane_base + 32, b);
@@ -299,13 +340,14 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
             }
             tc_fence_before();
-            cluster_sync();  // #1 partial projections of all CTAs are visible
+            cluster_arrive();  // #1 partial projections of all CTAs are visible
+            cluster_wait();
 
-            // ---- owner CTA: sum partials of its TPO rows, z = M y, scatter z hi|lo
-            // (one warp per row, one projection entry per lane)
+            // ---- owner CTA: sum the partials of its TPO rows (one warp per row, one
+            // projection entry per lane), z = M y, push z hi|lo to every CTA
             if (warp < TPO) {
-                const int mloc = warp, kq = lane;
-                const int mo = int(crank) * TPO + mloc;
+                const int kq = lane;
+                const int mo = int(crank) * TPO + warp;
                 const uint32_t row_addr = smem_u32(sz + mo * 128);
                 float pv[CS];
 #pragma unroll
@@ -314,46 +356,59 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 float y = 0.f;
 #pragma unroll
                 for (int c = 0; c < CS; ++c) y += pv[c];
-                syred[mloc * 32 + kq] = y;
-                __syncwarp();
                 float acc = 0.f;
 #pragma unroll
-                for (int k = 0; k < 32; ++k) acc = fmaf(sm[k * 32 + kq], syred[mloc * 32 + k], acc);
-                const uint16_t hi = bf16_bits(acc), lo = bf16_bits(acc - bf16_val(bf16_bits(acc)));
-                __syncwarp();
+                for (int k = 0; k < 32; ++k) acc = fmaf(sm[k * 32 + kq], __shfl_sync(0xFFFFFFFFu, y, k), acc);
+                const uint16_t hi = bf16_bits(acc), lo = bf16_bits(acc - bf16_val(hi));
+                const uint32_t hl = uint32_t(hi) | (uint32_t(lo) << 16);
+                // lane -> 16-byte chunk ch of the row (hi: z[8 ch ..], lo: z[8 (ch - 4) ..])
+                const int ch = lane & 7;
+                const int src0 = 8 * (ch & 3);
+                const int sh = ch >= 4 ? 16 : 0;
+                uint32_t hw[8];
 #pragma unroll
-                for (int c = 0; c < CS; ++c) {
-                    const uint32_t ra = mapa(row_addr, uint32_t(c));
-                    st_dsmem_u16(ra + swz(mo, kq >> 3) + 2 * (kq & 7), hi);
-                    st_dsmem_u16(ra + swz(mo, 4 + (kq >> 3)) + 2 * (kq & 7), lo);
-                }
+                for (int e = 0; e < 8; ++e) hw[e] = (__shfl_sync(0xFFFFFFFFu, hl, src0 + e) >> sh) & 0xFFFFu;
+                const uint32_t w0 = hw[0] | (hw[1] << 16), w1 = hw[2] | (hw[3] << 16);
+                const uint32_t w2 = hw[4] | (hw[5] << 16), w3 = hw[6] | (hw[7] << 16);
+                // the row goes into this CTA's operand buffer (its own partial has been
+                // read above), then by bulk copy (async proxy, like the tensor core that
+                // reads it) into the same row of every other CTA
+                if (lane < 8) *reinterpret_cast<uint4 *>(sz + mo * 128 + swz(mo, ch)) = make_uint4(w0, w1, w2, w3);
+                fence_proxy_async_cta();
+                __syncwarp();
+                if (lane < CS && lane != int(crank))
+                    bulk_copy_to_cluster(mapa(row_addr, uint32_t(lane)), row_addr, 128u,
+                                         mapa(bar(kBarZ), uint32_t(lane)));
+                if (lane == 0) mbar_arrive(bar(kBarZ));
             }
-            fence_proxy_async();
-            cluster_sync();  // #2 z of all rows is in every CTA's operand buffer
 
-            // ---- c = z Q^T (hi/lo split): half h into TMEM columns [256 h, 256 h + 256)
+            // ---- c = z Q^T (hi/lo split): quarter q into TMEM columns [128 q, 128 q + 128)
             if (tid == 0) {
+                if (!mbar_wait(bar(kBarZ), ph, err != 0)) err |= kErrMbarTimeout;
+                if (next) mbar_expect_tx(bar(kBarZ), uint32_t(kZTx));
                 tc_fence_after();
                 fence_proxy_async();
-                // (A K-step, B K-step) pairs: z_hi Q_hi^T, z_hi Q_lo^T, z_lo Q_hi^T; K-steps of 16
-                // columns are 32 bytes apart inside the 128-byte swizzled rows
                 const uint64_t ad0 = opaque(smem_desc_sw128(smem_u32(sz), 1024));
                 const uint64_t bd0 = opaque(smem_desc_sw128(smem_u32(sq), 1024));
+                // (A K-step, B K-step) pairs: z_hi Q_hi^T, z_hi Q_lo^T, z_lo Q_hi^T
                 constexpr uint32_t kA[6] = {0, 1, 0, 1, 2, 3}, kB[6] = {0, 1, 2, 3, 0, 1};
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int q = 0; q < 4; ++q) {
 #pragma unroll
                     for (int s = 0; s < 6; ++s)
-                        umma_f16(tmem + h * 256, ad0 + ((kA[s] * 32) >> 4),
-                                 bd0 + ((uint32_t(h) * 32768 + kB[s] * 32) >> 4), idesc_c, s != 0);
-                    umma_commit(h == 0 ? bar_c0 : bar_c1);
+                        umma_f16(tmem + q * 128, ad0 + ((kA[s] * 32) >> 4),
+                                 bd0 + ((uint32_t(q) * 16384 + kB[s] * 32) >> 4), idesc_c, s != 0);
+                    umma_commit(bar(kBarC + q));
                 }
             }
-            if (!mbar_wait(half == 0 ? bar_c0 : bar_c1, ph, err != 0)) err |= kErrMbarTimeout;
-            tc_fence_after();
+            __syncwarp();
 
             // ---- pass 1: x_out = x + c over this warp's 128 columns (TMEM loads pipelined:
             // the load of the next 32-column block overlaps the arithmetic of the current one)
+            if (!mbar_wait(bar(kBarLd + 2 * part), ph, err != 0)) err |= kErrMbarTimeout;
+            if (!mbar_wait(bar(kBarLd + 2 * part + 1), ph, err != 0)) err |= kErrMbarTimeout;
+            if (!mbar_wait(bar(kBarC + part), ph, err != 0)) err |= kErrMbarTimeout;
+            tc_fence_after();
             double ss = 0.0;
             float amax = 0.f;
             {
@@ -386,65 +441,80 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 amax = fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3]));
             }
             fence_proxy_async_cta();  // x_out (generic writes) -> TMA store (async proxy)
-            // statistics: fold the column parts of each row, publish one entry per row
+            // statistics: fold the column parts of each row; part 0 pushes the CTA's
+            // partial (ss, amax) of row m to the row's owner
             if (part > 0) {
                 reinterpret_cast<double *>(sloc + ((part - 1) * kTileM + m) * 16)[0] = ss;
                 reinterpret_cast<float *>(sloc + ((part - 1) * kTileM + m) * 16)[2] = amax;
             }
             named_sync(1, kConsumers);
+            if (warp == kConsumerWarps - 1) {
+                // x_out back to HBM, one bulk group per slab; each slab takes the next
+                // tile as soon as its store has read it (a warp with no statistics
+                // duty; the whole warp waits for its lane 0)
+                if (lane == 0) {
+#pragma unroll 1
+                    for (int s = 0; s < kSlabs; ++s) {
+                        tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
+                        bulk_commit();
+                    }
+                    if (next) {
+                        const int tn = int(tile_t0(it + 1));
+#pragma unroll 1
+                        for (int s = 0; s < kSlabs; ++s) {
+                            bulk_wait_read_n(kSlabs - 1 - s);
+                            mbar_expect_tx(bar(kBarLd + s), slab_tx);
+                            tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, tn,
+                                        bar(kBarLd + s));
+                        }
+                    }
+                }
+                __syncwarp();
+            }
             if (part == 0) {
 #pragma unroll
                 for (int k = 0; k < kParts - 1; ++k) {
                     ss += reinterpret_cast<const double *>(sloc + (k * kTileM + m) * 16)[0];
                     amax = fmaxf(amax, reinterpret_cast<const float *>(sloc + (k * kTileM + m) * 16)[2]);
                 }
-                reinterpret_cast<double *>(sstat + m * 16)[0] = ss;
-                reinterpret_cast<float *>(sstat + m * 16)[2] = amax;
-            }
-            tc_fence_before();
-            cluster_sync();  // #3 statistics visible; every thread's x_out is in the tile buffer
-            if (tid == 0) {  // x_out back to HBM (issued after the barrier, whose release
-                             // semantics would otherwise wait for this bulk store); one
-                             // bulk group per slab so the slabs can be refilled one by one
-#pragma unroll
-                for (int s = 0; s < kSlabs; ++s) {
-                    tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
-                    bulk_commit();
-                }
-                const long long tn = tile_t0(it + 1);
-                next_t0 = (it + 1 < p.tiles_per_cluster && tn < p.T) ? tn : -1;
-                if (next_t0 >= 0) mbar_expect_tx(bar_load, uint32_t(kSlabs * R * 128));
+                const uint32_t owner = uint32_t(m / TPO);
+                const uint32_t dst = smem_u32(sst + (int(crank) * TPO + m % TPO) * 16);
+                st_async_v4(mapa(dst, owner), uint32_t(__double2loint(ss)), uint32_t(__double2hiint(ss)),
+                            __float_as_uint(amax), 0u, mapa(bar(kBarSt), owner));
             }
 
-            // row totals over the cluster (fixed order: deterministic), computed by
-            // the part-0 thread of each row and handed to the other parts
-            if (part == 0) {
-                float4 sv[CS];
-#pragma unroll
-                for (int c = 0; c < CS; ++c) sv[c] = ld_dsmem_f4(mapa(smem_u32(sstat + m * 16), uint32_t(c)));
+            // ---- owner: totals of its rows over the cluster in a fixed order
+            // (deterministic), scale, row quantiser pushed to every CTA
+            constexpr int kStatThreads = TPO * CS;  // one per (own row, destination CTA)
+            if (tid < kStatThreads) {
+                const int rl = tid / CS, dst_cta = tid % CS;
+                if (!mbar_wait(bar(kBarSt), ph, err != 0)) err |= kErrMbarTimeout;
                 double ss_t = 0.0;
                 float am_t = 0.f;
 #pragma unroll
                 for (int c = 0; c < CS; ++c) {
-                    ss_t += __hiloint2double(__float_as_int(sv[c].y), __float_as_int(sv[c].x));
-                    am_t = fmaxf(am_t, sv[c].z);
+                    const float4 v = *reinterpret_cast<const float4 *>(sst + (c * TPO + rl) * 16);
+                    ss_t += __hiloint2double(__float_as_int(v.y), __float_as_int(v.x));
+                    am_t = fmaxf(am_t, v.z);
                 }
+                const int mo = int(crank) * TPO + rl;
                 const float ms = float(ss_t / double(p.D));
                 const float rs = 1.0f / sqrtf(ms + p.eps);
                 const RowQuant q = row_quant(am_t, qmax);
-                if (crank == 0 && m < nrows) p.scales[t0 + m] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
-                reinterpret_cast<float *>(sloc + m * 16)[0] = q.inv;
-                reinterpret_cast<float *>(sloc + m * 16)[1] = q.pre;
+                if (dst_cta == 0 && mo < nrows) p.scales[t0 + mo] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+                st_async_v2(mapa(smem_u32(sprm + mo * 8), uint32_t(dst_cta)), __float_as_uint(q.inv),
+                            __float_as_uint(q.pre), mapa(bar(kBarPrm), uint32_t(dst_cta)));
+                if (tid == 0 && next) mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
             }
-            named_sync(1, kConsumers);
+            if (!mbar_wait(bar(kBarPrm), ph, err != 0)) err |= kErrMbarTimeout;
+            if (tid == 0 && next) mbar_expect_tx(bar(kBarPrm), uint32_t(kTileM * 8));
             RowQuant rq;
-            rq.inv = reinterpret_cast<const float *>(sloc + m * 16)[0];
-            rq.pre = reinterpret_cast<const float *>(sloc + m * 16)[1];
+            rq.inv = reinterpret_cast<const float *>(sprm + m * 8)[0];
+            rq.pre = reinterpret_cast<const float *>(sprm + m * 8)[1];
             const bool scaled = rq.pre != 1.0f;
             const bool valid = m < nrows;
 
-            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined); thread 0
-            // also refills the tile buffer slab by slab as the x_out store drains
+            // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined)
             {
                 constexpr int kBlocks = kPartCols / 32;
                 const uint32_t taddr = tmem + lane_base + tcol;
@@ -473,21 +543,14 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                             reinterpret_cast<uint2 *>(dst)[2] = make_uint2(words[4], words[5]);
                         }
                     }
-                    if (tid == 0) {  // slabs 4j .. 4j+3 of x_out have been read: reload them
-                        const int j = b / 2;
-                        if (j == 0) bulk_wait_read<4>();
-                        else bulk_wait_read<0>();
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) refill(4 * j + q);
-                    }
                     tmem_wait_ld();
                 }
             }
             tc_fence_before();
-            named_sync(1, kConsumers);  // TMEM reads done before the next tile's MMAs
-            ph ^= 1;
+            named_sync(1, kConsumers);  // TMEM reads done before the next tile's products
+            tc_fence_after();
         }
-        if (tid == 0) bulk_wait0();
+        if (warp == kConsumerWarps - 1 && lane == 0) bulk_wait0();
     }
 
     tc_fence_before();

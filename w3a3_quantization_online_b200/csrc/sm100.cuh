@@ -254,6 +254,10 @@ __device__ __forceinline__ uint32_t ncluster_x() {
 __device__ __forceinline__ void cluster_arrive() {
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+// Arrive without release semantics: for threads that publish nothing at this barrier.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -305,6 +309,31 @@ __device__ __forceinline__ void st_dsmem_u16(uint32_t addr, uint16_t a) {
 
 __device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t a) {
     asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
+}
+
+// Bulk copy (async proxy) of `bytes` (a multiple of 16) from this CTA's shared
+// memory to the shared memory of a CTA of this cluster, counted (complete_tx) on
+// that CTA's mbarrier `mbar`.  dst and mbar come from mapa; 16-byte aligned.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "r"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+
+// Asynchronous store into the shared memory of a CTA of this cluster: the bytes
+// are counted (complete_tx) on the mbarrier `mbar` of that same CTA, whose
+// waiters then see the data.  Both addresses come from mapa.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_async_v2(uint32_t addr, uint32_t a, uint32_t b, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];"
+                 ::"r"(addr), "r"(a), "r"(b), "r"(mbar)
+                 : "memory");
 }
 
 }  // namespace sm100

@@ -129,9 +129,10 @@ uint64_t rsq_launch_count(void);
 int rsq_select_align_kernel(int which);
 
 /* Kernel used by rht_quant: 0 = automatic (tensor-core kernel for bf16,
- * d = 4096, m = 1; shared-memory radix-16 kernel otherwise), 1 = always the
- * radix-16 kernel, 2 = only the warp-per-row CUDA-core kernel, 3 = only the
- * tensor-core kernel (2 and 3 return RSQ_ERR_UNSUPPORTED for other shapes).
+ * d in {4096, 8192}, m = 1; shared-memory radix-16 kernel otherwise), 1 =
+ * always the radix-16 kernel, 2 = only the warp-per-row CUDA-core kernel
+ * (d = 4096), 3 = only the tensor-core kernel (2 and 3 return
+ * RSQ_ERR_UNSUPPORTED for other shapes).
  * Process-wide; returns the previous setting, -1 if invalid.  All compute the
  * same function; this exists for testing and measurement. */
 int rsq_select_rht_kernel(int which);

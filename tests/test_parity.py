@@ -272,26 +272,27 @@ def test_rht_shapes(d, m, dtype, bits):
     check_rht(h, label=f"d={d} m={m}")
 
 
-def test_rht_kernels_agree_with_the_oracle_at_4096():
+@pytest.mark.parametrize("d,kernels", [(4096, (3, 2, 1)), (8192, (3, 1))])
+def test_rht_kernels_agree_with_the_oracle(d, kernels):
     rsq = _rsq()
-    for which in (rsq.RHT_TENSOR_CORE, rsq.RHT_SPECIALISED, rsq.RHT_GENERIC):
+    for which in kernels:
         prev = rsq.select_rht_kernel(which)
         try:
             for T in (1, 7, 600):
                 for bits in (4, 3):
-                    h = inputs.rht_case(T, 4096, 1, 60 + T + bits, dtype="bf16", bits=bits, n_outliers=8,
+                    h = inputs.rht_case(T, d, 1, 60 + T + bits + d, dtype="bf16", bits=bits, n_outliers=8,
                                         outlier_scale=100.0)
-                    check_rht(h, label=f"rht kernel {which} T={T} bits={bits}")
+                    check_rht(h, label=f"rht d={d} kernel {which} T={T} bits={bits}")
         finally:
             rsq.select_rht_kernel(prev)
 
 
-@pytest.mark.parametrize("which", [1, 2, 3])
-def test_tiny_and_zero_rows_rht_4096(which):
+@pytest.mark.parametrize("d,which", [(4096, 1), (4096, 2), (4096, 3), (8192, 3)])
+def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()
     prev = rsq.select_rht_kernel(which)
     try:
-        h = inputs.rht_case(6, 4096, 1, 3, dtype="bf16")
+        h = inputs.rht_case(6, d, 1, 3, dtype="bf16")
         h.x[1] = 0.0
         h.x[2] *= np.float32(2.0 ** -120)      # absmax far below 2^-64: rescaled path
         h.x[3, :] = 0.0

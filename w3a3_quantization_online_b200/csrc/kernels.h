@@ -47,9 +47,10 @@ bool rht_fast_supports(int d, int m, int dtype, int bits, long long T);
 cudaError_t launch_rht_fast(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
                             int bits, cudaStream_t s);
 
-// Randomised Hadamard of order 4096 with the first 64-point stage on tcgen05
-// (m = 1, bf16, INT4/INT3; same support as rht_fast_supports).
-cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int bits,
-                          cudaStream_t s);
+// Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
+// (m = 1, bf16, INT4/INT3).
+bool rht_tc_supports(int d, int m, int dtype, int bits, long long T);
+cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
+                          int bits, cudaStream_t s);
 
 }  // namespace rsq

@@ -1,26 +1,28 @@
-// rht_tc.cu -- randomised Hadamard transform of order 4096 + per-token
-// symmetric quantiser, bf16 input; the first half of the transform runs on the
-// tensor cores.
+// rht_tc.cu -- randomised Hadamard transform of order 4096 or 8192 + per-token
+// symmetric quantiser, bf16 input; the first stage of the transform runs on
+// the tensor cores.
 //
 // Infra Quant II, QuaRot / Background: v = H diag(s) x / sqrt(d) with the
-// Sylvester H of order d = 2^12; QuaRot / Method: per-token symmetric absmax
-// quantisation.
+// Sylvester H of order d = 2^12 or 2^13; QuaRot / Method: per-token symmetric
+// absmax quantisation.
 //
-// A token row is the 64 x 64 matrix U[a][b] = s_i x_i (i = 64 a + b).  The
-// Sylvester matrix factors as H_4096 = H_64 (x) H_64, so the transform is
-// W = H_64 U H_64:
-//  * Y = H_64 U (along a) for four tokens at once is one tcgen05 product
+// A token row is the R x 64 matrix U[a][b] = s_i x_i (i = 64 a + b, R = d/64).
+// The Sylvester matrix factors as H_d = H_R (x) H_64, so the transform is
+// W = H_R U H_64:
+//  * Y = H_R U (along a) is one tcgen05 product per group of tokens, with
+//    M = N = K = 128.  For d = 4096 (R = 64) four tokens go at once:
 //        D[(p, a)][(q, b)] = sum_{(p', a')} diag(H_64, H_64)[(p, a)][(p', a')] B[(p', a')][(q, b)]
-//    with B the four TMA-loaded token tiles (token p + 2 q): M = 128, N = 128,
-//    K = 128.  The products are +-1 x bf16, exact; accumulation is fp32 in TMEM.
+//    with B the four TMA-loaded token tiles (token p + 2 q).  For d = 8192
+//    (R = 128) two tokens go at once: D[a][(q, b)] = sum_a' H_128[a][a'] B[a'][(q, b)]
+//    (token q).  The products are +-1 x bf16, exact; accumulation is fp32 in TMEM.
 //  * W = Y H_64 (along b): each thread reads one row a of one token (64
 //    columns) from TMEM and finishes it with register butterflies (packed
 //    f32x2), then owns the 64 contiguous outputs [64 a, 64 a + 64).
 // The signs are applied to the tiles in shared memory (XOR of the bf16 sign
-// bits) before the product.  The 1/sqrt(4096) = 1/64 factor goes to the scale.
+// bits) before the product.  The 1/sqrt(d) factor goes to the scale.
 //
-// Pipeline (one CTA per SM): a producer warp streams 4-token groups into 5
-// tile stages (32 KB each) by TMA; two consumer warp groups (8 warps each) take
+// Pipeline (one CTA per SM): a producer warp streams token groups (4 or 2
+// tokens) into 5 tile stages (32 KB each) by TMA; two consumer warp groups (8 warps each) take
 // alternate groups, each with two of the four 128-column TMEM slots, so one
 // group's product overlaps its own previous epilogue and the other warp group's
 // work.  A stage is released by the tcgen05 commit of the product that read
@@ -41,21 +43,30 @@ constexpr int kGroupWarps = 8;                // one consumer warp group
 constexpr int kGroupThreads = kGroupWarps * 32;
 constexpr int kConsumerGroups = 2;
 constexpr int kThreads = kConsumerGroups * kGroupThreads + 32;  // + producer warp
-constexpr int kTok = 4;                       // tokens per group (one MMA set)
-constexpr int kTileBytes = 64 * 128;          // one token: 64 rows x 128 B (bf16)
-constexpr int kStageBytes = kTok * kTileBytes;  // 32 KB
+constexpr int kStageBytes = 32768;            // one token group (4 x 8 KB or 2 x 16 KB)
 constexpr int kStages = 5;
 constexpr int kSlots = 4;                     // TMEM slots of 128 columns (two per warp group)
-constexpr int kOffA = 0;                      // diag(H_64, H_64), K-major SW128: 2 slabs x 16 KB
-constexpr int kOffMask = kOffA + 2 * 16384;   // 8 KB sign masks, laid out like a token tile
-constexpr int kOffStage = kOffMask + kTileBytes;
-constexpr int kOffRed = kOffStage + kStages * kStageBytes;  // [warp group][token 4][half-quadrant 2]
-constexpr int kOffBar = kOffRed + kConsumerGroups * kTok * 2 * 4;
-constexpr int kOffTmem = kOffBar + (2 * kStages + kSlots) * 8;  // full[], empty[], mma[]
-constexpr int kBytes = kOffTmem + 16;
-constexpr int kSmem = kBytes + 1024;
 
-__device__ __forceinline__ uint32_t tile_off(int a, int chunk) {  // SWIZZLE_128B 64 x 128 B tile
+// Shape constants for token rows of d = 64 * ROWS elements.
+template <int ROWS>
+struct Shape {
+    static constexpr int kRows = ROWS;                        // a: 64 (d = 4096) or 128 (d = 8192)
+    static constexpr int kD = 64 * ROWS;
+    static constexpr int kTileBytes = ROWS * 128;             // one token: ROWS rows x 128 B (bf16)
+    static constexpr int kTok = kStageBytes / kTileBytes;     // tokens per group: 4 or 2
+    static constexpr int kQuadsPerToken = ROWS / 32;          // TMEM lane quadrants holding one token
+    static constexpr int kOffA = 0;                           // H (block-diagonal for ROWS = 64), 2 x 16 KB
+    static constexpr int kOffMask = kOffA + 2 * 16384;        // sign masks, laid out like a token tile
+    static constexpr int kOffStage = kOffMask + kTileBytes;
+    static constexpr int kOffRed = kOffStage + kStages * kStageBytes;  // [warp group][token][quadrant]
+    static constexpr int kOffBar = kOffRed + kConsumerGroups * 8 * 4;
+    static constexpr int kOffTmem = kOffBar + (2 * kStages + kSlots) * 8;  // full[], empty[], mma[]
+    static constexpr int kBytes = kOffTmem + 16;
+    static constexpr int kSmem = kBytes + 1024;
+    static_assert(kTok * kQuadsPerToken == 8, "reduction slots");
+};
+
+__device__ __forceinline__ uint32_t tile_off(int a, int chunk) {  // SWIZZLE_128B token tile
     return uint32_t(a * 128 + ((chunk ^ (a & 7)) << 4));
 }
 
@@ -87,12 +98,17 @@ __device__ __forceinline__ void fwht64(float (&v)[64]) {
     }
 }
 
-template <int BITS>
+template <int ROWS, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
-k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ signs,
-             uint8_t *__restrict__ codes, float *__restrict__ scales, long long T, int *status) {
+k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ signs,
+         uint8_t *__restrict__ codes, float *__restrict__ scales, long long T, int *status) {
+    using S = Shape<ROWS>;
+    constexpr int kTok = S::kTok;
+    constexpr int kTileBytes = S::kTileBytes;
+    constexpr int kOffA = S::kOffA, kOffMask = S::kOffMask, kOffStage = S::kOffStage;
+    constexpr int kOffRed = S::kOffRed, kOffBar = S::kOffBar, kOffTmem = S::kOffTmem;
     constexpr int qmax = (1 << (BITS - 1)) - 1;
-    constexpr int row_bytes = 4096 * BITS / 8;
+    constexpr int row_bytes = S::kD * BITS / 8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sa = base + kOffA;
@@ -105,8 +121,9 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int err = 0;
 
-    // constants: A = diag(H_64, H_64) with H_64[a][a'] = (-1)^popcount(a & a'),
-    // bf16 +-1 (K-major, SWIZZLE_128B: slab kk holds K columns 64 kk .. 64 kk + 63)
+    // constants: A = diag(H_64, H_64) (ROWS = 64) or H_128 (ROWS = 128), with
+    // H_n[a][a'] = (-1)^popcount(a & a'), bf16 +-1 (K-major, SWIZZLE_128B: slab kk
+    // holds K columns 64 kk .. 64 kk + 63)
     for (int idx = tid; idx < 2 * 128 * 8; idx += kThreads) {
         const int kk = idx >> 10, m = (idx >> 3) & 127, ch = idx & 7;
         uint32_t w[4];
@@ -116,8 +133,9 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const int k = 64 * kk + ch * 8 + 2 * e + u;
-                uint32_t hv = 0;  // 0 outside the diagonal blocks
-                if ((m >> 6) == (k >> 6)) hv = (__popc((m & 63) & (k & 63)) & 1) ? 0xBF80u : 0x3F80u;
+                uint32_t hv = 0;  // 0 outside the diagonal blocks of diag(H_64, H_64)
+                if (ROWS == 128) hv = (__popc(m & k) & 1) ? 0xBF80u : 0x3F80u;
+                else if ((m >> 6) == (k >> 6)) hv = (__popc((m & 63) & (k & 63)) & 1) ? 0xBF80u : 0x3F80u;
                 pair |= hv << (16 * u);
             }
             w[e] = pair;
@@ -125,7 +143,7 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
         *reinterpret_cast<uint4 *>(sa + kk * 16384 + tile_off(m, ch)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     // sign masks: bit 15 / 31 of the word for (a, b-pair) flips elements 64a + 2j, 64a + 2j + 1
-    for (int idx = tid; idx < 64 * 32; idx += kThreads) {
+    for (int idx = tid; idx < ROWS * 32; idx += kThreads) {
         const int a = idx >> 5, j = idx & 31;
         const int i = 64 * a + 2 * j;
         const uint32_t mk = (signs[i] < 0 ? 0x8000u : 0u) | (signs[i + 1] < 0 ? 0x80000000u : 0u);
@@ -174,13 +192,15 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
         const int gtid = tid - wg * kGroupThreads;      // thread within the warp group
         const int gw = warp - wg * kGroupWarps;
         const uint32_t named = 1 + wg;
-        float *sred = reinterpret_cast<float *>(base + kOffRed) + wg * kTok * 2;
+        float *sred = reinterpret_cast<float *>(base + kOffRed) + wg * 8;
         const uint32_t idesc = idesc_bf16_f32(128, 128, false, true);
-        // epilogue mapping: TMEM lane (p, a) = 64 p + a, column half q
+        // epilogue mapping: TMEM lane (p, a) = 64 p + a (ROWS = 64) or a (ROWS = 128),
+        // column half q
         const int quad = gw & 3, q = gw >> 2;
         const int lrow = quad * 32 + lane;
-        const int p = lrow >> 6, a = lrow & 63;
-        const int tslot = p + 2 * q;  // token within the group
+        const int p = ROWS == 64 ? lrow >> 6 : 0, a = lrow & (ROWS - 1);
+        const int tslot = ROWS == 64 ? p + 2 * q : q;  // token within the group
+        constexpr int QPT = S::kQuadsPerToken;
 
         auto epilogue = [&](int it) {
             const int slot = it % kSlots;
@@ -204,10 +224,12 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
 #pragma unroll
             for (int k = 0; k < 64; k += 2) mx[(k >> 1) & 3] = max3(mx[(k >> 1) & 3], fabsf(v[k]), fabsf(v[k + 1]));
             const float wm = warp_max(max3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
-            // the 64 rows of a token live in quadrants 2p, 2p+1 of column half q
-            if (lane == 0) sred[tslot * 2 + (quad & 1)] = wm;
+            // the ROWS rows of a token live in QPT quadrants of column half q
+            if (lane == 0) sred[tslot * QPT + (quad & (QPT - 1))] = wm;
             named_sync(named, kGroupThreads);
-            const float amax = fmaxf(sred[tslot * 2], sred[tslot * 2 + 1]);
+            float amax = sred[tslot * QPT];
+#pragma unroll
+            for (int k = 1; k < QPT; ++k) amax = fmaxf(amax, sred[tslot * QPT + k]);
             const long long t = (g0 + (long long)it * gstep) * kTok + tslot;
             if (t < T) {
                 const RowQuant rq = row_quant(amax, qmax);
@@ -235,7 +257,7 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
 #pragma unroll
                     for (int h = 0; h < 3; ++h) reinterpret_cast<uint2 *>(dst)[h] = make_uint2(o[2 * h], o[2 * h + 1]);
                 }
-                if (a == 0) scales[t] = amax > 0.f ? amax / float(qmax * 64) : 0.f;
+                if (a == 0) scales[t] = amax > 0.f ? amax / (float(qmax) * sqrtf(float(S::kD))) : 0.f;
             }
             tc_fence_before();
             named_sync(named, kGroupThreads);  // sred reuse; TMEM slot reads done
@@ -245,7 +267,7 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
         for (int it = wg; it < nmine; it += kConsumerGroups) {
             const int s = it % kStages, slot = it % kSlots;
             if (!mbar_wait(bar_full + 8 * s, uint32_t((it / kStages) & 1), err != 0)) err |= kErrMbarTimeout;
-            // apply the random signs to the four tiles (XOR of bf16 sign bits)
+            // apply the random signs to the group's tiles (XOR of bf16 sign bits)
             uint8_t *st = sstage + s * kStageBytes;
 #pragma unroll
             for (int k = 0; k < (kStageBytes / 16) / kGroupThreads; ++k) {
@@ -265,8 +287,8 @@ k_rht4096_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict_
             if (gtid == 0) {
                 tc_fence_after();
                 // A: K-major, K-steps of 16 are 32 bytes apart within a slab, slabs 16 KB apart.
-                // B: MN-major, K rows (p', a') 128 B apart (16 per K-step: 2 KB), the two
-                //    64-column atoms (token pairs q = 0, 1) 16 KB apart.
+                // B: MN-major, K rows 128 B apart (16 per K-step: 2 KB), the two 64-column
+                //    atoms (column halves q = 0, 1) 16 KB apart.
                 const uint64_t ad0 = smem_desc_sw128(smem_u32(sa), 1024);
                 const uint64_t bd0 = smem_desc_sw128_lbo(smem_u32(st), 16384, 1024);
 #pragma unroll
@@ -309,16 +331,17 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int BITS>
-cudaError_t launch_bits(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
-                        cudaStream_t st) {
+template <int ROWS, int BITS>
+cudaError_t launch_shape(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
+                         cudaStream_t st) {
+    using S = Shape<ROWS>;
     static bool configured[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    auto kern = k_rht4096_tc<BITS>;
+    auto kern = k_rht_tc<ROWS, BITS>;
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kSmem);
         if (e != cudaSuccess) return e;
         configured[dev] = true;
     }
@@ -326,18 +349,18 @@ cudaError_t launch_bits(const void *x, const int8_t *signs, uint8_t *codes, floa
     int *status = device_status_word();
     if (!enc || !status) return cudaErrorInvalidValue;
     CUtensorMap map;
-    const cuuint64_t dims[3] = {64, 64, cuuint64_t(T)};
-    const cuuint64_t strides[2] = {128, 8192};
-    const cuuint32_t box[3] = {64, 64, kTok};
+    const cuuint64_t dims[3] = {64, cuuint64_t(ROWS), cuuint64_t(T)};
+    const cuuint64_t strides[2] = {128, cuuint64_t(S::kD) * 2};
+    const cuuint32_t box[3] = {64, cuuint32_t(ROWS), cuuint32_t(S::kTok)};
     const cuuint32_t estr[3] = {1, 1, 1};
     if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(x), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const long long ngroups = (T + kTok - 1) / kTok;
+    const long long ngroups = (T + S::kTok - 1) / S::kTok;
     long long grid = num_sms();
     if (grid > ngroups) grid = ngroups;
-    kern<<<int(grid), kThreads, kSmem, st>>>(map, signs, codes, scales, T, status);
+    kern<<<int(grid), kThreads, S::kSmem, st>>>(map, signs, codes, scales, T, status);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
@@ -345,9 +368,18 @@ cudaError_t launch_bits(const void *x, const int8_t *signs, uint8_t *codes, floa
 
 }  // namespace
 
-cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int bits,
-                          cudaStream_t s) {
-    return bits == 4 ? launch_bits<4>(x, signs, codes, scales, T, s) : launch_bits<3>(x, signs, codes, scales, T, s);
+bool rht_tc_supports(int d, int m, int dtype, int bits, long long T) {
+    return (d == 4096 || d == 8192) && m == 1 && dtype == 1 && (bits == 3 || bits == 4) && T >= 1 &&
+           T <= 0x7FFFFFFFLL;
+}
+
+cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
+                          int bits, cudaStream_t s) {
+    if (d == 8192)
+        return bits == 4 ? launch_shape<128, 4>(x, signs, codes, scales, T, s)
+                         : launch_shape<128, 3>(x, signs, codes, scales, T, s);
+    return bits == 4 ? launch_shape<64, 4>(x, signs, codes, scales, T, s)
+                     : launch_shape<64, 3>(x, signs, codes, scales, T, s);
 }
 
 }  // namespace rsq

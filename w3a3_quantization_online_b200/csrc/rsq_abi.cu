@@ -179,8 +179,8 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
     if (overlap(sc, sx) || overlap(sc, sg) || overlap(sc, ss) || overlap(ss, sx) || overlap(ss, sg))
         return RSQ_ERR_ALIAS;
     const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
-    if ((which == 0 || which == 3) && rsq::rht_fast_supports(d, m, dtype, bits, T))
-        return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
+    if ((which == 0 || which == 3) && rsq::rht_tc_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, d, bits, static_cast<cudaStream_t>(stream)));
     if (which == 2 && rsq::rht_fast_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_fast(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
     if (which == 2 || which == 3) return RSQ_ERR_UNSUPPORTED;

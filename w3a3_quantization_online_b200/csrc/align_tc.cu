@@ -170,15 +170,16 @@ __device__ __forceinline__ void bulk_wait_read_n(int n) {
 
 // Codes of one 32-column block (INT4: 4 words, INT3: 3 words).
 template <int BITS>
-__device__ __forceinline__ void code_block(const uint32_t (&v)[32], const RowQuant &rq, bool scaled,
-                                           uint32_t *words) {
+__device__ __forceinline__ void code_block(const uint32_t (&v)[32], const RowQuant &rq, uint32_t *words) {
     uint32_t g[4];
 #pragma unroll
     for (int gi = 0; gi < 4; ++gi) {
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[gi * 8 + e]);
-        g[gi] = pack8_fast<BITS>(f, rq.inv, rq.pre, scaled);
+        // the row factor pre (1, or 2^64 for a tiny row) is always applied: one
+        // packed multiply per pair is cheaper than a per-element predicate
+        g[gi] = pack8_fast<BITS>(f, rq.inv, rq.pre, true);
     }
     if (BITS == 4) {
 #pragma unroll
@@ -519,7 +520,6 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             RowQuant rq;
             rq.inv = reinterpret_cast<const float *>(sprm + m * 8)[0];
             rq.pre = reinterpret_cast<const float *>(sprm + m * 8)[1];
-            const bool scaled = rq.pre != 1.0f;
             const bool valid = m < nrows;
 
             // ---- pass 2: codes from the fp32 x_out in TMEM (loads pipelined)
@@ -534,10 +534,10 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 for (int b = 0; b < kBlocks; b += 2) {
                     uint32_t words[2 * BITS];  // 64 codes
                     tmem_ld32(taddr + (b + 1) * 32, vb);
-                    code_block<BITS>(va, rq, scaled, words);
+                    code_block<BITS>(va, rq, words);
                     tmem_wait_ld();
                     if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
-                    code_block<BITS>(vb, rq, scaled, words + BITS);
+                    code_block<BITS>(vb, rq, words + BITS);
                     if (valid) {
                         uint8_t *dst = crow + (b / 2) * (BITS * 8);
                         if (BITS == 4 && p.codes_v8) {

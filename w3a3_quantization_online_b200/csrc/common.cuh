@@ -104,6 +104,7 @@ __device__ __forceinline__ int quant_code(float v, const RowQuant &q, int qmax) 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // max(a, b, c) in one instruction (sm_100 three-input max).
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -131,7 +132,7 @@ __device__ __forceinline__ uint32_t pack8_fast(const float (&v)[8], float inv, f
 #pragma unroll
     for (int e = 0; e < 8; e += 2) {
         float2 t = make_float2(v[e], v[e + 1]);
-        if (scaled) t = make_float2(t.x * pre, t.y * pre);
+        if (scaled) t = mul2(t, make_float2(pre, pre));
         const float2 q = fma2(t, inv2, mag2);
         r[e] = __float_as_uint(q.x);
         r[e + 1] = __float_as_uint(q.y);

@@ -98,6 +98,20 @@ __device__ __forceinline__ void fwht64(float (&v)[64]) {
     }
 }
 
+// Codes of 64 values, 8 packed words (INT4) or 8 24-bit groups (INT3).  The
+// row factor `pre` (1, or 2^64 for a tiny row) is always applied: one packed
+// multiply per pair is cheaper than a per-element predicate.
+template <int BITS, bool SCALED>
+__device__ __forceinline__ void quant64s(const float (&v)[64], const RowQuant &rq, uint32_t (&w)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = v[8 * k + e];
+        w[k] = pack8_fast<BITS>(f, rq.inv, rq.pre, SCALED);
+    }
+}
+
 template <int ROWS, int BITS>
 __global__ void __launch_bounds__(kThreads, 1)
 k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ signs,
@@ -233,15 +247,8 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
             const long long t = (g0 + (long long)it * gstep) * kTok + tslot;
             if (t < T) {
                 const RowQuant rq = row_quant(amax, qmax);
-                const bool scaled = rq.pre != 1.0f;
                 uint32_t w[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = v[8 * k + e];
-                    w[k] = pack8_fast<BITS>(f, rq.inv, rq.pre, scaled);
-                }
+                quant64s<BITS, true>(v, rq, w);
                 uint8_t *dst = codes + t * row_bytes + a * (8 * BITS);
                 if (BITS == 4) {
                     reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);

@@ -138,12 +138,11 @@ __device__ __forceinline__ uint32_t pack8_fast(const float (&v)[8], float inv, f
         r[e + 1] = __float_as_uint(q.y);
     }
     if (BITS == 4) {
-        // byte k = low nibble of r[2k] | low nibble of r[2k+1] << 4 (bits above
-        // the byte are don't-care), then gather the four low bytes
-        uint32_t b[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) b[k] = (r[2 * k] & 0x0Fu) | ((r[2 * k + 1] << 4) & 0xF0u);
-        return prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+        // gather the low bytes of the even and of the odd elements, then byte k =
+        // low nibble of r[2k] | low nibble of r[2k+1] << 4
+        const uint32_t ev = prmt(prmt(r[0], r[2], 0x0040u), prmt(r[4], r[6], 0x0040u), 0x5410u);
+        const uint32_t od = prmt(prmt(r[1], r[3], 0x0040u), prmt(r[5], r[7], 0x0040u), 0x5410u);
+        return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
     } else {
         uint32_t w = 0;
 #pragma unroll

@@ -266,8 +266,10 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
                 }
                 if (a == 0) scales[t] = amax > 0.f ? amax / (float(qmax) * sqrtf(float(S::kD))) : 0.f;
             }
+            // no barrier here: the warp group's next epilogue follows its next
+            // pre-product barrier, which orders these sred reads and TMEM loads
+            // before any later write
             tc_fence_before();
-            named_sync(named, kGroupThreads);  // sred reuse; TMEM slot reads done
         };
 
         int prev = -1;
@@ -307,6 +309,7 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
                 umma_commit(bar_mma + 8 * slot);
                 umma_commit(bar_empty + 8 * s);  // the stage can be refilled once the product is done
             }
+            __syncwarp();  // the other lanes wait here, not in a poll that competes with lane 0
             if (prev >= 0) epilogue(prev);
             prev = it;
         }

@@ -21,10 +21,10 @@
 //    The same shared-memory Q buffer serves as the MN-major B operand of the
 //    first product and the K-major B operand of the second.
 //  * Sixteen warps, four per TMEM lane quadrant, each on 128 columns of its 32
-//    rows.  Thread 0 also issues the tensor-core products (those of the first
-//    contraction follow the tile's slabs as they land) and an L2 prefetch of
-//    the next tile; the last warp issues the x_out stores and the next tile's
-//    loads.
+//    rows.  Thread 0 also issues the first product (following the tile's slabs
+//    as they land) and an L2 prefetch of the next tile; a warp of the last
+//    column part issues the second product; the last warp issues the x_out
+//    stores and the next tile's loads.
 //  * Cross-CTA exchange.  After one cluster barrier the CTA that owns 128/CS
 //    token rows reads their CS partial projections through distributed shared
 //    memory, applies the r x r matrix M and copies z (split hi/lo) into every
@@ -67,6 +67,7 @@ constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kThreads = kConsumers;
 constexpr int kTmemCols = 512;
 constexpr int kPartCols = kCols / kParts;    // columns per consumer thread (128)
+constexpr int kMma2Warp = 4 * (kParts - 1);  // first warp of the last column part
 
 struct AlignTcArgs {
     const float *Q;
@@ -285,7 +286,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const uint32_t lane_base = uint32_t(quad * 32) << 16;
         const uint32_t tcol = uint32_t(part * kPartCols);
         const uint32_t idesc_y = idesc_bf16_f32(128, 64, false, true);
-        const uint32_t idesc_c = idesc_bf16_f32(128, 256, false, false);
+        const uint32_t idesc_c = idesc_bf16_f32(128, 128, false, false);
         const uint32_t slab_tx = uint32_t(R * 128);
         if (tid == 0 && has_tile(0)) {
 #pragma unroll 1
@@ -389,9 +390,10 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (lane == 0) mbar_arrive(bar(kBarZ));
             }
 
-            // ---- c = z Q^T (hi/lo split): half h into TMEM columns [256 h, 256 h + 256),
-            // its completion signalled to the two column parts that read it
-            if (tid == 0) {
+            // ---- c = z Q^T (hi/lo split): quarter q into TMEM columns [128 q, 128 q + 128),
+            // in column-part order, issued by a warp of the last part (whose quarter lands
+            // last anyway), so that parts 0-2 start pass 1 as soon as theirs is done
+            if (warp == kMma2Warp && lane == 0) {
                 if (!mbar_wait(bar(kBarZ), ph, err != 0)) err |= kErrMbarTimeout;
                 if (next) mbar_expect_tx(bar(kBarZ), uint32_t(kZTx));
                 tc_fence_after();
@@ -401,13 +403,12 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 // (A K-step, B K-step) pairs: z_hi Q_hi^T, z_hi Q_lo^T, z_lo Q_hi^T
                 constexpr uint32_t kA[6] = {0, 1, 0, 1, 2, 3}, kB[6] = {0, 1, 2, 3, 0, 1};
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int q = 0; q < 4; ++q) {
 #pragma unroll
                     for (int s = 0; s < 6; ++s)
-                        umma_f16(tmem + h * 256, ad0 + ((kA[s] * 32) >> 4),
-                                 bd0 + ((uint32_t(h) * 32768 + kB[s] * 32) >> 4), idesc_c, s != 0);
-                    umma_commit(bar(kBarC + 2 * h));
-                    umma_commit(bar(kBarC + 2 * h + 1));
+                        umma_f16(tmem + q * 128, ad0 + ((kA[s] * 32) >> 4),
+                                 bd0 + ((uint32_t(q) * 16384 + kB[s] * 32) >> 4), idesc_c, s != 0);
+                    umma_commit(bar(kBarC + q));
                 }
             }
             __syncwarp();

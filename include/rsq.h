@@ -118,14 +118,16 @@ int rsq_last_cuda_error(void);
 /* Number of kernels this library has launched in this process (all threads). */
 uint64_t rsq_launch_count(void);
 
-/* Kernel used by rsq_align_norm_quant: 0 = automatic (for bf16, D in
- * {4096, 8192} and r <= 32 the single-tile tensor-core cluster kernel; the
- * CUDA-core kernel otherwise),
- * 1 = always the CUDA-core kernel, 2 = only the single-tile tensor-core
- * kernel, 3 = only the double-buffered one (2 and 3 return RSQ_ERR_UNSUPPORTED
- * for calls they cannot serve).  Process-wide; returns the previous setting, or
- * -1 for an invalid value.  All compute the same function; this exists for
- * testing and measurement. */
+/* Kernel used by rsq_align_norm_quant: 0 = automatic (T <= 16 with
+ * 2048 <= D <= 8192, D % 128 == 0, r <= 32: the decode kernel, one cluster of
+ * 16 CTAs on FP32 FMAs, which takes up to 32 rows on request; otherwise, for
+ * bf16, D in {4096, 8192} and r <= 32,
+ * the single-tile tensor-core cluster kernel; the CUDA-core kernel for
+ * everything else), 1 = always the CUDA-core kernel, 2 = only the single-tile
+ * tensor-core kernel, 3 = only the double-buffered one, 4 = only the decode
+ * kernel (2, 3 and 4 return RSQ_ERR_UNSUPPORTED for calls they cannot serve).
+ * Process-wide; returns the previous setting, or -1 for an invalid value.  All
+ * compute the same function; this exists for testing and measurement. */
 int rsq_select_align_kernel(int which);
 
 /* Kernel used by rht_quant: 0 = automatic (tensor-core kernel for bf16,

@@ -246,6 +246,43 @@ def test_tensor_core_kernel_serves_the_hot_shapes(which):
         rsq.select_align_kernel(prev)
 
 
+def test_decode_kernel_serves_small_batches():
+    rsq = _rsq()
+    prev = rsq.select_align_kernel(rsq.ALIGN_DECODE)
+    try:
+        for T in (1, 5, 16, 32):
+            a, _ = inputs.llama7b_case(T=T)
+            check_align(a, label=f"decode hidden T={T}")
+        a, _ = inputs.w3a3_case(T=31)  # D = 8192, INT3
+        check_align(a, label="decode w3a3 T=31")
+        for r in (1, 7, 32):
+            a = inputs.align_case(16, 4096, r, 50 + r, dtype="bf16", n_outliers=8, outlier_scale=100.0)
+            check_align(a, label=f"decode r={r}")
+        a = inputs.align_case(9, 2048, 16, 9, dtype="f32", n_outliers=2, outlier_scale=20.0)
+        check_align(a, label="decode f32 D=2048")
+        a = inputs.align_case(12, 4096, 32, 11, dtype="bf16", dist="student_t3")
+        a.x[[0, 5]] = 0.0
+        a.x[7] *= np.float32(2.0 ** -120)  # absmax far below 2^-64: rescaled path
+        a.x = inputs.round_to_bf16(a.x)
+        xo, codes, scales = run_align(a)
+        assert np.all(scales[[0, 5]] == 0) and np.all(codes[[0, 5]] == 0)
+        check_align(a, label="decode zero and tiny rows")
+        # in place, as the chain runs it
+        a, _ = inputs.llama7b_case(T=16)
+        xo1, c1, s1 = run_align(a)
+        x = _to_dev(a.x, "bf16")
+        xo2, c2, s2 = run_align(a, x_dev=x, in_place=True)
+        np.testing.assert_array_equal(xo1, xo2)
+        np.testing.assert_array_equal(c1, c2)
+        np.testing.assert_array_equal(s1, s2)
+        # more rows than the decode kernel takes: refused, nothing launched
+        a, _ = inputs.llama7b_case(T=33)
+        with pytest.raises(rsq.RsqError):
+            run_align(a)
+    finally:
+        rsq.select_align_kernel(prev)
+
+
 def test_in_place_update_equals_out_of_place():
     a, _ = inputs.llama7b_case(T=77)
     xo1, c1, s1 = run_align(a)

@@ -1,0 +1,336 @@
+// align_decode.cu -- residual subspace alignment + RMSNorm + quantiser for a
+// handful of token rows (decode: T <= 32), where a per-tile pipeline cannot be
+// filled and the latency of the chain of reductions is all that counts.
+//
+// ReSpinQuant paper notes, key design 3: y = Q^T x, z = M y, x_out = x + Q z.
+// Infra Quant II, QuaRot / Method: scale-free RMSNorm in FP32, per-token
+// symmetric absmax quantisation.
+//
+// One cluster of 16 CTAs splits the hidden dimension (CTA c owns columns
+// [c D/16, (c+1) D/16)) and holds every token row of its slice, as float32, in
+// shared memory.  All arithmetic is FP32 FMA on the CUDA cores (the work is
+// tiny: 2 D r MACs per token); Q is read once from HBM/L2 straight as float32.
+//   1. partial y of the slice for every token (warp per column block, lane per
+//      rank index, one accumulator per token), cluster barrier;
+//   2. the owner CTA of token t (t mod 16) sums the 16 partials in CTA order,
+//      forms z = M y and stores it into every CTA (DSMEM), cluster barrier;
+//   3. x_out = x + Q z (thread per column, Q row in registers), bf16/fp32 store,
+//      fp32 kept in shared memory; per-token partial (sum of squares, absmax)
+//      of the slice, cluster barrier;
+//   4. every CTA reads the 16 partials of every token (fixed order: the same
+//      totals everywhere), forms the row quantiser; CTA 0 writes the scales;
+//   5. codes of the slice, one thread per token and group of eight columns.
+// Three exposed cluster barriers per call; the last one, which only keeps a CTA
+// from leaving while others read its statistics, is split around step 5.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rsq {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kDecCS = 16;        // CTAs per cluster: the hidden dimension is split 16 ways
+constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kDecMaxT = 32;
+constexpr int kR = 32;            // rank slots (r <= 32, zero padded)
+
+struct DecodeArgs {
+    const float *Q;
+    const float *M;
+    uint8_t *codes;
+    float *scales;
+    long long T;
+    int D;
+    int r;
+    float eps;
+};
+
+// Shared memory (floats unless noted), for T tokens and cw columns per CTA.
+struct DecLayout {
+    int cw, T;
+    __host__ __device__ int off_q() const { return 0; }                          // cw x 32
+    __host__ __device__ int off_x() const { return off_q() + cw * kR; }          // T x cw
+    __host__ __device__ int off_yp() const { return off_x() + T * cw; }          // T x 32 partial y
+    __host__ __device__ int off_z() const { return off_yp() + T * kR; }          // T x 32 z
+    __host__ __device__ int off_mt() const { return off_z() + T * kR; }          // 32 x 32 M^T
+    __host__ __device__ int off_st() const { return off_mt() + kR * kR; }        // T x float4 partial stats
+    __host__ __device__ int off_prm() const { return off_st() + 4 * T; }         // T x (inv, pre)
+    __host__ __device__ int off_wp() const { return off_prm() + 2 * T; }         // warps x T x 32
+    __host__ __device__ int floats() const { return off_wp() + kDecWarps * T * kR; }
+    __host__ __device__ size_t bytes() const { return size_t(floats()) * 4; }
+};
+
+template <class IO, int BITS>
+__global__ void __launch_bounds__(kDecThreads, 1)
+k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict__ x_out, const DecodeArgs p) {
+    extern __shared__ float4 dsm4[];
+    float *smf = reinterpret_cast<float *>(dsm4);
+    const int T = int(p.T), D = p.D, r = p.r;
+    const int cw = D / kDecCS;
+    const DecLayout L{cw, T};
+    float *sq = smf + L.off_q();
+    float *sx = smf + L.off_x();
+    float *syp = smf + L.off_yp();
+    float *sz = smf + L.off_z();
+    float *smt = smf + L.off_mt();
+    float4 *sst = reinterpret_cast<float4 *>(smf + L.off_st());
+    float2 *sprm = reinterpret_cast<float2 *>(smf + L.off_prm());
+    float *swp = smf + L.off_wp();
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t crank = cluster_ctarank();
+    const int col0 = int(crank) * cw;
+    constexpr int qmax = (1 << (BITS - 1)) - 1;
+    const long long row_bytes = (long long)D * BITS / 8;
+
+    // ---- stage Q rows of the slice (zero padded to 32), M^T, and the token rows
+    for (int i = tid; i < cw * kR; i += kDecThreads) {
+        const int c = i >> 5, j = i & 31;
+        sq[i] = j < r ? __ldg(p.Q + (size_t)(col0 + c) * r + j) : 0.f;
+    }
+    for (int i = tid; i < kR * kR; i += kDecThreads) {  // smt[k][j] = M[j][k]
+        const int k = i >> 5, j = i & 31;
+        smt[i] = (j < r && k < r) ? __ldg(p.M + j * r + k) : 0.f;
+    }
+    for (int e = tid; e < T * cw / 8; e += kDecThreads) {
+        const int t = (e * 8) / cw, c = (e * 8) % cw;
+        float v[8];
+        load8(x + (size_t)t * D + col0 + c, v);
+        store8(sx + t * cw + c, v);
+    }
+    __syncthreads();
+
+    // ---- 1. partial y of this slice: warp w takes columns [w cw/8, (w+1) cw/8), lane j
+    // the rank index, one accumulator per token (each Q entry loaded once); the
+    // eight warp partials are then summed in warp order
+    {
+        const int cpw = cw / kDecWarps;
+        const int c0 = warp * cpw;
+        for (int t0 = 0; t0 < T; t0 += 8) {  // eight tokens per pass: eight accumulators
+            const int nt = T - t0 < 8 ? T - t0 : 8;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const float *xs = sx + t0 * cw;
+            for (int c = c0; c < c0 + cpw; ++c) {
+                const float qv = sq[c * kR + lane];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < nt) acc[k] = fmaf(xs[k * cw + c], qv, acc[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (k < nt) swp[(warp * T + t0 + k) * kR + lane] = acc[k];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < T * kR; i += kDecThreads) {
+        float y = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecWarps; ++w) y += swp[w * T * kR + i];
+        syp[i] = y;
+    }
+    cluster_sync();  // #1 partial projections visible
+
+    // ---- 2. owner of token t (t mod 16): y, z = M y, z into every CTA
+    for (int t = int(crank) + kDecCS * warp; t < T; t += kDecCS * kDecWarps) {
+        const uint32_t a = smem_u32(syp + t * kR + lane);
+        float pv[kDecCS];
+#pragma unroll
+        for (int c = 0; c < kDecCS; ++c) pv[c] = ld_dsmem_f32(mapa(a, uint32_t(c)));
+        float y = 0.f;
+#pragma unroll
+        for (int c = 0; c < kDecCS; ++c) y += pv[c];
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kR; ++k) acc = fmaf(smt[k * kR + lane], __shfl_sync(0xFFFFFFFFu, y, k), acc);
+        const uint32_t dz = smem_u32(sz + t * kR + lane);
+#pragma unroll
+        for (int c = 0; c < kDecCS; ++c) st_dsmem_u32(mapa(dz, uint32_t(c)), __float_as_uint(acc));
+    }
+    cluster_sync();  // #2 z of every token in every CTA
+
+    // ---- 3. x_out = x + Q z for this thread's columns, every token
+    for (int c = tid; c < cw; c += kDecThreads) {
+        float qv[kR];
+#pragma unroll
+        for (int j = 0; j < kR; j += 4) {
+            const float4 f = *reinterpret_cast<const float4 *>(sq + c * kR + j);
+            qv[j] = f.x;
+            qv[j + 1] = f.y;
+            qv[j + 2] = f.z;
+            qv[j + 3] = f.w;
+        }
+        // four tokens at a time: four independent FMA chains (z read four entries per load)
+        for (int t0 = 0; t0 < T; t0 += 4) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < kR; j += 4) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    if (t0 + k < T) {
+                        const float4 zz = *reinterpret_cast<const float4 *>(sz + (t0 + k) * kR + j);
+                        acc[k] = fmaf(qv[j], zz.x, acc[k]);
+                        acc[k] = fmaf(qv[j + 1], zz.y, acc[k]);
+                        acc[k] = fmaf(qv[j + 2], zz.z, acc[k]);
+                        acc[k] = fmaf(qv[j + 3], zz.w, acc[k]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int t = t0 + k;
+                if (t < T) {
+                    const float v = sx[t * cw + c] + acc[k];
+                    sx[t * cw + c] = v;
+                    x_out[(size_t)t * D + col0 + c] = IO::from_f(v);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    // per-token partial statistics of the slice: warp per token, lanes over columns
+    for (int t = warp; t < T; t += kDecWarps) {
+        const float *xr = sx + t * cw;
+        float ss = 0.f, am = 0.f;
+        for (int c = lane; c < cw; c += 32) {
+            const float v = xr[c];
+            ss = fmaf(v, v, ss);
+            am = fmaxf(am, fabsf(v));
+        }
+        const double sd = warp_sum(double(ss));
+        am = warp_max(am);
+        if (lane == 0)
+            sst[t] = make_float4(__int_as_float(__double2loint(sd)), __int_as_float(__double2hiint(sd)), am, 0.f);
+    }
+    cluster_sync();  // #3 partial statistics visible
+
+    // ---- 4. row quantisers of every token from the 16 partials (fixed order)
+    if (tid < T) {
+        const int t = tid;
+        const uint32_t a = smem_u32(sst + t);
+        float4 sv[kDecCS];
+#pragma unroll
+        for (int c = 0; c < kDecCS; ++c) sv[c] = ld_dsmem_f4(mapa(a, uint32_t(c)));
+        double ss_t = 0.0;
+        float am_t = 0.f;
+#pragma unroll
+        for (int c = 0; c < kDecCS; ++c) {
+            ss_t += __hiloint2double(__float_as_int(sv[c].y), __float_as_int(sv[c].x));
+            am_t = fmaxf(am_t, sv[c].z);
+        }
+        const float ms = float(ss_t / double(D));
+        const float rs = 1.0f / sqrtf(ms + p.eps);
+        const RowQuant q = row_quant(am_t, qmax);
+        sprm[t] = make_float2(q.inv, q.pre);
+        if (crank == 0) p.scales[t] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
+    }
+    cluster_arrive();  // #4 (no CTA leaves while a peer may still read its statistics)
+    __syncthreads();
+
+    // ---- 5. codes: one thread per (token, group of eight columns)
+    for (int pidx = tid; pidx < T * (cw / 8); pidx += kDecThreads) {
+        const int t = pidx / (cw / 8), g = pidx % (cw / 8);
+        float f[8];
+        const float4 a0 = *reinterpret_cast<const float4 *>(sx + t * cw + 8 * g);
+        const float4 a1 = *reinterpret_cast<const float4 *>(sx + t * cw + 8 * g + 4);
+        f[0] = a0.x; f[1] = a0.y; f[2] = a0.z; f[3] = a0.w;
+        f[4] = a1.x; f[5] = a1.y; f[6] = a1.z; f[7] = a1.w;
+        const float2 pr = sprm[t];
+        // |v| <= amax, so |v qmax / amax| <= qmax: no clamp is needed
+        const uint32_t w = pack8_fast<BITS>(f, pr.x, pr.y, true);
+        uint8_t *dst = p.codes + (size_t)t * row_bytes + (size_t)(col0 + 8 * g) * BITS / 8;
+        if (BITS == 4) {
+            *reinterpret_cast<uint32_t *>(dst) = w;
+        } else {
+            dst[0] = uint8_t(w);
+            dst[1] = uint8_t(w >> 8);
+            dst[2] = uint8_t(w >> 16);
+        }
+    }
+    cluster_wait();
+}
+
+template <class IO, int BITS>
+cudaError_t launch_typed(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes, float *scales,
+                         long long T, int D, int r, float eps, cudaStream_t s) {
+    static bool configured[64];
+    static int max_clusters[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    auto kern = k_align_decode<IO, BITS>;
+    const DecLayout L{D / kDecCS, int(T)};
+    const DecLayout Lmax{8192 / kDecCS, kDecMaxT};
+    if (!configured[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Lmax.bytes()));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kDecCS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3(kDecCS, 1, 1);
+        cfg.blockDim = dim3(kDecThreads, 1, 1);
+        cfg.dynamicSmemBytes = Lmax.bytes();
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        max_clusters[dev] = n;
+        configured[dev] = true;
+    }
+    if (max_clusters[dev] < 1) return cudaErrorNotSupported;
+    DecodeArgs a;
+    a.Q = Q;
+    a.M = M;
+    a.codes = codes;
+    a.scales = scales;
+    a.T = T;
+    a.D = D;
+    a.r = r;
+    a.eps = eps;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kDecCS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(kDecCS, 1, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = L.bytes();
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, static_cast<const typename IO::T *>(x), static_cast<typename IO::T *>(x_out),
+                           a);
+    if (e == cudaSuccess) count_launch();
+    return e;
+}
+
+}  // namespace
+
+bool align_decode_supports(int D, int r, long long T) {
+    return T >= 1 && T <= kDecMaxT && D >= 2048 && D <= 8192 && D % (kDecCS * 8) == 0 && r >= 1 && r <= kR;
+}
+
+cudaError_t launch_align_decode(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                                float *scales, long long T, int D, int r, int bits, float eps, int dtype,
+                                cudaStream_t s) {
+    if (dtype == 0)
+        return bits == 4 ? launch_typed<F32, 4>(x, Q, M, x_out, codes, scales, T, D, r, eps, s)
+                         : launch_typed<F32, 3>(x, Q, M, x_out, codes, scales, T, D, r, eps, s);
+    return bits == 4 ? launch_typed<BF16, 4>(x, Q, M, x_out, codes, scales, T, D, r, eps, s)
+                     : launch_typed<BF16, 3>(x, Q, M, x_out, codes, scales, T, D, r, eps, s);
+}
+
+}  // namespace rsq

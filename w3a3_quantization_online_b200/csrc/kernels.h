@@ -42,6 +42,14 @@ cudaError_t launch_align_tc_db(const void *x, const float *Q, const float *M, vo
                                float *scales, long long T, int r, int bits, float eps, cudaStream_t s,
                                bool *launched);
 
+// Decode-size alignment + RMSNorm + quantiser: one cluster of 16 CTAs, FP32 FMAs
+// (T <= 32, 2048 <= D <= 8192, D % 128 == 0, r <= 32, bf16 or fp32 I/O).
+// Returns cudaErrorNotSupported if the cluster cannot be co-scheduled.
+bool align_decode_supports(int D, int r, long long T);
+cudaError_t launch_align_decode(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                                float *scales, long long T, int D, int r, int bits, float eps, int dtype,
+                                cudaStream_t s);
+
 // Warp-per-row randomised Hadamard of order 4096 (m = 1, bf16, INT4/INT3).
 bool rht_fast_supports(int d, int m, int dtype, int bits, long long T);
 cudaError_t launch_rht_fast(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,

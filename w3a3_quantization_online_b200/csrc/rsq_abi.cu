@@ -19,7 +19,7 @@ __device__ int g_device_status;
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
-std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 double-buffered
+std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 double-buffered, 4 decode
 std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 warp-per-row, 3 tensor core
 thread_local int g_last_cuda_error = 0;
 
@@ -146,6 +146,12 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         return RSQ_ERR_ALIAS;
     const int which = rsq::g_align_kernel.load(std::memory_order_relaxed);
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // decode kernel: chosen automatically up to 16 rows (measured: beyond that the
+    // tensor-core kernel's flat ~16 us per call is shorter), on request up to 32
+    if (((which == 0 && T <= 16) || which == 4) && rsq::align_decode_supports(D, r, T)) {
+        const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype, cs);
+        if (e != cudaErrorNotSupported) return finish(e);  // not co-schedulable: another kernel serves it
+    }
     if (which == 3 && rsq::align_tc_db_supports(D, r, dtype, T)) {
         bool launched = false;
         const cudaError_t e = rsq::launch_align_tc_db(x, Q, M, x_out, codes, scales, T, r, bits, eps, cs, &launched);
@@ -158,7 +164,7 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         if (e != cudaSuccess) return finish(e);
         if (launched) return RSQ_OK;
     }
-    if (which == 2 || which == 3) return RSQ_ERR_UNSUPPORTED;
+    if (which == 2 || which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
                                             true, static_cast<cudaStream_t>(stream)));
 }
@@ -207,7 +213,7 @@ const char *rsq_status_string(int status) {
 int rsq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int rsq_select_align_kernel(int which) {
-    if (which < 0 || which > 3) return -1;
+    if (which < 0 || which > 4) return -1;
     return rsq::g_align_kernel.exchange(which);
 }
 

@@ -131,9 +131,10 @@ uint64_t rsq_launch_count(void);
 int rsq_select_align_kernel(int which);
 
 /* Kernel used by rht_quant: 0 = automatic (tensor-core kernel for bf16,
- * d in {4096, 8192}, m = 1; shared-memory radix-16 kernel otherwise), 1 =
- * always the radix-16 kernel, 2 = only the warp-per-row CUDA-core kernel
- * (d = 4096), 3 = only the tensor-core kernel (2 and 3 return
+ * d in {4096, 8192}, m = 1; the Kronecker kernel for bf16, d = 12288, m = 12,
+ * INT4; shared-memory radix-16 kernel otherwise), 1 = always the radix-16
+ * kernel, 2 = only the warp-per-row CUDA-core kernel (d = 4096), 3 = only the
+ * tensor-core kernel, 4 = only the Kronecker kernel (2, 3 and 4 return
  * RSQ_ERR_UNSUPPORTED for other shapes).
  * Process-wide; returns the previous setting, -1 if invalid.  All compute the
  * same function; this exists for testing and measurement. */

@@ -324,6 +324,24 @@ def test_rht_kernels_agree_with_the_oracle(d, kernels):
             rsq.select_rht_kernel(prev)
 
 
+@pytest.mark.parametrize("which", [1, 4])
+def test_kronecker_12288_kernels(which):
+    rsq = _rsq()
+    prev = rsq.select_rht_kernel(which)
+    try:
+        for T in (1, 7, 300):
+            check_rht(inputs.down_proj_case(T=T), label=f"kron kernel {which} T={T}")
+        h = inputs.rht_case(6, 12288, 12, 5, dtype="bf16", n_outliers=4, outlier_scale=50.0)
+        h.x[1] = 0.0
+        h.x[2] *= np.float32(2.0 ** -120)  # absmax far below 2^-64: rescaled path
+        h.x = inputs.round_to_bf16(h.x)
+        codes, scales = run_rht(h)
+        assert scales[1] == 0 and np.all(codes[1] == 0)
+        check_rht(h, label=f"kron kernel {which} zero and tiny rows")
+    finally:
+        rsq.select_rht_kernel(prev)
+
+
 @pytest.mark.parametrize("d,which", [(4096, 1), (4096, 2), (4096, 3), (8192, 3)])
 def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()

@@ -55,6 +55,11 @@ bool rht_fast_supports(int d, int m, int dtype, int bits, long long T);
 cudaError_t launch_rht_fast(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
                             int bits, cudaStream_t s);
 
+// Randomised Hadamard H_1024 (x) H_12 of order 12288 (Paley H_12), bf16, INT4.
+bool rht_kron_supports(int d, int m, int dtype, int bits, long long T);
+cudaError_t launch_rht_kron(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
+                            cudaStream_t s);
+
 // Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
 // (m = 1, bf16, INT4/INT3).
 bool rht_tc_supports(int d, int m, int dtype, int bits, long long T);

@@ -20,7 +20,7 @@ __device__ int g_device_status;
 namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 double-buffered, 4 decode
-std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 warp-per-row, 3 tensor core
+std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 warp-per-row, 3 tensor core, 4 Kronecker 12288
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -187,9 +187,11 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
     const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
     if ((which == 0 || which == 3) && rsq::rht_tc_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, d, bits, static_cast<cudaStream_t>(stream)));
+    if ((which == 0 || which == 4) && rsq::rht_kron_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_kron(x, signs, codes, scales, T, static_cast<cudaStream_t>(stream)));
     if (which == 2 && rsq::rht_fast_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_fast(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
-    if (which == 2 || which == 3) return RSQ_ERR_UNSUPPORTED;
+    if (which == 2 || which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
                                           static_cast<cudaStream_t>(stream)));
 }
@@ -218,7 +220,7 @@ int rsq_select_align_kernel(int which) {
 }
 
 int rsq_select_rht_kernel(int which) {
-    if (which < 0 || which > 3) return -1;
+    if (which < 0 || which > 4) return -1;
     return rsq::g_rht_kernel.exchange(which);
 }
 

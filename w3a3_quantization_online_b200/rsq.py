@@ -47,7 +47,7 @@ EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_stat
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status")
 
 ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DOUBLE_BUFFERED, ALIGN_DECODE = 0, 1, 2, 3, 4
-RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED, RHT_TENSOR_CORE = 0, 1, 2, 3
+RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED, RHT_TENSOR_CORE, RHT_KRONECKER = 0, 1, 2, 3, 4
 
 
 class RsqError(RuntimeError):

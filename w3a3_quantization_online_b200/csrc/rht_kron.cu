@@ -43,17 +43,24 @@ __host__ __device__ constexpr int paley12(int i, int j) {
 }
 
 // out = H_12 u on two groups at once (u[k] = (group 0, group 1) entries k).
+// With s = u_1 + ... + u_11 and P_i = sum of u_j over the j (1..11) with
+// chi(j - i) = +1 (j - i a nonzero square mod 11), row i >= 1 of I + S gives
+//     out_i = u_i - u_0 + (P_i - (s - u_i - P_i)) = 2 (u_i + P_i) - (u_0 + s),
+// and row 0 (all ones) gives out_0 = u_0 + s: 6 packed operations per output
+// instead of 11.
 __device__ __forceinline__ void h12_pair(const float2 (&u)[12], float2 (&out)[12]) {
+    float2 s = u[1];
 #pragma unroll
-    for (int i = 0; i < 12; ++i) {
-        // start from the diagonal (+1), then add or subtract the other eleven
+    for (int k = 2; k < 12; ++k) s = add2(s, u[k]);
+    const float2 c = add2(u[0], s);
+    out[0] = c;
+    constexpr int kSquares[5] = {1, 3, 4, 5, 9};
+#pragma unroll
+    for (int i = 1; i < 12; ++i) {
         float2 acc = u[i];
 #pragma unroll
-        for (int k = 0; k < 12; ++k) {
-            if (k == i) continue;
-            acc = paley12(i, k) > 0 ? add2(acc, u[k]) : sub2(acc, u[k]);
-        }
-        out[i] = acc;
+        for (int q = 0; q < 5; ++q) acc = add2(acc, u[(i - 1 + kSquares[q]) % 11 + 1]);
+        out[i] = fma2(acc, make_float2(2.f, 2.f), make_float2(-c.x, -c.y));
     }
 }
 

@@ -297,6 +297,33 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
         }
 
+        // INT3 codes (three 8-byte stores per 64 codes) are stored while the next
+        // tile's first cluster barrier settles, so that its release does not wait
+        // for them (measured: faster for INT3, slower for the single 32-byte INT4
+        // store, which leaves at once)
+        uint32_t pend[4 * BITS];
+        uint8_t *pend_dst = nullptr;
+        auto store_pending = [&]() {
+            if (pend_dst) {
+#pragma unroll
+                for (int b2 = 0; b2 < 2; ++b2) {
+                    uint8_t *dst = pend_dst + b2 * (BITS * 8);
+                    const uint32_t *w = pend + b2 * 2 * BITS;
+                    if (BITS == 4 && p.codes_v8) {
+                        st_global_v8(dst, w);
+                    } else if (BITS == 4) {
+                        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    } else {
+                        reinterpret_cast<uint2 *>(dst)[0] = make_uint2(w[0], w[1]);
+                        reinterpret_cast<uint2 *>(dst)[1] = make_uint2(w[2], w[3]);
+                        reinterpret_cast<uint2 *>(dst)[2] = make_uint2(w[4], w[5]);
+                    }
+                }
+                pend_dst = nullptr;
+            }
+        };
+
         for (int it = 0; has_tile(it); ++it) {
             const uint32_t ph = uint32_t(it) & 1u;
             const long long t0 = tile_t0(it);
@@ -349,6 +376,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             }
             tc_fence_before();
             cluster_arrive();  // #1 partial projections of all CTAs are visible
+            store_pending();
             cluster_wait();
 
             // ---- owner CTA: sum the partials of its TPO rows (one warp per row, one
@@ -533,32 +561,30 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 tmem_wait_ld();
 #pragma unroll
                 for (int b = 0; b < kBlocks; b += 2) {
-                    uint32_t words[2 * BITS];  // 64 codes
+                    uint32_t *words = pend + (b / 2) * 2 * BITS;  // 64 codes
                     tmem_ld32(taddr + (b + 1) * 32, vb);
                     code_block<BITS>(va, rq, words);
                     tmem_wait_ld();
                     if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
                     code_block<BITS>(vb, rq, words + BITS);
-                    if (valid) {
+                    if (BITS == 4 && valid) {
                         uint8_t *dst = crow + (b / 2) * (BITS * 8);
-                        if (BITS == 4 && p.codes_v8) {
+                        if (p.codes_v8) {
                             st_global_v8(dst, words);
-                        } else if (BITS == 4) {
+                        } else {
                             reinterpret_cast<uint4 *>(dst)[0] = make_uint4(words[0], words[1], words[2], words[3]);
                             reinterpret_cast<uint4 *>(dst)[1] = make_uint4(words[4], words[5], words[6], words[7]);
-                        } else {
-                            reinterpret_cast<uint2 *>(dst)[0] = make_uint2(words[0], words[1]);
-                            reinterpret_cast<uint2 *>(dst)[1] = make_uint2(words[2], words[3]);
-                            reinterpret_cast<uint2 *>(dst)[2] = make_uint2(words[4], words[5]);
                         }
                     }
                     tmem_wait_ld();
                 }
+                if (BITS == 3 && valid) pend_dst = crow;
             }
             tc_fence_before();
             named_sync(1, kConsumers);  // TMEM reads done before the next tile's products
             tc_fence_after();
         }
+        store_pending();
         if (warp == kConsumerWarps - 1 && lane == 0) bulk_wait0();
     }
 

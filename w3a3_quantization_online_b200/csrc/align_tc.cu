@@ -292,7 +292,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 #pragma unroll 1
             for (int s = 0; s < kSlabs; ++s) {
                 mbar_expect_tx(bar(kBarLd + s), slab_tx);
-                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(0)),
+                if (!err) tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(0)),
                             bar(kBarLd + s));
             }
         }
@@ -343,10 +343,10 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                         const int i = 4 * s + k;
                         const uint32_t aoff = uint32_t(s * kSlabBytes + k * 32) >> 4;
                         const uint32_t boff = uint32_t(i * 2048) >> 4;
-                        umma_f16(tmem, ad0 + aoff, bd0 + boff, idesc_y, i != 0);
+                        if (!err) umma_f16(tmem, ad0 + aoff, bd0 + boff, idesc_y, i != 0);
                     }
                 }
-                umma_commit(bar(kBarY));
+                if (!err) umma_commit(bar(kBarY));
                 if (next) {  // the next tile into L2 while this one is processed
                     const int tn = int(tile_t0(it + 1));
 #pragma unroll 1
@@ -413,7 +413,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 fence_proxy_async_cta();
                 __syncwarp();
                 if (lane < CS && lane != int(crank))
-                    bulk_copy_to_cluster(mapa(row_addr, uint32_t(lane)), row_addr, 128u,
+                    if (!err) bulk_copy_to_cluster(mapa(row_addr, uint32_t(lane)), row_addr, 128u,
                                          mapa(bar(kBarZ), uint32_t(lane)));
                 if (lane == 0) mbar_arrive(bar(kBarZ));
             }
@@ -434,9 +434,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 for (int q = 0; q < 4; ++q) {
 #pragma unroll
                     for (int s = 0; s < 6; ++s)
-                        umma_f16(tmem + q * 128, ad0 + ((kA[s] * 32) >> 4),
+                        if (!err) umma_f16(tmem + q * 128, ad0 + ((kA[s] * 32) >> 4),
                                  bd0 + ((uint32_t(q) * 16384 + kB[s] * 32) >> 4), idesc_c, s != 0);
-                    umma_commit(bar(kBarC + q));
+                    if (!err) umma_commit(bar(kBarC + q));
                 }
             }
             __syncwarp();
@@ -493,7 +493,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (lane == 0) {
 #pragma unroll 1
                     for (int s = 0; s < kSlabs; ++s) {
-                        tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
+                        if (!err) tma_store_2d(&tm_xo, smem_u32(sx + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
                         bulk_commit();
                     }
                     if (next) {
@@ -502,7 +502,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                         for (int s = 0; s < kSlabs; ++s) {
                             bulk_wait_read_n(kSlabs - 1 - s);
                             mbar_expect_tx(bar(kBarLd + s), slab_tx);
-                            tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, tn,
+                            if (!err) tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, tn,
                                         bar(kBarLd + s));
                         }
                     }
@@ -517,7 +517,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
                 const uint32_t owner = uint32_t(m / TPO);
                 const uint32_t dst = smem_u32(sst + (int(crank) * TPO + m % TPO) * 16);
-                st_async_v4(mapa(dst, owner), uint32_t(__double2loint(ss)), uint32_t(__double2hiint(ss)),
+                if (!err) st_async_v4(mapa(dst, owner), uint32_t(__double2loint(ss)), uint32_t(__double2hiint(ss)),
                             __float_as_uint(amax), 0u, mapa(bar(kBarSt), owner));
             }
 
@@ -540,7 +540,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 const float rs = 1.0f / sqrtf(ms + p.eps);
                 const RowQuant q = row_quant(am_t, qmax);
                 if (dst_cta == 0 && mo < nrows) p.scales[t0 + mo] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
-                st_async_v2(mapa(smem_u32(sprm + mo * 8), uint32_t(dst_cta)), __float_as_uint(q.inv),
+                if (!err) st_async_v2(mapa(smem_u32(sprm + mo * 8), uint32_t(dst_cta)), __float_as_uint(q.inv),
                             __float_as_uint(q.pre), mapa(bar(kBarPrm), uint32_t(dst_cta)));
                 if (tid == 0 && next) mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
             }
@@ -589,7 +589,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     }
 
     tc_fence_before();
-    __syncthreads();
+    // after a failed wait no further asynchronous work was issued: let what was
+    // already in flight land before TMEM is freed and the CTA exits
+    if (__syncthreads_or(err)) drain_delay();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
     err = __reduce_or_sync(0xFFFFFFFFu, err);

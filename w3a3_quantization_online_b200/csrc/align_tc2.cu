@@ -219,7 +219,7 @@ k_align_tc_db(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         mbar_expect_tx(bar, uint32_t(kXBytes));
 #pragma unroll
         for (int s = 0; s < kSlabs; ++s)
-            tma_load_2d(smem_u32(xbuf(i) + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(i)), bar);
+            if (!err) tma_load_2d(smem_u32(xbuf(i) + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(i)), bar);
     };
 
     const int quad = warp & 3, half = warp >> 2;
@@ -235,9 +235,9 @@ k_align_tc_db(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         const uint64_t bd0 = opaque(smem_desc_sw128(smem_u32(sq), 1024));
 #pragma unroll
         for (int k = 0; k < kSlabs * 4; ++k)
-            umma_f16(tmem + region(i), ad0 + (uint32_t((k >> 2) * kSlabBytes + (k & 3) * 32) >> 4),
+            if (!err) umma_f16(tmem + region(i), ad0 + (uint32_t((k >> 2) * kSlabBytes + (k & 3) * 32) >> 4),
                      bd0 + (uint32_t(k * 2048) >> 4), idesc_y, k != 0);
-        umma_commit(bar_y);
+        if (!err) umma_commit(bar_y);
     };
     auto mma2 = [&](int i) {  // thread 0: c(i) = z_hi Q_hi^T + z_hi Q_lo^T + z_lo Q_hi^T into region(i)
         tc_fence_after();
@@ -247,8 +247,8 @@ k_align_tc_db(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         constexpr uint32_t kA[6] = {0, 1, 0, 1, 2, 3}, kB[6] = {0, 1, 2, 3, 0, 1};
 #pragma unroll
         for (int s = 0; s < 6; ++s)
-            umma_f16(tmem + region(i), ad0 + ((kA[s] * 32) >> 4), bd0 + ((kB[s] * 32) >> 4), idesc_c, s != 0);
-        umma_commit(bar_c);
+            if (!err) umma_f16(tmem + region(i), ad0 + ((kA[s] * 32) >> 4), bd0 + ((kB[s] * 32) >> 4), idesc_c, s != 0);
+        if (!err) umma_commit(bar_c);
     };
     auto yread = [&](int i) {  // warps 0-3: partial y of row m -> P rows (swizzled fp32)
         if (half == 0) {
@@ -382,7 +382,7 @@ k_align_tc_db(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
         if (tid == 0) {
 #pragma unroll
             for (int s = 0; s < kSlabs; ++s)
-                tma_store_2d(&tm_xo, smem_u32(xbuf(i) + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
+                if (!err) tma_store_2d(&tm_xo, smem_u32(xbuf(i) + s * kSlabBytes), col0 + s * kSlabCols, int(t0));
             bulk_commit();
         }
         cluster_wait();
@@ -468,7 +468,9 @@ k_align_tc_db(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ 
 
     if (tid == 0) bulk_wait0();
     tc_fence_before();
-    __syncthreads();
+    // after a failed wait no further asynchronous work was issued: let what was
+    // already in flight land before TMEM is freed and the CTA exits
+    if (__syncthreads_or(err)) drain_delay();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, 512);
     err = __reduce_or_sync(0xFFFFFFFFu, err);

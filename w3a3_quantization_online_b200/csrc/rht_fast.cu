@@ -166,7 +166,7 @@ k_rht4096(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ s
             const long long t = gw + s * nw;
             if (t < T) {
                 mbar_expect_tx(bar0 + 8 * s, kRowIn);
-                tma_load_3d(smem_u32(sin + s * kRowIn), &tm_x, 0, 0, int(t), bar0 + 8 * s);
+                if (!err) tma_load_3d(smem_u32(sin + s * kRowIn), &tm_x, 0, 0, int(t), bar0 + 8 * s);
             }
         }
     }
@@ -196,7 +196,7 @@ k_rht4096(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ s
             const long long tn = t + kStages * nw;
             if (tn < T) {
                 mbar_expect_tx(bar0 + 8 * s, kRowIn);
-                tma_load_3d(smem_u32(sin + s * kRowIn), &tm_x, 0, 0, int(tn), bar0 + 8 * s);
+                if (!err) tma_load_3d(smem_u32(sin + s * kRowIn), &tm_x, 0, 0, int(tn), bar0 + 8 * s);
             }
         }
         fwht64x2(v);  // along a for columns 2l, 2l+1
@@ -233,6 +233,7 @@ k_rht4096(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ s
             scales[t] = amax > 0.f ? amax / float(qmax * 64) : 0.f;  // sqrt(4096) = 64
         }
     }
+    if (__syncthreads_or(err)) drain_delay();  // a staged copy still in flight lands before the CTA exits
     err = __reduce_or_sync(0xFFFFFFFFu, err);
     if (err && lane == 0) atomicOr(status, err);
 }

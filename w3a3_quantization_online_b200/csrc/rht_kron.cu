@@ -93,7 +93,7 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs
         fence_mbar_init();
         if (blockIdx.x < T) {  // the first row (the next ones are staged while the previous is transformed)
             mbar_expect_tx(bar, kKd * 2);
-            bulk_load_1d(smem_u32(srow), x + (long long)blockIdx.x * kKd, kKd * 2, bar);
+            if (!err) bulk_load_1d(smem_u32(srow), x + (long long)blockIdx.x * kKd, kKd * 2, bar);
         }
     }
     __syncthreads();
@@ -174,7 +174,7 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs
         __syncthreads();  // the staged row is consumed: bring in the next one
         if (tid == 0 && t + gridDim.x < T) {
             mbar_expect_tx(bar, kKd * 2);
-            bulk_load_1d(smem_u32(srow), x + (t + gridDim.x) * kKd, kKd * 2, bar);
+            if (!err) bulk_load_1d(smem_u32(srow), x + (t + gridDim.x) * kKd, kKd * 2, bar);
         }
         // thread (a0, hb) now takes a = a0 + 128 k (k < 8), b = 6 hb .. 6 hb + 5
         float2 r[8][3];
@@ -234,6 +234,7 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs
         if (tid == 0) scales[t] = amax > 0.f ? amax / (float(qmax) * sqrtf(float(kKd))) : 0.f;
         __syncthreads();  // red[] and the transpose buffer are reused by the next row
     }
+    if (__syncthreads_or(err)) drain_delay();  // a staged copy still in flight lands before the CTA exits
     err = __reduce_or_sync(0xFFFFFFFFu, err);
     if (err && lane == 0) atomicOr(status, err);
 }

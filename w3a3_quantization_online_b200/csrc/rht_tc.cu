@@ -195,7 +195,7 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
                     if (!mbar_wait(bar_empty + 8 * s, uint32_t((it / kStages - 1) & 1), err != 0))
                         err |= kErrMbarTimeout;
                 mbar_expect_tx(bar_full + 8 * s, kStageBytes);
-                tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok),
+                if (!err) tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok),
                             bar_full + 8 * s);
             }
         }
@@ -304,10 +304,10 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
                 for (int k = 0; k < 8; ++k) {
                     const uint32_t aoff = uint32_t((k >> 2) * 16384 + (k & 3) * 32) >> 4;
                     const uint32_t boff = uint32_t(k * 2048) >> 4;
-                    umma_f16(tmem + uint32_t(slot * 128), ad0 + aoff, bd0 + boff, idesc, k != 0);
+                    if (!err) umma_f16(tmem + uint32_t(slot * 128), ad0 + aoff, bd0 + boff, idesc, k != 0);
                 }
-                umma_commit(bar_mma + 8 * slot);
-                umma_commit(bar_empty + 8 * s);  // the stage can be refilled once the product is done
+                if (!err) umma_commit(bar_mma + 8 * slot);
+                if (!err) umma_commit(bar_empty + 8 * s);  // the stage can be refilled once the product is done
             }
             __syncwarp();  // the other lanes wait here, not in a poll that competes with lane 0
             if (prev >= 0) epilogue(prev);
@@ -317,7 +317,9 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     }
 
     tc_fence_before();
-    __syncthreads();
+    // after a failed wait no further asynchronous work was issued: let what was
+    // already in flight land before TMEM is freed and the CTA exits
+    if (__syncthreads_or(err)) drain_delay();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, kSlots * 128);
     err = __reduce_or_sync(0xFFFFFFFFu, err);

@@ -68,6 +68,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool fa
     }
 }
 
+// After a failed wait: spin for a bounded time so that asynchronous work issued
+// before the failure (tensor-core products, bulk copies into this CTA) lands
+// before TMEM is freed and the CTA exits.
+constexpr uint64_t kDrainNs = 20000000ull;
+__device__ __forceinline__ void drain_delay() {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kDrainNs) { }
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }

@@ -21,12 +21,14 @@
 // The signs are applied to the tiles in shared memory (XOR of the bf16 sign
 // bits) before the product.  The 1/sqrt(d) factor goes to the scale.
 //
-// Pipeline (one CTA per SM): a producer warp streams token groups (4 or 2
-// tokens) into 5 tile stages (32 KB each) by TMA; two consumer warp groups (8 warps each) take
+// Pipeline (one CTA per SM, 16 warps): token groups (4 or 2 tokens) stream
+// into 5 tile stages (32 KB each) by TMA; two warp groups (8 warps each) take
 // alternate groups, each with two of the four 128-column TMEM slots, so one
 // group's product overlaps its own previous epilogue and the other warp group's
-// work.  A stage is released by the tcgen05 commit of the product that read
-// it.  Waits are bounded (device status word).
+// work.  A stage is refilled, five groups ahead, by the warp group whose
+// product read it, as soon as that product is done (no producer warp: with 16
+// warps a thread may hold 128 registers).  The row maximum is combined only
+// among the warps that hold the token.  Waits are bounded (device status word).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -42,7 +44,7 @@ namespace {
 constexpr int kGroupWarps = 8;                // one consumer warp group
 constexpr int kGroupThreads = kGroupWarps * 32;
 constexpr int kConsumerGroups = 2;
-constexpr int kThreads = kConsumerGroups * kGroupThreads + 32;  // + producer warp
+constexpr int kThreads = kConsumerGroups * kGroupThreads;  // 16 warps: 128 registers each
 constexpr int kStageBytes = 32768;            // one token group (4 x 8 KB or 2 x 16 KB)
 constexpr int kStages = 5;
 constexpr int kSlots = 4;                     // TMEM slots of 128 columns (two per warp group)
@@ -60,7 +62,7 @@ struct Shape {
     static constexpr int kOffStage = kOffMask + kTileBytes;
     static constexpr int kOffRed = kOffStage + kStages * kStageBytes;  // [warp group][token][quadrant]
     static constexpr int kOffBar = kOffRed + kConsumerGroups * 8 * 4;
-    static constexpr int kOffTmem = kOffBar + (2 * kStages + kSlots) * 8;  // full[], empty[], mma[]
+    static constexpr int kOffTmem = kOffBar + (kStages + kSlots) * 8;  // full[], mma[]
     static constexpr int kBytes = kOffTmem + 16;
     static constexpr int kSmem = kBytes + 1024;
     static_assert(kTok * kQuadsPerToken == 8, "reduction slots");
@@ -129,8 +131,7 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     uint8_t *smask = base + kOffMask;
     uint8_t *sstage = base + kOffStage;
     const uint32_t bar_full = smem_u32(base + kOffBar);   // kStages: tile landed
-    const uint32_t bar_empty = bar_full + 8 * kStages;    // kStages: tile consumed by its product
-    const uint32_t bar_mma = bar_empty + 8 * kStages;     // kSlots: product done
+    const uint32_t bar_mma = bar_full + 8 * kStages;      // kSlots: product done (its stage is free again)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTmem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int err = 0;
@@ -164,10 +165,7 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
         *reinterpret_cast<uint32_t *>(smask + tile_off(a, j >> 2) + (j & 3) * 4) = mk;
     }
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1);
-        }
+        for (int s = 0; s < kStages; ++s) mbar_init(bar_full + 8 * s, 1);
         for (int s = 0; s < kSlots; ++s) mbar_init(bar_mma + 8 * s, 1);
         fence_mbar_init();
         prefetch_tmap(&tm_x);
@@ -186,21 +184,18 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     const long long g0 = blockIdx.x, gstep = gridDim.x;
     const int nmine = g0 < ngroups ? int((ngroups - 1 - g0) / gstep + 1) : 0;
 
-    if (warp == kConsumerGroups * kGroupWarps) {
-        // ------------------------------------------------ producer warp
-        if (lane == 0) {
-            for (int it = 0; it < nmine; ++it) {
-                const int s = it % kStages;
-                if (it >= kStages)  // the product of group it - kStages has read this stage
-                    if (!mbar_wait(bar_empty + 8 * s, uint32_t((it / kStages - 1) & 1), err != 0))
-                        err |= kErrMbarTimeout;
-                mbar_expect_tx(bar_full + 8 * s, kStageBytes);
-                if (!err) tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok),
-                            bar_full + 8 * s);
-            }
-        }
-        __syncwarp();
-    } else {
+    // group it goes to stage it % kStages; the first kStages are issued here, the
+    // others by the epilogue of the group that last used the stage
+    auto load_group = [&](int it) {
+        const int s = it % kStages;
+        mbar_expect_tx(bar_full + 8 * s, kStageBytes);
+        if (!err) tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok),
+                              bar_full + 8 * s);
+    };
+    if (tid == 0)
+        for (int it = 0; it < kStages && it < nmine; ++it) load_group(it);
+    __syncwarp();
+    {
         // ------------------------------------------------ consumer warp groups
         const int wg = warp / kGroupWarps;              // takes local groups wg, wg + 2, ...
         const int gtid = tid - wg * kGroupThreads;      // thread within the warp group
@@ -215,10 +210,20 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
         const int p = ROWS == 64 ? lrow >> 6 : 0, a = lrow & (ROWS - 1);
         const int tslot = ROWS == 64 ? p + 2 * q : q;  // token within the group
         constexpr int QPT = S::kQuadsPerToken;
+        const uint32_t named_tok = 3 + 4 * wg + tslot;  // barrier of the QPT warps holding one token
+        // sign masks of this thread's chunks (the same positions in every group)
+        constexpr int kChunksPerThread = (kStageBytes / 16) / kGroupThreads;
+        constexpr int kMasks = (kTileBytes / 16) / kGroupThreads;  // distinct positions: 2 or 4
+        uint4 mk[kMasks];
+#pragma unroll
+        for (int k = 0; k < kMasks; ++k) mk[k] = reinterpret_cast<const uint4 *>(smask)[gtid + k * kGroupThreads];
 
         auto epilogue = [&](int it) {
             const int slot = it % kSlots;
             if (!mbar_wait(bar_mma + 8 * slot, uint32_t((it / kSlots) & 1), err != 0)) err |= kErrMbarTimeout;
+            // the product has read stage it % kStages: refill it
+            if (gtid == 0 && it + kStages < nmine) load_group(it + kStages);
+            __syncwarp();
             tc_fence_after();
             float v[64];
             {
@@ -240,7 +245,7 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
             const float wm = warp_max(max3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
             // the ROWS rows of a token live in QPT quadrants of column half q
             if (lane == 0) sred[tslot * QPT + (quad & (QPT - 1))] = wm;
-            named_sync(named, kGroupThreads);
+            named_sync(named_tok, 32 * QPT);  // only the warps that hold this token
             float amax = sred[tslot * QPT];
 #pragma unroll
             for (int k = 1; k < QPT; ++k) amax = fmaxf(amax, sred[tslot * QPT + k]);
@@ -248,7 +253,10 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
             if (t < T) {
                 const RowQuant rq = row_quant(amax, qmax);
                 uint32_t w[8];
-                quant64s<BITS, true>(v, rq, w);
+                if (rq.pre == 1.0f)  // the same for the whole warp (one token)
+                    quant64s<BITS, false>(v, rq, w);
+                else
+                    quant64s<BITS, true>(v, rq, w);
                 uint8_t *dst = codes + t * row_bytes + a * (8 * BITS);
                 if (BITS == 4) {
                     reinterpret_cast<uint4 *>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -279,11 +287,10 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
             // apply the random signs to the group's tiles (XOR of bf16 sign bits)
             uint8_t *st = sstage + s * kStageBytes;
 #pragma unroll
-            for (int k = 0; k < (kStageBytes / 16) / kGroupThreads; ++k) {
-                const int c = gtid + k * kGroupThreads;        // 16-byte chunk within the stage
-                const int within = c & (kTileBytes / 16 - 1);  // same position in the mask tile
+            for (int k = 0; k < kChunksPerThread; ++k) {
+                const int c = gtid + k * kGroupThreads;  // 16-byte chunk within the stage
                 uint4 xv = reinterpret_cast<uint4 *>(st)[c];
-                const uint4 mv = reinterpret_cast<const uint4 *>(smask)[within];
+                const uint4 mv = mk[k % kMasks];         // same position in the mask tile
                 xv.x ^= mv.x;
                 xv.y ^= mv.y;
                 xv.z ^= mv.z;
@@ -307,7 +314,6 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
                     if (!err) umma_f16(tmem + uint32_t(slot * 128), ad0 + aoff, bd0 + boff, idesc, k != 0);
                 }
                 if (!err) umma_commit(bar_mma + 8 * slot);
-                if (!err) umma_commit(bar_empty + 8 * s);  // the stage can be refilled once the product is done
             }
             __syncwarp();  // the other lanes wait here, not in a poll that competes with lane 0
             if (prev >= 0) epilogue(prev);

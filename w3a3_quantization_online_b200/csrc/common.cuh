@@ -190,6 +190,12 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Maximum over the warp of a non-negative float in one integer reduction: the
+// bit patterns of non-negative IEEE floats order like unsigned integers.
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+    return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(v)));
+}
+
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);

@@ -52,7 +52,6 @@ constexpr int kSlots = 4;                     // TMEM slots of 128 columns (two 
 // Shape constants for token rows of d = 64 * ROWS elements.
 template <int ROWS>
 struct Shape {
-    static constexpr int kRows = ROWS;                        // a: 64 (d = 4096) or 128 (d = 8192)
     static constexpr int kD = 64 * ROWS;
     static constexpr int kTileBytes = ROWS * 128;             // one token: ROWS rows x 128 B (bf16)
     static constexpr int kTok = kStageBytes / kTileBytes;     // tokens per group: 4 or 2
@@ -72,11 +71,12 @@ __device__ __forceinline__ uint32_t tile_off(int a, int chunk) {  // SWIZZLE_128
     return uint32_t(a * 128 + ((chunk ^ (a & 7)) << 4));
 }
 
-// In-place 64-point Sylvester transform of v[0..63].  Adjacent elements form
-// the packed pairs (v[2j], v[2j+1]) -- the register pairs the TMEM load
-// delivers -- so the stages for index bits 1..5 are packed two-wide
-// butterflies between pairs and the stage for bit 0 works inside each pair.
-__device__ __forceinline__ void fwht64(float (&v)[64]) {
+// In-place 64-point Sylvester transform of v[0..63], all stages but the last.
+// Adjacent elements form the packed pairs (v[2j], v[2j+1]) -- the register
+// pairs the TMEM load delivers -- so the stages for index bits 1..5 are packed
+// two-wide butterflies between pairs; the stage for bit 0 works inside each
+// pair (fwht64_last_absmax).
+__device__ __forceinline__ void fwht64_outer(float (&v)[64]) {
 #pragma unroll
     for (int hv = 1; hv < 32; hv <<= 1) {  // pair stride: element stride 2 hv
 #pragma unroll
@@ -92,12 +92,27 @@ __device__ __forceinline__ void fwht64(float (&v)[64]) {
             }
         }
     }
+}
+
+// The last stage (inside each pair) and the largest magnitude of its outputs.
+// max(|u + w|, |u - w|) = |u| + |w|, and rounding keeps the equality (the
+// larger of the two rounded results is the rounded |u| + |w|), so the maximum
+// is taken over the 32 pairs instead of the 64 outputs.
+__device__ __forceinline__ float fwht64_last_absmax(float (&v)[64]) {
+    float mx[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains of three-input maxima
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+        const float s0 = fabsf(v[2 * j]) + fabsf(v[2 * j + 1]);
+        const float s1 = fabsf(v[2 * j + 2]) + fabsf(v[2 * j + 3]);
+        mx[(j >> 1) & 3] = max3(mx[(j >> 1) & 3], s0, s1);
+    }
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         const float u = v[2 * j], w = v[2 * j + 1];
         v[2 * j] = u + w;
         v[2 * j + 1] = u - w;
     }
+    return max3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
 }
 
 // Codes of 64 values, 8 packed words (INT4) or 8 24-bit groups (INT3).  The
@@ -238,11 +253,8 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
                     v[k + 32] = __uint_as_float(r1[k]);
                 }
             }
-            fwht64(v);  // along b: row a of token tslot is now final
-            float mx[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains of three-input maxima
-#pragma unroll
-            for (int k = 0; k < 64; k += 2) mx[(k >> 1) & 3] = max3(mx[(k >> 1) & 3], fabsf(v[k]), fabsf(v[k + 1]));
-            const float wm = warp_max(max3(mx[0], mx[1], fmaxf(mx[2], mx[3])));
+            fwht64_outer(v);  // along b; then the last stage, which also gives the row's largest magnitude
+            const float wm = warp_max_nonneg(fwht64_last_absmax(v));
             // the ROWS rows of a token live in QPT quadrants of column half q
             if (lane == 0) sred[tslot * QPT + (quad & (QPT - 1))] = wm;
             named_sync(named_tok, 32 * QPT);  // only the warps that hold this token

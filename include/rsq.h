@@ -88,6 +88,15 @@ typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
  *               n = d / m a power of two with 16 <= n <= 16384, d <= 32768,
  *               d % 16 == 0. */
 
+/* Programmatic dependent launch.  The default kernels of rsq_align_norm_quant
+ * (tensor-core, decode) and rht_quant (tensor-core) are launched so that they
+ * may start while the kernel before them on `stream` is still running: they
+ * read their constant operands (Q and M; signs) at once, and wait for that
+ * kernel to complete before they read x or write any output.  So Q, M and
+ * signs must not be written by the immediately preceding kernel when that
+ * kernel itself lets its successor start early (as these kernels do); an
+ * ordinary launch, a copy or an event between them always completes first. */
+
 /* Residual subspace alignment only: x_out = x + Q (M (Q^T x)) per token row.
  * ReSpinQuant paper notes, key design 3.  x_out may equal x. */
 int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_out,
@@ -97,7 +106,8 @@ int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_ou
  * per-token symmetric absmax quantisation of n -> packed codes.
  * ReSpinQuant key design 3; Infra Quant II, QuaRot / Method and SpinQuant /
  * Motivation.  Writes x_out (rounded to dtype), codes and scales
- * (scales[t] = max_i |n_ti| / qmax).  x_out may equal x. */
+ * (scales[t] = max_i |n_ti| / qmax).  x_out may equal x.
+ * Launch ordering: see "Programmatic dependent launch" above. */
 int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_out,
                          uint8_t *codes, float *scales, int64_t T, int D, int r,
                          int bits, float eps, int dtype, void *stream);

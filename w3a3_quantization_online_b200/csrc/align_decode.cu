@@ -22,6 +22,12 @@
 //   5. codes of the slice, one thread per token and group of eight columns.
 // Three exposed cluster barriers per call; the last one, which only keeps a CTA
 // from leaving while others read its statistics, is split around step 5.
+// The launch allows programmatic dependent launch: a call may start while the
+// previous kernel of the stream still runs, stages its Q slice (one 16-byte
+// load per thread and round, all in flight) and M, and waits for that kernel
+// before it touches x or any output; it lets its own successor start at once.
+// In a chain of layers this hides the launch and the Q read of each layer
+// behind the previous one.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -88,16 +94,41 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
     const int col0 = int(crank) * cw;
     constexpr int qmax = (1 << (BITS - 1)) - 1;
     const long long row_bytes = (long long)D * BITS / 8;
+    // the next kernel of the stream may start staging its own Q and M now
+    asm volatile("griddepcontrol.launch_dependents;");
 
     // ---- stage Q rows of the slice (zero padded to 32), M^T, and the token rows
-    for (int i = tid; i < cw * kR; i += kDecThreads) {
-        const int c = i >> 5, j = i & 31;
-        sq[i] = j < r ? __ldg(p.Q + (size_t)(col0 + c) * r + j) : 0.f;
+    if (r == kR && (reinterpret_cast<uintptr_t>(p.Q) & 15u) == 0) {
+        // the slice is contiguous: all of a thread's 16-byte loads in flight at once
+        const float4 *q4 = reinterpret_cast<const float4 *>(p.Q + (size_t)col0 * kR);
+        float4 *s4 = reinterpret_cast<float4 *>(sq);
+        const int n4 = cw * kR / 4;
+        for (int i0 = 0; i0 < n4; i0 += 8 * kDecThreads) {
+            float4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int i = i0 + tid + k * kDecThreads;
+                if (i < n4) v[k] = __ldg(q4 + i);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int i = i0 + tid + k * kDecThreads;
+                if (i < n4) s4[i] = v[k];
+            }
+        }
+    } else {
+        for (int i = tid; i < cw * kR; i += kDecThreads) {
+            const int c = i >> 5, j = i & 31;
+            sq[i] = j < r ? __ldg(p.Q + (size_t)(col0 + c) * r + j) : 0.f;
+        }
     }
     for (int i = tid; i < kR * kR; i += kDecThreads) {  // smt[k][j] = M[j][k]
         const int k = i >> 5, j = i & 31;
         smt[i] = (j < r && k < r) ? __ldg(p.M + j * r + k) : 0.f;
     }
+    // x may be written by the previous kernel of the stream: wait for it (a no-op
+    // unless this grid was launched early, programmatic dependent launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int e = tid; e < T * cw / 8; e += kDecThreads) {
         const int t = (e * 8) / cw, c = (e * 8) % cw;
         float v[8];
@@ -300,17 +331,19 @@ cudaError_t launch_typed(const void *x, const float *Q, const float *M, void *x_
     a.r = r;
     a.eps = eps;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kDecCS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(kDecCS, 1, 1);
     cfg.blockDim = dim3(kDecThreads, 1, 1);
     cfg.dynamicSmemBytes = L.bytes();
     cfg.stream = s;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, static_cast<const typename IO::T *>(x), static_cast<typename IO::T *>(x_out),
                            a);
     if (e == cudaSuccess) count_launch();

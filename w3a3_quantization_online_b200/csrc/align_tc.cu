@@ -225,6 +225,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     const int R = p.rows_per_tile;
     int err = 0;
 
+    // programmatic dependent launch: the next kernel of the stream may start and
+    // stage its constants now; it waits for this grid before it touches data
+    asm volatile("griddepcontrol.launch_dependents;");
     auto tile_t0 = [&](int it) { return ((long long)cid + (long long)it * ncl) * R; };
     auto has_tile = [&](int it) { return it < p.tiles_per_cluster && tile_t0(it) < p.T; };
 
@@ -279,6 +282,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     cluster_sync();  // barriers initialised in every CTA before any push
+    // Q and M are staged above while the previous kernel of the stream may still
+    // run; x and every output only after it has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     {
         const int quad = warp & 3, part = warp >> 2;
@@ -695,17 +701,19 @@ struct TcKernel {
         a.codes_v8 = (reinterpret_cast<uintptr_t>(codes) & 31u) == 0;
         a.eps = eps;
         cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = CS;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.gridDim = dim3(CS * ncl, 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
         cfg.dynamicSmemBytes = Layout<CS>::kSmem;
         cfg.stream = s;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         e = cudaLaunchKernelEx(&cfg, k_align_tc<CS, BITS>, mx, mxo, a);
         if (e == cudaSuccess) {
             *launched = true;

@@ -150,6 +150,9 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTmem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int err = 0;
+    // programmatic dependent launch: the next kernel of the stream may start and
+    // stage its constants now; it waits for this grid before it touches data
+    asm volatile("griddepcontrol.launch_dependents;");
 
     // constants: A = diag(H_64, H_64) (ROWS = 64) or H_128 (ROWS = 128), with
     // H_n[a][a'] = (-1)^popcount(a & a'), bf16 +-1 (K-major, SWIZZLE_128B: slab kk
@@ -194,6 +197,9 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // H and the sign masks are built above while the previous kernel of the
+    // stream may still run; x and every output only after it has completed
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const long long ngroups = (T + kTok - 1) / kTok;
     const long long g0 = blockIdx.x, gstep = gridDim.x;
@@ -390,8 +396,17 @@ cudaError_t launch_shape(const void *x, const int8_t *signs, uint8_t *codes, flo
     const long long ngroups = (T + S::kTok - 1) / S::kTok;
     long long grid = num_sms();
     if (grid > ngroups) grid = ngroups;
-    kern<<<int(grid), kThreads, S::kSmem, st>>>(map, signs, codes, scales, T, status);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(unsigned(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = S::kSmem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, map, signs, codes, scales, T, status);
     if (e == cudaSuccess) count_launch();
     return e;
 }

@@ -132,6 +132,44 @@ def test_chain_32_layers_teacher_forced(T):
     np.testing.assert_allclose(n1, np.linalg.norm(xr, axis=1), rtol=2e-3)
 
 
+@pytest.mark.parametrize("T", [16, 300])
+def test_back_to_back_layers_match_the_synchronised_run(T):
+    """The default kernels may start before the previous kernel of the stream
+    has finished (they stage Q and M first); every layer's input is the previous
+    layer's in-place output, so the unsynchronised chain must reproduce the
+    synchronised one bit for bit -- also when rht_quant reads the stream that
+    the alignment just wrote."""
+    rsq = _rsq()
+    x0, qs, ms, _, _ = inputs.chain_case(T=T)
+    signs = torch.from_numpy(inputs.rht_case(1, 4096, 1, 7).signs).to(DEV)
+    Qd = [torch.from_numpy(q).to(DEV) for q in qs]
+    Md = [torch.from_numpy(m).to(DEV) for m in ms]
+
+    def run(sync):
+        x = _to_dev(x0, "bf16")
+        outs = []
+        for i in range(len(qs)):
+            codes = torch.empty((T, 2048), dtype=torch.uint8, device=DEV)
+            scales = torch.empty((T,), dtype=torch.float32, device=DEV)
+            rsq.rsq_align_norm_quant(x, Qd[i], Md[i], x_out=x, codes=codes, scales=scales, bits=4)
+            if sync:
+                torch.cuda.synchronize()
+            hc, hs = rsq.rht_quant(x, signs, bits=4)
+            if sync:
+                torch.cuda.synchronize()
+            outs.append((codes, scales, hc, hs))
+        torch.cuda.synchronize()
+        return _host(x), [tuple(t.cpu().numpy() for t in o) for o in outs]
+
+    x_sync, o_sync = run(True)
+    x_fast, o_fast = run(False)
+    assert np.array_equal(x_sync.view(np.uint32), x_fast.view(np.uint32))
+    for i, (a, b) in enumerate(zip(o_sync, o_fast)):
+        for u, v in zip(a, b):
+            assert np.array_equal(u, v), f"layer {i}"
+    assert rsq.device_status() == 0
+
+
 # --------------------------------------------------------------------------
 # full sizes, sampled rows
 # --------------------------------------------------------------------------

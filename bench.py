@@ -63,9 +63,6 @@ def workload_config(T: int, n: int) -> dict:
         "T_per_gpu": T, "D": D, "r": R, "bits": BITS, "io_dtype": "bf16", "eps": EPS,
         "global_tokens": T * n, "parallelism": f"token-sharded replicas x{n}, no data-path collective",
         "l2": f"no flush: the bf16 input batch alone ({T * D * 2 / 1e6:.0f} MB) exceeds the {L2_BYTES / 1e6:.0f} MB L2; per-step traffic {ws / 1e6:.0f} MB",
-        "kernel_timing": f"CUDA events around each kernel on every {KERNEL_EVERY}th step of the timed region; "
-                         "the other steps run back to back (programmatic dependent launch lets a kernel start "
-                         "while the previous one finishes)",
     }
 
 
@@ -432,6 +429,9 @@ def run_gpu(args) -> None:
         "config": workload_config(T, n),
         "roofline": roof,
         "kernels": kern,
+        "kernel_timing": f"CUDA events around each kernel on every {KERNEL_EVERY}th step of the timed region; "
+                         "the other steps run back to back (programmatic dependent launch lets a kernel start "
+                         "while the previous one finishes)",
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "pipeline": f"{E2E_CHUNKS} row chunks on three streams: H2D, kernels, D2H"},
         "gpu_launches": launches,

@@ -10,18 +10,23 @@
 // [c D/16, (c+1) D/16)) and holds every token row of its slice, as float32, in
 // shared memory.  All arithmetic is FP32 FMA on the CUDA cores (the work is
 // tiny: 2 D r MACs per token); Q is read once from HBM/L2 straight as float32.
+// The exchanges are pushed (st.async into the receiving CTA, completing bytes
+// on one of its mbarriers), so every wait ends when the data has arrived rather
+// than at a cluster-wide barrier:
 //   1. partial y of the slice for every token (warp per column block, lane per
-//      rank index, one accumulator per token), cluster barrier;
-//   2. the owner CTA of token t (t mod 16) sums the 16 partials in CTA order,
-//      forms z = M y and stores it into every CTA (DSMEM), cluster barrier;
+//      rank index, one accumulator per token), pushed to the token's owner CTA
+//      (t mod 16);
+//   2. the owner sums the 16 partials in CTA order, forms z = M y and pushes it
+//      into every CTA;
 //   3. x_out = x + Q z (thread per column, Q row in registers), bf16/fp32 store,
 //      fp32 kept in shared memory; per-token partial (sum of squares, absmax)
-//      of the slice, cluster barrier;
-//   4. every CTA reads the 16 partials of every token (fixed order: the same
-//      totals everywhere), forms the row quantiser; CTA 0 writes the scales;
+//      of the slice, pushed into every CTA;
+//   4. every CTA sums the 16 partials of every token in CTA order (the same
+//      totals everywhere) and forms the row quantiser; CTA 0 writes the scales;
 //   5. codes of the slice, one thread per token and group of eight columns.
-// Three exposed cluster barriers per call; the last one, which only keeps a CTA
-// from leaving while others read its statistics, is split around step 5.
+// Two cluster barriers remain, both split: the first (every CTA's mbarriers
+// armed before any push) around the partial projection, the last (no CTA
+// leaves while its pushes may be in flight) around steps 4 and 5.
 // The launch allows programmatic dependent launch: a call may start while the
 // previous kernel of the stream still runs, stages its Q slice (one 16-byte
 // load per thread and round, all in flight) and M, and waits for that kernel
@@ -45,12 +50,14 @@ constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kDecMaxT = 32;
 constexpr int kR = 32;            // rank slots (r <= 32, zero padded)
+constexpr int kOwnMax = kDecMaxT / kDecCS;  // token rows owned by one CTA (t mod 16)
 
 struct DecodeArgs {
     const float *Q;
     const float *M;
     uint8_t *codes;
     float *scales;
+    int *status;
     long long T;
     int D;
     int r;
@@ -58,19 +65,30 @@ struct DecodeArgs {
 };
 
 // Shared memory (floats unless noted), for T tokens and cw columns per CTA.
+// Every float2 / float4 region starts on a multiple of 2 / 4 floats whatever
+// T is (cw is a multiple of 8).
 struct DecLayout {
     int cw, T;
     __host__ __device__ int off_q() const { return 0; }                          // cw x 32
     __host__ __device__ int off_x() const { return off_q() + cw * kR; }          // T x cw
-    __host__ __device__ int off_yp() const { return off_x() + T * cw; }          // T x 32 partial y
-    __host__ __device__ int off_z() const { return off_yp() + T * kR; }          // T x 32 z
+    __host__ __device__ int off_z() const { return off_x() + T * cw; }           // T x 32 z (float4 reads)
     __host__ __device__ int off_mt() const { return off_z() + T * kR; }          // 32 x 32 M^T
-    __host__ __device__ int off_st() const { return off_mt() + kR * kR; }        // T x float4 partial stats
-    __host__ __device__ int off_prm() const { return off_st() + 4 * T; }         // T x (inv, pre)
+    __host__ __device__ int off_prm() const { return off_mt() + kR * kR; }       // T x (inv, pre)
     __host__ __device__ int off_wp() const { return off_prm() + 2 * T; }         // warps x T x 32
-    __host__ __device__ int floats() const { return off_wp() + kDecWarps * T * kR; }
+    __host__ __device__ int off_yin() const { return off_wp() + kDecWarps * T * kR; }  // [source CTA][own row][32]
+    __host__ __device__ int off_stin() const { return (off_yin() + kDecCS * kOwnMax * kR + 3) & ~3; }  // [source][T] float4
+    __host__ __device__ int off_bar() const { return off_stin() + kDecCS * 4 * T; }  // 3 mbarriers (8 B each)
+    __host__ __device__ int floats() const { return off_bar() + 3 * 2; }
     __host__ __device__ size_t bytes() const { return size_t(floats()) * 4; }
 };
+
+// Asynchronous 4-byte store into the shared memory of a CTA of this cluster,
+// completing `bytes` on its mbarrier.
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(mbar)
+                 : "memory");
+}
 
 template <class IO, int BITS>
 __global__ void __launch_bounds__(kDecThreads, 1)
@@ -82,10 +100,8 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
     const DecLayout L{cw, T};
     float *sq = smf + L.off_q();
     float *sx = smf + L.off_x();
-    float *syp = smf + L.off_yp();
     float *sz = smf + L.off_z();
     float *smt = smf + L.off_mt();
-    float4 *sst = reinterpret_cast<float4 *>(smf + L.off_st());
     float2 *sprm = reinterpret_cast<float2 *>(smf + L.off_prm());
     float *swp = smf + L.off_wp();
 
@@ -96,6 +112,23 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
     const long long row_bytes = (long long)D * BITS / 8;
     // the next kernel of the stream may start staging its own Q and M now
     asm volatile("griddepcontrol.launch_dependents;");
+    float *syin = smf + L.off_yin();
+    float4 *sstin = reinterpret_cast<float4 *>(smf + L.off_stin());
+    const uint32_t bar_y = smem_u32(smf + L.off_bar());  // own rows: partial y from every CTA
+    const uint32_t bar_z = bar_y + 8;                      // z of every row from its owner
+    const uint32_t bar_st = bar_y + 16;                    // partial statistics of every row from every CTA
+    const int n_own = T > int(crank) ? (T - 1 - int(crank)) / kDecCS + 1 : 0;
+    int err = 0;
+    if (tid == 0) {
+        mbar_init(bar_y, 1);
+        mbar_init(bar_z, 1);
+        mbar_init(bar_st, 1);
+        fence_mbar_init();
+        mbar_expect_tx(bar_y, uint32_t(n_own * kDecCS * kR * 4));
+        mbar_expect_tx(bar_z, uint32_t(T * kR * 4));
+        mbar_expect_tx(bar_st, uint32_t(kDecCS * T * 16));
+    }
+    cluster_arrive();  // #1 (waited before the first push)
 
     // ---- stage Q rows of the slice (zero padded to 32), M^T, and the token rows
     if (r == kR && (reinterpret_cast<uintptr_t>(p.Q) & 15u) == 0) {
@@ -159,31 +192,35 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         }
     }
     __syncthreads();
+    cluster_wait();  // #1: every CTA's barriers are armed before the first push
+    // own rows of token t live in CTA t mod 16; push this slice's partial y there
     for (int i = tid; i < T * kR; i += kDecThreads) {
         float y = 0.f;
 #pragma unroll
         for (int w = 0; w < kDecWarps; ++w) y += swp[w * T * kR + i];
-        syp[i] = y;
+        const int t = i / kR, k = i % kR;
+        const uint32_t owner = uint32_t(t % kDecCS);
+        const uint32_t dst = smem_u32(syin + (int(crank) * kOwnMax + t / kDecCS) * kR + k);
+        if (!err) st_async_b32(mapa(dst, owner), __float_as_uint(y), mapa(bar_y, owner));
     }
-    cluster_sync();  // #1 partial projections visible
 
-    // ---- 2. owner of token t (t mod 16): y, z = M y, z into every CTA
-    for (int t = int(crank) + kDecCS * warp; t < T; t += kDecCS * kDecWarps) {
-        const uint32_t a = smem_u32(syp + t * kR + lane);
-        float pv[kDecCS];
-#pragma unroll
-        for (int c = 0; c < kDecCS; ++c) pv[c] = ld_dsmem_f32(mapa(a, uint32_t(c)));
+    // ---- 2. owner of token t (t mod 16): y from the 16 partials in CTA order,
+    // z = M y, pushed into every CTA
+    for (int j = warp; j < n_own; j += kDecWarps) {
+        const int t = int(crank) + kDecCS * j;
+        if (!mbar_wait(bar_y, 0, err != 0)) err |= kErrMbarTimeout;
         float y = 0.f;
 #pragma unroll
-        for (int c = 0; c < kDecCS; ++c) y += pv[c];
+        for (int c = 0; c < kDecCS; ++c) y += syin[(c * kOwnMax + j) * kR + lane];
         float acc = 0.f;
 #pragma unroll
         for (int k = 0; k < kR; ++k) acc = fmaf(smt[k * kR + lane], __shfl_sync(0xFFFFFFFFu, y, k), acc);
         const uint32_t dz = smem_u32(sz + t * kR + lane);
 #pragma unroll
-        for (int c = 0; c < kDecCS; ++c) st_dsmem_u32(mapa(dz, uint32_t(c)), __float_as_uint(acc));
+        for (int c = 0; c < kDecCS; ++c)
+            if (!err) st_async_b32(mapa(dz, uint32_t(c)), __float_as_uint(acc), mapa(bar_z, uint32_t(c)));
     }
-    cluster_sync();  // #2 z of every token in every CTA
+    if (!mbar_wait(bar_z, 0, err != 0)) err |= kErrMbarTimeout;  // z of every token from its owner
 
     // ---- 3. x_out = x + Q z for this thread's columns, every token
     for (int c = tid; c < cw; c += kDecThreads) {
@@ -224,7 +261,8 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         }
     }
     __syncthreads();
-    // per-token partial statistics of the slice: warp per token, lanes over columns
+    // per-token partial statistics of the slice (warp per token, lanes over
+    // columns), pushed into every CTA
     for (int t = warp; t < T; t += kDecWarps) {
         const float *xr = sx + t * cw;
         float ss = 0.f, am = 0.f;
@@ -235,24 +273,24 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         }
         const double sd = warp_sum(double(ss));
         am = warp_max(am);
-        if (lane == 0)
-            sst[t] = make_float4(__int_as_float(__double2loint(sd)), __int_as_float(__double2hiint(sd)), am, 0.f);
+        if (lane < kDecCS && !err)
+            st_async_v4(mapa(smem_u32(sstin + int(crank) * T + t), uint32_t(lane)), uint32_t(__double2loint(sd)),
+                        uint32_t(__double2hiint(sd)), __float_as_uint(am), 0u, mapa(bar_st, uint32_t(lane)));
     }
-    cluster_sync();  // #3 partial statistics visible
+    cluster_arrive();  // #2 (waited at the end): no CTA leaves while its pushes may be in flight
+    if (!mbar_wait(bar_st, 0, err != 0)) err |= kErrMbarTimeout;
 
-    // ---- 4. row quantisers of every token from the 16 partials (fixed order)
+    // ---- 4. row quantisers of every token from the 16 partials (CTA order: the
+    // same totals everywhere)
     if (tid < T) {
         const int t = tid;
-        const uint32_t a = smem_u32(sst + t);
-        float4 sv[kDecCS];
-#pragma unroll
-        for (int c = 0; c < kDecCS; ++c) sv[c] = ld_dsmem_f4(mapa(a, uint32_t(c)));
         double ss_t = 0.0;
         float am_t = 0.f;
 #pragma unroll
         for (int c = 0; c < kDecCS; ++c) {
-            ss_t += __hiloint2double(__float_as_int(sv[c].y), __float_as_int(sv[c].x));
-            am_t = fmaxf(am_t, sv[c].z);
+            const float4 sv = sstin[c * T + t];
+            ss_t += __hiloint2double(__float_as_int(sv.y), __float_as_int(sv.x));
+            am_t = fmaxf(am_t, sv.z);
         }
         const float ms = float(ss_t / double(D));
         const float rs = 1.0f / sqrtf(ms + p.eps);
@@ -260,7 +298,6 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         sprm[t] = make_float2(q.inv, q.pre);
         if (crank == 0) p.scales[t] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
     }
-    cluster_arrive();  // #4 (no CTA leaves while a peer may still read its statistics)
     __syncthreads();
 
     // ---- 5. codes: one thread per (token, group of eight columns)
@@ -283,6 +320,9 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
             dst[2] = uint8_t(w >> 16);
         }
     }
+    if (__syncthreads_or(err)) drain_delay();
+    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    if (err && lane == 0) atomicOr(p.status, err);
     cluster_wait();
 }
 
@@ -326,6 +366,8 @@ cudaError_t launch_typed(const void *x, const float *Q, const float *M, void *x_
     a.M = M;
     a.codes = codes;
     a.scales = scales;
+    a.status = device_status_word();
+    if (!a.status) return cudaErrorInvalidValue;
     a.T = T;
     a.D = D;
     a.r = r;

@@ -156,6 +156,15 @@ int rsq_select_rht_kernel(int which);
  * outputs are invalid).  Returns an rsq_status. */
 int rsq_device_status(void *stream, int *status);
 
+/* Test of the error path of the bounded waits: enqueues on `stream` a
+ * one-thread kernel that waits, through the same bounded wait the kernels use,
+ * on an mbarrier that nothing arrives on, with a limit of limit_ms
+ * milliseconds (1..1000, else RSQ_ERR_VALUE).  The wait gives up, the kernel
+ * sets bit 1 of the device status word and returns: no fault, the context
+ * stays usable, and rsq_device_status() then reports the bit.  No counterpart
+ * in the method; it exists for testing. */
+int rsq_selftest_wait_timeout(int limit_ms, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

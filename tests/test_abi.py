@@ -50,6 +50,12 @@ def test_library_exports_every_declared_symbol():
             assert n in syms
 
 
+def test_selftest_rejects_out_of_range_limits():
+    # host-side validation: nothing is enqueued (no GPU needed)
+    for bad in (0, -5, 1001):
+        assert L.rsq_selftest_wait_timeout(bad, None) == 9  # RSQ_ERR_VALUE
+
+
 def test_status_strings():
     for s in range(10):
         assert rsq.status_string(s)

@@ -170,6 +170,20 @@ def test_back_to_back_layers_match_the_synchronised_run(T):
     assert rsq.device_status() == 0
 
 
+def test_bounded_wait_runs_out_and_reports():
+    """The kernels' bounded wait, on an mbarrier that nothing arrives on, gives
+    up after its limit; the kernel returns and sets the timeout bit of the
+    device status word; the context stays usable (no fault, no hang)."""
+    rsq = _rsq()
+    assert rsq.device_status() == 0
+    rsq.selftest_wait_timeout(20)
+    assert rsq.device_status() == 1
+    assert rsq.device_status() == 0  # read and cleared
+    a, _ = inputs.llama7b_case(T=64)
+    check_align(a, label="after the timeout self test")
+    assert rsq.device_status() == 0
+
+
 # --------------------------------------------------------------------------
 # full sizes, sampled rows
 # --------------------------------------------------------------------------

@@ -10,6 +10,7 @@
 
 #include "kernels.h"
 #include "rsq.h"
+#include "sm100.cuh"
 
 namespace rsq {
 
@@ -35,6 +36,19 @@ int cur_device() {
 }  // namespace
 
 void count_launch(int n) { g_launches.fetch_add(uint64_t(n), std::memory_order_relaxed); }
+
+namespace {
+// One thread waits, through the same bounded wait the kernels use, on an
+// mbarrier that nothing arrives on: the wait gives up after limit_ns and the
+// timeout bit goes into the device status word; the kernel then returns.
+__global__ void k_selftest_wait(int *status, unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = sm100::smem_u32(&bar);
+    sm100::mbar_init(b, 1);
+    sm100::fence_mbar_init();
+    if (!sm100::mbar_wait(b, 0u, false, limit_ns)) atomicOr(status, sm100::kErrMbarTimeout);
+}
+}  // namespace
 
 int num_sms() {
     const int dev = cur_device();
@@ -236,5 +250,15 @@ int rsq_device_status(void *stream, int *status) {
 }
 
 uint64_t rsq_launch_count(void) { return rsq::g_launches.load(std::memory_order_relaxed); }
+
+int rsq_selftest_wait_timeout(int limit_ms, void *stream) {
+    if (limit_ms < 1 || limit_ms > 1000) return RSQ_ERR_VALUE;
+    int *word = rsq::device_status_word();
+    if (!word) return finish(cudaErrorInvalidDevice);
+    rsq::k_selftest_wait<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(word, (unsigned long long)limit_ms * 1000000ull);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) rsq::count_launch(1);
+    return finish(e);
+}
 
 }  // extern "C"

@@ -57,14 +57,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // first failure a kernel stops waiting, so it ends quickly).  The caller keeps
 // executing the same control flow so that cluster barriers stay matched, and
 // reports the failure through the device status word.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool failed = false) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, bool failed = false,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (failed) return false;
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
     }
 }
 

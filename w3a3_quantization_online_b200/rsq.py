@@ -42,9 +42,12 @@ _lib.rsq_select_rht_kernel.argtypes = [_i32]
 _lib.rsq_select_rht_kernel.restype = _i32
 _lib.rsq_device_status.argtypes = [_vp, ctypes.POINTER(_i32)]
 _lib.rsq_device_status.restype = _i32
+_lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
+_lib.rsq_selftest_wait_timeout.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_status_string",
-            "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status")
+            "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
+            "rsq_selftest_wait_timeout")
 
 ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DOUBLE_BUFFERED, ALIGN_DECODE = 0, 1, 2, 3, 4
 RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED, RHT_TENSOR_CORE, RHT_KRONECKER = 0, 1, 2, 3, 4
@@ -88,6 +91,12 @@ def device_status(stream=None) -> int:
     out = _i32(0)
     _check(_lib.rsq_device_status(_stream(stream), ctypes.byref(out)))
     return int(out.value)
+
+
+def selftest_wait_timeout(limit_ms: int = 20, stream=None) -> None:
+    """Enqueue the bounded-wait self test (a wait that runs out after limit_ms
+    and sets the timeout bit of the device status word)."""
+    _check(_lib.rsq_selftest_wait_timeout(int(limit_ms), _stream(stream)))
 
 
 def status_string(status: int) -> str:

@@ -42,6 +42,25 @@ __host__ __device__ constexpr int paley12(int i, int j) {
     return i == j ? 1 : (i == 0 ? 1 : (j == 0 ? -1 : (((0x23A >> ((j - i + 11) % 11)) & 1) ? 1 : -1)));
 }
 
+// The residue neighbours used below are exactly the +1 entries of the Paley
+// rows 1..11 off the diagonal and column 0: checked at compile time.
+__host__ __device__ constexpr int square_mod11(int q) {  // the nonzero squares mod 11: 1, 3, 4, 5, 9
+    return q == 0 ? 1 : (q == 1 ? 3 : (q == 2 ? 4 : (q == 3 ? 5 : 9)));
+}
+constexpr bool paley_rows_match_residues() {
+    for (int i = 1; i < 12; ++i) {
+        int plus = 0;
+        for (int j = 1; j < 12; ++j)
+            if (j != i && paley12(i, j) == 1) ++plus;
+        if (plus != 5) return false;
+        for (int q = 0; q < 5; ++q)
+            if (paley12(i, (i - 1 + square_mod11(q)) % 11 + 1) != 1) return false;
+        if (paley12(i, 0) != -1 || paley12(0, i) != 1 || paley12(i, i) != 1) return false;
+    }
+    return paley12(0, 0) == 1;
+}
+static_assert(paley_rows_match_residues(), "Paley H_12 structure");
+
 // out = H_12 u on two groups at once (u[k] = (group 0, group 1) entries k).
 // With s = u_1 + ... + u_11 and P_i = sum of u_j over the j (1..11) with
 // chi(j - i) = +1 (j - i a nonzero square mod 11), row i >= 1 of I + S gives
@@ -54,12 +73,11 @@ __device__ __forceinline__ void h12_pair(const float2 (&u)[12], float2 (&out)[12
     for (int k = 2; k < 12; ++k) s = add2(s, u[k]);
     const float2 c = add2(u[0], s);
     out[0] = c;
-    constexpr int kSquares[5] = {1, 3, 4, 5, 9};
 #pragma unroll
     for (int i = 1; i < 12; ++i) {
         float2 acc = u[i];
 #pragma unroll
-        for (int q = 0; q < 5; ++q) acc = add2(acc, u[(i - 1 + kSquares[q]) % 11 + 1]);
+        for (int q = 0; q < 5; ++q) acc = add2(acc, u[(i - 1 + square_mod11(q)) % 11 + 1]);
         out[i] = fma2(acc, make_float2(2.f, 2.f), make_float2(-c.x, -c.y));
     }
 }

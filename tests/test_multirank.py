@@ -69,3 +69,16 @@ def test_single_process_helpers():
     assert bench.max_over_ranks(3.25) == 3.25
     assert bench.whole_job_rate(100, 1, 10, 1000.0) == pytest.approx(1000.0)
     assert bench.shard_seed(0) != bench.shard_seed(1)
+
+
+def test_traffic_record_follows_code_not_comments(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("// a kernel\n__global__ void k(int *p) { p[0] = 1; }  /* store */\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_sha(["k.cu"])
+    src.write_text("// the same kernel, reworded comment\n__global__ void k(int *p) {\n    p[0] = 1;\n}\n")
+    assert bench.kernel_source_sha(["k.cu"]) == h0
+    src.write_text("__global__ void k(int *p) { p[0] = 2; }\n")
+    assert bench.kernel_source_sha(["k.cu"]) != h0

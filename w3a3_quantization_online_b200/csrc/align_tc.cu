@@ -38,9 +38,14 @@
 //    tile as soon as its store has read it, so the load overlaps the statistics
 //    exchange and the codes.  The fp32 value goes back to TMEM, from which the
 //    codes are computed once the row quantiser arrives.
+//  * Programmatic dependent launch: the kernel lets the next kernel of the
+//    stream start at once, and stages its own Q slice and M while the previous
+//    kernel may still run; it waits for that kernel before touching x or any
+//    output.
 // Every mbarrier wait is bounded; a timeout sets a bit in the device status
 // word and the kernel keeps its barrier sequence so that no CTA is left
-// waiting.
+// waiting; after a failed wait a thread issues no further asynchronous work,
+// and the CTA drains what is in flight before freeing TMEM.
 #include <cuda.h>
 
 #include "common.cuh"

@@ -28,7 +28,10 @@
 // work.  A stage is refilled, five groups ahead, by the warp group whose
 // product read it, as soon as that product is done (no producer warp: with 16
 // warps a thread may hold 128 registers).  The row maximum is combined only
-// among the warps that hold the token.  Waits are bounded (device status word).
+// among the warps that hold the token.  Programmatic dependent launch: the
+// Hadamard operand and the sign masks are built while the previous kernel of
+// the stream may still run; x and the outputs only after it completes.  Waits
+// are bounded (device status word).
 #include <cuda.h>
 
 #include "common.cuh"

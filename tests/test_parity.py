@@ -170,6 +170,33 @@ def test_back_to_back_layers_match_the_synchronised_run(T):
     assert rsq.device_status() == 0
 
 
+@pytest.mark.parametrize("T", [7, 17, 1000])
+def test_repeated_back_to_back_launches_are_deterministic(T):
+    """Hundreds of launches of the default kernels back to back on one stream
+    (each may start before the previous one ends) reproduce the first outputs
+    bit for bit and leave the device status word clean."""
+    rsq = _rsq()
+    a, h = inputs.llama7b_case(T=T)
+    x = torch.from_numpy(a.x).to(DEV).to(torch.bfloat16)
+    Q = torch.from_numpy(a.Q).to(DEV)
+    M = torch.from_numpy(a.M).to(DEV)
+    xh = torch.from_numpy(h.x).to(DEV).to(torch.bfloat16)
+    sg = torch.from_numpy(h.signs).to(DEV)
+
+    def run():
+        xo, ca, sa = rsq.rsq_align_norm_quant(x, Q, M, bits=4)
+        ch, sh = rsq.rht_quant(xh, sg, bits=4)
+        return xo.view(torch.int16), ca, sa, ch, sh
+
+    ref = [t.clone() for t in run()]
+    for i in range(300):
+        out = run()
+        if i % 100 == 99:
+            for u, v in zip(out, ref):
+                assert torch.equal(u, v), f"launch {i}"
+    assert rsq.device_status() == 0
+
+
 def test_bounded_wait_runs_out_and_reports():
     """The kernels' bounded wait, on an mbarrier that nothing arrives on, gives
     up after its limit; the kernel returns and sets the timeout bit of the

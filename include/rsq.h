@@ -98,7 +98,10 @@ typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
  * ordinary launch, a copy or an event between them always completes first. */
 
 /* Residual subspace alignment only: x_out = x + Q (M (Q^T x)) per token row.
- * ReSpinQuant paper notes, key design 3.  x_out may equal x. */
+ * ReSpinQuant paper notes, key design 3.  x_out may equal x.  Served by the
+ * kernels of rsq_align_norm_quant (same selection, see
+ * rsq_select_align_kernel) without the norm and the codes; x_out is the same
+ * bit for bit. */
 int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_out,
                        int64_t T, int D, int r, int dtype, void *stream);
 

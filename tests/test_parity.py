@@ -449,6 +449,40 @@ def test_residual_align_only_matches_oracle():
         H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, dtype, f"align {dtype}")
 
 
+@pytest.mark.parametrize("which", [0, 1, 2, 4])
+def test_residual_align_kernels(which):
+    """rsq_residual_align through the decode kernel (small T), the tensor-core
+    kernel (bf16, D = 4096 / 8192) and the CUDA-core kernel, each without the
+    norm and the codes; x_out must equal the alignment of rsq_align_norm_quant
+    bit for bit where both use the same kernel."""
+    rsq = _rsq()
+    prev = rsq.select_align_kernel(which)
+    try:
+        shapes = {0: [(1, 4096), (16, 4096), (17, 4096), (1000, 4096), (300, 8192)],
+                  1: [(16, 4096), (300, 4096)],
+                  2: [(1, 4096), (200, 4096), (3001, 4096), (129, 8192)],
+                  4: [(1, 4096), (16, 4096), (32, 2048), (31, 8192)]}[which]
+        for T, D in shapes:
+            a = inputs.align_case(T, D, 32, T + D, dtype="bf16", n_outliers=8, outlier_scale=100.0)
+            x = _to_dev(a.x, "bf16")
+            Q = torch.from_numpy(a.Q).to(DEV)
+            M = torch.from_numpy(a.M).to(DEV)
+            xo = rsq.rsq_residual_align(x, Q, M)
+            torch.cuda.synchronize()
+            H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, "bf16", f"kernel {which} T={T} D={D}")
+            xo2, _, _ = rsq.rsq_align_norm_quant(x, Q, M, bits=4)
+            torch.cuda.synchronize()
+            assert torch.equal(xo.view(torch.int16), xo2.view(torch.int16)), f"kernel {which} T={T} D={D}"
+        if which == 4:  # decode kernel with fp32 I/O
+            a = inputs.align_case(9, 2048, 16, 9, dtype="f32", n_outliers=2, outlier_scale=20.0)
+            xo = rsq.rsq_residual_align(_to_dev(a.x, "f32"), torch.from_numpy(a.Q).to(DEV), torch.from_numpy(a.M).to(DEV))
+            torch.cuda.synchronize()
+            H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, "f32", "decode f32")
+        assert rsq.device_status() == 0
+    finally:
+        rsq.select_align_kernel(prev)
+
+
 def test_exact_ties_round_half_to_even():
     """w = H x with small integers chosen so that v/alpha hits exact ties; both
     sides must round them to even with no exemption."""

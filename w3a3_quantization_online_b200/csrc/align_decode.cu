@@ -108,7 +108,8 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t crank = cluster_ctarank();
     const int col0 = int(crank) * cw;
-    constexpr int qmax = (1 << (BITS - 1)) - 1;
+    constexpr bool kQuant = BITS > 0;  // BITS = 0: alignment only (x_out), no norm / codes
+    constexpr int qmax = kQuant ? (1 << (BITS - 1)) - 1 : 1;
     const long long row_bytes = (long long)D * BITS / 8;
     // the next kernel of the stream may start staging its own Q and M now
     asm volatile("griddepcontrol.launch_dependents;");
@@ -126,7 +127,7 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         fence_mbar_init();
         mbar_expect_tx(bar_y, uint32_t(n_own * kDecCS * kR * 4));
         mbar_expect_tx(bar_z, uint32_t(T * kR * 4));
-        mbar_expect_tx(bar_st, uint32_t(kDecCS * T * 16));
+        if (kQuant) mbar_expect_tx(bar_st, uint32_t(kDecCS * T * 16));
     }
     cluster_arrive();  // #1 (waited before the first push)
 
@@ -261,6 +262,7 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         }
     }
     __syncthreads();
+    if constexpr (kQuant) {
     // per-token partial statistics of the slice (warp per token, lanes over
     // columns), pushed into every CTA
     for (int t = warp; t < T; t += kDecWarps) {
@@ -277,7 +279,9 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
             st_async_v4(mapa(smem_u32(sstin + int(crank) * T + t), uint32_t(lane)), uint32_t(__double2loint(sd)),
                         uint32_t(__double2hiint(sd)), __float_as_uint(am), 0u, mapa(bar_st, uint32_t(lane)));
     }
+    }
     cluster_arrive();  // #2 (waited at the end): no CTA leaves while its pushes may be in flight
+    if constexpr (kQuant) {
     if (!mbar_wait(bar_st, 0, err != 0)) err |= kErrMbarTimeout;
 
     // ---- 4. row quantisers of every token from the 16 partials (CTA order: the
@@ -319,6 +323,7 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
             dst[1] = uint8_t(w >> 8);
             dst[2] = uint8_t(w >> 16);
         }
+    }
     }
     if (__syncthreads_or(err)) drain_delay();
     err = __reduce_or_sync(0xFFFFFFFFu, err);
@@ -401,9 +406,12 @@ bool align_decode_supports(int D, int r, long long T) {
 cudaError_t launch_align_decode(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
                                 float *scales, long long T, int D, int r, int bits, float eps, int dtype,
                                 cudaStream_t s) {
-    if (dtype == 0)
+    if (dtype == 0) {
+        if (bits == 0) return launch_typed<F32, 0>(x, Q, M, x_out, codes, scales, T, D, r, eps, s);
         return bits == 4 ? launch_typed<F32, 4>(x, Q, M, x_out, codes, scales, T, D, r, eps, s)
                          : launch_typed<F32, 3>(x, Q, M, x_out, codes, scales, T, D, r, eps, s);
+    }
+    if (bits == 0) return launch_typed<BF16, 0>(x, Q, M, x_out, codes, scales, T, D, r, eps, s);
     return bits == 4 ? launch_typed<BF16, 4>(x, Q, M, x_out, codes, scales, T, D, r, eps, s)
                      : launch_typed<BF16, 3>(x, Q, M, x_out, codes, scales, T, D, r, eps, s);
 }

@@ -225,7 +225,8 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     const uint32_t cid = cluster_id_x(), ncl = ncluster_x();
     const int col0 = int(crank) * kCols;
     const int r = p.r;
-    const int qmax = (1 << (BITS - 1)) - 1;
+    constexpr bool kQuant = BITS > 0;  // BITS = 0: alignment only (x_out), no norm / codes
+    const int qmax = kQuant ? (1 << (BITS - 1)) - 1 : 1;
     const long long row_bytes = (long long)p.D * BITS / 8;
     const int R = p.rows_per_tile;
     int err = 0;
@@ -243,8 +244,10 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         // waiter once the previous phase has completed)
         if (has_tile(0)) {
             mbar_expect_tx(bar(kBarZ), uint32_t(kZTx));
-            mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
-            mbar_expect_tx(bar(kBarPrm), uint32_t(kTileM * 8));
+            if (kQuant) {
+                mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
+                mbar_expect_tx(bar(kBarPrm), uint32_t(kTileM * 8));
+            }
         }
     }
     if (warp == 0) {
@@ -312,7 +315,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         // tile's first cluster barrier settles, so that its release does not wait
         // for them (measured: faster for INT3, slower for the single 32-byte INT4
         // store, which leaves at once)
-        uint32_t pend[4 * BITS];
+        uint32_t pend[4 * (kQuant ? BITS : 1)];
         uint8_t *pend_dst = nullptr;
         auto store_pending = [&]() {
             if (pend_dst) {
@@ -475,12 +478,12 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     tmem_wait_st();
                     tmem_ld32(taddr + (b + 1) * 32, vb);
                     xout_block(va, xbase + (cb >> 1) * kSlabBytes, m, (cb & 1) * 4, s2, am);
-                    tmem_st32(taddr + b * 32, va);
+                    if (kQuant) tmem_st32(taddr + b * 32, va);  // fp32 x_out for the codes
                     tmem_wait_ld();
                     tmem_wait_st();
                     if (b + 2 < kBlocks) tmem_ld32(taddr + (b + 2) * 32, va);
                     xout_block(vb, xbase + ((cb + 1) >> 1) * kSlabBytes, m, ((cb + 1) & 1) * 4, s2, am);
-                    tmem_st32(taddr + (b + 1) * 32, vb);
+                    if (kQuant) tmem_st32(taddr + (b + 1) * 32, vb);
                     tmem_wait_ld();
                     // fold the fp32 pair sums of these 64 columns into float64
                     ss += double(s2.x) + double(s2.y);
@@ -492,7 +495,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             fence_proxy_async_cta();  // x_out (generic writes) -> TMA store (async proxy)
             // statistics: fold the column parts of each row; part 0 pushes the CTA's
             // partial (ss, amax) of row m to the row's owner
-            if (part > 0) {
+            if (kQuant && part > 0) {
                 reinterpret_cast<double *>(sloc + ((part - 1) * kTileM + m) * 16)[0] = ss;
                 reinterpret_cast<float *>(sloc + ((part - 1) * kTileM + m) * 16)[2] = amax;
             }
@@ -520,6 +523,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 }
                 __syncwarp();
             }
+            if constexpr (kQuant) {
             if (part == 0) {
 #pragma unroll
                 for (int k = 0; k < kParts - 1; ++k) {
@@ -590,6 +594,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     tmem_wait_ld();
                 }
                 if (BITS == 3 && valid) pend_dst = crow;
+            }
             }
             tc_fence_before();
             named_sync(1, kConsumers);  // TMEM reads done before the next tile's products
@@ -744,9 +749,12 @@ cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void 
                             bool *launched) {
     int *status = device_status_word();
     if (!status) return cudaErrorInvalidDevice;
-    if (D == 4096)
+    if (D == 4096) {
+        if (bits == 0) return TcKernel<8, 0>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched);
         return bits == 4 ? TcKernel<8, 4>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched)
                          : TcKernel<8, 3>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched);
+    }
+    if (bits == 0) return TcKernel<16, 0>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched);
     return bits == 4 ? TcKernel<16, 4>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched)
                      : TcKernel<16, 3>::launch(x, Q, M, x_out, codes, scales, T, D, r, eps, status, s, launched);
 }

@@ -137,8 +137,22 @@ int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_ou
                        int D, int r, int dtype, void *stream) {
     int st = check_align_args(x, Q, M, x_out, T, D, r, dtype);
     if (st != RSQ_OK || T == 0) return st;
-    return finish(rsq::launch_align_generic(x, Q, M, x_out, nullptr, nullptr, T, D, r, 4, 0.f, dtype,
-                                            false, static_cast<cudaStream_t>(stream)));
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // the kernels of rsq_align_norm_quant instantiated without the norm and the
+    // codes (bits = 0), chosen the same way
+    const int which = rsq::g_align_kernel.load(std::memory_order_relaxed);
+    if (((which == 0 && T <= 16) || which == 4) && rsq::align_decode_supports(D, r, T)) {
+        const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, dtype, cs);
+        if (e != cudaErrorNotSupported) return finish(e);
+    }
+    if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
+        bool launched = false;
+        const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, cs, &launched);
+        if (e != cudaSuccess) return finish(e);
+        if (launched) return RSQ_OK;
+    }
+    if (which >= 2) return RSQ_ERR_UNSUPPORTED;
+    return finish(rsq::launch_align_generic(x, Q, M, x_out, nullptr, nullptr, T, D, r, 4, 0.f, dtype, false, cs));
 }
 
 int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_out,

@@ -197,6 +197,18 @@ def test_repeated_back_to_back_launches_are_deterministic(T):
     assert rsq.device_status() == 0
 
 
+@pytest.mark.parametrize("T", [1, 129, 3001])
+def test_int3_at_4096_on_the_tensor_core_kernels(T):
+    """INT3 at D = d = 4096 (cluster-of-8 alignment kernel with the deferred
+    INT3 code stores; the RHT tensor-core kernel) against the oracle."""
+    a = inputs.align_case(T, 4096, 32, 300 + T, dtype="bf16", bits=3, dist="student_t3", n_outliers=8,
+                          outlier_scale=100.0)
+    check_align(a, label=f"int3 align T={T}")
+    h = inputs.rht_case(T, 4096, 1, 400 + T, dtype="bf16", bits=3, dist="student_t3", n_outliers=8,
+                        outlier_scale=100.0)
+    check_rht(h, label=f"int3 rht T={T}")
+
+
 def test_bounded_wait_runs_out_and_reports():
     """The kernels' bounded wait, on an mbarrier that nothing arrives on, gives
     up after its limit; the kernel returns and sets the timeout bit of the

@@ -441,7 +441,7 @@ def run_gpu(args) -> None:
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; see DESIGN.md input recipe)",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded: N(0,1) activations with 8 outlier channels x100; random orthonormal Q, Cayley M, random signs)",
         "config": workload_config(T, n),
         "roofline": roof,
         "kernels": kern,

@@ -77,7 +77,8 @@ struct DecLayout {
     __host__ __device__ int off_wp() const { return off_prm() + 2 * T; }         // warps x T x 32
     __host__ __device__ int off_yin() const { return off_wp() + kDecWarps * T * kR; }  // [source CTA][own row][32]
     __host__ __device__ int off_stin() const { return (off_yin() + kDecCS * kOwnMax * kR + 3) & ~3; }  // [source][T] float4
-    __host__ __device__ int off_bar() const { return off_stin() + kDecCS * 4 * T; }  // 3 mbarriers (8 B each)
+    __host__ __device__ int off_ys() const { return off_stin() + kDecCS * 4 * T; }  // warps x 32: owner's y
+    __host__ __device__ int off_bar() const { return off_ys() + kDecWarps * kR; }  // 3 mbarriers (8 B each)
     __host__ __device__ int floats() const { return off_bar() + 3 * 2; }
     __host__ __device__ size_t bytes() const { return size_t(floats()) * 4; }
 };
@@ -213,9 +214,22 @@ k_align_decode(const typename IO::T *__restrict__ x, typename IO::T *__restrict_
         float y = 0.f;
 #pragma unroll
         for (int c = 0; c < kDecCS; ++c) y += syin[(c * kOwnMax + j) * kR + lane];
-        float acc = 0.f;
+        // z = M y: y through shared memory, read back whole by every lane
+        // (broadcast), four independent FMA chains
+        float *ys = smf + L.off_ys() + warp * kR;
+        __syncwarp();  // this warp's reads of its previous row are done
+        ys[lane] = y;
+        __syncwarp();
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < kR; ++k) acc = fmaf(smt[k * kR + lane], __shfl_sync(0xFFFFFFFFu, y, k), acc);
+        for (int k4 = 0; k4 < kR / 4; ++k4) {
+            const float4 yv = reinterpret_cast<const float4 *>(ys)[k4];
+            a4[0] = fmaf(smt[(4 * k4 + 0) * kR + lane], yv.x, a4[0]);
+            a4[1] = fmaf(smt[(4 * k4 + 1) * kR + lane], yv.y, a4[1]);
+            a4[2] = fmaf(smt[(4 * k4 + 2) * kR + lane], yv.z, a4[2]);
+            a4[3] = fmaf(smt[(4 * k4 + 3) * kR + lane], yv.w, a4[3]);
+        }
+        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
         const uint32_t dz = smem_u32(sz + t * kR + lane);
 #pragma unroll
         for (int c = 0; c < kDecCS; ++c)

@@ -252,6 +252,41 @@ def test_full_w3a3_sampled():
     check_rht(h, rows, "w3a3 rht T=8192")
 
 
+def test_batch_past_32_bit_byte_offsets():
+    """T = 2^19 rows at D = 4096: 4 GiB of bf16 input, so x_out reaches past
+    every 32-bit byte offset (codes up to 1 GiB).  The batch is one seeded
+    8192-row block repeated 64 times on the device, so every block of every
+    output must equal the first block bit for bit; sampled rows of the last
+    block are also checked against the oracle on their source rows."""
+    rsq = _rsq()
+    blk, reps = 8192, 64
+    a, h = inputs.llama7b_case(T=blk)
+    x = _to_dev(a.x, "bf16").repeat(reps, 1)
+    Q = torch.from_numpy(a.Q).to(DEV)
+    M = torch.from_numpy(a.M).to(DEV)
+    s = torch.from_numpy(h.signs).to(DEV)
+    xo, codes, scales = rsq.rsq_align_norm_quant(x, Q, M, bits=4, eps=a.eps)
+    hcodes, hscales = rsq.rht_quant(x, s, 1, bits=4)
+    torch.cuda.synchronize()
+    assert rsq.device_status() == 0
+    for k in (1, reps // 2, reps - 1):
+        sl = slice(k * blk, (k + 1) * blk)
+        assert torch.equal(xo[sl].view(torch.int16), xo[:blk].view(torch.int16)), k
+        assert torch.equal(codes[sl], codes[:blk]) and torch.equal(scales[sl], scales[:blk]), k
+        assert torch.equal(hcodes[sl], hcodes[:blk]) and torch.equal(hscales[sl], hscales[:blk]), k
+    rows = _sample(blk, 16)
+    last = torch.from_numpy((reps - 1) * blk + rows).to(DEV)
+    ref = oracle.align_norm_quant(a.x[rows], a.Q, a.M, 4, a.eps)
+    H.check_aligned(_host(xo[last]), ref["x_out"], a.x[rows], "bf16", "T=2^19 align")
+    H.check_scales(scales[last].cpu().numpy(), ref["scales"], "T=2^19 align")
+    H.check_codes(codes[last].cpu().numpy(), ref["q"], ref["pre"], 4, "T=2^19 align")
+    refh = oracle.rht_quant(a.x[rows], h.signs, 1, 4)
+    H.check_scales(hscales[last].cpu().numpy(), refh["scales"], "T=2^19 rht")
+    H.check_codes(hcodes[last].cpu().numpy(), refh["q"], refh["pre"], 4, "T=2^19 rht")
+    del x, xo, codes, scales, hcodes, hscales
+    torch.cuda.empty_cache()
+
+
 # --------------------------------------------------------------------------
 # edge cases
 # --------------------------------------------------------------------------

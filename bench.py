@@ -34,9 +34,16 @@ if ROOT not in sys.path:
 METRIC = "tokens/s & HBM GB/s (frac of B200 peak), fused align+FWHT+INT4 quant, D=4096"
 T_TOK, D, R, BITS, EPS = 16384, 4096, 32, 4, 1e-5
 E2E_CHUNKS = 8
-KERNEL_EVERY = 8  # per-kernel CUDA events on every 8th step of the timed region
+KERNEL_LOOP = 200  # isolated launches per kernel in the kernel-timing loop after the timed region
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0  # B200 HBM3e datasheet figure (HGX)
 L2_BYTES = 126 * 10 ** 6
+ARITHMETIC = ("bf16 I/O; alignment products on tcgen05 tensor cores as split-bf16 (hi/lo) operands with fp32 "
+              "accumulation in TMEM; RMSNorm, absmax and quantiser in fp32 (sum of squares folded into fp64); "
+              "Hadamard first stage as exact +-1 x bf16 tensor-core products, fp32 accumulate, fp32 butterflies")
+CONTEXT = ("ReSpinQuant pages: ~0.2% online overhead of the alignment at r~32 relative to the base model's "
+           "compute (hardware not stated for that figure; the end-to-end latency figures on the pages are "
+           "from an H100)")
 
 
 def algorithmic_bytes(T: int) -> dict:
@@ -226,9 +233,15 @@ def cpu_baseline(target_s: float = 10.0) -> dict:
     if T_s == T_TOK:
         reps = max(1, int(round(target_s / max(per_tok * T_TOK, 1e-9))))
     r = oracle_sample_rate(T_s, cores, reps)
+    # single-threaded: the same oracle on one core, a sample of about target_s / 2
+    T_1 = int(max(8, min(T_TOK, (target_s / 2) / max(per_tok * r["cores"], 1e-9))))
+    r1 = oracle_sample_rate(T_1, 1)
     return {"value": r["tokens"] / r["seconds"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
             "sample": f"{T_s} tokens of the same workload x {reps} pass(es) (both pipelines, float64 C "
-                      f"oracle, OpenMP over tokens), {r['seconds']:.1f} s"}
+                      f"oracle, OpenMP over tokens), {r['seconds']:.1f} s",
+            "single_thread": {"value": r1["tokens"] / r1["seconds"], "unit": "tokens/s", "cores": r1["cores"],
+                              "sample": f"{T_1} tokens of the same workload (both pipelines, float64 C oracle, "
+                                        f"one thread), {r1['seconds']:.1f} s"}}
 
 
 def run_reference(args) -> None:
@@ -307,21 +320,33 @@ def run_gpu(args) -> None:
         if n > 1:
             dist.barrier()
 
+    # Clock samples cover the warm-up, the timed region and the kernel-timing
+    # loop; the warm-up runs right before the timed region (no idle gap, so the
+    # timed steps start at the clocks the warm-up brought up).
+    sampler = ClockSampler(smi_id(dev))
+    sampler.start()
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
     torch.cuda.synchronize(dev)
+    # nvidia-smi takes a moment to report its first sample: until it does (2 s at
+    # most) the GPU keeps running untimed steps, so that the device is under load,
+    # not idle, when the timed region starts and while the sampler comes up
+    preroll, t_pre = 0, time.time()
+    while not sampler.samples and sampler.proc is not None and time.time() - t_pre < 2.0:
+        with torch.cuda.stream(stream):
+            for _ in range(8):
+                step()
+        torch.cuda.synchronize(dev)
+        preroll += 8
 
-    # Kernel durations: CUDA events around each kernel on every KERNEL_EVERY-th
-    # step of the timed region.  The other steps run back to back, as a user's
-    # stream does, so that the next kernel may start early (programmatic
-    # dependent launch); an event between two kernels would serialise them.
-    sampled = set(range(0, args.steps, KERNEL_EVERY))
-    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for k in sorted(sampled)}
+    # Timed region: K steps; CUDA events on the launching stream around each
+    # kernel of every step give the per-kernel durations inside the timed
+    # region (an event between two kernels also stops the next one from
+    # starting early by programmatic dependent launch, so the step time
+    # includes that small cost).
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(smi_id(dev))
-    sampler.start()
-    time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
     launches0 = rsq.launch_count()
@@ -329,25 +354,40 @@ def run_gpu(args) -> None:
     with torch.cuda.stream(stream):
         e_start.record(stream)
         for k in range(args.steps):
-            if k in sampled:
-                ev[k][0].record(stream)
+            ev[k][0].record(stream)
             rsq.rsq_align_norm_quant(x, Q, M, x_out, codes_a, scales_a, bits=BITS, eps=EPS, stream=stream)
-            if k in sampled:
-                ev[k][1].record(stream)
+            ev[k][1].record(stream)
             rsq.rht_quant(x, signs, 1, codes_h, scales_h, bits=BITS, stream=stream)
-            if k in sampled:
-                ev[k][2].record(stream)
+            ev[k][2].record(stream)
         e_end.record(stream)
     torch.cuda.synchronize(dev)
-    t_wall1 = time.time()
     barrier()
     launches = rsq.launch_count() - launches0
-    time.sleep(0.2)
+    total_ms = e_start.elapsed_time(e_end)
+    align_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    rht_ms = [e[1].elapsed_time(e[2]) for e in ev]
+
+    # Kernel-timing loop right after the timed region: KERNEL_LOOP launches of
+    # each kernel, each between its own pair of events (isolated launches, as
+    # ncu times them), for a per-launch figure resting on many samples.
+    def isolated(fn):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(KERNEL_LOOP)]
+        with torch.cuda.stream(stream):
+            for a0, a1 in evs:
+                a0.record(stream)
+                fn()
+                a1.record(stream)
+        torch.cuda.synchronize(dev)
+        return [a0.elapsed_time(a1) for a0, a1 in evs]
+
+    loop_ms = {
+        "align_norm_quant": isolated(lambda: rsq.rsq_align_norm_quant(x, Q, M, x_out, codes_a, scales_a, bits=BITS,
+                                                                      eps=EPS, stream=stream)),
+        "rht_quant": isolated(lambda: rsq.rht_quant(x, signs, 1, codes_h, scales_h, bits=BITS, stream=stream)),
+    }
+    t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
 
-    total_ms = e_start.elapsed_time(e_end)
-    align_ms = [e[0].elapsed_time(e[1]) for e in ev.values()]
-    rht_ms = [e[1].elapsed_time(e[2]) for e in ev.values()]
     total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     value = whole_job_rate(T, n, args.steps, total_ms)
@@ -429,30 +469,43 @@ def run_gpu(args) -> None:
     ab = algorithmic_bytes(T)
     kern = {}
     for name, ms in (("align_norm_quant", align_ms), ("rht_quant", rht_ms)):
-        avg = statistics.mean(ms)
+        lm = loop_ms[name]
+        avg = statistics.mean(lm)
         gbs = ab[name] / (avg / 1e3) / 1e9
-        kern[name] = {"avg_us": avg * 1e3, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"],
-                      "tokens_per_s": T / (avg / 1e3)}
+        in_step = statistics.mean(ms)
+        kern[name] = {"avg_us": avg * 1e3, "median_us": statistics.median(lm) * 1e3, "min_us": min(lm) * 1e3,
+                      "samples": len(lm), "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"],
+                      "frac_nominal": gbs / NOMINAL_HBM_GBS, "tokens_per_s": T / (avg / 1e3),
+                      "in_step_avg_us": in_step * 1e3, "in_step_samples": len(ms),
+                      "in_step_frac": ab[name] / (in_step / 1e3) / 1e9 / pk["hbm_gbs"],
+                      "algorithmic_bytes_per_launch": ab[name]}
     dom = max(kern, key=lambda k: kern[k]["avg_us"])
     roof = {"bound": "hbm", "kernel": dom, "achieved": kern[dom]["achieved_gbs"], "peak": pk["hbm_gbs"],
             "unit": "GB/s", "frac": kern[dom]["frac"], "traffic": recorded_traffic(dom),
             "algorithmic_bytes_per_launch": ab[dom],
-            "peak_source": f"{pk['source']} (STREAM-style copy, burst)"}
+            "peak_source": f"{pk['source']} (STREAM-style copy, burst)",
+            "frac_nominal": kern[dom]["frac_nominal"],
+            "nominal_peak": {"value": NOMINAL_HBM_GBS, "unit": "GB/s", "source": "B200 HBM3e datasheet (HGX)"}}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded: N(0,1) activations with 8 outlier channels x100; random orthonormal Q, Cayley M, random signs)",
+        "vs_baseline": None, "dtype": "bf16", "arithmetic": ARITHMETIC,
+        "data": "synthetic (seeded: N(0,1) activations with 8 outlier channels x100; random orthonormal Q, Cayley M, random signs)",
         "config": workload_config(T, n),
         "roofline": roof,
         "kernels": kern,
-        "kernel_timing": f"CUDA events around each kernel on every {KERNEL_EVERY}th step of the timed region; "
-                         "the other steps run back to back (programmatic dependent launch lets a kernel start "
-                         "while the previous one finishes)",
+        "kernel_timing": f"avg_us: {KERNEL_LOOP} isolated launches of each kernel, each between its own pair "
+                         "of CUDA events on the launching stream, right after the timed region (same clock "
+                         "window); in_step_avg_us: CUDA events around each kernel of every timed step",
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "pipeline": f"{E2E_CHUNKS} row chunks on three streams: H2D, kernels, D2H"},
         "gpu_launches": launches,
         "clocks": clocks,
+        "clock_preroll_steps": preroll,
+        "context": CONTEXT,
     }
+    if n == 1 and not args.no_secondary:
+        line["secondary"] = secondary_metrics(dev, stream, pk)
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
@@ -460,13 +513,116 @@ def run_gpu(args) -> None:
         dist.destroy_process_group()
 
 
-def run_secondary(args) -> None:
-    """Secondary workloads (one JSON line each, rank 0 only, 1 GPU): the 32-layer
-    chain at decode (T=16) and prefill (T=16384) sizes, timed as one CUDA graph
-    per pass, and the W3A3 / down_proj parity workloads."""
+def chain_metrics(dev, stream, T: int, steps: int, warmup: int, pk: dict) -> dict:
+    """The 32-layer chain (config of the chain workload: D=4096, r=32, bf16,
+    INT4, in place) at T rows, timed as one CUDA graph of the 32 layer calls."""
     import torch
     from w3a3_quantization_online_b200 import inputs, rsq
+    x0, qs, ms, _, _ = inputs.chain_case(T=T)
+    x = torch.from_numpy(x0).to(dev).to(torch.bfloat16)
+    Qd = [torch.from_numpy(q).to(dev) for q in qs]
+    Md = [torch.from_numpy(m).to(dev) for m in ms]
+    codes = torch.empty((T, 2048), dtype=torch.uint8, device=dev)
+    scales = torch.empty((T,), dtype=torch.float32, device=dev)
+    L = len(qs)
 
+    def chain():
+        for i in range(L):
+            rsq.rsq_align_norm_quant(x, Qd[i], Md[i], x, codes, scales, bits=4, stream=stream)
+
+    with torch.cuda.stream(stream):
+        chain()  # configure kernels outside capture
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        chain()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_pass = e0.elapsed_time(e1) / steps
+    per_layer_us = ms_pass * 1e3 / L
+    bytes_layer = T * (2 * 4096 * 2 + 2048 + 4) + 4096 * 32 * 4 + 32 * 32 * 4
+    gbs = bytes_layer / (per_layer_us * 1e-6) / 1e9
+    del g
+    return {"T": T, "layers": L, "us_per_layer": per_layer_us, "achieved_gbs": gbs, "frac": gbs / pk["hbm_gbs"],
+            "tokens_per_s_per_layer": T / (per_layer_us * 1e-6), "passes": steps,
+            "timing": "CUDA graph of the 32 in-place layer calls, CUDA events over the replays"}
+
+
+def kernel_metrics(dev, stream, workload: str, steps: int, warmup: int, pk: dict) -> dict:
+    """Back-to-back launches of each kernel of the W3A3 or down_proj workload."""
+    import torch
+    from w3a3_quantization_online_b200 import inputs, rsq
+    if workload == "w3a3":
+        a, h = inputs.w3a3_case(T=8192)
+    elif workload == "downproj":
+        a, h = None, inputs.down_proj_case(T=4096)
+    else:
+        raise SystemExit(f"unknown workload {workload}")
+    res = {}
+    if a is not None:
+        x = torch.from_numpy(a.x).to(dev).to(torch.bfloat16)
+        Q, M = torch.from_numpy(a.Q).to(dev), torch.from_numpy(a.M).to(dev)
+        xo = torch.empty_like(x)
+        c = torch.empty((a.T, a.D * a.bits // 8), dtype=torch.uint8, device=dev)
+        sc = torch.empty((a.T,), dtype=torch.float32, device=dev)
+        f = lambda: rsq.rsq_align_norm_quant(x, Q, M, xo, c, sc, bits=a.bits, stream=stream)
+        byts = a.T * (2 * a.D * 2 + a.D * a.bits // 8 + 4) + a.D * a.r * 4
+        res["align_norm_quant"] = (f, byts, a.T, f"T={a.T}, D={a.D}, r={a.r}, INT{a.bits}")
+    xh = torch.from_numpy(h.x).to(dev).to(torch.bfloat16)
+    sg = torch.from_numpy(h.signs).to(dev)
+    ch = torch.empty((h.T, h.d * h.bits // 8), dtype=torch.uint8, device=dev)
+    sh = torch.empty((h.T,), dtype=torch.float32, device=dev)
+    fr = lambda: rsq.rht_quant(xh, sg, h.m, ch, sh, bits=h.bits, stream=stream)
+    res["rht_quant"] = (fr, h.T * (h.d * 2 + h.d * h.bits // 8 + 4) + h.d, h.T,
+                        f"T={h.T}, d={h.d} = {h.d // h.m}*{h.m}, INT{h.bits}")
+    kern = {}
+    for name, (f, byts, T, shape) in res.items():
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                f()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(steps):
+                f()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) * 1e3 / steps
+        kern[name] = {"shape": shape, "avg_us": us, "achieved_gbs": byts / (us * 1e-6) / 1e9,
+                      "frac": byts / (us * 1e-6) / 1e9 / pk["hbm_gbs"], "tokens_per_s": T / (us * 1e-6),
+                      "launches": steps, "timing": "back-to-back launches, CUDA events over the loop"}
+    return kern
+
+
+def secondary_metrics(dev, stream, pk: dict) -> dict:
+    """The other configurations, bounded to a few seconds of GPU time: W3A3
+    (T=8192, D=8192, INT3: alignment and RHT 2^13), the down_proj RHT
+    (T=4096, d=12288 Kronecker) and the 32-layer chain at T=16 and T=16384."""
+    import torch
+    out = {"w3a3": kernel_metrics(dev, stream, "w3a3", 100, 5, pk)}
+    torch.cuda.empty_cache()
+    out["downproj"] = kernel_metrics(dev, stream, "downproj", 100, 5, pk)
+    torch.cuda.empty_cache()
+    out["chain16"] = chain_metrics(dev, stream, 16, 50, 5, pk)
+    out["chain16384"] = chain_metrics(dev, stream, 16384, 10, 3, pk)
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_secondary(args) -> None:
+    """One secondary workload on its own line (rank 0, 1 GPU), with the
+    requested steps: the 32-layer chain at decode (T=16) or prefill (T=16384)
+    size, or the W3A3 / down_proj kernels."""
+    import torch
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     pk = peaks()
@@ -474,83 +630,11 @@ def run_secondary(args) -> None:
     out = {"workload": args.workload, "steps": args.steps, "warmup": args.warmup, "data": "synthetic"}
     if args.workload.startswith("chain"):
         T = 16 if args.workload == "chain16" else 16384
-        x0, qs, ms, _, _ = inputs.chain_case(T=T)
-        x = torch.from_numpy(x0).to(dev).to(torch.bfloat16)
-        Qd = [torch.from_numpy(q).to(dev) for q in qs]
-        Md = [torch.from_numpy(m).to(dev) for m in ms]
-        codes = torch.empty((T, 2048), dtype=torch.uint8, device=dev)
-        scales = torch.empty((T,), dtype=torch.float32, device=dev)
-        L = len(qs)
-
-        def chain():
-            for i in range(L):
-                rsq.rsq_align_norm_quant(x, Qd[i], Md[i], x, codes, scales, bits=4, stream=stream)
-
-        with torch.cuda.stream(stream):
-            chain()  # configure kernels outside capture
-        torch.cuda.synchronize(dev)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            chain()
-        for _ in range(args.warmup):
-            g.replay()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        with torch.cuda.stream(stream):
-            for _ in range(args.steps):
-                g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms_pass = e0.elapsed_time(e1) / args.steps
-        per_layer_us = ms_pass * 1e3 / L
-        bytes_layer = T * (2 * 4096 * 2 + 2048 + 4) + 4096 * 32 * 4 + 32 * 32 * 4
-        gbs = bytes_layer / (per_layer_us * 1e-6) / 1e9
-        out.update({"metric": "per-layer latency and HBM GB/s, 32-layer align+norm+INT4 chain, D=4096",
-                    "T": T, "layers": L, "us_per_layer": per_layer_us, "achieved_gbs": gbs,
-                    "frac": gbs / pk["hbm_gbs"], "tokens_per_s_per_layer": T / (per_layer_us * 1e-6),
-                    "timing": "CUDA graph of the 32 in-place layer calls, CUDA events over the replays"})
-        del g
+        out.update({"metric": "per-layer latency and HBM GB/s, 32-layer align+norm+INT4 chain, D=4096"})
+        out.update(chain_metrics(dev, stream, T, args.steps, args.warmup, pk))
     else:
-        if args.workload == "w3a3":
-            a, h = inputs.w3a3_case(T=8192)
-        elif args.workload == "downproj":
-            a, h = None, inputs.down_proj_case(T=4096)
-        else:
-            raise SystemExit(f"unknown workload {args.workload}")
-        res = {}
-        if a is not None:
-            x = torch.from_numpy(a.x).to(dev).to(torch.bfloat16)
-            Q, M = torch.from_numpy(a.Q).to(dev), torch.from_numpy(a.M).to(dev)
-            xo = torch.empty_like(x)
-            c = torch.empty((a.T, a.D * a.bits // 8), dtype=torch.uint8, device=dev)
-            sc = torch.empty((a.T,), dtype=torch.float32, device=dev)
-            f = lambda: rsq.rsq_align_norm_quant(x, Q, M, xo, c, sc, bits=a.bits, stream=stream)
-            byts = a.T * (2 * a.D * 2 + a.D * a.bits // 8 + 4) + a.D * a.r * 4
-            res["align_norm_quant"] = (f, byts, a.T)
-        xh = torch.from_numpy(h.x).to(dev).to(torch.bfloat16)
-        sg = torch.from_numpy(h.signs).to(dev)
-        ch = torch.empty((h.T, h.d * h.bits // 8), dtype=torch.uint8, device=dev)
-        sh = torch.empty((h.T,), dtype=torch.float32, device=dev)
-        fr = lambda: rsq.rht_quant(xh, sg, h.m, ch, sh, bits=h.bits, stream=stream)
-        res["rht_quant"] = (fr, h.T * (h.d * 2 + h.d * h.bits // 8 + 4) + h.d, h.T)
-        kern = {}
-        for name, (f, byts, T) in res.items():
-            with torch.cuda.stream(stream):
-                for _ in range(args.warmup):
-                    f()
-            torch.cuda.synchronize(dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            with torch.cuda.stream(stream):
-                for _ in range(args.steps):
-                    f()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            us = e0.elapsed_time(e1) * 1e3 / args.steps
-            kern[name] = {"avg_us": us, "achieved_gbs": byts / (us * 1e-6) / 1e9,
-                          "frac": byts / (us * 1e-6) / 1e9 / pk["hbm_gbs"], "tokens_per_s": T / (us * 1e-6)}
-        out.update({"metric": "tokens/s and HBM GB/s per kernel", "kernels": kern})
+        out.update({"metric": "tokens/s and HBM GB/s per kernel",
+                    "kernels": kernel_metrics(dev, stream, args.workload, args.steps, args.warmup, pk)})
     out["peak_gbs"] = pk["hbm_gbs"]
     print(json.dumps(out), flush=True)
 
@@ -563,6 +647,8 @@ def main():
     ap.add_argument("--impl", choices=["rsq", "reference"], default="rsq")
     ap.add_argument("--tokens", type=int, default=T_TOK, help="tokens per GPU (default 16384)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="leave out the secondary workloads (W3A3, down_proj, 32-layer chain) of the headline line")
     ap.add_argument("--workload", default="hidden",
                     choices=["hidden", "chain16", "chain16384", "w3a3", "downproj"],
                     help="hidden = the headline step (default); the others print a secondary line")

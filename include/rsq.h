@@ -134,29 +134,34 @@ uint64_t rsq_launch_count(void);
 /* Kernel used by rsq_align_norm_quant: 0 = automatic (T <= 16 with
  * 2048 <= D <= 8192, D % 128 == 0, r <= 32: the decode kernel, one cluster of
  * 16 CTAs on FP32 FMAs, which takes up to 32 rows on request; otherwise, for
- * bf16, D in {4096, 8192} and r <= 32,
- * the single-tile tensor-core cluster kernel; the CUDA-core kernel for
- * everything else), 1 = always the CUDA-core kernel, 2 = only the single-tile
- * tensor-core kernel, 3 = only the double-buffered one, 4 = only the decode
- * kernel (2, 3 and 4 return RSQ_ERR_UNSUPPORTED for calls they cannot serve).
- * Process-wide; returns the previous setting, or -1 for an invalid value.  All
- * compute the same function; this exists for testing and measurement. */
+ * bf16, D in {4096, 8192} and r <= 32, the tensor-core cluster kernel; the
+ * CUDA-core kernel for everything else), 1 = always the CUDA-core kernel,
+ * 2 = only the tensor-core cluster kernel, 4 = only the decode kernel (2 and 4
+ * return RSQ_ERR_UNSUPPORTED for calls they cannot serve).  Process-wide;
+ * returns the previous setting, or -1 for an invalid value.  All compute the
+ * same function; this exists for testing and measurement. */
 int rsq_select_align_kernel(int which);
 
 /* Kernel used by rht_quant: 0 = automatic (tensor-core kernel for bf16,
  * d in {4096, 8192}, m = 1; the Kronecker kernel for bf16, d = 12288, m = 12,
  * INT4; shared-memory radix-16 kernel otherwise), 1 = always the radix-16
- * kernel, 2 = only the warp-per-row CUDA-core kernel (d = 4096), 3 = only the
- * tensor-core kernel, 4 = only the Kronecker kernel (2, 3 and 4 return
- * RSQ_ERR_UNSUPPORTED for other shapes).
- * Process-wide; returns the previous setting, -1 if invalid.  All compute the
- * same function; this exists for testing and measurement. */
+ * kernel, 3 = only the tensor-core kernel, 4 = only the Kronecker kernel (3 and
+ * 4 return RSQ_ERR_UNSUPPORTED for other shapes).  Process-wide; returns the
+ * previous setting, -1 if invalid.  All compute the same function; this exists
+ * for testing and measurement. */
 int rsq_select_rht_kernel(int which);
 
-/* Synchronise `stream`, then read and clear the device status word of the
- * current device into *status: 0 if no kernel reported a problem, otherwise the
- * OR of error bits (1 = a bounded wait inside a kernel timed out; that call's
- * outputs are invalid).  Returns an rsq_status. */
+/* Device status word.  Kernels of this library report problems by OR-ing error
+ * bits into one word per device (1 = a bounded wait inside a kernel timed out;
+ * that call's outputs are invalid).  The word is shared by every stream, host
+ * thread and call on the device.  rsq_device_status enqueues on `stream` a
+ * one-thread kernel that takes the word and clears it in one atomic exchange,
+ * synchronises `stream` and stores the value taken in *status (0 = no problem).
+ * Work queued on `stream` before the call is therefore covered; a kernel still
+ * running on another stream may set a bit after the exchange, and that bit then
+ * stays in the word for the next call (it is never lost, but it may be
+ * reported by a later call than the one whose kernel set it).  Returns an
+ * rsq_status. */
 int rsq_device_status(void *stream, int *status);
 
 /* Test of the error path of the bounded waits: enqueues on `stream` a

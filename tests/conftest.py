@@ -24,3 +24,12 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def near_tie_session_rule():
+    """At the end of the session: near-tie code mismatches over every parity
+    check of the session are at most 1e-5 of all codes compared."""
+    from tests import helpers
+    yield
+    helpers.tie_tally_check()

@@ -2,13 +2,20 @@
 
 Tolerances (written here once, used by every parity test):
   * aligned values, float32 I/O: max |gpu - oracle| <= 1e-4 * max|x| per row;
-  * aligned values, bf16 I/O:    max |gpu - oracle| <= 4e-3 * max|oracle| per row;
+  * aligned values, bf16 I/O: element by element, |gpu - oracle| <= 4e-3 * |oracle|
+    + 1e-5 * max|oracle of the row| (the relative bound itself, plus a floor for
+    elements near zero, where a relative error means nothing: the floor is far
+    below the 4e-3 bound on every ordinary element of a row with outliers);
   * scales: relative error <= 1e-6 (both exactly 0 for an all-zero row); a
     scale below the float32 normal range cannot carry that relative precision,
     so the bound is 1e-6 * scale + 2^-149 (half the float32 subnormal spacing);
   * codes: equal, except +-1 where the oracle's pre-round value v/alpha lies
-    within 1e-4 of a rounding tie (|frac(|v/alpha|) - 0.5| < 1e-4); such
-    mismatches may number at most 1e-5 of all codes, rounded up to a whole code.
+    within 1e-4 of a rounding tie (|frac(|v/alpha|) - 0.5| < 1e-4).  Such
+    mismatches are added up over the whole test session together with the
+    number of codes compared, and the session total may be at most 1e-5 of all
+    codes (checked once at the end of the session, tests/conftest.py); a single
+    check outside a session (smoke) applies the same fraction to its own codes,
+    rounded down.
 """
 from __future__ import annotations
 
@@ -18,9 +25,19 @@ import numpy as np
 
 ALIGN_F32_ABS = 1e-4
 ALIGN_BF16_REL = 4e-3
+ALIGN_BF16_FLOOR = 1e-5
 SCALE_REL = 1e-6
 TIE_BAND = 1e-4
 TIE_FRACTION = 1e-5
+
+# near-tie mismatches and codes compared, over the test session
+TIE_TALLY = {"mismatches": 0, "codes": 0}
+
+
+def tie_tally_check() -> None:
+    """The session rule: near-tie mismatches <= 1e-5 of all codes compared."""
+    m, n = TIE_TALLY["mismatches"], TIE_TALLY["codes"]
+    assert m <= TIE_FRACTION * n, f"{m} near-tie code mismatches over {n} codes > {TIE_FRACTION:g} of them"
 
 
 def unpack_int4(b: np.ndarray, n: int) -> np.ndarray:
@@ -46,13 +63,18 @@ def unpack(b: np.ndarray, n: int, bits: int) -> np.ndarray:
 
 
 def check_codes(gpu_bytes: np.ndarray, ora_q: np.ndarray, ora_pre: np.ndarray, bits: int,
-                label: str = "") -> int:
-    """Assert the code rule; returns the number of (allowed) near-tie mismatches."""
+                label: str = "", session: bool = True) -> int:
+    """Assert the code rule; returns the number of (allowed) near-tie mismatches.
+
+    session=True adds the counts to the session tally (checked at the end of
+    the session); session=False checks the fraction on this call's codes."""
     n = ora_q.shape[-1]
     g = unpack(np.asarray(gpu_bytes), n, bits)
     qmax = 2 ** (bits - 1) - 1
-    assert g.min() >= -qmax and g.max() <= qmax, f"{label}: code out of range"
+    assert g.size == 0 or (g.min() >= -qmax and g.max() <= qmax), f"{label}: code out of range"
     mism = g != ora_q
+    if session:
+        TIE_TALLY["codes"] += int(ora_q.size)
     if not mism.any():
         return 0
     a = np.abs(ora_pre)
@@ -64,8 +86,11 @@ def check_codes(gpu_bytes: np.ndarray, ora_q: np.ndarray, ora_pre: np.ndarray, b
         info = [(tuple(i), int(g[tuple(i)]), int(ora_q[tuple(i)]), float(ora_pre[tuple(i)])) for i in idx]
         raise AssertionError(f"{label}: {int(bad.sum())} code mismatches outside the tie band, e.g. {info}")
     count = int(mism.sum())
-    allowed = math.ceil(TIE_FRACTION * ora_q.size)
-    assert count <= allowed, f"{label}: {count} near-tie mismatches > {allowed} allowed"
+    if session:
+        TIE_TALLY["mismatches"] += count
+    else:
+        allowed = math.floor(TIE_FRACTION * ora_q.size)
+        assert count <= allowed, f"{label}: {count} near-tie mismatches > {allowed} allowed"
     return count
 
 
@@ -82,14 +107,22 @@ def check_scales(gpu: np.ndarray, ora: np.ndarray, label: str = "") -> float:
 
 
 def check_aligned(gpu: np.ndarray, ora: np.ndarray, x: np.ndarray, dtype: str, label: str = "") -> float:
+    """Assert the aligned-value rule; returns the largest error / bound ratio."""
     gpu = np.asarray(gpu, dtype=np.float64)
-    err = np.abs(gpu - ora).max(axis=1)
+    ora = np.asarray(ora, dtype=np.float64)
+    if gpu.size == 0:
+        return 0.0
+    err = np.abs(gpu - ora)
     if dtype == "f32":
-        bound = ALIGN_F32_ABS * np.abs(np.asarray(x, dtype=np.float64)).max(axis=1)
+        bound = ALIGN_F32_ABS * np.abs(np.asarray(x, dtype=np.float64)).max(axis=1, keepdims=True)
+        err = err.max(axis=1, keepdims=True)
     else:
-        bound = ALIGN_BF16_REL * np.abs(ora).max(axis=1)
+        bound = ALIGN_BF16_REL * np.abs(ora) + ALIGN_BF16_FLOOR * np.abs(ora).max(axis=1, keepdims=True)
     ok = err <= bound
-    assert ok.all(), f"{label}: aligned-value error {err[~ok].max():.3e} above bound in {int((~ok).sum())} rows"
+    if not ok.all():
+        i = np.unravel_index(np.argmax(np.where(ok, 0.0, err - bound)), err.shape)
+        raise AssertionError(f"{label}: aligned-value error above bound at {int((~ok).sum())} places, "
+                             f"e.g. {tuple(int(v) for v in i)}: err {float(err[i]):.3e} > {float(bound[i]):.3e}")
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = np.where(bound > 0, err / bound, 0.0)
-    return float(ratio.max()) if ratio.size else 0.0
+    return float(ratio.max())

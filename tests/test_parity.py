@@ -132,6 +132,34 @@ def test_chain_32_layers_teacher_forced(T):
     np.testing.assert_allclose(n1, np.linalg.norm(xr, axis=1), rtol=2e-3)
 
 
+def test_chain_32_layers_prefill_16384_sampled():
+    """The 32-layer chain at prefill size (T = 16384, in place, bench launch
+    configuration): every layer runs on the whole stream on the GPU; before
+    each layer the sampled rows of the GPU's bf16 stream are taken as that
+    layer's oracle input (teacher forcing), and after it that layer's x_out,
+    codes and scales of those rows are checked against the oracle."""
+    rsq = _rsq()
+    T = 16384
+    x0, qs, ms, _, _ = inputs.chain_case(T=T)
+    rows = _sample(T, 40, seed=4)
+    rows_dev = torch.from_numpy(rows).to(DEV)
+    x = _to_dev(x0, "bf16")
+    codes = torch.empty((T, 2048), dtype=torch.uint8, device=DEV)
+    scales = torch.empty((T,), dtype=torch.float32, device=DEV)
+    for i in range(len(qs)):
+        x_in = _host(x[rows_dev])
+        Q = torch.from_numpy(qs[i]).to(DEV)
+        M = torch.from_numpy(ms[i]).to(DEV)
+        rsq.rsq_align_norm_quant(x, Q, M, x_out=x, codes=codes, scales=scales, bits=4)
+        ref = oracle.align_norm_quant(x_in, qs[i], ms[i], 4, 1e-5)
+        H.check_aligned(_host(x[rows_dev]), ref["x_out"], x_in, "bf16", f"prefill layer {i}")
+        H.check_scales(scales[rows_dev].cpu().numpy(), ref["scales"], f"prefill layer {i}")
+        H.check_codes(codes[rows_dev].cpu().numpy(), ref["q"], ref["pre"], 4, f"prefill layer {i}")
+    assert rsq.device_status() == 0
+    del x, codes, scales
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("T", [16, 300])
 def test_back_to_back_layers_match_the_synchronised_run(T):
     """The default kernels may start before the previous kernel of the stream
@@ -334,7 +362,7 @@ def test_generic_kernel_at_the_tensor_core_shapes(generic_align, T):
     check_align(a, label=f"generic w3a3 T={T}")
 
 
-@pytest.mark.parametrize("which", [2, 3])
+@pytest.mark.parametrize("which", [2])
 def test_tensor_core_kernel_serves_the_hot_shapes(which):
     rsq = _rsq()
     prev = rsq.select_align_kernel(which)
@@ -435,7 +463,7 @@ def test_rht_shapes(d, m, dtype, bits):
     check_rht(h, label=f"d={d} m={m}")
 
 
-@pytest.mark.parametrize("d,kernels", [(4096, (3, 2, 1)), (8192, (3, 1))])
+@pytest.mark.parametrize("d,kernels", [(4096, (3, 1)), (8192, (3, 1))])
 def test_rht_kernels_agree_with_the_oracle(d, kernels):
     rsq = _rsq()
     for which in kernels:
@@ -468,7 +496,7 @@ def test_kronecker_12288_kernels(which):
         rsq.select_rht_kernel(prev)
 
 
-@pytest.mark.parametrize("d,which", [(4096, 1), (4096, 2), (4096, 3), (8192, 3)])
+@pytest.mark.parametrize("d,which", [(4096, 1), (4096, 3), (8192, 3)])
 def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()
     prev = rsq.select_rht_kernel(which)

@@ -27,6 +27,8 @@ cudaError_t launch_rht_generic(const void *x, const int8_t *signs, int m, uint8_
 // Device-side status word of the current device (bits from sm100::kErr*), or
 // nullptr if its address cannot be obtained.
 int *device_status_word();
+// Device word that rsq_device_status() takes the status into (same device).
+int *status_taken_word();
 
 // Tensor-core alignment + RMSNorm + quantiser (bf16, D in {4096, 8192}, r <= 32).
 bool align_tc_supports(int D, int r, int dtype, long long T);
@@ -36,12 +38,6 @@ cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void 
                             float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
                             bool *launched);
 
-// Double-buffered tensor-core alignment kernel for D = 4096 (cluster of 16).
-bool align_tc_db_supports(int D, int r, int dtype, long long T);
-cudaError_t launch_align_tc_db(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
-                               float *scales, long long T, int r, int bits, float eps, cudaStream_t s,
-                               bool *launched);
-
 // Decode-size alignment + RMSNorm + quantiser: one cluster of 16 CTAs, FP32 FMAs
 // (T <= 32, 2048 <= D <= 8192, D % 128 == 0, r <= 32, bf16 or fp32 I/O).
 // Returns cudaErrorNotSupported if the cluster cannot be co-scheduled.
@@ -49,11 +45,6 @@ bool align_decode_supports(int D, int r, long long T);
 cudaError_t launch_align_decode(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
                                 float *scales, long long T, int D, int r, int bits, float eps, int dtype,
                                 cudaStream_t s);
-
-// Warp-per-row randomised Hadamard of order 4096 (m = 1, bf16, INT4/INT3).
-bool rht_fast_supports(int d, int m, int dtype, int bits, long long T);
-cudaError_t launch_rht_fast(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
-                            int bits, cudaStream_t s);
 
 // Randomised Hadamard H_1024 (x) H_12 of order 12288 (Paley H_12), bf16, INT4.
 bool rht_kron_supports(int d, int m, int dtype, int bits, long long T);

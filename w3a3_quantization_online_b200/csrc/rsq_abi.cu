@@ -15,13 +15,15 @@
 namespace rsq {
 
 // Device-side status word: kernels OR error bits into it (bounded waits that
-// timed out); rsq_device_status() reads and clears it.
+// timed out); rsq_device_status() takes it (atomic exchange with 0) into
+// g_status_taken on the caller's stream and copies that to the host.
 __device__ int g_device_status;
+__device__ int g_status_taken;
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
-std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 double-buffered, 4 decode
-std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 2 warp-per-row, 3 tensor core, 4 Kronecker 12288
+std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 4 decode
+std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 3 tensor core, 4 Kronecker 12288
 thread_local int g_last_cuda_error = 0;
 
 constexpr int kMaxDevices = 64;
@@ -48,7 +50,22 @@ __global__ void k_selftest_wait(int *status, unsigned long long limit_ns) {
     sm100::fence_mbar_init();
     if (!sm100::mbar_wait(b, 0u, false, limit_ns)) atomicOr(status, sm100::kErrMbarTimeout);
 }
+
+// Takes the status word in one atomic step, so that a bit a kernel on another
+// stream sets at the same moment is either taken now or left for the next call.
+__global__ void k_take_status(int *word, int *out) { *out = atomicExch(word, 0); }
 }  // namespace
+
+int *status_taken_word() {
+    static int *addr[kMaxDevices];
+    const int dev = cur_device();
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_taken) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
 
 int num_sms() {
     const int dev = cur_device();
@@ -180,19 +197,13 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype, cs);
         if (e != cudaErrorNotSupported) return finish(e);  // not co-schedulable: another kernel serves it
     }
-    if (which == 3 && rsq::align_tc_db_supports(D, r, dtype, T)) {
-        bool launched = false;
-        const cudaError_t e = rsq::launch_align_tc_db(x, Q, M, x_out, codes, scales, T, r, bits, eps, cs, &launched);
-        if (e != cudaSuccess) return finish(e);
-        if (launched) return RSQ_OK;
-    }
     if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
         bool launched = false;
         const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, cs, &launched);
         if (e != cudaSuccess) return finish(e);
         if (launched) return RSQ_OK;
     }
-    if (which == 2 || which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
+    if (which == 2 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
                                             true, static_cast<cudaStream_t>(stream)));
 }
@@ -217,9 +228,7 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
         return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, d, bits, static_cast<cudaStream_t>(stream)));
     if ((which == 0 || which == 4) && rsq::rht_kron_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_kron(x, signs, codes, scales, T, static_cast<cudaStream_t>(stream)));
-    if (which == 2 && rsq::rht_fast_supports(d, m, dtype, bits, T))
-        return finish(rsq::launch_rht_fast(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
-    if (which == 2 || which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
+    if (which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
                                           static_cast<cudaStream_t>(stream)));
 }
@@ -243,23 +252,28 @@ const char *rsq_status_string(int status) {
 int rsq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int rsq_select_align_kernel(int which) {
-    if (which < 0 || which > 4) return -1;
+    if (which < 0 || which > 4 || which == 3) return -1;
     return rsq::g_align_kernel.exchange(which);
 }
 
 int rsq_select_rht_kernel(int which) {
-    if (which < 0 || which > 4) return -1;
+    if (which < 0 || which > 4 || which == 2) return -1;
     return rsq::g_rht_kernel.exchange(which);
 }
 
 int rsq_device_status(void *stream, int *status) {
     if (!status) return RSQ_ERR_NULL;
     int *word = rsq::device_status_word();
-    if (!word) return finish(cudaErrorInvalidDevice);
+    int *taken = rsq::status_taken_word();
+    if (!word || !taken) return finish(cudaErrorInvalidDevice);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaStreamSynchronize(s);
-    if (e == cudaSuccess) e = cudaMemcpy(status, word, sizeof(int), cudaMemcpyDeviceToHost);
-    if (e == cudaSuccess) e = cudaMemset(word, 0, sizeof(int));
+    rsq::k_take_status<<<1, 1, 0, s>>>(word, taken);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) rsq::count_launch(1);
+    int v = 0;
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&v, taken, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess) *status = v;
     return finish(e);
 }
 

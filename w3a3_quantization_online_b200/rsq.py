@@ -49,8 +49,8 @@ EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_stat
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
 
-ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DOUBLE_BUFFERED, ALIGN_DECODE = 0, 1, 2, 3, 4
-RHT_AUTO, RHT_GENERIC, RHT_SPECIALISED, RHT_TENSOR_CORE, RHT_KRONECKER = 0, 1, 2, 3, 4
+ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DECODE = 0, 1, 2, 4
+RHT_AUTO, RHT_GENERIC, RHT_TENSOR_CORE, RHT_KRONECKER = 0, 1, 3, 4
 
 
 class RsqError(RuntimeError):
@@ -71,7 +71,7 @@ def launch_count() -> int:
 
 
 def select_align_kernel(which: int) -> int:
-    """0 auto, 1 CUDA-core, 2 single-tile tensor-core, 3 double-buffered tensor-core; returns the previous setting."""
+    """0 auto, 1 CUDA-core, 2 tensor-core cluster kernel, 4 decode kernel; returns the previous setting."""
     prev = int(_lib.rsq_select_align_kernel(int(which)))
     if prev < 0:
         raise ValueError(which)
@@ -79,7 +79,7 @@ def select_align_kernel(which: int) -> int:
 
 
 def select_rht_kernel(which: int) -> int:
-    """0 auto, 1 radix-16 SMEM kernel, 2 warp-per-row kernel, 3 tensor-core kernel; returns the previous setting."""
+    """0 auto, 1 radix-16 SMEM kernel, 3 tensor-core kernel, 4 Kronecker kernel; returns the previous setting."""
     prev = int(_lib.rsq_select_rht_kernel(int(which)))
     if prev < 0:
         raise ValueError(which)
@@ -87,7 +87,9 @@ def select_rht_kernel(which: int) -> int:
 
 
 def device_status(stream=None) -> int:
-    """Synchronise the stream and return (and clear) the device status word (0 = healthy)."""
+    """Take (and clear) the device status word on the stream, after the work
+    queued on it; returns it (0 = healthy).  The word is per device and shared
+    by all streams."""
     out = _i32(0)
     _check(_lib.rsq_device_status(_stream(stream), ctypes.byref(out)))
     return int(out.value)

@@ -46,6 +46,8 @@ def lib():
             L.ora_pack.argtypes = [i64, i32, i32, _I8, _U8]
             L.ora_align_norm_quant.argtypes = [i64, i32, i32, i32, f64, _D, _D, _D, _D, _I8, _U8, _D, _D]
             L.ora_rht_quant.argtypes = [i64, i32, i32, i32, _D, _D, _I8, _I8, _U8, _D, _D]
+            L.ora_silu_gate.argtypes = [i64, i32, _D, _D, _D]
+            L.ora_rht_quant_gate.argtypes = [i64, i32, i32, i32, _D, _D, _D, _I8, _I8, _U8, _D, _D]
             _lib = L
     return _lib
 
@@ -179,6 +181,32 @@ def rht_quant(x, signs, m: int, bits: int, want_pre: bool = True) -> dict:
     pre = np.empty_like(x) if want_pre else None
     rc = lib().ora_rht_quant(T, d, m, bits, _p(Hm, _D), _p(x, _D), _p(s, _I8), _p(q, _I8),
                              _p(codes, _U8), _p(scales, _D), _p(pre, _D))
+    if rc:
+        raise ValueError(f"oracle rejected d={d}, m={m}, bits={bits} (rc={rc})")
+    return {"q": q, "codes": codes, "scales": scales, "pre": pre}
+
+
+def silu_gate(a, b) -> np.ndarray:
+    """g = SiLU(a) * b = a / (1 + exp(-a)) * b, element by element (the gated FFN product)."""
+    a, b = _f64(a), _f64(b)
+    T, d = a.shape
+    g = np.empty_like(a)
+    lib().ora_silu_gate(T, d, _p(a, _D), _p(b, _D), _p(g, _D))
+    return g
+
+
+def rht_quant_gate(a, b, signs, m: int, bits: int, want_pre: bool = True) -> dict:
+    """SiLU(a) * b -> randomised Hadamard -> symmetric per-token quantisation -> pack."""
+    a, b = _f64(a), _f64(b)
+    T, d = a.shape
+    s = np.ascontiguousarray(signs, dtype=np.int8)
+    Hm = _f64(kron_factor(m))
+    q = np.empty((T, d), dtype=np.int8)
+    codes = np.empty((T, d * bits // 8), dtype=np.uint8)
+    scales = np.empty(T, dtype=np.float64)
+    pre = np.empty_like(a) if want_pre else None
+    rc = lib().ora_rht_quant_gate(T, d, m, bits, _p(Hm, _D), _p(a, _D), _p(b, _D), _p(s, _I8), _p(q, _I8),
+                                  _p(codes, _U8), _p(scales, _D), _p(pre, _D))
     if rc:
         raise ValueError(f"oracle rejected d={d}, m={m}, bits={bits} (rc={rc})")
     return {"q": q, "codes": codes, "scales": scales, "pre": pre}

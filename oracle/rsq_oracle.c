@@ -26,6 +26,8 @@
  *          quantisation, row absmax / 7, scale-free RMSNorm in FP32), and
  *          SpinQuant / Motivation (symmetric quantiser
  *          alpha = max|X| / (2^(N-1) - 1), X_Q = alpha * round(X / alpha)).
+ *          QuaRot / Method also places an online Hadamard on the down_proj
+ *          input, which is the FFN's gated product SiLU(gate) * up.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - rounding is to nearest, ties to even (rint in the default mode);
@@ -239,6 +241,14 @@ static void pack_int3_row(int n, const int8_t *q, uint8_t *out)
     }
 }
 
+/* [IQ2] QuaRot / Method: the down_proj input is the gated FFN product
+ * g = SiLU(a) * b, SiLU(a) = a / (1 + exp(-a)) (a = gate projection, b = up
+ * projection).  Computed in double from the exact input values. */
+static void silu_gate_row(int d, const double *a, const double *b, double *g)
+{
+    for (int i = 0; i < d; ++i) g[i] = a[i] / (1.0 + exp(-a[i])) * b[i];
+}
+
 /* ------------------------------------------------------------------------ */
 /* exported batched entry points (OpenMP over independent token rows)       */
 /* ------------------------------------------------------------------------ */
@@ -375,6 +385,51 @@ int ora_rht_quant(int64_t T, int d, int m, int bits, const double *Hm, const dou
                 else pack_int3_row(d, q + t * d, codes + t * row_bytes);
             }
         }
+        free(u);
+        free(v);
+    }
+    return err;
+}
+
+int ora_silu_gate(int64_t T, int d, const double *a, const double *b, double *g)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) silu_gate_row(d, a + t * d, b + t * d, g + t * d);
+    return 0;
+}
+
+/* Gated FFN product -> randomised Hadamard -> quantise -> pack: the down_proj
+ * input path with the gate fused (the product is never rounded to the I/O
+ * type).  Same outputs as ora_rht_quant on x = SiLU(a) * b. */
+int ora_rht_quant_gate(int64_t T, int d, int m, int bits, const double *Hm, const double *a,
+                       const double *b, const int8_t *s, int8_t *q, uint8_t *codes, double *scales,
+                       double *pre)
+{
+    if ((bits != 3 && bits != 4) || (d * bits) % 8 || (bits == 3 && d % 8)) return -1;
+    if (m < 1 || d % m) return -1;
+    int n2 = d / m;
+    if (n2 & (n2 - 1)) return -1;
+    int err = 0;
+    int row_bytes = d * bits / 8;
+#pragma omp parallel
+    {
+        double *g = (double *)malloc(sizeof(double) * (size_t)d);
+        double *u = (double *)malloc(sizeof(double) * (size_t)d);
+        double *v = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!g || !u || !v) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                silu_gate_row(d, a + t * d, b + t * d, g);
+                rht_row(d, m, Hm, g, s, u, v);
+                scales[t] = quant_row(d, bits, v, q + t * d, pre ? pre + t * d : NULL);
+                if (bits == 4) pack_int4_row(d, q + t * d, codes + t * row_bytes);
+                else pack_int3_row(d, q + t * d, codes + t * row_bytes);
+            }
+        }
+        free(g);
         free(u);
         free(v);
     }

@@ -314,3 +314,62 @@ def test_inputs_are_deterministic_and_on_the_bf16_grid():
     u = a1.x.view(np.uint32)
     assert np.all(u & 0xFFFF == 0)
     np.testing.assert_allclose(a1.Q64.T @ a1.Q64, np.eye(32), atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# The gated down_proj input: SiLU(a) * b fused in front of the Hadamard
+# --------------------------------------------------------------------------
+
+def test_silu_gate_matches_the_logistic_function_of_the_library():
+    """g = a * sigmoid(a) * b against scipy's logistic sigmoid (an independent
+    library routine); closed forms: sigmoid(0) = 1/2, sigmoid(ln 3) = 3/4."""
+    import scipy.special
+    rng = np.random.default_rng(5)
+    a = rng.normal(0.0, 3.0, size=(7, 64))
+    b = rng.normal(0.0, 1.0, size=(7, 64))
+    np.testing.assert_allclose(oracle.silu_gate(a, b), a * scipy.special.expit(a) * b, rtol=1e-14, atol=1e-300)
+    a2 = np.array([[0.0, math.log(3.0), -math.log(3.0), 1.0]])
+    b2 = np.ones_like(a2)
+    np.testing.assert_allclose(oracle.silu_gate(a2, b2)[0],
+                               [0.0, 0.75 * math.log(3.0), -0.25 * math.log(3.0), 1.0 / (1.0 + math.exp(-1.0))],
+                               rtol=1e-15)
+
+
+def test_silu_gate_odd_part_and_limits():
+    """SiLU(a) - SiLU(-a) = a for every a (sigmoid(a) + sigmoid(-a) = 1); SiLU
+    tends to a for large a and to 0 for large negative a; b scales linearly."""
+    a = np.linspace(-30.0, 30.0, 241)[None, :]
+    one = np.ones_like(a)
+    np.testing.assert_allclose(oracle.silu_gate(a, one) - oracle.silu_gate(-a, one), a, rtol=1e-14, atol=1e-13)
+    big = np.array([[60.0, -60.0, 745.0, -745.0]])
+    g = oracle.silu_gate(big, np.ones_like(big))[0]
+    assert g[0] == 60.0 and abs(g[1]) < 1e-24 and g[2] == 745.0 and g[3] == 0.0
+    np.testing.assert_array_equal(oracle.silu_gate(a, 2.0 * one), 2.0 * oracle.silu_gate(a, one))
+
+
+def test_rht_quant_gate_is_the_rht_of_the_gated_product():
+    """The fused path equals the randomised Hadamard quantiser applied to the
+    gate values (no rounding in between); a zero up-projection row gives scale
+    0 and all codes 0."""
+    g = inputs.gate_case(5, 12 * 64, 12, 9, dtype="bf16", bits=4)
+    g.b[2] = 0.0
+    fused = oracle.rht_quant_gate(g.a, g.b, g.signs, 12, 4)
+    plain = oracle.rht_quant(oracle.silu_gate(g.a, g.b), g.signs, 12, 4)
+    np.testing.assert_array_equal(fused["codes"], plain["codes"])
+    np.testing.assert_array_equal(fused["scales"], plain["scales"])
+    assert fused["scales"][2] == 0.0 and np.all(fused["codes"][2] == 0)
+    h = inputs.gate_case(3, 256, 1, 4, dtype="f32", bits=3)
+    f3 = oracle.rht_quant_gate(h.a, h.b, h.signs, 1, 3)
+    p3 = oracle.rht_quant(oracle.silu_gate(h.a, h.b), h.signs, 1, 3)
+    np.testing.assert_array_equal(f3["codes"], p3["codes"])
+
+
+def test_gate_inputs_match_the_down_proj_activations():
+    """The two projections are the same seeded draws whose gated product the
+    unfused down_proj workload stores: a from the activation stream, b from the
+    gate stream of the same seed."""
+    a, b = inputs.gate_inputs(4, 12288, 2, dtype="f32")
+    ra = np.random.Generator(np.random.PCG64(np.random.SeedSequence([2, 0]))).standard_normal((4, 12288))
+    rb = np.random.Generator(np.random.PCG64(np.random.SeedSequence([2, 5]))).standard_normal((4, 12288))
+    np.testing.assert_array_equal(a, ra.astype(np.float32))
+    np.testing.assert_array_equal(b, rb.astype(np.float32))

@@ -143,6 +143,26 @@ class AlignCase:
 
 
 @dataclasses.dataclass
+class GateCase:
+    """Inputs of one gated down_proj problem: SiLU(a) * b -> randomised Hadamard -> codes."""
+    name: str
+    a: np.ndarray          # T x d float32 holding the exact I/O values (gate projection)
+    b: np.ndarray          # T x d float32 holding the exact I/O values (up projection)
+    signs: np.ndarray      # d int8 +-1
+    m: int
+    dtype: str
+    bits: int
+
+    @property
+    def T(self) -> int:
+        return self.a.shape[0]
+
+    @property
+    def d(self) -> int:
+        return self.a.shape[1]
+
+
+@dataclasses.dataclass
 class RhtCase:
     """Inputs of one randomised-Hadamard problem."""
     name: str
@@ -198,6 +218,30 @@ def llama7b_case(T: int = 2048):
     h = rht_case(T, 4096, 1, 1, dtype="bf16", bits=4, n_outliers=8, outlier_scale=100.0,
                  name=f"rht_T{T}_d4096")
     return a, h
+
+
+def gate_inputs(T: int, d: int, seed: int, dtype: str = "bf16"):
+    """The two FFN projections a (gate) and b (up), each N(0, 1), cast once to the
+    I/O type; the same draws as the "silu_gate" activations of that seed."""
+    rx = _rng(seed, _S_X)
+    rg = _rng(seed, _S_GATE)
+    a = np.empty((T, d), dtype=np.float32)
+    b = np.empty((T, d), dtype=np.float32)
+    for r0 in range(0, T, _CHUNK_ROWS):
+        n = min(_CHUNK_ROWS, T - r0)
+        a[r0:r0 + n] = _cast_io(rx.standard_normal((n, d)), dtype)
+        b[r0:r0 + n] = _cast_io(rg.standard_normal((n, d)), dtype)
+    return a, b
+
+
+def gate_case(T: int, d: int, m: int, seed: int, *, dtype: str = "bf16", bits: int = 4, name: str = "") -> GateCase:
+    a, b = gate_inputs(T, d, seed, dtype)
+    return GateCase(name or f"gate_T{T}_d{d}_m{m}", a, b, random_signs(d, seed), m, dtype, bits)
+
+
+def down_proj_gate_case(T: int = 4096) -> GateCase:
+    """FFN down_proj with the gate fused: a, b ~ N(0, 1) in bf16, d=12288=1024*12, INT4."""
+    return gate_case(T, 12288, 12, 2, dtype="bf16", bits=4, name=f"downproj_gate_T{T}_d12288")
 
 
 def down_proj_case(T: int = 4096):

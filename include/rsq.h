@@ -122,6 +122,23 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
 int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *scales,
               int64_t T, int d, int bits, int dtype, void *stream);
 
+/* The gated down_proj input fused in front of rht_quant: v = H_d diag(signs) g /
+ * sqrt(d) with g = SiLU(a) * b = a * b / (1 + exp(-a)), element by element, then
+ * the same per-token symmetric absmax quantisation and packing as rht_quant.
+ * Infra Quant II, QuaRot / Method (the online Hadamard on the down_proj input,
+ * the FFN's gated product of the gate projection a and the up projection b).
+ * a, b: T x d elements of `dtype`, row-major; g is formed in float32 and never
+ * rounded to `dtype` (so the result equals rht_quant of g, not of g rounded).
+ * Where exp(-a) overflows float32 (a below about -87) the factor SiLU(a)
+ * contributes 0 (its true magnitude is below 1e-35).
+ * a and b may overlap each other (both are only read); the outputs may not
+ * overlap anything (RSQ_ERR_ALIAS).  Shapes, m, bits, signs, codes, scales,
+ * stream and errors as for rht_quant.  Kernels: bf16, d = 12288, m = 12, INT4
+ * on the Kronecker kernel; every other supported shape on the radix-16
+ * kernel (rsq_select_rht_kernel: 0 automatic, 1 radix-16, 4 Kronecker only). */
+int rht_quant_silu_gate(const void *a, const void *b, const int8_t *signs, int m, uint8_t *codes,
+                        float *scales, int64_t T, int d, int bits, int dtype, void *stream);
+
 /* Human-readable name of an rsq_status value (static storage; never NULL). */
 const char *rsq_status_string(int status);
 

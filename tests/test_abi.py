@@ -24,7 +24,7 @@ OK, NULL, SHAPE, DTYPE, BITS, ALIGN, ALIAS, UNSUP, CUDA, VALUE = range(10)
 F32, BF16 = 0, 1
 
 # fake device addresses, far apart and 16-byte aligned
-X, Q, M, XO, C, S, SG = (0x10_0000_0000 + i * 0x1_0000_0000 for i in range(7))
+X, Q, M, XO, C, S, SG, XB = (0x10_0000_0000 + i * 0x1_0000_0000 for i in range(8))
 
 
 def declared_functions():
@@ -119,11 +119,41 @@ def test_rht_quant_rejects(kw, want):
     assert rsq.launch_count() == before
 
 
+def _gate(a=X, b=XB, sg=SG, m=12, c=C, s=S, T=4, d=12288, bits=4, dt=BF16):
+    return L.rht_quant_silu_gate(a, b, sg, m, c, s, T, d, bits, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(a=None), NULL), (dict(b=None), NULL), (dict(sg=None), NULL), (dict(c=None), NULL), (dict(s=None), NULL),
+    (dict(m=3), UNSUP), (dict(d=12 * 48), SHAPE), (dict(d=96, m=1), SHAPE), (dict(T=-1), SHAPE),
+    (dict(bits=2), BITS), (dict(dt=5), DTYPE),
+    (dict(a=X + 4), ALIGN), (dict(b=XB + 8), ALIGN), (dict(s=S + 2), ALIGN),
+    (dict(c=XB + 4096), ALIAS),          # codes inside b
+    (dict(s=X + 64), ALIAS),             # scales inside a
+    (dict(c=SG), ALIAS),                 # codes over the signs
+    (dict(s=C + 32), ALIAS),             # scales inside codes
+])
+def test_rht_quant_silu_gate_rejects(kw, want):
+    before = rsq.launch_count()
+    assert _gate(**kw) == want
+    assert rsq.launch_count() == before
+
+
+def test_rht_quant_silu_gate_inputs_may_overlap():
+    # a == b (SiLU(a) * a) passes validation; without a GPU the call then fails
+    # at the first CUDA call (nothing launched); never run on fake pointers on a GPU
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("would launch on fake pointers")
+    assert _gate(b=X) == CUDA
+
+
 def test_empty_batch_is_a_no_op():
     before = rsq.launch_count()
     assert _anq(x=None, xo=None, c=None, s=None, T=0) == OK
     assert _ra(x=None, xo=None, T=0) == OK
     assert _rht(x=None, c=None, s=None, T=0) == OK
+    assert _gate(a=None, b=None, c=None, s=None, T=0) == OK
     assert rsq.launch_count() == before
 
 

@@ -362,7 +362,7 @@ def test_generic_kernel_at_the_tensor_core_shapes(generic_align, T):
     check_align(a, label=f"generic w3a3 T={T}")
 
 
-@pytest.mark.parametrize("which", [2])
+@pytest.mark.parametrize("which", [2, 3])
 def test_tensor_core_kernel_serves_the_hot_shapes(which):
     rsq = _rsq()
     prev = rsq.select_align_kernel(which)
@@ -370,9 +370,8 @@ def test_tensor_core_kernel_serves_the_hot_shapes(which):
         for T in (1, 128, 129, 1000):
             a, _ = inputs.llama7b_case(T=T)
             check_align(a, label=f"tc hidden T={T}")
-        if which == 2:
-            a, _ = inputs.w3a3_case(T=257)
-            check_align(a, label="tc w3a3 T=257")
+        a, _ = inputs.w3a3_case(T=257)
+        check_align(a, label="tc w3a3 T=257")
         for r in (1, 7, 32):
             a = inputs.align_case(300, 4096, r, 40 + r, dtype="bf16", n_outliers=8, outlier_scale=100.0)
             check_align(a, label=f"tc r={r}")
@@ -496,6 +495,49 @@ def test_kronecker_12288_kernels(which):
         rsq.select_rht_kernel(prev)
 
 
+def check_gate(case, rows=None, label=""):
+    rsq = _rsq()
+    a = _to_dev(case.a, case.dtype)
+    b = _to_dev(case.b, case.dtype)
+    s = torch.from_numpy(case.signs).to(DEV)
+    codes, scales = rsq.rht_quant_silu_gate(a, b, s, case.m, bits=case.bits)
+    assert rsq.device_status() == 0
+    codes, scales = codes.cpu().numpy(), scales.cpu().numpy()
+    sel = slice(None) if rows is None else rows
+    ref = oracle.rht_quant_gate(case.a[sel], case.b[sel], case.signs, case.m, case.bits)
+    H.check_scales(scales[sel], ref["scales"], label)
+    return H.check_codes(codes[sel], ref["q"], ref["pre"], case.bits, label)
+
+
+@pytest.mark.parametrize("which", [0, 1, 4])
+def test_silu_gate_down_proj_12288(which):
+    """The gated down_proj input (SiLU(a) * b formed in fp32 in the kernel) at
+    d = 12288 = 1024 * 12: the Kronecker kernel (default) and the radix-16 one."""
+    rsq = _rsq()
+    prev = rsq.select_rht_kernel(which)
+    try:
+        for T in (1, 7, 300):
+            check_gate(inputs.down_proj_gate_case(T=T), label=f"gate kernel {which} T={T}")
+        g = inputs.down_proj_gate_case(T=6)
+        g.b[1] = 0.0                         # zero row
+        g.a[2] = np.float32(-30.0)           # strongly negative gate: a row of tiny values
+        g.a[3, :7] = np.float32(100.0)       # large gate: SiLU(a) -> a
+        check_gate(g, label=f"gate kernel {which} edge rows")
+    finally:
+        rsq.select_rht_kernel(prev)
+
+
+@pytest.mark.parametrize("d,m,dtype,bits", [(4096, 1, "bf16", 4), (8192, 1, "bf16", 3), (256, 1, "f32", 4),
+                                             (192, 12, "f32", 3), (16, 1, "bf16", 4)])
+def test_silu_gate_other_shapes(d, m, dtype, bits):
+    check_gate(inputs.gate_case(37, d, m, d + m + bits, dtype=dtype, bits=bits), label=f"gate d={d} m={m}")
+
+
+def test_silu_gate_full_down_proj_sampled():
+    g = inputs.down_proj_gate_case(T=4096)
+    check_gate(g, _sample(4096, 24), "gate T=4096")
+
+
 @pytest.mark.parametrize("d,which", [(4096, 1), (4096, 3), (8192, 3)])
 def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()
@@ -524,7 +566,7 @@ def test_residual_align_only_matches_oracle():
         H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, dtype, f"align {dtype}")
 
 
-@pytest.mark.parametrize("which", [0, 1, 2, 4])
+@pytest.mark.parametrize("which", [0, 1, 2, 3, 4])
 def test_residual_align_kernels(which):
     """rsq_residual_align through the decode kernel (small T), the tensor-core
     kernel (bf16, D = 4096 / 8192) and the CUDA-core kernel, each without the
@@ -536,6 +578,7 @@ def test_residual_align_kernels(which):
         shapes = {0: [(1, 4096), (16, 4096), (17, 4096), (1000, 4096), (300, 8192)],
                   1: [(16, 4096), (300, 4096)],
                   2: [(1, 4096), (200, 4096), (3001, 4096), (129, 8192)],
+                  3: [(1, 4096), (65, 4096), (200, 4096), (3001, 4096), (129, 8192)],
                   4: [(1, 4096), (16, 4096), (32, 2048), (31, 8192)]}[which]
         for T, D in shapes:
             a = inputs.align_case(T, D, 32, T + D, dtype="bf16", n_outliers=8, outlier_scale=100.0)

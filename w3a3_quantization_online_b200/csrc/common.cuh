@@ -63,6 +63,15 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8]) {
 }
 
 // ---------------------------------------------------------------------------
+// Gated FFN product SiLU(a) * b = a * sigmoid(a) * b in fp32 (the down_proj
+// input), sigmoid(a) = 1 / (1 + e^-a).  For a below about -88, e^-a overflows
+// to +inf and the reciprocal gives 0, the limit of the product.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float silu_gate(float a, float b) {
+    return (a * __frcp_rn(1.0f + __expf(-a))) * b;
+}
+
+// ---------------------------------------------------------------------------
 // Quantiser: code = clamp(round_half_even(v * inv), -qmax, qmax).
 // fmaf(v, inv, 1.5 * 2^23) rounds the exact product v*inv to the nearest
 // integer (ties to even) because the float grid has unit spacing there; the

@@ -38,6 +38,13 @@ cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void 
                             float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
                             bool *launched);
 
+// Tensor-core alignment + RMSNorm + quantiser with two 64-row tiles in flight
+// per CTA (bf16, D in {4096, 8192}, r <= 32); same contract as launch_align_tc.
+bool align_pipe_supports(int D, int r, int dtype, long long T);
+cudaError_t launch_align_pipe(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
+                              float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
+                              bool *launched);
+
 // Decode-size alignment + RMSNorm + quantiser: one cluster of 16 CTAs, FP32 FMAs
 // (T <= 32, 2048 <= D <= 8192, D % 128 == 0, r <= 32, bf16 or fp32 I/O).
 // Returns cudaErrorNotSupported if the cluster cannot be co-scheduled.
@@ -46,10 +53,15 @@ cudaError_t launch_align_decode(const void *x, const float *Q, const float *M, v
                                 float *scales, long long T, int D, int r, int bits, float eps, int dtype,
                                 cudaStream_t s);
 
+// The generic kernel with the input formed as SiLU(a) * b in fp32.
+cudaError_t launch_rht_gate_generic(const void *a, const void *b, const int8_t *signs, int m, uint8_t *codes,
+                                    float *scales, int64_t T, int d, int bits, int dtype, cudaStream_t s);
+
 // Randomised Hadamard H_1024 (x) H_12 of order 12288 (Paley H_12), bf16, INT4.
+// With b != nullptr the input is SiLU(x) * b (the gated down_proj input).
 bool rht_kron_supports(int d, int m, int dtype, int bits, long long T);
-cudaError_t launch_rht_kron(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
-                            cudaStream_t s);
+cudaError_t launch_rht_kron(const void *x, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
+                            long long T, cudaStream_t s);
 
 // Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
 // (m = 1, bf16, INT4/INT3).

@@ -5,6 +5,11 @@
 // or H_d = H_{2^n} (x) H_m for d = 2^n m with m = 12 (Paley type I, q = 11).
 // QuaRot / Method: per-token symmetric absmax quantisation.
 //
+// With GATE the input is the FFN's gated product SiLU(a) * b (QuaRot / Method:
+// the online Hadamard on the down_proj input), formed in fp32 from the two
+// projections a (x) and b as they are loaded; it is never rounded to the I/O
+// type.
+//
 // One CTA per token row; the row lives in shared memory as float32 and the
 // butterflies run in radix-16 register passes (4 stages per pass).  The
 // 1/sqrt(d) factor never touches the data: codes do not depend on a positive
@@ -28,9 +33,10 @@ __host__ __device__ constexpr int paley12_entry(int i, int j) {
 // padded shared-memory index (one float of padding per 16) against bank conflicts
 __device__ __forceinline__ int pidx(int i) { return i + (i >> 4); }
 
-template <class IO, int kM>
+template <class IO, int kM, bool GATE>
 __global__ void __launch_bounds__(kRhtThreads)
-k_rht_generic(const typename IO::T *__restrict__ x, const int8_t *__restrict__ signs,
+k_rht_generic(const typename IO::T *__restrict__ x, const typename IO::T *__restrict__ xb,
+              const int8_t *__restrict__ signs,
               uint8_t *__restrict__ codes, float *__restrict__ scales, int64_t T, int d,
               int logn, int bits) {
     extern __shared__ float4 smem4[];
@@ -45,10 +51,16 @@ k_rht_generic(const typename IO::T *__restrict__ x, const int8_t *__restrict__ s
 
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         const typename IO::T *xr = x + t * d;
-        // load, apply the random signs
+        // load (and gate), apply the random signs
         for (int e = tid; e < d / 8; e += blockDim.x) {
             float a[8];
             load8(xr + 8 * e, a);
+            if (GATE) {
+                float bv[8];
+                load8(xb + t * d + 8 * e, bv);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a[k] = silu_gate(a[k], bv[k]);
+            }
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[pidx(8 * e + k)] = signs[8 * e + k] < 0 ? -a[k] : a[k];
         }
@@ -125,22 +137,23 @@ k_rht_generic(const typename IO::T *__restrict__ x, const int8_t *__restrict__ s
     }
 }
 
-template <class IO, int kM>
-static cudaError_t launch_typed(const void *x, const int8_t *signs, uint8_t *codes, float *scales,
+template <class IO, int kM, bool GATE>
+static cudaError_t launch_typed(const void *x, const void *xb, const int8_t *signs, uint8_t *codes, float *scales,
                                 int64_t T, int d, int bits, cudaStream_t st) {
     const int n2 = d / kM;
     int logn = 0;
     while ((1 << logn) < n2) ++logn;
     const size_t smem = size_t(d + d / 16 + 16) * sizeof(float);
-    auto kern = k_rht_generic<IO, kM>;
+    auto kern = k_rht_generic<IO, kM, GATE>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
     }
     const int64_t cap = int64_t(num_sms()) * 8;
     const int grid = int(T < cap ? T : cap);
-    kern<<<grid, kRhtThreads, smem, st>>>(static_cast<const typename IO::T *>(x), signs, codes,
-                                          scales, T, d, logn, bits);
+    kern<<<grid, kRhtThreads, smem, st>>>(static_cast<const typename IO::T *>(x),
+                                          static_cast<const typename IO::T *>(xb), signs, codes, scales, T, d,
+                                          logn, bits);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
@@ -150,10 +163,19 @@ cudaError_t launch_rht_generic(const void *x, const int8_t *signs, int m, uint8_
                                float *scales, int64_t T, int d, int bits, int dtype,
                                cudaStream_t s) {
     if (dtype == 0)
-        return m == 12 ? launch_typed<F32, 12>(x, signs, codes, scales, T, d, bits, s)
-                       : launch_typed<F32, 1>(x, signs, codes, scales, T, d, bits, s);
-    return m == 12 ? launch_typed<BF16, 12>(x, signs, codes, scales, T, d, bits, s)
-                   : launch_typed<BF16, 1>(x, signs, codes, scales, T, d, bits, s);
+        return m == 12 ? launch_typed<F32, 12, false>(x, nullptr, signs, codes, scales, T, d, bits, s)
+                       : launch_typed<F32, 1, false>(x, nullptr, signs, codes, scales, T, d, bits, s);
+    return m == 12 ? launch_typed<BF16, 12, false>(x, nullptr, signs, codes, scales, T, d, bits, s)
+                   : launch_typed<BF16, 1, false>(x, nullptr, signs, codes, scales, T, d, bits, s);
+}
+
+cudaError_t launch_rht_gate_generic(const void *a, const void *b, const int8_t *signs, int m, uint8_t *codes,
+                                    float *scales, int64_t T, int d, int bits, int dtype, cudaStream_t s) {
+    if (dtype == 0)
+        return m == 12 ? launch_typed<F32, 12, true>(a, b, signs, codes, scales, T, d, bits, s)
+                       : launch_typed<F32, 1, true>(a, b, signs, codes, scales, T, d, bits, s);
+    return m == 12 ? launch_typed<BF16, 12, true>(a, b, signs, codes, scales, T, d, bits, s)
+                   : launch_typed<BF16, 1, true>(a, b, signs, codes, scales, T, d, bits, s);
 }
 
 }  // namespace rsq

@@ -21,6 +21,11 @@
 //      bank conflicts) so that thread (a0, h) owns a = a0 + 128 k (k < 8) and
 //      b = 6h..6h+5; FWHT bits 7-9 in the thread;
 //   4. block absmax, codes of 6 consecutive columns per (thread, k) = 3 bytes.
+// With GATE the input row is the gated FFN product SiLU(a) * b (QuaRot /
+// Method: the online Hadamard sits on the down_proj input), formed in fp32
+// from the two staged projection rows in step 1 and never rounded to bf16; the
+// signs are then applied to the fp32 sign bit (one bit per element, 48 per
+// thread).
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -82,15 +87,19 @@ __device__ __forceinline__ void h12_pair(const float2 (&u)[12], float2 (&out)[12
     }
 }
 
-template <int BITS>
+template <int BITS, bool GATE>
 __global__ void __launch_bounds__(kKThreads, 2)
-k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs, uint8_t *__restrict__ codes,
+k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ xb,
+           const int8_t *__restrict__ signs, uint8_t *__restrict__ codes,
            float *__restrict__ scales, long long T, int *status) {
     static_assert(BITS == 4, "6 codes of 4 bits make 3 whole bytes");
     extern __shared__ float4 km4[];
     float *buf = reinterpret_cast<float *>(km4);                    // 256 x 52 floats
-    uint4 *smask = reinterpret_cast<uint4 *>(buf + kKThreads * kKBlk);  // bf16 sign masks, 8 per uint4
-    uint4 *srow = smask + kKd / 8;                                  // the row being processed (bf16)
+    // without GATE: bf16 sign masks, 8 per uint4; with GATE: 48 sign bits per thread
+    uint4 *smask = reinterpret_cast<uint4 *>(buf + kKThreads * kKBlk);
+    uint64_t *sbits = reinterpret_cast<uint64_t *>(smask);
+    uint4 *srow = GATE ? smask + kKThreads / 2 : smask + kKd / 8;  // the row being processed (bf16)
+    uint4 *srow_b = srow + kKd / 8;                                 // GATE: the second projection row
     __shared__ float red[kKThreads / 32];
     __shared__ __align__(8) uint64_t bar_row;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -99,19 +108,26 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs
     constexpr int qmax = 7;
     constexpr int row_bytes = kKd / 2;
 
-    for (int i = tid; i < kKd / 8; i += kKThreads) {
-        uint32_t w[4];
+    if (GATE) {
+        uint64_t w = 0;  // bit e: sign of element 48 tid + e
+        for (int e = 0; e < 48; ++e) w |= uint64_t(signs[48 * tid + e] < 0) << e;
+        sbits[tid] = w;
+    } else {
+        for (int i = tid; i < kKd / 8; i += kKThreads) {
+            uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            w[e] = (signs[8 * i + 2 * e] < 0 ? 0x8000u : 0u) | (signs[8 * i + 2 * e + 1] < 0 ? 0x80000000u : 0u);
-        smask[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 4; ++e)
+                w[e] = (signs[8 * i + 2 * e] < 0 ? 0x8000u : 0u) | (signs[8 * i + 2 * e + 1] < 0 ? 0x80000000u : 0u);
+            smask[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
     if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
         if (blockIdx.x < T) {  // the first row (the next ones are staged while the previous is transformed)
-            mbar_expect_tx(bar, kKd * 2);
+            mbar_expect_tx(bar, GATE ? 2 * kKd * 2 : kKd * 2);
             if (!err) bulk_load_1d(smem_u32(srow), x + (long long)blockIdx.x * kKd, kKd * 2, bar);
+            if (GATE && !err) bulk_load_1d(smem_u32(srow_b), xb + (long long)blockIdx.x * kKd, kKd * 2, bar);
         }
     }
     __syncthreads();
@@ -124,7 +140,26 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs
         // ---- 1. 48 values (groups a = 4 tid + g) from the staged row, signs, H_12
         if (!mbar_wait(bar, uint32_t(it) & 1u, err != 0)) err |= kErrMbarTimeout;
         float2 p[2][12];  // p[h][k] = (group 2h, group 2h+1) entry k
-        {
+        if (GATE) {
+            const uint4 *src = srow + 6 * tid, *srcb = srow_b + 6 * tid;
+            const uint64_t sb = sbits[tid];
+#pragma unroll
+            for (int c = 0; c < 6; ++c) {
+                const uint4 u = src[c], ub = srcb[c];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int e = 8 * c + q, g = e / 12, k = e % 12;
+                    const float fa = __uint_as_float(q & 1 ? (w[q >> 1] & 0xFFFF0000u) : (w[q >> 1] << 16));
+                    const float fb = __uint_as_float(q & 1 ? (wb[q >> 1] & 0xFFFF0000u) : (wb[q >> 1] << 16));
+                    const float f = __uint_as_float(__float_as_uint(silu_gate(fa, fb)) ^
+                                                    (uint32_t((sb >> e) & 1u) << 31));
+                    if (g & 1) p[g >> 1][k].y = f;
+                    else p[g >> 1][k].x = f;
+                }
+            }
+            fence_proxy_async_cta();  // these reads before the next row's bulk copies
+        } else {
             const uint4 *src = srow + 6 * tid;
 #pragma unroll
             for (int c = 0; c < 6; ++c) {
@@ -191,8 +226,9 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const int8_t *__restrict__ signs
         }
         __syncthreads();  // the staged row is consumed: bring in the next one
         if (tid == 0 && t + gridDim.x < T) {
-            mbar_expect_tx(bar, kKd * 2);
+            mbar_expect_tx(bar, GATE ? 2 * kKd * 2 : kKd * 2);
             if (!err) bulk_load_1d(smem_u32(srow), x + (t + gridDim.x) * kKd, kKd * 2, bar);
+            if (GATE && !err) bulk_load_1d(smem_u32(srow_b), xb + (t + gridDim.x) * kKd, kKd * 2, bar);
         }
         // thread (a0, hb) now takes a = a0 + 128 k (k < 8), b = 6 hb .. 6 hb + 5
         float2 r[8][3];
@@ -263,24 +299,28 @@ bool rht_kron_supports(int d, int m, int dtype, int bits, long long T) {
     return d == kKd && m == 12 && dtype == 1 && bits == 4 && T >= 1 && T <= 0x7FFFFFFFLL;
 }
 
-cudaError_t launch_rht_kron(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
-                            cudaStream_t s) {
-    static bool configured[64];
+cudaError_t launch_rht_kron(const void *x, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
+                            long long T, cudaStream_t s) {
+    static bool configured[2][64];
+    const bool gate = b != nullptr;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const size_t smem = size_t(kKThreads) * kKBlk * 4 + size_t(kKd / 8) * 16 + size_t(kKd) * 2;
+    // transpose buffer; sign masks (bf16 masks, or 48 sign bits per thread); the staged row(s)
+    const size_t smem = size_t(kKThreads) * kKBlk * 4 + (gate ? size_t(kKThreads) * 8 : size_t(kKd / 8) * 16) +
+                        size_t(kKd) * 2 * (gate ? 2 : 1);
     int *status = device_status_word();
     if (!status) return cudaErrorInvalidValue;
-    if (dev >= 0 && dev < 64 && !configured[dev]) {
-        e = cudaFuncSetAttribute(k_rht_kron<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    auto kern = gate ? k_rht_kron<4, true> : k_rht_kron<4, false>;
+    if (dev >= 0 && dev < 64 && !configured[gate][dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        configured[dev] = true;
+        configured[gate][dev] = true;
     }
     const long long cap = (long long)num_sms() * 2;
     const int grid = int(T < cap ? T : cap);
-    k_rht_kron<4><<<grid, kKThreads, smem, s>>>(static_cast<const __nv_bfloat16 *>(x), signs, codes, scales, T,
-                                                 status);
+    kern<<<grid, kKThreads, smem, s>>>(static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(b),
+                                       signs, codes, scales, T, status);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;

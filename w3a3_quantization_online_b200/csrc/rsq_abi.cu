@@ -22,7 +22,7 @@ __device__ int g_status_taken;
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
-std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 4 decode
+std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 pipelined, 4 decode
 std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 3 tensor core, 4 Kronecker 12288
 thread_local int g_last_cuda_error = 0;
 
@@ -162,6 +162,12 @@ int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_ou
         const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, dtype, cs);
         if (e != cudaErrorNotSupported) return finish(e);
     }
+    if (which == 3 && rsq::align_pipe_supports(D, r, dtype, T)) {
+        bool launched = false;
+        const cudaError_t e = rsq::launch_align_pipe(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, cs, &launched);
+        if (e != cudaSuccess) return finish(e);
+        if (launched) return RSQ_OK;
+    }
     if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
         bool launched = false;
         const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, cs, &launched);
@@ -197,13 +203,19 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype, cs);
         if (e != cudaErrorNotSupported) return finish(e);  // not co-schedulable: another kernel serves it
     }
+    if (which == 3 && rsq::align_pipe_supports(D, r, dtype, T)) {
+        bool launched = false;
+        const cudaError_t e = rsq::launch_align_pipe(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, cs, &launched);
+        if (e != cudaSuccess) return finish(e);
+        if (launched) return RSQ_OK;
+    }
     if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
         bool launched = false;
         const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, cs, &launched);
         if (e != cudaSuccess) return finish(e);
         if (launched) return RSQ_OK;
     }
-    if (which == 2 || which == 4) return RSQ_ERR_UNSUPPORTED;
+    if (which == 2 || which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
                                             true, static_cast<cudaStream_t>(stream)));
 }
@@ -227,10 +239,37 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
     if ((which == 0 || which == 3) && rsq::rht_tc_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, d, bits, static_cast<cudaStream_t>(stream)));
     if ((which == 0 || which == 4) && rsq::rht_kron_supports(d, m, dtype, bits, T))
-        return finish(rsq::launch_rht_kron(x, signs, codes, scales, T, static_cast<cudaStream_t>(stream)));
+        return finish(rsq::launch_rht_kron(x, nullptr, signs, codes, scales, T, static_cast<cudaStream_t>(stream)));
     if (which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+int rht_quant_silu_gate(const void *a, const void *b, const int8_t *signs, int m, uint8_t *codes, float *scales,
+                        int64_t T, int d, int bits, int dtype, void *stream) {
+    if (bits != 3 && bits != 4) return RSQ_ERR_BITS;
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (m != 1 && m != 12) return RSQ_ERR_UNSUPPORTED;
+    if (T < 0 || d < 16 || d > 32768 || d % 16 != 0 || d % m != 0) return RSQ_ERR_SHAPE;
+    const int n2 = d / m;
+    if (!is_pow2(n2) || n2 < 16 || n2 > 16384) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!a || !b || !signs || !codes || !scales) return RSQ_ERR_NULL;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(signs) || !aligned16(codes) || !aligned16(scales))
+        return RSQ_ERR_ALIGN;
+    const uint64_t in_bytes = uint64_t(T) * d * elem_bytes(dtype);
+    const Span sa = span(a, in_bytes), sb = span(b, in_bytes), sg = span(signs, uint64_t(d));
+    const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * 4);
+    // the inputs may overlap each other (read only); no output may overlap anything
+    if (overlap(sc, sa) || overlap(sc, sb) || overlap(sc, sg) || overlap(sc, ss) || overlap(ss, sa) ||
+        overlap(ss, sb) || overlap(ss, sg))
+        return RSQ_ERR_ALIAS;
+    const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if ((which == 0 || which == 4) && rsq::rht_kron_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_kron(a, b, signs, codes, scales, T, cs));
+    if (which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
+    return finish(rsq::launch_rht_gate_generic(a, b, signs, m, codes, scales, T, d, bits, dtype, cs));
 }
 
 const char *rsq_status_string(int status) {
@@ -252,7 +291,7 @@ const char *rsq_status_string(int status) {
 int rsq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int rsq_select_align_kernel(int which) {
-    if (which < 0 || which > 4 || which == 3) return -1;
+    if (which < 0 || which > 4) return -1;
     return rsq::g_align_kernel.exchange(which);
 }
 

@@ -30,6 +30,8 @@ _lib.rsq_align_norm_quant.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, 
 _lib.rsq_align_norm_quant.restype = _i32
 _lib.rht_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.rht_quant.restype = _i32
+_lib.rht_quant_silu_gate.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.rht_quant_silu_gate.restype = _i32
 _lib.rsq_status_string.argtypes = [_i32]
 _lib.rsq_status_string.restype = ctypes.c_char_p
 _lib.rsq_last_cuda_error.argtypes = []
@@ -45,11 +47,11 @@ _lib.rsq_device_status.restype = _i32
 _lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
 _lib.rsq_selftest_wait_timeout.restype = _i32
 
-EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rsq_status_string",
+EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
 
-ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DECODE = 0, 1, 2, 4
+ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_PIPELINED, ALIGN_DECODE = 0, 1, 2, 3, 4
 RHT_AUTO, RHT_GENERIC, RHT_TENSOR_CORE, RHT_KRONECKER = 0, 1, 3, 4
 
 
@@ -71,7 +73,8 @@ def launch_count() -> int:
 
 
 def select_align_kernel(which: int) -> int:
-    """0 auto, 1 CUDA-core, 2 tensor-core cluster kernel, 4 decode kernel; returns the previous setting."""
+    """0 auto, 1 CUDA-core, 2 tensor-core cluster kernel (one 128-row tile per CTA), 3 pipelined
+    tensor-core cluster kernel (two 64-row tiles per CTA), 4 decode kernel; returns the previous setting."""
     prev = int(_lib.rsq_select_align_kernel(int(which)))
     if prev < 0:
         raise ValueError(which)
@@ -188,4 +191,24 @@ def rht_quant(x: torch.Tensor, signs: torch.Tensor, m: int = 1, codes: Optional[
     _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
     _check(_lib.rht_quant(_ptr(x), _ptr(signs), m, _ptr(codes), _ptr(scales), T, d, bits,
                           _dtype_code(x), _stream(stream)))
+    return codes, scales
+
+
+def rht_quant_silu_gate(a: torch.Tensor, b: torch.Tensor, signs: torch.Tensor, m: int = 1,
+                        codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None,
+                        bits: int = 4, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """SiLU(a) * b -> randomised Hadamard H_d diag(signs) / sqrt(d) -> per-token INT{bits} codes.
+
+    Returns (codes uint8 T x d*bits/8, scales float32 T)."""
+    _need(a, "a"); _need(b, "b", a.dtype); _need(signs, "signs", torch.int8)
+    T, d = a.shape
+    if tuple(b.shape) != (T, d):
+        raise ValueError(f"b has shape {tuple(b.shape)}, expected {(T, d)}")
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=a.device)
+    if scales is None:
+        scales = torch.empty((T,), dtype=torch.float32, device=a.device)
+    _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
+    _check(_lib.rht_quant_silu_gate(_ptr(a), _ptr(b), _ptr(signs), m, _ptr(codes), _ptr(scales), T, d, bits,
+                                    _dtype_code(a), _stream(stream)))
     return codes, scales

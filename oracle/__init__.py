@@ -47,6 +47,10 @@ def lib():
             L.ora_align_norm_quant.argtypes = [i64, i32, i32, i32, f64, _D, _D, _D, _D, _I8, _U8, _D, _D]
             L.ora_rht_quant.argtypes = [i64, i32, i32, i32, _D, _D, _I8, _I8, _U8, _D, _D]
             L.ora_silu_gate.argtypes = [i64, i32, _D, _D, _D]
+            L.ora_head_rht.argtypes = [i64, i32, i32, _D, _I8, _D]
+            L.ora_head_mix.argtypes = [i64, i32, i32, _D, _I8, _D]
+            L.ora_head_rht_quant.argtypes = [i64, i32, i32, i32, _D, _I8, _I8, _U8, _D, _D]
+            L.ora_head_mix_quant.argtypes = [i64, i32, i32, i32, _D, _I8, _I8, _U8, _D, _D]
             L.ora_rht_quant_gate.argtypes = [i64, i32, i32, i32, _D, _D, _D, _I8, _I8, _U8, _D, _D]
             _lib = L
     return _lib
@@ -209,4 +213,62 @@ def rht_quant_gate(a, b, signs, m: int, bits: int, want_pre: bool = True) -> dic
                                   _p(codes, _U8), _p(scales, _D), _p(pre, _D))
     if rc:
         raise ValueError(f"oracle rejected d={d}, m={m}, bits={bits} (rc={rc})")
+    return {"q": q, "codes": codes, "scales": scales, "pre": pre}
+
+
+def _signs_or_none(signs):
+    return None if signs is None else np.ascontiguousarray(signs, dtype=np.int8)
+
+
+def head_rht(x, signs, n_heads: int) -> np.ndarray:
+    """Per-head randomised Hadamard (I_{n_h} (x) H_{d_h}) diag(s) x / sqrt(d_h) (signs may be None)."""
+    x = _f64(x)
+    T, d = x.shape
+    s = _signs_or_none(signs)
+    v = np.empty_like(x)
+    if lib().ora_head_rht(T, d, n_heads, _p(x, _D), _p(s, _I8), _p(v, _D)):
+        raise ValueError(f"d={d}, n_heads={n_heads}")
+    return v
+
+
+def head_mix(x, signs, n_heads: int) -> np.ndarray:
+    """Head-mixing randomised Hadamard (H_{n_h} (x) I_{d_h}) diag(s) x / sqrt(n_h) (signs may be None)."""
+    x = _f64(x)
+    T, d = x.shape
+    s = _signs_or_none(signs)
+    v = np.empty_like(x)
+    if lib().ora_head_mix(T, d, n_heads, _p(x, _D), _p(s, _I8), _p(v, _D)):
+        raise ValueError(f"d={d}, n_heads={n_heads}")
+    return v
+
+
+def head_rht_quant(x, signs, n_heads: int, bits: int, want_pre: bool = True) -> dict:
+    """Per-head rotation -> symmetric quantisation per (token, head) -> pack; scales T x n_heads."""
+    x = _f64(x)
+    T, d = x.shape
+    s = _signs_or_none(signs)
+    q = np.empty((T, d), dtype=np.int8)
+    codes = np.empty((T, d * bits // 8), dtype=np.uint8)
+    scales = np.empty((T, n_heads), dtype=np.float64)
+    pre = np.empty_like(x) if want_pre else None
+    rc = lib().ora_head_rht_quant(T, d, n_heads, bits, _p(x, _D), _p(s, _I8), _p(q, _I8), _p(codes, _U8),
+                                  _p(scales, _D), _p(pre, _D))
+    if rc:
+        raise ValueError(f"oracle rejected d={d}, n_heads={n_heads}, bits={bits} (rc={rc})")
+    return {"q": q, "codes": codes, "scales": scales, "pre": pre}
+
+
+def head_mix_quant(x, signs, n_heads: int, bits: int, want_pre: bool = True) -> dict:
+    """Head mixing -> symmetric per-token quantisation -> pack."""
+    x = _f64(x)
+    T, d = x.shape
+    s = _signs_or_none(signs)
+    q = np.empty((T, d), dtype=np.int8)
+    codes = np.empty((T, d * bits // 8), dtype=np.uint8)
+    scales = np.empty(T, dtype=np.float64)
+    pre = np.empty_like(x) if want_pre else None
+    rc = lib().ora_head_mix_quant(T, d, n_heads, bits, _p(x, _D), _p(s, _I8), _p(q, _I8), _p(codes, _U8),
+                                  _p(scales, _D), _p(pre, _D))
+    if rc:
+        raise ValueError(f"oracle rejected d={d}, n_heads={n_heads}, bits={bits} (rc={rc})")
     return {"q": q, "codes": codes, "scales": scales, "pre": pre}

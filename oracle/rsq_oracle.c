@@ -27,7 +27,12 @@
  *          SpinQuant / Motivation (symmetric quantiser
  *          alpha = max|X| / (2^(N-1) - 1), X_Q = alpha * round(X / alpha)).
  *          QuaRot / Method also places an online Hadamard on the down_proj
- *          input, which is the FFN's gated product SiLU(gate) * up.
+ *          input, which is the FFN's gated product SiLU(gate) * up; and, in
+ *          attention, a per-head Hadamard on the queries and keys after the
+ *          position transform (post-RoPE key cache, quantised per head) and
+ *          the head-mixing product Z (H_{n_h} (x) I) on the attention output,
+ *          with (I (x) H_{d_h}) (H_{n_h} (x) I) = H_{n_h d_h} when n_h and
+ *          d_h are powers of two.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - rounding is to nearest, ties to even (rint in the default mode);
@@ -431,6 +436,119 @@ int ora_rht_quant_gate(int64_t T, int d, int m, int bits, const double *Hm, cons
         }
         free(g);
         free(u);
+        free(v);
+    }
+    return err;
+}
+
+
+/* [IQ2] QuaRot / Method, key rotation: the per-head Hadamard of the queries and
+ * keys, v = (I_{n_h} (x) H_{d_h}) diag(s) x / sqrt(d_h): head h occupies
+ * columns [h d_h, (h+1) d_h) and is transformed on its own.  s may be NULL
+ * (all +1). */
+static void head_rht_row(int d, int n_heads, const double *x, const int8_t *s, double *v)
+{
+    int dh = d / n_heads;
+    for (int i = 0; i < d; ++i) v[i] = (s ? (double)s[i] : 1.0) * x[i];
+    for (int h = 0; h < n_heads; ++h) ora_fwht(dh, 1, v + (int64_t)h * dh);
+    double c = 1.0 / sqrt((double)dh);
+    for (int i = 0; i < d; ++i) v[i] = v[i] * c;
+}
+
+/* [IQ2] QuaRot / Method, value projection: the online head-mixing product on
+ * the attention output, z <- z (H_{n_h} (x) I_{d_h}), here with random signs
+ * first: v[h d_h + j] = sum_h' H[h][h'] s[h' d_h + j] z[h' d_h + j] / sqrt(n_h)
+ * (H symmetric: the row-vector form of the pages is the same map).  s may be
+ * NULL (all +1). */
+static void head_mix_row(int d, int n_heads, const double *x, const int8_t *s, double *v)
+{
+    int dh = d / n_heads;
+    for (int i = 0; i < d; ++i) v[i] = (s ? (double)s[i] : 1.0) * x[i];
+    for (int j = 0; j < dh; ++j) ora_fwht(n_heads, dh, v + j);
+    double c = 1.0 / sqrt((double)n_heads);
+    for (int i = 0; i < d; ++i) v[i] = v[i] * c;
+}
+
+static int heads_ok(int d, int n_heads, int need_pow2_dh, int need_pow2_nh)
+{
+    if (n_heads < 1 || d % n_heads) return 0;
+    int dh = d / n_heads;
+    if (need_pow2_dh && (dh & (dh - 1))) return 0;
+    if (need_pow2_nh && (n_heads & (n_heads - 1))) return 0;
+    return 1;
+}
+
+int ora_head_rht(int64_t T, int d, int n_heads, const double *x, const int8_t *s, double *v)
+{
+    if (!heads_ok(d, n_heads, 1, 0)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) head_rht_row(d, n_heads, x + t * d, s, v + t * d);
+    return 0;
+}
+
+int ora_head_mix(int64_t T, int d, int n_heads, const double *x, const int8_t *s, double *v)
+{
+    if (!heads_ok(d, n_heads, 0, 1)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) head_mix_row(d, n_heads, x + t * d, s, v + t * d);
+    return 0;
+}
+
+/* Per-head rotation -> symmetric quantisation of each (token, head) group of
+ * d_h values (the key cache is quantised per head) -> pack.  scales: T x n_heads. */
+int ora_head_rht_quant(int64_t T, int d, int n_heads, int bits, const double *x, const int8_t *s,
+                       int8_t *q, uint8_t *codes, double *scales, double *pre)
+{
+    if ((bits != 3 && bits != 4) || !heads_ok(d, n_heads, 1, 0)) return -1;
+    int dh = d / n_heads;
+    if ((dh * bits) % 8 || (bits == 3 && dh % 8)) return -1;
+    int err = 0;
+    int row_bytes = d * bits / 8;
+#pragma omp parallel
+    {
+        double *v = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!v) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                head_rht_row(d, n_heads, x + t * d, s, v);
+                for (int h = 0; h < n_heads; ++h)
+                    scales[t * n_heads + h] = quant_row(dh, bits, v + (int64_t)h * dh, q + t * d + (int64_t)h * dh,
+                                                        pre ? pre + t * d + (int64_t)h * dh : NULL);
+                if (bits == 4) pack_int4_row(d, q + t * d, codes + t * row_bytes);
+                else pack_int3_row(d, q + t * d, codes + t * row_bytes);
+            }
+        }
+        free(v);
+    }
+    return err;
+}
+
+/* Head mixing -> per-token symmetric quantisation -> pack (the out_proj input). */
+int ora_head_mix_quant(int64_t T, int d, int n_heads, int bits, const double *x, const int8_t *s,
+                       int8_t *q, uint8_t *codes, double *scales, double *pre)
+{
+    if ((bits != 3 && bits != 4) || (d * bits) % 8 || (bits == 3 && d % 8)) return -1;
+    if (!heads_ok(d, n_heads, 0, 1)) return -1;
+    int err = 0;
+    int row_bytes = d * bits / 8;
+#pragma omp parallel
+    {
+        double *v = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!v) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                head_mix_row(d, n_heads, x + t * d, s, v);
+                scales[t] = quant_row(d, bits, v, q + t * d, pre ? pre + t * d : NULL);
+                if (bits == 4) pack_int4_row(d, q + t * d, codes + t * row_bytes);
+                else pack_int3_row(d, q + t * d, codes + t * row_bytes);
+            }
+        }
         free(v);
     }
     return err;

@@ -373,3 +373,89 @@ def test_gate_inputs_match_the_down_proj_activations():
     rb = np.random.Generator(np.random.PCG64(np.random.SeedSequence([2, 5]))).standard_normal((4, 12288))
     np.testing.assert_array_equal(a, ra.astype(np.float32))
     np.testing.assert_array_equal(b, rb.astype(np.float32))
+
+
+# --------------------------------------------------------------------------
+# Attention: per-head Hadamard of queries and keys, head mixing of the output
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n_heads,dh", [(1, 16), (4, 8), (3, 32), (8, 4)])
+def test_head_rht_equals_the_dense_block_diagonal_map(n_heads, dh):
+    """(I_{n_h} (x) H_{d_h}) diag(s) / sqrt(d_h) built densely from the library
+    Hadamard matrix and np.kron."""
+    rng = np.random.default_rng(n_heads * 100 + dh)
+    d = n_heads * dh
+    x = rng.normal(size=(5, d))
+    s = np.where(rng.integers(0, 2, size=d) == 1, 1, -1).astype(np.int8)
+    dense = np.kron(np.eye(n_heads), scipy.linalg.hadamard(dh)) @ np.diag(s.astype(np.float64)) / math.sqrt(dh)
+    np.testing.assert_allclose(oracle.head_rht(x, s, n_heads), x @ dense.T, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(oracle.head_rht(x, None, n_heads), oracle.head_rht(x, np.ones(d, np.int8), n_heads),
+                               rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("n_heads,dh", [(2, 3), (4, 8), (8, 5), (16, 2)])
+def test_head_mix_equals_the_dense_kronecker_map(n_heads, dh):
+    """(H_{n_h} (x) I_{d_h}) diag(s) / sqrt(n_h) built densely; d_h need not be a
+    power of two (it is only the stride)."""
+    rng = np.random.default_rng(n_heads * 10 + dh)
+    d = n_heads * dh
+    x = rng.normal(size=(4, d))
+    s = np.where(rng.integers(0, 2, size=d) == 1, 1, -1).astype(np.int8)
+    dense = np.kron(scipy.linalg.hadamard(n_heads), np.eye(dh)) @ np.diag(s.astype(np.float64)) / math.sqrt(n_heads)
+    np.testing.assert_allclose(oracle.head_mix(x, s, n_heads), x @ dense.T, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("n_heads,dh", [(4, 16), (32, 128), (8, 64)])
+def test_head_mix_after_per_head_rotation_is_the_full_hadamard(n_heads, dh):
+    """The identity the pages state for powers of two: (H_{n_h} (x) I)(I (x) H_{d_h})
+    = H_{n_h d_h}, so mixing the heads of per-head-rotated activations equals
+    the full Sylvester transform of order n_h d_h (normalised)."""
+    rng = np.random.default_rng(dh)
+    d = n_heads * dh
+    x = rng.normal(size=(3, d))
+    both = oracle.head_mix(oracle.head_rht(x, None, n_heads), None, n_heads)
+    np.testing.assert_allclose(both, oracle.rht(x, np.ones(d, np.int8), 1), rtol=1e-11, atol=1e-11)
+
+
+def test_per_head_rotation_keeps_the_attention_scores():
+    """Rotating queries and keys with the same per-head Hadamard leaves every
+    per-head dot product q_h . k_h unchanged (the pages: the scores P_1..P_{n_h}
+    do not change), and every head keeps its norm."""
+    rng = np.random.default_rng(3)
+    n_heads, dh = 8, 64
+    q = rng.normal(size=(6, n_heads * dh))
+    k = rng.normal(size=(9, n_heads * dh))
+    s = np.where(rng.integers(0, 2, size=n_heads * dh) == 1, 1, -1).astype(np.int8)
+    qr, kr = oracle.head_rht(q, s, n_heads), oracle.head_rht(k, s, n_heads)
+    for h in range(n_heads):
+        sl = slice(h * dh, (h + 1) * dh)
+        np.testing.assert_allclose(qr[:, sl] @ kr[:, sl].T, q[:, sl] @ k[:, sl].T, rtol=1e-12, atol=1e-11)
+        np.testing.assert_allclose(np.linalg.norm(kr[:, sl], axis=1), np.linalg.norm(k[:, sl], axis=1), rtol=1e-13)
+
+
+def test_head_rht_quant_is_per_head():
+    """Each (token, head) group has its own step max|v_head| / qmax; a head of
+    zeros gets scale 0 and zero codes while the other heads of the row do not;
+    the worked example (20, 0, 0, 0) -> (10, 10, 10, 10), step 10/7, codes 7."""
+    x = np.zeros((1, 3 * 4))
+    x[0, 4] = 20.0                       # head 1: the worked example
+    x[0, 8:12] = [1.0, -2.0, 3.0, 0.5]   # head 2: something else; head 0 stays zero
+    r = oracle.head_rht_quant(x, None, 3, 4)
+    np.testing.assert_array_equal(r["q"][0, 0:4], 0)
+    assert r["scales"][0, 0] == 0.0
+    np.testing.assert_array_equal(r["q"][0, 4:8], [7, 7, 7, 7])
+    assert r["scales"][0, 1] == pytest.approx(10.0 / 7.0, rel=1e-15)
+    v2 = oracle.head_rht(x, None, 3)[0, 8:12]
+    assert r["scales"][0, 2] == pytest.approx(np.abs(v2).max() / 7.0, rel=1e-15)
+    q, a, _ = oracle.quant_sym(v2[None, :], 4)
+    np.testing.assert_array_equal(r["q"][0, 8:12], q[0])
+
+
+def test_head_mix_quant_is_the_composition_of_its_steps():
+    g = inputs.rht_case(5, 32 * 24, 1, 13, dtype="bf16", bits=3, n_outliers=4, outlier_scale=30.0)
+    r = oracle.head_mix_quant(g.x, g.signs, 32, 3)
+    v = oracle.head_mix(g.x, g.signs, 32)
+    q, a, pre = oracle.quant_sym(v, 3)
+    np.testing.assert_array_equal(r["q"], q)
+    np.testing.assert_array_equal(r["scales"], a)
+    np.testing.assert_array_equal(r["codes"], oracle.pack(q, 3))

@@ -139,6 +139,39 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
 int rht_quant_silu_gate(const void *a, const void *b, const int8_t *signs, int m, uint8_t *codes,
                         float *scales, int64_t T, int d, int bits, int dtype, void *stream);
 
+/* Attention-side online Hadamards.  Infra Quant II, QuaRot / Method (key
+ * rotation; value projection).  x: T x d elements of `dtype`, row-major, with
+ * head h in columns [h d_h, (h+1) d_h), d = n_heads * d_h.  signs: d int8 +-1,
+ * or NULL for the plain (unrandomised) Hadamard.  Streams, errors, alignment
+ * as above. */
+
+/* Per-head rotation of queries (and keys) after the position transform:
+ * x_out = (I_{n_heads} (x) H_{d_h}) diag(signs) x / sqrt(d_h), rounded to
+ * `dtype`.  d_h = d / n_heads must be a power of two in [16, 256]
+ * (RSQ_ERR_SHAPE otherwise).  x_out may equal x; any other overlap with x or
+ * signs is RSQ_ERR_ALIAS.  Rotating queries and keys with the same signs
+ * leaves every per-head dot product q_h . k_h unchanged. */
+int rht_heads(const void *x, const int8_t *signs, int n_heads, void *x_out, int64_t T, int d, int dtype,
+              void *stream);
+
+/* Per-head rotation as rht_heads, then symmetric absmax quantisation of each
+ * (token, head) group of d_h values (the post-RoPE key cache, quantised per
+ * head): scales[t * n_heads + h] = max_i |v_{t,h,i}| / qmax with v the
+ * normalised rotated values; codes: T rows of d * bits / 8 bytes, packed as
+ * for rht_quant along the row (head h in its own whole bytes). */
+int rht_heads_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales,
+                    int64_t T, int d, int bits, int dtype, void *stream);
+
+/* Head mixing of the attention output (the out_proj input):
+ * v = (H_{n_heads} (x) I_{d_h}) diag(signs) x / sqrt(n_heads), i.e. the
+ * n_heads-point transform along the head index at stride d_h, then per-token
+ * symmetric absmax quantisation and packing as for rht_quant
+ * (scales[t] = max_i |v_ti| / qmax).  n_heads a power of two in [2, 64];
+ * d % 16 == 0; d_h = d / n_heads (any, it is the stride) with
+ * d_h <= 512 (n_heads <= 16) or d_h <= 256 (n_heads >= 32). */
+int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales,
+                       int64_t T, int d, int bits, int dtype, void *stream);
+
 /* Human-readable name of an rsq_status value (static storage; never NULL). */
 const char *rsq_status_string(int status);
 

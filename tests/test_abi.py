@@ -148,12 +148,55 @@ def test_rht_quant_silu_gate_inputs_may_overlap():
     assert _gate(b=X) == CUDA
 
 
+def _heads(x=X, sg=SG, nh=32, xo=XO, T=4, d=4096, dt=BF16):
+    return L.rht_heads(x, sg, nh, xo, T, d, dt, None)
+
+
+def _heads_q(x=X, sg=SG, nh=32, c=C, s=S, T=4, d=4096, bits=4, dt=BF16):
+    return L.rht_heads_quant(x, sg, nh, c, s, T, d, bits, dt, None)
+
+
+def _mix_q(x=X, sg=SG, nh=32, c=C, s=S, T=4, d=4096, bits=4, dt=BF16):
+    return L.rht_head_mix_quant(x, sg, nh, c, s, T, d, bits, dt, None)
+
+
+@pytest.mark.parametrize("fn,kw,want", [
+    (_heads, dict(x=None), NULL), (_heads, dict(xo=None), NULL), (_heads, dict(nh=0), SHAPE),
+    (_heads, dict(nh=3), SHAPE),                      # d_h = 4096 / 3 is not whole
+    (_heads, dict(nh=512), SHAPE),                    # d_h = 8 < 16
+    (_heads, dict(nh=8), SHAPE),                      # d_h = 512 > 256
+    (_heads, dict(d=96 * 32), SHAPE),                 # d_h = 96 is not a power of two
+    (_heads, dict(dt=4), DTYPE), (_heads, dict(x=X + 2), ALIGN), (_heads, dict(sg=SG + 8), ALIGN),
+    (_heads, dict(xo=X + 16), ALIAS), (_heads, dict(xo=SG - 64), ALIAS),
+    (_heads_q, dict(c=None), NULL), (_heads_q, dict(s=None), NULL), (_heads_q, dict(bits=5), BITS),
+    (_heads_q, dict(nh=64, d=4096 + 64), SHAPE), (_heads_q, dict(c=X + 512), ALIAS), (_heads_q, dict(s=C + 16), ALIAS),
+    (_mix_q, dict(nh=3, d=48 * 3), SHAPE), (_mix_q, dict(nh=1), SHAPE), (_mix_q, dict(nh=128), SHAPE),
+    (_mix_q, dict(nh=2, d=2 * 1024), SHAPE),          # d_h = 1024: more columns than threads per row
+    (_mix_q, dict(d=4096 + 8), SHAPE), (_mix_q, dict(bits=1), BITS), (_mix_q, dict(c=C + 4), ALIGN),
+    (_mix_q, dict(s=X + 32), ALIAS), (_mix_q, dict(c=SG), ALIAS),
+])
+def test_head_transforms_reject(fn, kw, want):
+    before = rsq.launch_count()
+    assert fn(**kw) == want
+    assert rsq.launch_count() == before
+
+
+def test_head_transforms_accept_null_signs():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("would launch on fake pointers")
+    assert _heads(sg=None) == CUDA and _heads_q(sg=None) == CUDA and _mix_q(sg=None) == CUDA
+
+
 def test_empty_batch_is_a_no_op():
     before = rsq.launch_count()
     assert _anq(x=None, xo=None, c=None, s=None, T=0) == OK
     assert _ra(x=None, xo=None, T=0) == OK
     assert _rht(x=None, c=None, s=None, T=0) == OK
     assert _gate(a=None, b=None, c=None, s=None, T=0) == OK
+    assert _heads(x=None, xo=None, T=0) == OK
+    assert _heads_q(x=None, c=None, s=None, T=0) == OK
+    assert _mix_q(x=None, c=None, s=None, T=0) == OK
     assert rsq.launch_count() == before
 
 

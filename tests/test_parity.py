@@ -538,6 +538,105 @@ def test_silu_gate_full_down_proj_sampled():
     check_gate(g, _sample(4096, 24), "gate T=4096")
 
 
+def _signs_dev(case, use):
+    return torch.from_numpy(case.signs).to(DEV) if use else None
+
+
+@pytest.mark.parametrize("n_heads,d_head", [(32, 128), (1, 16), (7, 64), (3, 256), (64, 32)])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_heads_rotation(n_heads, d_head, dtype):
+    """Per-head rotation of queries / keys against the oracle (rotated values:
+    the same tolerance as aligned values), with and without signs, and in place."""
+    rsq = _rsq()
+    c = inputs.rht_case(33, n_heads * d_head, 1, n_heads + d_head, dtype=dtype, n_outliers=3, outlier_scale=20.0)
+    for use_signs in (True, False):
+        x = _to_dev(c.x, dtype)
+        out = rsq.rht_heads(x, _signs_dev(c, use_signs), n_heads)
+        torch.cuda.synchronize()
+        ref = oracle.head_rht(c.x, c.signs if use_signs else None, n_heads)
+        H.check_aligned(_host(out), ref, c.x, dtype, f"heads {n_heads}x{d_head} {dtype} signs={use_signs}")
+        rsq.rht_heads(x, _signs_dev(c, use_signs), n_heads, x_out=x)  # in place
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(_host(x), _host(out))
+    assert rsq.device_status() == 0
+
+
+def test_heads_rotation_keeps_the_scores():
+    """Queries and keys rotated on the GPU (fp32 I/O) with the same signs give
+    the same per-head dot products as the unrotated ones."""
+    rsq = _rsq()
+    n_heads, d_head = 32, 128
+    q = inputs.rht_case(16, n_heads * d_head, 1, 61, dtype="f32", n_outliers=4, outlier_scale=20.0)
+    k = inputs.rht_case(40, n_heads * d_head, 1, 62, dtype="f32", n_outliers=4, outlier_scale=20.0)
+    s = torch.from_numpy(q.signs).to(DEV)
+    qr = _host(rsq.rht_heads(_to_dev(q.x, "f32"), s, n_heads)).astype(np.float64)
+    kr = _host(rsq.rht_heads(_to_dev(k.x, "f32"), s, n_heads)).astype(np.float64)
+    for h in range(n_heads):
+        sl = slice(h * d_head, (h + 1) * d_head)
+        ref = q.x[:, sl].astype(np.float64) @ k.x[:, sl].astype(np.float64).T
+        np.testing.assert_allclose(qr[:, sl] @ kr[:, sl].T, ref, rtol=1e-5, atol=1e-4 * np.abs(ref).max())
+
+
+def check_heads_quant(case, n_heads, use_signs=True, rows=None, label=""):
+    rsq = _rsq()
+    codes, scales = rsq.rht_heads_quant(_to_dev(case.x, case.dtype), _signs_dev(case, use_signs), n_heads,
+                                        bits=case.bits)
+    assert rsq.device_status() == 0
+    sel = slice(None) if rows is None else rows
+    ref = oracle.head_rht_quant(case.x[sel], case.signs if use_signs else None, n_heads, case.bits)
+    H.check_scales(scales.cpu().numpy()[sel].ravel(), ref["scales"].ravel(), label)
+    return H.check_codes(codes.cpu().numpy()[sel], ref["q"], ref["pre"], case.bits, label)
+
+
+def check_head_mix(case, n_heads, use_signs=True, rows=None, label=""):
+    rsq = _rsq()
+    codes, scales = rsq.rht_head_mix_quant(_to_dev(case.x, case.dtype), _signs_dev(case, use_signs), n_heads,
+                                           bits=case.bits)
+    assert rsq.device_status() == 0
+    sel = slice(None) if rows is None else rows
+    ref = oracle.head_mix_quant(case.x[sel], case.signs if use_signs else None, n_heads, case.bits)
+    H.check_scales(scales.cpu().numpy()[sel], ref["scales"], label)
+    return H.check_codes(codes.cpu().numpy()[sel], ref["q"], ref["pre"], case.bits, label)
+
+
+@pytest.mark.parametrize("n_heads,d_head,dtype,bits", [(32, 128, "bf16", 4), (32, 128, "bf16", 3), (5, 16, "f32", 4),
+                                                       (8, 256, "f32", 3), (64, 64, "bf16", 4)])
+def test_heads_quant_per_head(n_heads, d_head, dtype, bits):
+    c = inputs.rht_case(29, n_heads * d_head, 1, 7 + d_head, dtype=dtype, bits=bits, n_outliers=3,
+                        outlier_scale=20.0)
+    c.x[4] = 0.0                               # a zero row: every head scale 0
+    c.x[5, :d_head] = 0.0                      # a zero head in an otherwise nonzero row
+    check_heads_quant(c, n_heads, True, label=f"heads quant {n_heads}x{d_head}")
+    check_heads_quant(c, n_heads, False, label=f"heads quant {n_heads}x{d_head} no signs")
+
+
+@pytest.mark.parametrize("n_heads,d_head,dtype,bits", [(32, 128, "bf16", 4), (32, 128, "f32", 3), (2, 8, "bf16", 4),
+                                                       (4, 96, "bf16", 3), (16, 512, "f32", 4), (64, 64, "bf16", 4),
+                                                       (64, 256, "bf16", 3)])
+def test_head_mix_quant(n_heads, d_head, dtype, bits):
+    c = inputs.rht_case(23, n_heads * d_head, 1, 3 + n_heads, dtype=dtype, bits=bits, n_outliers=3,
+                        outlier_scale=20.0)
+    c.x[2] = 0.0
+    check_head_mix(c, n_heads, True, label=f"head mix {n_heads}x{d_head}")
+    check_head_mix(c, n_heads, False, label=f"head mix {n_heads}x{d_head} no signs")
+
+
+def test_attention_transforms_full_size_sampled():
+    """T = 16384 tokens of 32 x 128 attention activations: per-head rotation,
+    per-head key quantisation and head mixing with per-token quantisation, in
+    the bench's launch configuration, sampled rows against the oracle."""
+    rsq = _rsq()
+    c = inputs.attention_case(T=16384)
+    rows = _sample(16384, 32, seed=7)
+    x = _to_dev(c.x, "bf16")
+    s = torch.from_numpy(c.signs).to(DEV)
+    out = rsq.rht_heads(x, s, 32)
+    torch.cuda.synchronize()
+    H.check_aligned(_host(out)[rows], oracle.head_rht(c.x[rows], c.signs, 32), c.x[rows], "bf16", "heads T=16384")
+    check_heads_quant(c, 32, True, rows, "heads quant T=16384")
+    check_head_mix(c, 32, True, rows, "head mix T=16384")
+
+
 @pytest.mark.parametrize("d,which", [(4096, 1), (4096, 3), (8192, 3)])
 def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()

@@ -63,6 +63,16 @@ bool rht_kron_supports(int d, int m, int dtype, int bits, long long T);
 cudaError_t launch_rht_kron(const void *x, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
                             long long T, cudaStream_t s);
 
+// Attention: per-head randomised Hadamard (I (x) H_dh), rotation only (x_out)
+// or with per-(token, head) quantisation (quant), and head mixing (H_nh (x) I)
+// with per-token quantisation.  signs may be nullptr (all +1).
+bool head_rht_supports(int d, int n_heads);
+bool head_mix_supports(int d, int n_heads);
+cudaError_t launch_head_rht(const void *x, const int8_t *signs, void *x_out, uint8_t *codes, float *scales,
+                            long long T, int d, int n_heads, int bits, bool quant, int dtype, cudaStream_t s);
+cudaError_t launch_head_mix(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
+                            int n_heads, int bits, int dtype, cudaStream_t s);
+
 // Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
 // (m = 1, bf16, INT4/INT3).
 bool rht_tc_supports(int d, int m, int dtype, int bits, long long T);

@@ -272,6 +272,61 @@ int rht_quant_silu_gate(const void *a, const void *b, const int8_t *signs, int m
     return finish(rsq::launch_rht_gate_generic(a, b, signs, m, codes, scales, T, d, bits, dtype, cs));
 }
 
+int rht_heads(const void *x, const int8_t *signs, int n_heads, void *x_out, int64_t T, int d, int dtype,
+              void *stream) {
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (T < 0 || d < 16 || d > 32768 || !rsq::head_rht_supports(d, n_heads)) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!x || !x_out) return RSQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(x_out) || (signs && !aligned16(signs))) return RSQ_ERR_ALIGN;
+    const uint64_t bytes = uint64_t(T) * d * elem_bytes(dtype);
+    const Span sx = span(x, bytes), so = span(x_out, bytes);
+    if (x != x_out && overlap(sx, so)) return RSQ_ERR_ALIAS;
+    if (signs && overlap(so, span(signs, uint64_t(d)))) return RSQ_ERR_ALIAS;
+    return finish(rsq::launch_head_rht(x, signs, x_out, nullptr, nullptr, T, d, n_heads, 4, false, dtype,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int rht_heads_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales, int64_t T,
+                    int d, int bits, int dtype, void *stream) {
+    if (bits != 3 && bits != 4) return RSQ_ERR_BITS;
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (T < 0 || d < 16 || d > 32768 || !rsq::head_rht_supports(d, n_heads)) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!x || !codes || !scales) return RSQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (signs && !aligned16(signs)))
+        return RSQ_ERR_ALIGN;
+    const Span sx = span(x, uint64_t(T) * d * elem_bytes(dtype));
+    const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * n_heads * 4);
+    if (overlap(sc, sx) || overlap(ss, sx) || overlap(sc, ss)) return RSQ_ERR_ALIAS;
+    if (signs) {
+        const Span sg = span(signs, uint64_t(d));
+        if (overlap(sc, sg) || overlap(ss, sg)) return RSQ_ERR_ALIAS;
+    }
+    return finish(rsq::launch_head_rht(x, signs, nullptr, codes, scales, T, d, n_heads, bits, true, dtype,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales, int64_t T,
+                       int d, int bits, int dtype, void *stream) {
+    if (bits != 3 && bits != 4) return RSQ_ERR_BITS;
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (T < 0 || d < 16 || d > 32768 || d % 16 != 0 || !rsq::head_mix_supports(d, n_heads)) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!x || !codes || !scales) return RSQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || (signs && !aligned16(signs)))
+        return RSQ_ERR_ALIGN;
+    const Span sx = span(x, uint64_t(T) * d * elem_bytes(dtype));
+    const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * 4);
+    if (overlap(sc, sx) || overlap(ss, sx) || overlap(sc, ss)) return RSQ_ERR_ALIAS;
+    if (signs) {
+        const Span sg = span(signs, uint64_t(d));
+        if (overlap(sc, sg) || overlap(ss, sg)) return RSQ_ERR_ALIAS;
+    }
+    return finish(rsq::launch_head_mix(x, signs, codes, scales, T, d, n_heads, bits, dtype,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 const char *rsq_status_string(int status) {
     switch (status) {
         case RSQ_OK: return "RSQ_OK";

@@ -239,6 +239,16 @@ def gate_case(T: int, d: int, m: int, seed: int, *, dtype: str = "bf16", bits: i
     return GateCase(name or f"gate_T{T}_d{d}_m{m}", a, b, random_signs(d, seed), m, dtype, bits)
 
 
+def attention_case(T: int = 16384, n_heads: int = 32, d_head: int = 128, seed: int = 5, *, dtype: str = "bf16",
+                   bits: int = 4) -> RhtCase:
+    """Attention activations (queries / keys after the position transform, or the
+    attention output), Llama-7B-like: n_heads x d_head = 32 x 128 columns, N(0, 1)
+    with 8 outlier channels x20 (a key cache has a few large channels), random
+    signs; INT4 per head / per token."""
+    return rht_case(T, n_heads * d_head, 1, seed, dtype=dtype, bits=bits, n_outliers=8, outlier_scale=20.0,
+                    name=f"attn_T{T}_h{n_heads}x{d_head}")
+
+
 def down_proj_gate_case(T: int = 4096) -> GateCase:
     """FFN down_proj with the gate fused: a, b ~ N(0, 1) in bf16, d=12288=1024*12, INT4."""
     return gate_case(T, 12288, 12, 2, dtype="bf16", bits=4, name=f"downproj_gate_T{T}_d12288")

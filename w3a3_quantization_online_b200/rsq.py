@@ -32,6 +32,12 @@ _lib.rht_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp
 _lib.rht_quant.restype = _i32
 _lib.rht_quant_silu_gate.argtypes = [_vp, _vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.rht_quant_silu_gate.restype = _i32
+_lib.rht_heads.argtypes = [_vp, _vp, _i32, _vp, _i64, _i32, _i32, _vp]
+_lib.rht_heads.restype = _i32
+_lib.rht_heads_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.rht_heads_quant.restype = _i32
+_lib.rht_head_mix_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.rht_head_mix_quant.restype = _i32
 _lib.rsq_status_string.argtypes = [_i32]
 _lib.rsq_status_string.restype = ctypes.c_char_p
 _lib.rsq_last_cuda_error.argtypes = []
@@ -47,7 +53,8 @@ _lib.rsq_device_status.restype = _i32
 _lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
 _lib.rsq_selftest_wait_timeout.restype = _i32
 
-EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rsq_status_string",
+EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rht_heads",
+            "rht_heads_quant", "rht_head_mix_quant", "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
 
@@ -211,4 +218,55 @@ def rht_quant_silu_gate(a: torch.Tensor, b: torch.Tensor, signs: torch.Tensor, m
     _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
     _check(_lib.rht_quant_silu_gate(_ptr(a), _ptr(b), _ptr(signs), m, _ptr(codes), _ptr(scales), T, d, bits,
                                     _dtype_code(a), _stream(stream)))
+    return codes, scales
+
+
+def _signs_ptr(signs: Optional[torch.Tensor]) -> Optional[int]:
+    if signs is None:
+        return None
+    _need(signs, "signs", torch.int8)
+    return signs.data_ptr()
+
+
+def rht_heads(x: torch.Tensor, signs: Optional[torch.Tensor], n_heads: int,
+              x_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per-head rotation (I (x) H_{d_h}) diag(signs) x / sqrt(d_h) of queries or keys (in place if x_out is x)."""
+    _need(x, "x")
+    T, d = x.shape
+    if x_out is None:
+        x_out = torch.empty_like(x)
+    _need(x_out, "x_out", x.dtype)
+    _check(_lib.rht_heads(_ptr(x), _signs_ptr(signs), n_heads, _ptr(x_out), T, d, _dtype_code(x), _stream(stream)))
+    return x_out
+
+
+def rht_heads_quant(x: torch.Tensor, signs: Optional[torch.Tensor], n_heads: int, codes: Optional[torch.Tensor] = None,
+                    scales: Optional[torch.Tensor] = None, bits: int = 4,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-head rotation, then per-(token, head) INT{bits} codes.  Returns (codes T x d*bits/8, scales T x n_heads)."""
+    _need(x, "x")
+    T, d = x.shape
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T, n_heads), dtype=torch.float32, device=x.device)
+    _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
+    _check(_lib.rht_heads_quant(_ptr(x), _signs_ptr(signs), n_heads, _ptr(codes), _ptr(scales), T, d, bits,
+                                _dtype_code(x), _stream(stream)))
+    return codes, scales
+
+
+def rht_head_mix_quant(x: torch.Tensor, signs: Optional[torch.Tensor], n_heads: int,
+                       codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, bits: int = 4,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Head mixing (H_{n_h} (x) I) diag(signs) x / sqrt(n_h), then per-token INT{bits} codes."""
+    _need(x, "x")
+    T, d = x.shape
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
+    _check(_lib.rht_head_mix_quant(_ptr(x), _signs_ptr(signs), n_heads, _ptr(codes), _ptr(scales), T, d, bits,
+                                   _dtype_code(x), _stream(stream)))
     return codes, scales

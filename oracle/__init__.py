@@ -51,6 +51,7 @@ def lib():
             L.ora_head_mix.argtypes = [i64, i32, i32, _D, _I8, _D]
             L.ora_head_rht_quant.argtypes = [i64, i32, i32, i32, _D, _I8, _I8, _U8, _D, _D]
             L.ora_head_mix_quant.argtypes = [i64, i32, i32, i32, _D, _I8, _I8, _U8, _D, _D]
+            L.ora_w4a4_gemm.argtypes = [i64, i32, i32, _U8, _D, _U8, _D, ctypes.POINTER(ctypes.c_int32), _D]
             L.ora_rht_quant_gate.argtypes = [i64, i32, i32, i32, _D, _D, _D, _I8, _I8, _U8, _D, _D]
             _lib = L
     return _lib
@@ -272,3 +273,29 @@ def head_mix_quant(x, signs, n_heads: int, bits: int, want_pre: bool = True) -> 
     if rc:
         raise ValueError(f"oracle rejected d={d}, n_heads={n_heads}, bits={bits} (rc={rc})")
     return {"q": q, "codes": codes, "scales": scales, "pre": pre}
+
+
+def w4a4_gemm(codes_a, scales_a, codes_w, scales_w) -> dict:
+    """INT4 GEMM: acc = unpack(codes_a) unpack(codes_w)^T exactly (int32), y = acc * sa[t] * sw[n] (float64)."""
+    ca = np.ascontiguousarray(codes_a, dtype=np.uint8)
+    cw = np.ascontiguousarray(codes_w, dtype=np.uint8)
+    T, kb = ca.shape
+    N = cw.shape[0]
+    K = 2 * kb
+    sa, sw = _f64(scales_a), _f64(scales_w)
+    acc = np.empty((T, N), dtype=np.int32)
+    y = np.empty((T, N), dtype=np.float64)
+    rc = lib().ora_w4a4_gemm(T, N, K, _p(ca, _U8), _p(sa, _D), _p(cw, _U8), _p(sw, _D),
+                             acc.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), _p(y, _D))
+    if rc:
+        raise ValueError(f"oracle rejected T={T}, N={N}, K={K} (rc={rc})")
+    return {"acc": acc, "y": y}
+
+
+def quant_weights_rtn(W, bits: int = 4) -> dict:
+    """Per-output-channel symmetric round-to-nearest weight quantisation (the
+    simple RTN option the pages name for QuaRot's weights): each row n of W
+    (an output channel) gets scale max|W[n]| / qmax; codes packed like the
+    activation codes."""
+    q, a, _ = quant_sym(W, bits)
+    return {"codes": pack(q, bits), "scales": a, "q": q}

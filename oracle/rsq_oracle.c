@@ -32,7 +32,9 @@
  *          position transform (post-RoPE key cache, quantised per head) and
  *          the head-mixing product Z (H_{n_h} (x) I) on the attention output,
  *          with (I (x) H_{d_h}) (H_{n_h} (x) I) = H_{n_h d_h} when n_h and
- *          d_h are powers of two.
+ *          d_h are powers of two.  The quantised activations feed an INT4
+ *          GEMM whose INT32 output is turned into FP16 and multiplied by the
+ *          activation's per-row scale and the weight's per-column scale.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - rounding is to nearest, ties to even (rint in the default mode);
@@ -551,5 +553,58 @@ int ora_head_mix_quant(int64_t T, int d, int n_heads, int bits, const double *x,
         }
         free(v);
     }
+    return err;
+}
+
+
+/* ------------------------------------------------------------------------ */
+/* the INT4 consumer GEMM                                                   */
+/* ------------------------------------------------------------------------ */
+
+/* Packed INT4 codes of one row (element 2i in the low nibble of byte i,
+ * two's complement) -> integers. */
+static void unpack_int4_row(int n, const uint8_t *in, int32_t *q)
+{
+    for (int i = 0; i < n / 2; ++i) {
+        int lo = in[i] & 0xF, hi = (in[i] >> 4) & 0xF;
+        q[2 * i] = lo >= 8 ? lo - 16 : lo;
+        q[2 * i + 1] = hi >= 8 ? hi - 16 : hi;
+    }
+}
+
+/* [IQ2] QuaRot / Method: Y = X W^T from INT4 codes.  acc[t][n] = sum_k
+ * qa[t][k] qw[n][k] (exact integers), y[t][n] = acc[t][n] * sa[t] * sw[n] in
+ * double: the dequantised product before its rounding to the 16-bit output.
+ * ca: T x K/2 bytes, cw: N x K/2 bytes (weight row n = output column n). */
+int ora_w4a4_gemm(int64_t T, int N, int K, const uint8_t *ca, const double *sa, const uint8_t *cw,
+                  const double *sw, int32_t *acc, double *y)
+{
+    if (K % 2 || K < 2 || N < 1) return -1;
+    int32_t *qw = (int32_t *)malloc(sizeof(int32_t) * (size_t)N * (size_t)K);
+    if (!qw) return -2;
+    for (int n = 0; n < N; ++n) unpack_int4_row(K, cw + (int64_t)n * (K / 2), qw + (int64_t)n * K);
+    int err = 0;
+#pragma omp parallel
+    {
+        int32_t *qa = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
+        if (!qa) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                unpack_int4_row(K, ca + t * (K / 2), qa);
+                for (int n = 0; n < N; ++n) {
+                    int64_t s = 0;
+                    const int32_t *w = qw + (int64_t)n * K;
+                    for (int k = 0; k < K; ++k) s += (int64_t)qa[k] * w[k];
+                    acc[t * N + n] = (int32_t)s;
+                    y[t * N + n] = (double)s * sa[t] * sw[n];
+                }
+            }
+        }
+        free(qa);
+    }
+    free(qw);
     return err;
 }

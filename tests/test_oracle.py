@@ -459,3 +459,54 @@ def test_head_mix_quant_is_the_composition_of_its_steps():
     np.testing.assert_array_equal(r["q"], q)
     np.testing.assert_array_equal(r["scales"], a)
     np.testing.assert_array_equal(r["codes"], oracle.pack(q, 3))
+
+
+# --------------------------------------------------------------------------
+# The INT4 consumer GEMM: INT32 accumulation, then row scale x column scale
+# --------------------------------------------------------------------------
+
+def test_w4a4_gemm_integer_products_are_exact():
+    """acc = qa qw^T over the full 4-bit two's complement range, against an
+    independent unpacker and numpy's int64 matrix product; the extreme case
+    K x (-8)(-8) stays exact."""
+    from tests import helpers as H
+    rng = np.random.default_rng(11)
+    qa = rng.integers(-8, 8, size=(9, 256)).astype(np.int8)
+    qw = rng.integers(-8, 8, size=(13, 256)).astype(np.int8)
+    ca, cw = oracle.pack(qa, 4), oracle.pack(qw, 4)
+    np.testing.assert_array_equal(H.unpack_int4(ca, 256), qa)
+    r = oracle.w4a4_gemm(ca, np.ones(9), cw, np.ones(13))
+    np.testing.assert_array_equal(r["acc"], qa.astype(np.int64) @ qw.astype(np.int64).T)
+    big = np.full((1, 4096), -8, np.int8)
+    rb = oracle.w4a4_gemm(oracle.pack(big, 4), [1.0], oracle.pack(big, 4), [1.0])
+    assert rb["acc"][0, 0] == 64 * 4096
+
+
+def test_w4a4_gemm_equals_the_product_of_the_dequantised_operands():
+    """y[t][n] = (sa[t] qa[t]) . (sw[n] qw[n]): the same number as dequantising
+    both operands first and multiplying them (a different order of the same
+    exact arithmetic)."""
+    rng = np.random.default_rng(12)
+    qa = rng.integers(-7, 8, size=(6, 128)).astype(np.int8)
+    qw = rng.integers(-7, 8, size=(5, 128)).astype(np.int8)
+    sa, sw = rng.uniform(0.01, 2.0, 6), rng.uniform(0.001, 0.1, 5)
+    r = oracle.w4a4_gemm(oracle.pack(qa, 4), sa, oracle.pack(qw, 4), sw)
+    deq = (sa[:, None] * qa) @ (sw[:, None] * qw).T
+    np.testing.assert_allclose(r["y"], deq, rtol=1e-13, atol=1e-13 * np.abs(deq).max())
+
+
+def test_w4a4_gemm_stays_within_the_quantisation_error_bound():
+    """Quantise real activations per token and weights per output channel
+    (round to nearest, steps a and w); the GEMM of the codes approximates X W^T
+    within sum_k (|x_k| w/2 + |w_k| a/2 + a w / 4)."""
+    rng = np.random.default_rng(13)
+    X = rng.normal(size=(8, 512))
+    W = rng.normal(scale=0.05, size=(16, 512))
+    qa, sa, _ = oracle.quant_sym(X, 4)
+    qwt = oracle.quant_weights_rtn(W, 4)
+    r = oracle.w4a4_gemm(oracle.pack(qa, 4), sa, qwt["codes"], qwt["scales"])
+    exact = X @ W.T
+    bound = (np.abs(X) @ np.ones((512, 16))) * (qwt["scales"][None, :] / 2) + \
+            (np.ones((8, 512)) @ np.abs(W).T) * (sa[:, None] / 2) + 512 * sa[:, None] * qwt["scales"][None, :] / 4
+    assert np.all(np.abs(r["y"] - exact) <= bound)
+    assert np.abs(r["y"] - exact).max() < 0.5 * np.abs(exact).max()

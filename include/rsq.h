@@ -79,7 +79,7 @@ typedef enum {
     RSQ_ERR_VALUE = 9        /* eps negative or not finite                        */
 } rsq_status;
 
-typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
+typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1, RSQ_F16 = 2 } rsq_dtype;  /* RSQ_F16: w4a4_gemm output only */
 
 /* Supported shapes (RSQ_ERR_SHAPE otherwise):
  *   alignment:  D % 16 == 0, 16 <= D <= 32768, 1 <= r <= 64;
@@ -171,6 +171,24 @@ int rht_heads_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *co
  * d_h <= 512 (n_heads <= 16) or d_h <= 256 (n_heads >= 32). */
 int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales,
                        int64_t T, int d, int bits, int dtype, void *stream);
+
+/* The INT4 consumer GEMM of the quantised activations (W4A4).  Infra Quant II,
+ * QuaRot / Method: the INT4 GEMM's INT32 output becomes 16-bit float and is
+ * multiplied by the activation's per-row scale and the weight's per-column
+ * scale.  With qa the T x K activation codes (as written by the quantising
+ * entry points with bits = 4: T rows of K/2 bytes) and qw the N x K weight codes
+ * (N rows of K/2 bytes, row n = output column n, same packing; any 4-bit two's
+ * complement value):
+ *     acc[t][n] = sum_k qa[t][k] qw[n][k]                 (exact, int32)
+ *     y[t][n]   = round(float(acc[t][n]) * scales_a[t] * scales_w[n])
+ * in float32, rounded once to out_dtype: RSQ_F16 (the pages' FP16) or
+ * RSQ_BF16.  y: T x N row-major.  acc: optional (NULL to skip) T x N int32
+ * copy of the accumulators.  K % 128 == 0 (128 <= K <= 65536), N % 8 == 0
+ * (8 <= N <= 65536), T <= 8388480 (RSQ_ERR_SHAPE otherwise).  Outputs may not
+ * overlap any input or each other (RSQ_ERR_ALIAS).  Streams, errors and
+ * alignment as above. */
+int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *codes_w, const float *scales_w,
+              void *y, int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream);
 
 /* Human-readable name of an rsq_status value (static storage; never NULL). */
 const char *rsq_status_string(int status);

@@ -126,3 +126,24 @@ def check_aligned(gpu: np.ndarray, ora: np.ndarray, x: np.ndarray, dtype: str, l
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = np.where(bound > 0, err / bound, 0.0)
     return float(ratio.max())
+
+
+GEMM_OUT_UNIT = {"f16": 2.0 ** -11, "bf16": 2.0 ** -8}
+
+
+def check_gemm(y_gpu: np.ndarray, y_ora: np.ndarray, out: str, label: str = "") -> float:
+    """16-bit GEMM outputs against the float64 oracle: one rounding to the output
+    type (unit roundoff u: 2^-11 fp16, 2^-8 bf16) after three float32 operations
+    (int32 -> float conversion, two scale products: <= 3 * 2^-24 relative), plus
+    the output type's smallest subnormal spacing for results near zero."""
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    u = GEMM_OUT_UNIT[out]
+    tiny = 2.0 ** -24 if out == "f16" else 2.0 ** -133
+    bound = (u + 4 * 2.0 ** -24) * np.abs(y_ora) + tiny
+    err = np.abs(y_gpu - y_ora)
+    ok = err <= bound
+    if not ok.all():
+        i = np.unravel_index(np.argmax(np.where(ok, 0.0, err - bound)), err.shape)
+        raise AssertionError(f"{label}: GEMM output error above bound at {int((~ok).sum())} places, e.g. "
+                             f"{tuple(int(v) for v in i)}: gpu {float(y_gpu[i])!r} oracle {float(y_ora[i])!r}")
+    return float((err / np.maximum(bound, 1e-300)).max()) if err.size else 0.0

@@ -188,6 +188,23 @@ def test_head_transforms_accept_null_signs():
     assert _heads(sg=None) == CUDA and _heads_q(sg=None) == CUDA and _mix_q(sg=None) == CUDA
 
 
+def _gemm(ca=X, sa=S, cw=Q, sw=M, y=XO, acc=C, T=4, N=256, K=4096, dt=2):
+    return L.w4a4_gemm(ca, sa, cw, sw, y, acc, T, N, K, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(ca=None), NULL), (dict(sa=None), NULL), (dict(cw=None), NULL), (dict(sw=None), NULL), (dict(y=None), NULL),
+    (dict(dt=0), DTYPE), (dict(dt=3), DTYPE), (dict(T=-1), SHAPE), (dict(N=4), SHAPE), (dict(N=260), SHAPE),
+    (dict(K=64), SHAPE), (dict(K=4096 + 64), SHAPE), (dict(T=65536 * 128), SHAPE),
+    (dict(ca=X + 1), ALIGN), (dict(y=XO + 2), ALIGN), (dict(acc=C + 8), ALIGN),
+    (dict(y=X + 1024), ALIAS), (dict(acc=XO + 16), ALIAS), (dict(acc=Q), ALIAS), (dict(y=S), ALIAS),
+])
+def test_w4a4_gemm_rejects(kw, want):
+    before = rsq.launch_count()
+    assert _gemm(**kw) == want
+    assert rsq.launch_count() == before
+
+
 def test_empty_batch_is_a_no_op():
     before = rsq.launch_count()
     assert _anq(x=None, xo=None, c=None, s=None, T=0) == OK
@@ -197,6 +214,7 @@ def test_empty_batch_is_a_no_op():
     assert _heads(x=None, xo=None, T=0) == OK
     assert _heads_q(x=None, c=None, s=None, T=0) == OK
     assert _mix_q(x=None, c=None, s=None, T=0) == OK
+    assert _gemm(ca=None, sa=None, y=None, acc=None, T=0) == OK
     assert rsq.launch_count() == before
 
 

@@ -637,6 +637,75 @@ def test_attention_transforms_full_size_sampled():
     check_head_mix(c, 32, True, rows, "head mix T=16384")
 
 
+def run_gemm(case, out="f16", with_acc=True, rows=None):
+    rsq = _rsq()
+    ca = torch.from_numpy(case.codes_a).to(DEV)
+    cw = torch.from_numpy(case.codes_w).to(DEV)
+    sa = torch.from_numpy(case.scales_a).to(DEV)
+    sw = torch.from_numpy(case.scales_w).to(DEV)
+    acc = torch.empty((case.T, case.N), dtype=torch.int32, device=DEV) if with_acc else None
+    y = rsq.w4a4_gemm(ca, sa, cw, sw, acc=acc, out_dtype=torch.float16 if out == "f16" else torch.bfloat16)
+    assert rsq.device_status() == 0
+    sel = slice(None) if rows is None else rows
+    ref = oracle.w4a4_gemm(case.codes_a[sel], case.scales_a[sel], case.codes_w, case.scales_w)
+    if with_acc:
+        np.testing.assert_array_equal(acc.cpu().numpy()[sel], ref["acc"])  # integer products: bit-exact
+    H.check_gemm(y.float().cpu().numpy()[sel], ref["y"], out, case.name)
+    return y
+
+
+@pytest.mark.parametrize("T,N,K", [(1, 8, 128), (128, 256, 128), (127, 264, 256), (300, 512, 1024),
+                                   (129, 4096, 4096), (515, 1000, 384)])
+@pytest.mark.parametrize("out", ["f16", "bf16"])
+def test_w4a4_gemm(T, N, K, out):
+    """The INT4 GEMM on tcgen05 (kind::i8): exact int32 products over the full
+    4-bit range, then the scale epilogue, against the oracle; several tiles and
+    ragged edges in both output dimensions."""
+    run_gemm(inputs.gemm_case(T, N, K, T + N + K), out)
+
+
+def test_w4a4_gemm_without_accumulator_copy_matches():
+    c = inputs.gemm_case(200, 768, 512, 3)
+    y1 = run_gemm(c, "f16", with_acc=True)
+    y2 = run_gemm(c, "f16", with_acc=False)
+    assert torch.equal(y1, y2)
+
+
+def test_w4a4_gemm_consumes_the_quantiser_codes():
+    """The consumer of the path, both chains independent: on the GPU the
+    alignment quantiser's INT4 codes and scales feed the GEMM; in the oracle
+    its own codes feed its own GEMM.  The codes agree up to the tie rule, and
+    on every row whose codes agree exactly the GEMM outputs agree within the
+    output rounding."""
+    rsq = _rsq()
+    a, _ = inputs.llama7b_case(T=256)
+    x = _to_dev(a.x, "bf16")
+    _, codes, scales = rsq.rsq_align_norm_quant(x, torch.from_numpy(a.Q).to(DEV), torch.from_numpy(a.M).to(DEV), bits=4)
+    W = np.random.default_rng(9).normal(scale=0.02, size=(512, 4096))
+    wq = oracle.quant_weights_rtn(W, 4)
+    sw = wq["scales"].astype(np.float32)
+    y = rsq.w4a4_gemm(codes, scales, torch.from_numpy(wq["codes"]).to(DEV), torch.from_numpy(sw).to(DEV))
+    ref_a = oracle.align_norm_quant(a.x, a.Q, a.M, 4, a.eps)
+    c_gpu = codes.cpu().numpy()
+    H.check_codes(c_gpu, ref_a["q"], ref_a["pre"], 4, "quantiser codes")
+    H.check_scales(scales.cpu().numpy(), ref_a["scales"], "quantiser scales")
+    ref = oracle.w4a4_gemm(ref_a["codes"], ref_a["scales"].astype(np.float32), wq["codes"], sw)
+    same = np.all(c_gpu == ref_a["codes"], axis=1)
+    assert same.sum() >= 250
+    # the activation scales may differ by the scale tolerance (1e-6): two more
+    # float32-sized terms in the bound
+    yg = y.float().cpu().numpy()[same].astype(np.float64)
+    bound = (2.0 ** -11 + 4 * 2.0 ** -24 + 2e-6) * np.abs(ref["y"][same]) + 2.0 ** -24
+    assert np.all(np.abs(yg - ref["y"][same]) <= bound)
+
+
+def test_w4a4_gemm_full_size_sampled():
+    """T = 16384, N = K = 4096 (the hidden stream through a 4096 x 4096 INT4
+    projection), sampled rows against the oracle."""
+    c = inputs.gemm_case(16384, 4096, 4096, 21)
+    run_gemm(c, "f16", with_acc=True, rows=_sample(16384, 24, seed=3))
+
+
 @pytest.mark.parametrize("d,which", [(4096, 1), (4096, 3), (8192, 3)])
 def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()

@@ -73,6 +73,12 @@ cudaError_t launch_head_rht(const void *x, const int8_t *signs, void *x_out, uin
 cudaError_t launch_head_mix(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
                             int n_heads, int bits, int dtype, cudaStream_t s);
 
+// INT4 consumer GEMM: y = round16(float(codes_a codes_w^T) * sa[t] * sw[n]),
+// fp16 (out_f16) or bf16 out, optional raw int32 accumulators.
+bool w4a4_gemm_supports(long long T, int N, int K);
+cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const uint8_t *codes_w, const float *sw,
+                             void *y, int32_t *acc, long long T, int N, int K, int out_f16, cudaStream_t s);
+
 // Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
 // (m = 1, bf16, INT4/INT3).
 bool rht_tc_supports(int d, int m, int dtype, int bits, long long T);

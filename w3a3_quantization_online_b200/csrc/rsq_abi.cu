@@ -327,6 +327,31 @@ int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t 
                                        static_cast<cudaStream_t>(stream)));
 }
 
+int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *codes_w, const float *scales_w, void *y,
+              int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream) {
+    if (out_dtype != RSQ_BF16 && out_dtype != RSQ_F16) return RSQ_ERR_DTYPE;
+    if (T < 0 || N < 8 || N % 8 != 0 || N > 65536 || K < 128 || K % 128 != 0 || K > 65536) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!rsq::w4a4_gemm_supports(T, N, K)) return RSQ_ERR_SHAPE;
+    if (!codes_a || !scales_a || !codes_w || !scales_w || !y) return RSQ_ERR_NULL;
+    if (!aligned16(codes_a) || !aligned16(scales_a) || !aligned16(codes_w) || !aligned16(scales_w) || !aligned16(y) ||
+        (acc && !aligned16(acc)))
+        return RSQ_ERR_ALIGN;
+    const Span in[4] = {span(codes_a, uint64_t(T) * (K / 2)), span(scales_a, uint64_t(T) * 4),
+                        span(codes_w, uint64_t(N) * (K / 2)), span(scales_w, uint64_t(N) * 4)};
+    const Span sy = span(y, uint64_t(T) * N * 2);
+    for (const Span &i : in)
+        if (overlap(sy, i)) return RSQ_ERR_ALIAS;
+    if (acc) {
+        const Span sacc = span(acc, uint64_t(T) * N * 4);
+        if (overlap(sacc, sy)) return RSQ_ERR_ALIAS;
+        for (const Span &i : in)
+            if (overlap(sacc, i)) return RSQ_ERR_ALIAS;
+    }
+    return finish(rsq::launch_w4a4_gemm(codes_a, scales_a, codes_w, scales_w, y, acc, T, N, K, out_dtype == RSQ_F16,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 const char *rsq_status_string(int status) {
     switch (status) {
         case RSQ_OK: return "RSQ_OK";

@@ -1,0 +1,352 @@
+// w4a4_gemm.cu -- the INT4 consumer GEMM of the quantised activations (W4A4).
+//
+// Infra Quant II, QuaRot / Method: the INT4 GEMM's INT32 output is converted to
+// 16-bit float and multiplied by the activation's per-row scale and the weight's
+// per-column scale.  Here Y[t][n] = round16(float(acc[t][n]) * sa[t] * sw[n])
+// with acc = qa qw^T exact in int32 (|acc| <= 64 K), qa the packed per-token
+// activation codes written by the quantising entry points and qw the packed
+// per-output-channel weight codes (element 2i in the low nibble of byte i,
+// two's complement, any 4-bit value).
+//
+// Design (B200, sm_100a): one CTA per 128 x 256 output tile, 10 warps.
+//  * Warp 0 (one thread): TMA loads of the packed tiles, 128 rows of A and 256
+//    rows of B by 64 bytes (128 K values), into a 3-stage ring.
+//  * Warps 2-9: unpack.  A 16-byte chunk of packed codes (32 values) becomes
+//    two 16-byte chunks of int8 in the SWIZZLE_128B K-major layout of a
+//    tcgen05 operand (nibbles masked into bytes, sign-extended by a multiply
+//    that cannot carry across bytes, even/odd elements interleaved by byte
+//    permutes); four consecutive threads take the four chunks of one packed
+//    row, so both the reads and the swizzled writes are free of bank
+//    conflicts.  2-stage ring of unpacked operands.
+//  * Warp 1 (one thread): tcgen05.mma kind::i8 (s8 x s8 -> s32, M = 128,
+//    N = 256, K = 32), four per stage, accumulating in 256 TMEM columns.
+//  * Epilogue, warps 2-9: TMEM -> registers, float(acc) * sa * sw, rounded to
+//    fp16 or bf16 into a swizzled staging tile, written by TMA (4 slabs of 64
+//    columns); optionally the raw int32 accumulators as well.
+// Every mbarrier wait is bounded; a timeout sets a bit in the device status
+// word, no further asynchronous work is issued, and the CTA drains what is in
+// flight before freeing TMEM.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace rsq {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kBM = 128, kBN = 256, kBK = 128;
+constexpr int kPA = kBM * kBK / 2;  // packed A bytes per stage (8 KB)
+constexpr int kPB = kBN * kBK / 2;  // packed B bytes per stage (16 KB)
+constexpr int kUA = kBM * kBK;      // unpacked A bytes per stage (16 KB)
+constexpr int kUB = kBN * kBK;      // unpacked B bytes per stage (32 KB)
+constexpr int kP = 3, kU = 2;       // ring depths
+constexpr int kUnpackWarps = 8;
+constexpr int kGThreads = (2 + kUnpackWarps) * 32;
+constexpr int kGTmemCols = 256;
+
+constexpr int kOffPk = 0;                           // packed ring
+constexpr int kOffUn = kOffPk + kP * (kPA + kPB);   // unpacked ring (1024-aligned: 73728)
+constexpr int kOffSw = kOffUn + kU * (kUA + kUB);   // 256 column scales
+constexpr int kOffBar = kOffSw + kBN * 4;
+enum : int { kPFull = 0, kPEmpty = kPFull + kP, kUFull = kPEmpty + kP, kUEmpty = kUFull + kU, kAcc = kUEmpty + kU,
+             kGBars = kAcc + 1 };
+constexpr int kOffTm = kOffBar + kGBars * 8;
+constexpr int kGSmem = kOffTm + 16 + 1024;
+static_assert(kOffUn % 1024 == 0 && (kUA + kUB) % 1024 == 0, "swizzle atoms");
+static_assert(kU * (kUA + kUB) >= kBM * kBN * 2, "epilogue staging fits in the unpacked ring");
+
+struct GemmArgs {
+    const float *sa;
+    const float *sw;
+    int32_t *acc;  // optional raw accumulators (T x N)
+    int *status;
+    long long T;
+    int N;
+    int K;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return uint32_t(((chunk ^ (row & 7)) << 4)); }
+
+// Instruction descriptor, kind::i8: s8 x s8 -> s32, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+    return (2u << 4)      // D format: s32
+           | (1u << 7)    // A format: signed 8-bit
+           | (1u << 10)   // B format: signed 8-bit
+           | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 8 packed 4-bit codes (one word) -> 8 int8 (two words), element order kept.
+__device__ __forceinline__ void unpack8(uint32_t w, uint32_t &o0, uint32_t &o1) {
+    uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    lo |= (lo & 0x08080808u) * 0x1Eu;  // bit 3 of a byte -> bits 4-7 of the same byte
+    hi |= (hi & 0x08080808u) * 0x1Eu;
+    o0 = prmt(lo, hi, 0x5140u);        // elements 0, 1, 2, 3
+    o1 = prmt(lo, hi, 0x7362u);        // elements 4, 5, 6, 7
+}
+
+// One packed row chunk (16 bytes: K values 32 c .. 32 c + 31 of row r) -> the
+// two unpacked 16-byte chunks 2 c and 2 c + 1 of row r.
+__device__ __forceinline__ void unpack_chunk(const uint8_t *pk, uint8_t *un, int r, int c) {
+    const uint4 p = *reinterpret_cast<const uint4 *>(pk + r * 64 + c * 16);
+    uint32_t o[8];
+    unpack8(p.x, o[0], o[1]);
+    unpack8(p.y, o[2], o[3]);
+    unpack8(p.z, o[4], o[5]);
+    unpack8(p.w, o[6], o[7]);
+    uint8_t *row = un + r * 128;
+    *reinterpret_cast<uint4 *>(row + swz(r, 2 * c)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4 *>(row + swz(r, 2 * c + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <class OUT>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+    return pack_bf16x2(a, b);
+}
+
+template <class OUT>
+__global__ void __launch_bounds__(kGThreads, 1)
+k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+            const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
+    extern __shared__ uint8_t gsm_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
+    float *ssw = reinterpret_cast<float *>(base + kOffSw);
+    const uint32_t bars = smem_u32(base + kOffBar);
+    auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTm);
+    auto pk_a = [&](int s) { return base + kOffPk + s * (kPA + kPB); };
+    auto pk_b = [&](int s) { return base + kOffPk + s * (kPA + kPB) + kPA; };
+    auto un_a = [&](int s) { return base + kOffUn + s * (kUA + kUB); };
+    auto un_b = [&](int s) { return base + kOffUn + s * (kUA + kUB) + kUA; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n0 = blockIdx.x * kBN;
+    const long long m0 = (long long)blockIdx.y * kBM;
+    const int KS = p.K / kBK;
+    int err = 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < kGBars; ++i)
+            mbar_init(bar(i), (i >= kPEmpty && i < kPEmpty + kP) || (i >= kUFull && i < kUFull + kU) ? kUnpackWarps : 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_a);
+        prefetch_tmap(&tm_b);
+        prefetch_tmap(&tm_y);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kGTmemCols);
+        tmem_relinquish();
+    }
+    for (int i = tid; i < kBN; i += kGThreads) ssw[i] = n0 + i < p.N ? p.sw[n0 + i] : 0.f;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- TMA producer
+        if (lane == 0) {
+            for (int ks = 0; ks < KS; ++ks) {
+                const int s = ks % kP;
+                if (!mbar_wait(bar(kPEmpty + s), uint32_t((ks / kP) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
+                mbar_expect_tx(bar(kPFull + s), uint32_t(kPA + kPB));
+                if (!err) {
+                    tma_load_2d(smem_u32(pk_a(s)), &tm_a, ks * (kBK / 2), int(m0), bar(kPFull + s));
+                    tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---- tensor-core issue
+        if (lane == 0) {
+            const uint32_t idesc = idesc_s8_s32(kBM, kBN);
+            for (int ks = 0; ks < KS; ++ks) {
+                const int u = ks % kU;
+                if (!mbar_wait(bar(kUFull + u), uint32_t((ks / kU) & 1), err != 0)) err |= kErrMbarTimeout;
+                tc_fence_after();
+                const uint64_t ad = smem_desc_sw128(smem_u32(un_a(u)), 1024);
+                const uint64_t bd = smem_desc_sw128(smem_u32(un_b(u)), 1024);
+#pragma unroll
+                for (int k = 0; k < kBK / 32; ++k)  // K steps of 32 int8 = 32 bytes
+                    if (!err) umma_i8(tmem, ad + uint64_t((k * 32) >> 4), bd + uint64_t((k * 32) >> 4), idesc,
+                                      (ks | k) != 0);
+                if (!err) umma_commit(bar(kUEmpty + u));
+            }
+            if (!err) umma_commit(bar(kAcc));
+        }
+        __syncwarp();
+    } else {
+        // ---- unpack
+        const int u_tid = tid - 64;  // 0..255
+        for (int ks = 0; ks < KS; ++ks) {
+            const int s = ks % kP, u = ks % kU;
+            if (!mbar_wait(bar(kPFull + s), uint32_t((ks / kP) & 1), err != 0)) err |= kErrMbarTimeout;
+            if (!mbar_wait(bar(kUEmpty + u), uint32_t((ks / kU) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
+            const uint8_t *pa = pk_a(s), *pb = pk_b(s);
+            uint8_t *ua = un_a(u), *ub = un_b(u);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // A: 512 chunks
+                const int i = u_tid + 256 * j;
+                unpack_chunk(pa, ua, i >> 2, i & 3);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // B: 1024 chunks
+                const int i = u_tid + 256 * j;
+                unpack_chunk(pb, ub, i >> 2, i & 3);
+            }
+            fence_proxy_async_cta();  // unpacked operands (generic writes) -> tensor core (async proxy)
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar(kPEmpty + s));
+                mbar_arrive(bar(kUFull + u));
+            }
+        }
+
+        // ---- epilogue: quadrant of TMEM lanes, half of the 256 columns
+        if (!mbar_wait(bar(kAcc), 0u, err != 0)) err |= kErrMbarTimeout;
+        tc_fence_after();
+        const int q = warp & 3, ch = (warp - 2) >> 2;
+        const int r = 32 * q + lane;
+        const long long row = m0 + r;
+        const float sa = row < p.T ? p.sa[row] : 0.f;
+        uint8_t *stage = base + kOffUn;  // 4 slabs of 128 rows x 64 columns (128 B per row, SWIZZLE_128B)
+#pragma unroll 1
+        for (int b = 0; b < 4; ++b) {  // 32-column blocks of this thread's 128 columns
+            uint32_t v[32];
+            tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(128 * ch + 32 * b), v);
+            tmem_wait_ld();
+            const int c0 = 128 * ch + 32 * b;  // first column of the block within the tile
+            if (p.acc && row < p.T) {
+                int32_t *dst = p.acc + row * p.N + n0 + c0;
+                if (n0 + c0 + 32 <= p.N) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<int4 *>(dst + e) = make_int4(int(v[e]), int(v[e + 1]), int(v[e + 2]), int(v[e + 3]));
+                } else {
+                    for (int e = 0; e < 32; ++e)
+                        if (n0 + c0 + e < p.N) dst[e] = int(v[e]);
+                }
+            }
+            uint32_t o[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                o[e] = pack2<OUT>(float(int(v[2 * e])) * sa * ssw[c0 + 2 * e],
+                                  float(int(v[2 * e + 1])) * sa * ssw[c0 + 2 * e + 1]);
+            uint8_t *slab = stage + (c0 >> 6) * (kBM * 128) + r * 128;
+            const int ck0 = (c0 & 63) >> 3;  // first 16-byte chunk (8 outputs) within the slab row
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4 *>(slab + swz(r, ck0 + c)) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        }
+        fence_proxy_async_cta();
+        named_sync(1, kUnpackWarps * 32);
+        if (u_tid == 0) {
+            if (!err)
+                for (int s = 0; s < 4; ++s)
+                    if (n0 + 64 * s < p.N) tma_store_2d(&tm_y, smem_u32(stage + s * (kBM * 128)), n0 + 64 * s, int(m0));
+            bulk_commit();
+            bulk_wait0();
+        }
+    }
+
+    tc_fence_before();
+    if (__syncthreads_or(err)) drain_delay();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kGTmemCols);
+    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    if (err && lane == 0) atomicOr(p.status, err);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *q = nullptr;
+        cudaDriverEntryPointQueryResult res;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &res) == cudaSuccess &&
+            res == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(q);
+    }
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap *mp, const void *ptr, CUtensorMapDataType dt, int esize, long long rows, long long cols,
+                 int box_cols, int box_rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+    const cuuint64_t strides[1] = {cuuint64_t(cols) * esize};
+    const cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(mp, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool w4a4_gemm_supports(long long T, int N, int K) {
+    return T >= 1 && T <= 65535LL * kBM && N >= 8 && N % 8 == 0 && K >= kBK && K % kBK == 0 && K <= 65536;
+}
+
+cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const uint8_t *codes_w, const float *sw,
+                             void *y, int32_t *acc, long long T, int N, int K, int out_f16, cudaStream_t s) {
+    static bool configured[2][64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int *status = device_status_word();
+    if (!status) return cudaErrorInvalidDevice;
+    auto kern = out_f16 ? k_w4a4_gemm<__half> : k_w4a4_gemm<__nv_bfloat16>;
+    if (dev >= 0 && dev < 64 && !configured[out_f16 ? 1 : 0][dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
+        if (e != cudaSuccess) return e;
+        configured[out_f16 ? 1 : 0][dev] = true;
+    }
+    CUtensorMap ma, mb, my;
+    if (!make_map_2d(&ma, codes_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&mb, codes_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, kBK / 2, kBN, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map_2d(&my, y, out_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, N, 64,
+                     kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    GemmArgs a;
+    a.sa = sa;
+    a.sw = sw;
+    a.acc = acc;
+    a.status = status;
+    a.T = T;
+    a.N = N;
+    a.K = K;
+    const dim3 grid(unsigned((N + kBN - 1) / kBN), unsigned((T + kBM - 1) / kBM));
+    kern<<<grid, kGThreads, kGSmem, s>>>(ma, mb, my, a);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch();
+    return e;
+}
+
+}  // namespace rsq

@@ -249,6 +249,41 @@ def attention_case(T: int = 16384, n_heads: int = 32, d_head: int = 128, seed: i
                     name=f"attn_T{T}_h{n_heads}x{d_head}")
 
 
+@dataclasses.dataclass
+class GemmCase:
+    """Inputs of one INT4 GEMM: packed activation and weight codes and their scales."""
+    name: str
+    codes_a: np.ndarray    # T x K/2 uint8 (two 4-bit codes per byte)
+    scales_a: np.ndarray   # T float32
+    codes_w: np.ndarray    # N x K/2 uint8
+    scales_w: np.ndarray   # N float32
+
+    @property
+    def T(self) -> int:
+        return self.codes_a.shape[0]
+
+    @property
+    def N(self) -> int:
+        return self.codes_w.shape[0]
+
+    @property
+    def K(self) -> int:
+        return 2 * self.codes_a.shape[1]
+
+
+def gemm_case(T: int, N: int, K: int, seed: int) -> GemmCase:
+    """Uniformly random bytes as packed 4-bit codes (every 4-bit two's complement
+    value, -8 .. 7, equally likely), activation scales ~ U(0.01, 1) and weight
+    scales ~ U(0.001, 0.02), float32 (the magnitudes of per-token activation
+    steps and per-channel weight steps)."""
+    r = _rng(seed, _S_X)
+    ca = r.integers(0, 256, size=(T, K // 2), dtype=np.uint8)
+    cw = _rng(seed, _S_Q).integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    sa = _rng(seed, _S_A).uniform(0.01, 1.0, size=T).astype(np.float32)
+    sw = _rng(seed, _S_SIGNS).uniform(0.001, 0.02, size=N).astype(np.float32)
+    return GemmCase(f"gemm_T{T}_N{N}_K{K}", ca, sa, cw, sw)
+
+
 def down_proj_gate_case(T: int = 4096) -> GateCase:
     """FFN down_proj with the gate fused: a, b ~ N(0, 1) in bf16, d=12288=1024*12, INT4."""
     return gate_case(T, 12288, 12, 2, dtype="bf16", bits=4, name=f"downproj_gate_T{T}_d12288")

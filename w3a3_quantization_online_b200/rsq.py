@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "librsq.so")
 
-RSQ_F32, RSQ_BF16 = 0, 1
+RSQ_F32, RSQ_BF16, RSQ_F16 = 0, 1, 2
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -38,6 +38,8 @@ _lib.rht_heads_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i3
 _lib.rht_heads_quant.restype = _i32
 _lib.rht_head_mix_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.rht_head_mix_quant.restype = _i32
+_lib.w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.w4a4_gemm.restype = _i32
 _lib.rsq_status_string.argtypes = [_i32]
 _lib.rsq_status_string.restype = ctypes.c_char_p
 _lib.rsq_last_cuda_error.argtypes = []
@@ -54,7 +56,7 @@ _lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
 _lib.rsq_selftest_wait_timeout.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rht_heads",
-            "rht_heads_quant", "rht_head_mix_quant", "rsq_status_string",
+            "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
 
@@ -270,3 +272,28 @@ def rht_head_mix_quant(x: torch.Tensor, signs: Optional[torch.Tensor], n_heads: 
     _check(_lib.rht_head_mix_quant(_ptr(x), _signs_ptr(signs), n_heads, _ptr(codes), _ptr(scales), T, d, bits,
                                    _dtype_code(x), _stream(stream)))
     return codes, scales
+
+
+def w4a4_gemm(codes_a: torch.Tensor, scales_a: torch.Tensor, codes_w: torch.Tensor, scales_w: torch.Tensor,
+              y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None, out_dtype=torch.float16,
+              stream=None) -> torch.Tensor:
+    """Y = (INT4 codes_a @ INT4 codes_w^T) * scales_a[:, None] * scales_w[None, :] in fp16 / bf16.
+
+    codes_a: T x K/2 uint8, codes_w: N x K/2 uint8 (packed INT4); acc (optional) receives the int32 products."""
+    _need(codes_a, "codes_a", torch.uint8); _need(codes_w, "codes_w", torch.uint8)
+    _need(scales_a, "scales_a", torch.float32); _need(scales_w, "scales_w", torch.float32)
+    T, kb = codes_a.shape
+    N = codes_w.shape[0]
+    if codes_w.shape[1] != kb:
+        raise ValueError("codes_a and codes_w disagree on K")
+    if out_dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("out_dtype must be float16 or bfloat16")
+    if y is None:
+        y = torch.empty((T, N), dtype=out_dtype, device=codes_a.device)
+    _need(y, "y", out_dtype)
+    if acc is not None:
+        _need(acc, "acc", torch.int32)
+    code = RSQ_F16 if out_dtype == torch.float16 else RSQ_BF16
+    _check(_lib.w4a4_gemm(_ptr(codes_a), _ptr(scales_a), _ptr(codes_w), _ptr(scales_w), _ptr(y), _ptr(acc), T, N,
+                          2 * kb, code, _stream(stream)))
+    return y

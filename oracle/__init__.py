@@ -299,3 +299,35 @@ def quant_weights_rtn(W, bits: int = 4) -> dict:
     activation codes."""
     q, a, _ = quant_sym(W, bits)
     return {"codes": pack(q, bits), "scales": a, "q": q}
+
+
+def qm_construct(R_in, R_out, r: int) -> dict:
+    """The offline (Q, M) construction of ReSpinQuant (paper notes, key design 2), in float64.
+
+    T = R_out R_in^T is the transition matrix at a residual connection; its
+    deviation dT = T - I is decomposed by SVD and Q takes the top-r left
+    singular vectors; T_sub = Q^T T Q is the transition restricted to that
+    subspace; the polar factor U V^T of T_sub (SVD T_sub = U S V^T), pulled
+    back into SO(r) (when det(U V^T) = -1 the singular pair of the smallest
+    singular value flips sign, the nearest rotation), is R_sub; M = R_sub - I.
+    The low-rank approximation T_hat = I + Q M Q^T is then in SO(D).  numpy's
+    SVD and matrix products are the library steps."""
+    R_in = np.asarray(R_in, dtype=np.float64)
+    R_out = np.asarray(R_out, dtype=np.float64)
+    D = R_in.shape[0]
+    T = R_out @ R_in.T
+    U, S, _ = np.linalg.svd(T - np.eye(D))
+    Q = U[:, :r]
+    T_sub = Q.T @ T @ Q
+    U2, S2, Vt2 = np.linalg.svd(T_sub)
+    if np.linalg.det(U2 @ Vt2) < 0:
+        U2 = U2.copy()
+        U2[:, -1] = -U2[:, -1]
+    R_sub = U2 @ Vt2
+    return {"Q": Q, "R_sub": R_sub, "M": R_sub - np.eye(r), "T": T, "T_sub": T_sub, "sv": S}
+
+
+def t_hat(Q, M) -> np.ndarray:
+    """The dense D x D T_hat = I + Q M Q^T (tests only: the online path never forms it)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    return np.eye(Q.shape[0]) + Q @ np.asarray(M, dtype=np.float64) @ Q.T

@@ -510,3 +510,73 @@ def test_w4a4_gemm_stays_within_the_quantisation_error_bound():
             (np.ones((8, 512)) @ np.abs(W).T) * (sa[:, None] / 2) + 512 * sa[:, None] * qwt["scales"][None, :] / 4
     assert np.all(np.abs(r["y"] - exact) <= bound)
     assert np.abs(r["y"] - exact).max() < 0.5 * np.abs(exact).max()
+
+
+# --------------------------------------------------------------------------
+# The offline (Q, M) construction: SVD of T - I, subspace, polar factor
+# --------------------------------------------------------------------------
+
+def test_qm_reproduces_a_transition_whose_deviation_has_rank_r():
+    """range(T - I) is invariant under an orthogonal T, so when T - I has rank k
+    the top-k subspace captures all of it and T_hat = T exactly; r = D is the
+    trivial case."""
+    R_in, R_out = inputs.near_hadamard_pair(128, 5, n_planes=8)   # deviation of rank 16
+    for r in (16, 128):
+        c = oracle.qm_construct(R_in, R_out, r)
+        np.testing.assert_allclose(oracle.t_hat(c["Q"], c["M"]), c["T"], rtol=0, atol=1e-12)
+    assert np.linalg.norm(oracle.t_hat(*[oracle.qm_construct(R_in, R_out, 8)[k] for k in ("Q", "M")]) -
+                          R_out @ R_in.T) > 0.1
+
+
+@pytest.mark.parametrize("r", [2, 8, 32])
+def test_qm_t_hat_is_a_rotation(r):
+    """The pages: after the polar step T_hat = I + Q (R_sub - I) Q^T is in SO(D)."""
+    R_in, R_out = inputs.near_hadamard_pair(256, 7)
+    c = oracle.qm_construct(R_in, R_out, r)
+    Th = oracle.t_hat(c["Q"], c["M"])
+    np.testing.assert_allclose(Th.T @ Th, np.eye(256), rtol=0, atol=1e-10)
+    sign, _ = np.linalg.slogdet(Th)
+    assert sign == 1.0
+    np.testing.assert_allclose(c["R_sub"].T @ c["R_sub"], np.eye(r), rtol=0, atol=1e-12)
+    assert np.linalg.det(c["R_sub"]) > 0
+    np.testing.assert_allclose(c["Q"].T @ c["Q"], np.eye(r), rtol=0, atol=1e-12)
+
+
+def test_qm_error_does_not_grow_with_the_rank():
+    """||T - T_hat||_F over r = 2, 4, ..., D (even r: the singular values of the
+    deviation of a rotation come in pairs) is non-increasing, as in the pages'
+    rank ablation, and zero at full rank."""
+    R_in, R_out = inputs.near_hadamard_pair(256, 9)
+    errs = []
+    for r in (2, 4, 8, 16, 32, 64, 128, 256):
+        c = oracle.qm_construct(R_in, R_out, r)
+        errs.append(np.linalg.norm(oracle.t_hat(c["Q"], c["M"]) - c["T"]))
+    assert all(b <= a + 1e-12 for a, b in zip(errs, errs[1:])), errs
+    assert errs[-1] < 1e-12
+
+
+def test_qm_polar_factor_is_the_nearest_rotation():
+    """R_sub = U V^T is the rotation nearest to T_sub: R_sub^T T_sub is symmetric
+    positive semidefinite, and small rotations of R_sub are farther from T_sub."""
+    R_in, R_out = inputs.near_hadamard_pair(128, 11)
+    c = oracle.qm_construct(R_in, R_out, 16)
+    P = c["R_sub"].T @ c["T_sub"]
+    np.testing.assert_allclose(P, P.T, rtol=0, atol=1e-12)
+    assert np.linalg.eigvalsh((P + P.T) / 2).min() > -1e-12
+    rng = np.random.default_rng(1)
+    base = np.linalg.norm(c["R_sub"] - c["T_sub"])
+    for _ in range(20):
+        A = rng.normal(scale=0.01, size=(16, 16))
+        A = A - A.T
+        G = np.linalg.solve(np.eye(16) - A, np.eye(16) + A)
+        assert np.linalg.norm(c["R_sub"] @ G - c["T_sub"]) >= base - 1e-12
+
+
+def test_qm_feeds_the_online_path():
+    """The constructed (Q, M) in the three-step online path equals the dense
+    T_hat applied to the rows."""
+    R_in, R_out = inputs.near_hadamard_pair(256, 13)
+    c = oracle.qm_construct(R_in, R_out, 32)
+    x = np.random.default_rng(2).normal(size=(7, 256))
+    np.testing.assert_allclose(oracle.residual_align(x, c["Q"], c["M"]), x @ oracle.t_hat(c["Q"], c["M"]).T,
+                               rtol=1e-12, atol=1e-12)

@@ -284,6 +284,36 @@ def gemm_case(T: int, N: int, K: int, seed: int) -> GemmCase:
     return GemmCase(f"gemm_T{T}_N{N}_K{K}", ca, sa, cw, sw)
 
 
+def sylvester_signed(D: int, seed: int) -> np.ndarray:
+    """Randomised Hadamard rotation H_D diag(s) / sqrt(D) (float64), the
+    initialisation the pages' rotations start from; D a power of two."""
+    H = np.ones((1, 1))
+    while H.shape[0] < D:
+        H = np.block([[H, H], [H, -H]])
+    return H * random_signs(D, seed)[None, :].astype(np.float64) / np.sqrt(D)
+
+
+def near_hadamard_pair(D: int, seed: int, n_planes: Optional[int] = None, theta0: float = 0.6,
+                       decay: float = 0.85):
+    """Two rotations R_in, R_out (float64 D x D) near the Hadamard start: R_in =
+    H_D diag(s) / sqrt(D), R_out = R_in G with G a product of commuting plane
+    rotations in the planes of an orthonormal D x 2m basis (QR of a Gaussian),
+    angles theta0 * decay^i (i < m, m = D/4 unless given): T = R_out R_in^T =
+    R_in G R_in^T deviates from I along few principal directions, with a
+    decaying tail, as the pages observe for Cayley-trained rotations."""
+    m = D // 4 if n_planes is None else n_planes
+    g = _rng(seed, _S_Q).standard_normal((D, 2 * m))
+    Ub, rr = np.linalg.qr(g)
+    Ub = Ub * np.where(np.diag(rr) < 0, -1.0, 1.0)[None, :]
+    th = theta0 * decay ** np.arange(m)
+    c, s = np.cos(th), np.sin(th)
+    u, v = Ub[:, 0::2], Ub[:, 1::2]
+    # G = I + sum_i (c_i - 1)(u u^T + v v^T) + s_i (v u^T - u v^T)
+    G = np.eye(D) + (u * (c - 1)) @ u.T + (v * (c - 1)) @ v.T + (v * s) @ u.T - (u * s) @ v.T
+    R_in = sylvester_signed(D, seed)
+    return R_in, R_in @ G
+
+
 def down_proj_gate_case(T: int = 4096) -> GateCase:
     """FFN down_proj with the gate fused: a, b ~ N(0, 1) in bf16, d=12288=1024*12, INT4."""
     return gate_case(T, 12288, 12, 2, dtype="bf16", bits=4, name=f"downproj_gate_T{T}_d12288")

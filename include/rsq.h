@@ -76,7 +76,7 @@ typedef enum {
     RSQ_ERR_ALIAS = 6,       /* buffers overlap other than x_out == x             */
     RSQ_ERR_UNSUPPORTED = 7, /* valid in principle but not built (e.g. m != 1, 12)*/
     RSQ_ERR_CUDA = 8,        /* a CUDA call failed; see rsq_last_cuda_error()     */
-    RSQ_ERR_VALUE = 9        /* eps negative or not finite                        */
+    RSQ_ERR_VALUE = 9        /* a scalar argument out of range (eps, iters, sizes)*/
 } rsq_status;
 
 typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1, RSQ_F16 = 2 } rsq_dtype;  /* RSQ_F16: w4a4_gemm output only */
@@ -189,6 +189,35 @@ int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t 
  * alignment as above. */
 int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *codes_w, const float *scales_w,
               void *y, int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream);
+
+/* Offline construction of the alignment's (Q, M) from the rotations on both
+ * sides of a residual connection.  ReSpinQuant paper notes, key design 2:
+ * T = R_out R_in^T; Q = the top-r left singular vectors of T - I (D x r,
+ * orthonormal, float32, Q[i*r + k]); T_sub = Q^T T Q; R_sub = the polar factor
+ * U V^T of T_sub (SVD T_sub = U S V^T), pulled into SO(r) by flipping the
+ * singular pair of the smallest singular value when det(U V^T) = -1;
+ * M = R_sub - I_r (r x r float32, row-major).  R_in, R_out: D x D float32,
+ * row-major, orthogonal up to rounding.  T - I is never formed: its products
+ * with D x p blocks come from the two inputs.  The subspace comes from `iters`
+ * steps (1..1000, RSQ_ERR_VALUE otherwise) of subspace iteration on
+ * (T - I)(T - I)^T with p = 64 (r <= 32) or 96 (r <= 64) columns and a
+ * Rayleigh-Ritz step; 8 to 20 steps suffice when the r-th and (r+1)-th
+ * singular values differ by 10 % or more.  Q is unique only up to rotations
+ * within equal singular values: the singular values of the deviation of a
+ * rotation come in pairs, so use an even r.  Float64 accumulation throughout.
+ * Shapes: D % 64 == 0, 64 <= D <= 16384, 1 <= r <= min(64, D/2)
+ * (RSQ_ERR_SHAPE).  workspace: device memory of at least
+ * rsq_qm_workspace_bytes(D, r) bytes (RSQ_ERR_VALUE if smaller), owned by the
+ * caller, 16-byte aligned; its contents on entry do not matter.  Outputs and
+ * workspace may not overlap the inputs or each other (RSQ_ERR_ALIAS).  Device
+ * status bits (rsq_device_status): 2 = a Gram matrix of the iteration was not
+ * positive definite (R_in or R_out not orthogonal, or T - I of rank below p),
+ * 4 = T_sub singular; the outputs are then invalid. */
+int rsq_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
+                 void *workspace, uint64_t workspace_bytes, void *stream);
+
+/* Workspace bytes rsq_qm_build needs for (D, r); 0 for an unsupported shape. */
+uint64_t rsq_qm_workspace_bytes(int D, int r);
 
 /* Human-readable name of an rsq_status value (static storage; never NULL). */
 const char *rsq_status_string(int status);

@@ -205,6 +205,30 @@ def test_w4a4_gemm_rejects(kw, want):
     assert rsq.launch_count() == before
 
 
+def _qm(ri=X, ro=XB, D=4096, r=32, it=16, q=Q, m=M, ws=C, wsb=1 << 30):
+    return L.rsq_qm_build(ri, ro, D, r, it, q, m, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(ri=None), NULL), (dict(ro=None), NULL), (dict(q=None), NULL), (dict(m=None), NULL), (dict(ws=None), NULL),
+    (dict(D=4000), SHAPE), (dict(D=32), SHAPE), (dict(D=32768), SHAPE), (dict(r=0), SHAPE), (dict(r=65), SHAPE),
+    (dict(D=64, r=33), SHAPE), (dict(it=0), VALUE), (dict(it=1001), VALUE), (dict(wsb=1024), VALUE),
+    (dict(ri=X + 4), ALIGN), (dict(ws=C + 8), ALIGN), (dict(q=X + 4096), ALIAS), (dict(ws=XB + 64), ALIAS),
+    (dict(m=Q + 256), ALIAS),
+])
+def test_qm_build_rejects(kw, want):
+    before = rsq.launch_count()
+    assert _qm(**kw) == want
+    assert rsq.launch_count() == before
+
+
+def test_qm_workspace_bytes():
+    assert L.rsq_qm_workspace_bytes(4000, 32) == 0 and L.rsq_qm_workspace_bytes(4096, 65) == 0
+    small, big = L.rsq_qm_workspace_bytes(256, 8), L.rsq_qm_workspace_bytes(4096, 32)
+    assert 0 < small < big < 64 << 20                                # a few D x 64 float64 blocks
+    assert L.rsq_qm_workspace_bytes(4096, 64) > big                  # 96 columns for r > 32
+
+
 def test_empty_batch_is_a_no_op():
     before = rsq.launch_count()
     assert _anq(x=None, xo=None, c=None, s=None, T=0) == OK

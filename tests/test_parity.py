@@ -706,6 +706,64 @@ def test_w4a4_gemm_full_size_sampled():
     run_gemm(c, "f16", with_acc=True, rows=_sample(16384, 24, seed=3))
 
 
+def run_qm(D, r, seed, iters=16, **kw):
+    rsq = _rsq()
+    R_in, R_out = inputs.near_hadamard_pair(D, seed, **kw)
+    Ri = torch.from_numpy(R_in.astype(np.float32)).to(DEV)
+    Ro = torch.from_numpy(R_out.astype(np.float32)).to(DEV)
+    Q, M = rsq.qm_build(Ri, Ro, r, iters=iters)
+    torch.cuda.synchronize()
+    assert rsq.device_status() == 0
+    # the oracle on the same float32 rotations the GPU read
+    ref = oracle.qm_construct(R_in.astype(np.float32), R_out.astype(np.float32), r)
+    return Q.cpu().numpy().astype(np.float64), M.cpu().numpy().astype(np.float64), ref
+
+
+# T_hat from the GPU's float32 (Q, M) against the oracle's float64 one: the
+# outputs are rounded once to float32 (relative 2^-24 on Q entries ~ 1/sqrt(D)
+# and on M entries <= 2), so T_hat entries differ by a few 1e-8; 2e-6 leaves
+# room for the subspace iteration's residual after `iters` steps.
+QM_TOL = 2e-6
+
+
+@pytest.mark.parametrize("D,r", [(128, 2), (256, 8), (256, 32), (512, 16), (1024, 64)])
+def test_qm_build_matches_the_oracle(D, r):
+    Q, M, ref = run_qm(D, r, D + r)
+    Th = oracle.t_hat(Q, M)
+    Th_ref = oracle.t_hat(ref["Q"], ref["M"])
+    np.testing.assert_allclose(Th, Th_ref, rtol=0, atol=QM_TOL)
+    np.testing.assert_allclose(Q.T @ Q, np.eye(r), rtol=0, atol=1e-6)      # orthonormal basis
+    np.testing.assert_allclose(Th.T @ Th, np.eye(D), rtol=0, atol=1e-5)    # a rotation (float32 outputs)
+    e_gpu = np.linalg.norm(Th - ref["T"])
+    e_ref = np.linalg.norm(Th_ref - ref["T"])
+    assert e_gpu <= e_ref * (1 + 1e-4) + 1e-5
+
+
+def test_qm_build_reproduces_an_exact_rank_deviation():
+    Q, M, ref = run_qm(256, 16, 5, n_planes=8)     # T - I of rank 16
+    np.testing.assert_allclose(oracle.t_hat(Q, M), ref["T"], rtol=0, atol=1e-5)
+
+
+def test_qm_build_full_size_feeds_the_alignment_kernels():
+    """D = 4096, r = 32 (the hidden stream's shape): T_hat against the oracle on
+    random directions, then the constructed (Q, M) through the alignment path on
+    the GPU against the oracle's path with the oracle's (Q, M)."""
+    rsq = _rsq()
+    Q, M, ref = run_qm(4096, 32, 77)
+    rng = np.random.default_rng(4)
+    V = rng.normal(size=(4096, 8))
+    np.testing.assert_allclose(V + Q @ (M @ (Q.T @ V)), V + ref["Q"] @ (ref["M"] @ (ref["Q"].T @ V)),
+                               rtol=0, atol=QM_TOL * np.abs(V).max() * 8)
+    a, _ = inputs.llama7b_case(T=200)
+    x = _to_dev(a.x, "bf16")
+    xo, codes, scales = rsq.rsq_align_norm_quant(x, torch.from_numpy(Q.astype(np.float32)).to(DEV),
+                                                 torch.from_numpy(M.astype(np.float32)).to(DEV), bits=4)
+    torch.cuda.synchronize()
+    r = oracle.align_norm_quant(a.x, ref["Q"].astype(np.float32), ref["M"].astype(np.float32), 4, a.eps)
+    H.check_aligned(_host(xo), r["x_out"], a.x, "bf16", "qm -> align")
+    H.check_codes(codes.cpu().numpy(), r["q"], r["pre"], 4, "qm -> align")
+
+
 @pytest.mark.parametrize("d,which", [(4096, 1), (4096, 3), (8192, 3)])
 def test_tiny_and_zero_rows_rht(d, which):
     rsq = _rsq()

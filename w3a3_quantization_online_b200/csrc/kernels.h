@@ -79,6 +79,12 @@ bool w4a4_gemm_supports(long long T, int N, int K);
 cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const uint8_t *codes_w, const float *sw,
                              void *y, int32_t *acc, long long T, int N, int K, int out_f16, cudaStream_t s);
 
+// Offline (Q, M) construction from two rotations; workspace from the caller.
+bool qm_supports(int D, int r);
+size_t qm_workspace_bytes(int D, int r);
+cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
+                            void *workspace, cudaStream_t s);
+
 // Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
 // (m = 1, bf16, INT4/INT3).
 bool rht_tc_supports(int d, int m, int dtype, int bits, long long T);

@@ -1,0 +1,482 @@
+// qm.cu -- the offline construction of the online alignment's (Q, M).
+//
+// ReSpinQuant paper notes, key design 2: at a residual connection the
+// transition T = R_out R_in^T between two layers' rotations stays close to I;
+// its deviation dT = T - I is decomposed by SVD, Q (D x r) takes the top-r left
+// singular vectors, T_sub = Q^T T Q is the transition inside that subspace,
+// and its polar factor U V^T, pulled back into SO(r), is R_sub; M = R_sub - I.
+//
+// Design: dT is never formed.  dT X = R_out (R_in^T X) - X and
+// dT^T X = R_in (R_out^T X) - X are skinny products with the two input
+// rotations (D x D float32, read as stored), so the workspace is a few D x p
+// blocks.  The top-r left singular subspace comes from subspace iteration on
+// dT dT^T with a block of p = 64 (r <= 32) or 96 (r <= 64) columns, each
+// iteration re-orthonormalised by CholeskyQR2, then a Rayleigh-Ritz step
+// (eigenvectors of (dT^T X)^T (dT^T X)) picks the r leading directions.
+// T_sub = (R_out^T Q)^T (R_in^T Q); its polar factor comes from the symmetric
+// eigen-decomposition T_sub^T T_sub = V S^2 V^T (well conditioned: T_sub is
+// close to a rotation): U = T_sub V S^-1, R_sub = U V^T, with the singular
+// pair of the smallest singular value flipped when det(R_sub) = -1.
+// All accumulation is float64 (the inputs are float32; Q and M are written as
+// float32).  The small dense steps (Cholesky, Jacobi eigen-decompositions,
+// the polar factor) run in one CTA each; the D-sized steps are tiled kernels.
+// No atomics: the result is bitwise reproducible.
+#include <algorithm>
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rsq {
+
+namespace {
+
+constexpr int kQmThreads = 256;
+constexpr int kGemmBM = 32, kGemmBN = 64, kGemmBK = 32;
+constexpr int kGramRows = 128;  // rows of X per partial Gram block
+
+// C[i][c] = sum_j op(A)[i][j] B[j][c] (- S[i][c]), A D x D float32 row-major
+// (op(A) = A or A^T), B, C, S D x ncols float64 with row stride ld.
+template <bool TRANS>
+__global__ void __launch_bounds__(kQmThreads)
+k_qm_gemm(const float *__restrict__ A, const double *__restrict__ B, double *__restrict__ C,
+          const double *__restrict__ S, int D, int ncols, int ld) {
+    __shared__ double sa[kGemmBK][kGemmBM + 1];  // sa[j][i] = op(A)[i0 + i][j0 + j]
+    __shared__ double sb[kGemmBK][kGemmBN];
+    const int tid = threadIdx.x;
+    const int i0 = blockIdx.x * kGemmBM, c0 = blockIdx.y * kGemmBN;
+    const int ty = tid >> 4, tx = tid & 15;  // rows ty, ty + 16; columns tx + 16 k
+    double acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+    for (int j0 = 0; j0 < D; j0 += kGemmBK) {
+        for (int e = tid; e < kGemmBM * kGemmBK; e += kQmThreads) {
+            if (TRANS) {  // op(A)[i][j] = A[j][i]: rows j of A, contiguous in i
+                const int jj = e / kGemmBM, ii = e % kGemmBM;
+                sa[jj][ii] = double(A[(size_t)(j0 + jj) * D + i0 + ii]);
+            } else {      // A[i][j], contiguous in j
+                const int ii = e / kGemmBK, jj = e % kGemmBK;
+                sa[jj][ii] = double(A[(size_t)(i0 + ii) * D + j0 + jj]);
+            }
+        }
+        for (int e = tid; e < kGemmBK * kGemmBN; e += kQmThreads) {
+            const int jj = e / kGemmBN, cc = e % kGemmBN;
+            sb[jj][cc] = c0 + cc < ncols ? B[(size_t)(j0 + jj) * ld + c0 + cc] : 0.0;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int jj = 0; jj < kGemmBK; ++jj) {
+            const double a0 = sa[jj][ty], a1 = sa[jj][ty + 16];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const double b = sb[jj][tx + 16 * k];
+                acc[0][k] = fma(a0, b, acc[0][k]);
+                acc[1][k] = fma(a1, b, acc[1][k]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = i0 + ty + 16 * h, c = c0 + tx + 16 * k;
+            if (c < ncols) C[(size_t)i * ld + c] = S ? acc[h][k] - S[(size_t)i * ld + c] : acc[h][k];
+        }
+}
+
+// Partial cross-Gram of a block of kGramRows rows: P[blk][a][b] = sum_i X[i][a] Y[i][b].
+__global__ void __launch_bounds__(kQmThreads)
+k_qm_gram(const double *__restrict__ X, const double *__restrict__ Y, double *__restrict__ P, int D, int p, int q,
+          int ld) {
+    const int blk = blockIdx.x;
+    const int r0 = blk * kGramRows, r1 = min(D, r0 + kGramRows);
+    for (int e = threadIdx.x; e < p * q; e += kQmThreads) {
+        const int a = e / q, b = e % q;
+        double s = 0.0;
+        for (int i = r0; i < r1; ++i) s = fma(X[(size_t)i * ld + a], Y[(size_t)i * ld + b], s);
+        P[(size_t)blk * p * q + e] = s;
+    }
+}
+
+// G = sum over blocks of P (fixed order).
+__global__ void k_qm_gram_reduce(const double *__restrict__ P, double *__restrict__ G, int nblk, int n) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n; e += gridDim.x * blockDim.x) {
+        double s = 0.0;
+        for (int b = 0; b < nblk; ++b) s += P[(size_t)b * n + e];
+        G[e] = s;
+    }
+}
+
+// out[i][c] = sum_j X[i][j] W[j][c], j < p (W p x q, row stride q); tri: W upper
+// triangular (only j <= c).
+__global__ void __launch_bounds__(kQmThreads)
+k_qm_apply(const double *__restrict__ X, const double *__restrict__ W, double *__restrict__ out, int D, int p, int q,
+           int ld_in, int ld_out, int tri) {
+    const long long n = (long long)D * q;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+        const int i = int(e / q), c = int(e % q);
+        const int jmax = tri ? c + 1 : p;
+        double s = 0.0;
+        for (int j = 0; j < jmax; ++j) s = fma(X[(size_t)i * ld_in + j], W[(size_t)j * q + c], s);
+        out[(size_t)i * ld_out + c] = s;
+    }
+}
+
+// Deterministic starting block: splitmix64 of the element index, mapped to [-1, 1).
+__global__ void k_qm_init(double *__restrict__ X, int D, int p, int ld) {
+    const long long n = (long long)D * p;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+        uint64_t z = uint64_t(e) + 0x9E3779B97F4A7C15ull;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        z ^= z >> 31;
+        X[(size_t)(e / p) * ld + e % p] = double(z >> 11) * 0x1p-52 - 1.0;
+    }
+}
+
+// ---- small dense linear algebra in one CTA (n <= 128), shared-memory matrices
+
+// Cyclic Jacobi on the symmetric n x n matrix a (row stride n): on return a is
+// (nearly) diagonal and v holds the eigenvectors in its columns.  Disjoint
+// pairs of one round-robin step rotate in parallel.  Fixed number of sweeps.
+__device__ void qm_jacobi(double *a, double *v, int n, double *cs, int *pr) {
+    const int tid = threadIdx.x;
+    for (int e = tid; e < n * n; e += blockDim.x) v[e] = (e / n == e % n) ? 1.0 : 0.0;
+    const int m = n + (n & 1);  // players of the round robin (one dummy when n is odd)
+    __syncthreads();
+    for (int sweep = 0; sweep < 12; ++sweep) {
+        for (int step = 0; step < m - 1; ++step) {
+            // pair k: players (k, m - 1 - k) of the rotated schedule
+            for (int k = tid; k < m / 2; k += blockDim.x) {
+                auto player = [&](int idx) { return idx == 0 ? 0 : 1 + (idx - 1 + step) % (m - 1); };
+                int p = player(k), q = player(m - 1 - k);
+                if (p > q) { const int t = p; p = q; q = t; }
+                pr[2 * k] = p;
+                pr[2 * k + 1] = q;
+                double c = 1.0, s = 0.0;
+                if (q < n) {
+                    const double apq = a[p * n + q];
+                    if (apq != 0.0) {
+                        const double theta = (a[q * n + q] - a[p * n + p]) / (2.0 * apq);
+                        const double t = (theta >= 0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+                        c = 1.0 / sqrt(t * t + 1.0);
+                        s = t * c;
+                    }
+                }
+                cs[2 * k] = c;
+                cs[2 * k + 1] = s;
+            }
+            __syncthreads();
+            // columns: a <- a J, v <- v J (J rotates columns p, q of each pair)
+            for (int e = tid; e < (m / 2) * n; e += blockDim.x) {
+                const int k = e / n, row = e % n;
+                const int p = pr[2 * k], q = pr[2 * k + 1];
+                if (q >= n) continue;
+                const double c = cs[2 * k], s = cs[2 * k + 1];
+                const double ap = a[row * n + p], aq = a[row * n + q];
+                a[row * n + p] = c * ap - s * aq;
+                a[row * n + q] = s * ap + c * aq;
+                const double vp = v[row * n + p], vq = v[row * n + q];
+                v[row * n + p] = c * vp - s * vq;
+                v[row * n + q] = s * vp + c * vq;
+            }
+            __syncthreads();
+            // rows: a <- J^T a
+            for (int e = tid; e < (m / 2) * n; e += blockDim.x) {
+                const int k = e / n, col = e % n;
+                const int p = pr[2 * k], q = pr[2 * k + 1];
+                if (q >= n) continue;
+                const double c = cs[2 * k], s = cs[2 * k + 1];
+                const double ap = a[p * n + col], aq = a[q * n + col];
+                a[p * n + col] = c * ap - s * aq;
+                a[q * n + col] = s * ap + c * aq;
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// Order of the eigenvalues (diagonal of a) from largest to smallest, ties by index.
+__device__ void qm_order_desc(const double *a, int n, int *order) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const double di = a[i * n + i];
+        int rank = 0;
+        for (int j = 0; j < n; ++j) {
+            const double dj = a[j * n + j];
+            rank += (dj > di) || (dj == di && j < i);
+        }
+        order[rank] = i;
+    }
+    __syncthreads();
+}
+
+// CHOL: G (p x p) = Rc^T Rc; out = Rc^-1 (upper triangular).  status bit 2 if G
+// is not positive definite.  One p x p shared array: the Cholesky factor L
+// (Rc = L^T) fills the lower triangle, then L^-1 is written transposed into the
+// strict upper triangle (entry (i, c), i > c, of L^-1 at (c, i)).
+__global__ void __launch_bounds__(kQmThreads) k_qm_chol_inv(const double *__restrict__ G, double *__restrict__ out,
+                                                            int p, int *status) {
+    extern __shared__ double sm[];
+    double *L = sm;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < p * p; e += blockDim.x) L[e] = G[e];
+    __shared__ int bad;
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    for (int j = 0; j < p; ++j) {  // right-looking Cholesky, column j (lower triangle only)
+        if (tid == 0) {
+            const double d = L[j * p + j];
+            if (!(d > 0.0)) bad = 1;
+            L[j * p + j] = d > 0.0 ? sqrt(d) : 1.0;
+        }
+        __syncthreads();
+        const double djj = L[j * p + j];
+        for (int i = j + 1 + tid; i < p; i += blockDim.x) L[i * p + j] /= djj;
+        __syncthreads();
+        const int w = p - j - 1;
+        for (int e = tid; e < w * w; e += blockDim.x) {
+            const int i = j + 1 + e / w, k = j + 1 + e % w;
+            if (k <= i) L[i * p + k] -= L[i * p + j] * L[k * p + j];
+        }
+        __syncthreads();
+    }
+    // column c of L^-1 by forward substitution (one column per thread); its
+    // entries below the diagonal go to row c of the strict upper triangle
+    for (int c = tid; c < p; c += blockDim.x) {
+        for (int i = c + 1; i < p; ++i) {
+            double s = -L[i * p + c] / L[c * p + c];
+            for (int k = c + 1; k < i; ++k) s -= L[i * p + k] * L[c * p + k];
+            L[c * p + i] = s / L[i * p + i];
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < p * p; e += blockDim.x) {  // Rc^-1 = (L^-1)^T: entry (i, c) = L^-1 (c, i)
+        const int i = e / p, c = e % p;
+        out[e] = i < c ? L[i * p + c] : (i == c ? 1.0 / L[c * p + c] : 0.0);
+    }
+    if (tid == 0 && bad) atomicOr(status, 2);
+}
+
+// EIG: S (p x p) symmetric -> W (p x r): eigenvectors of the r largest eigenvalues.
+__global__ void __launch_bounds__(kQmThreads) k_qm_top_eig(const double *__restrict__ S, double *__restrict__ W, int p,
+                                                           int r) {
+    extern __shared__ double sm[];
+    double *a = sm, *v = sm + p * p, *cs = sm + 2 * p * p;
+    int *pr = reinterpret_cast<int *>(cs + p + 2);
+    int *order = pr + p + 2;
+    for (int e = threadIdx.x; e < p * p; e += blockDim.x) a[e] = S[e];
+    __syncthreads();
+    qm_jacobi(a, v, p, cs, pr);
+    qm_order_desc(a, p, order);
+    for (int e = threadIdx.x; e < p * r; e += blockDim.x) {
+        const int j = e / r, c = e % r;
+        W[e] = v[j * p + order[c]];
+    }
+}
+
+// POLAR: T_sub (r x r) -> M = R_sub - I (float32, r x r row-major) with
+// R_sub = U V^T the polar factor in SO(r).
+__global__ void __launch_bounds__(kQmThreads) k_qm_polar(const double *__restrict__ Ts, float *__restrict__ M, int r,
+                                                         int *status) {
+    extern __shared__ double sm[];
+    double *t = sm, *a = sm + r * r, *v = sm + 2 * r * r, *u = sm + 3 * r * r, *rs = sm + 4 * r * r;
+    double *cs = rs + r * r;
+    int *pr = reinterpret_cast<int *>(cs + r + 2);
+    int *order = pr + r + 2;
+    __shared__ double sg[64];
+    __shared__ int neg;
+    const int tid = threadIdx.x;
+    for (int e = tid; e < r * r; e += blockDim.x) t[e] = Ts[e];
+    __syncthreads();
+    for (int e = tid; e < r * r; e += blockDim.x) {  // a = T^T T
+        const int i = e / r, j = e % r;
+        double s = 0.0;
+        for (int k = 0; k < r; ++k) s = fma(t[k * r + i], t[k * r + j], s);
+        a[e] = s;
+    }
+    __syncthreads();
+    qm_jacobi(a, v, r, cs, pr);
+    qm_order_desc(a, r, order);
+    for (int c = tid; c < r; c += blockDim.x) sg[c] = sqrt(fmax(a[c * r + c], 0.0));
+    __syncthreads();
+    for (int e = tid; e < r * r; e += blockDim.x) {  // u = T v diag(1/sigma)
+        const int i = e / r, c = e % r;
+        double s = 0.0;
+        for (int k = 0; k < r; ++k) s = fma(t[i * r + k], v[k * r + c], s);
+        u[e] = sg[c] > 0.0 ? s / sg[c] : 0.0;
+    }
+    __syncthreads();
+    for (int e = tid; e < r * r; e += blockDim.x) {  // R = U V^T
+        const int i = e / r, j = e % r;
+        double s = 0.0;
+        for (int k = 0; k < r; ++k) s = fma(u[i * r + k], v[j * r + k], s);
+        rs[e] = s;
+    }
+    __syncthreads();
+    // det(R) sign by Gaussian elimination with partial pivoting (one thread; r <= 64)
+    if (tid == 0) {
+        double *w = a;  // a is free now
+        for (int e = 0; e < r * r; ++e) w[e] = rs[e];
+        int sign = 1;
+        for (int c = 0; c < r; ++c) {
+            int piv = c;
+            for (int i = c + 1; i < r; ++i)
+                if (fabs(w[i * r + c]) > fabs(w[piv * r + c])) piv = i;
+            if (piv != c) {
+                sign = -sign;
+                for (int k = 0; k < r; ++k) {
+                    const double x = w[c * r + k];
+                    w[c * r + k] = w[piv * r + k];
+                    w[piv * r + k] = x;
+                }
+            }
+            const double d = w[c * r + c];
+            if (d < 0) sign = -sign;
+            if (d == 0.0) {
+                sign = 0;
+                break;
+            }
+            for (int i = c + 1; i < r; ++i) {
+                const double f = w[i * r + c] / d;
+                for (int k = c; k < r; ++k) w[i * r + k] -= f * w[c * r + k];
+            }
+        }
+        neg = sign < 0;
+        if (sign == 0) atomicOr(status, 4);
+    }
+    __syncthreads();
+    if (neg) {  // flip the singular pair of the smallest singular value
+        const int cmin = order[r - 1];
+        for (int e = tid; e < r * r; e += blockDim.x) {
+            const int i = e / r, j = e % r;
+            rs[e] -= 2.0 * u[i * r + cmin] * v[j * r + cmin];
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < r * r; e += blockDim.x) M[e] = float(rs[e] - ((e / r == e % r) ? 1.0 : 0.0));
+}
+
+__global__ void k_qm_out(const double *__restrict__ Qd, float *__restrict__ Q, int D, int r, int ld) {
+    const long long n = (long long)D * r;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+        Q[e] = float(Qd[(size_t)(e / r) * ld + e % r]);
+}
+
+struct QmWork {
+    double *X, *Y, *Z, *P, *G, *Wt;
+    int p, nblk;
+};
+
+size_t qm_layout(int D, int r, QmWork *w, void *base) {
+    const int p = r <= 32 ? 64 : 96;
+    const int nblk = (D + kGramRows - 1) / kGramRows;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    };
+    const size_t oX = take(size_t(D) * p * 8), oY = take(size_t(D) * p * 8), oZ = take(size_t(D) * p * 8);
+    const size_t oP = take(size_t(nblk) * p * p * 8), oG = take(size_t(p) * p * 8), oW = take(size_t(p) * p * 8);
+    if (w) {
+        char *b = static_cast<char *>(base);
+        w->X = reinterpret_cast<double *>(b + oX);
+        w->Y = reinterpret_cast<double *>(b + oY);
+        w->Z = reinterpret_cast<double *>(b + oZ);
+        w->P = reinterpret_cast<double *>(b + oP);
+        w->G = reinterpret_cast<double *>(b + oG);
+        w->Wt = reinterpret_cast<double *>(b + oW);
+        w->p = p;
+        w->nblk = nblk;
+    }
+    return off;
+}
+
+cudaError_t qm_check(int n) {
+    count_launch(n);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t qm_workspace_bytes(int D, int r) { return qm_layout(D, r, nullptr, nullptr); }
+
+bool qm_supports(int D, int r) { return D >= 64 && D <= 16384 && D % 64 == 0 && r >= 1 && r <= 64 && r <= D / 2; }
+
+cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
+                            void *workspace, cudaStream_t s) {
+    int *status = device_status_word();
+    if (!status) return cudaErrorInvalidDevice;
+    QmWork w;
+    qm_layout(D, r, &w, workspace);
+    const int p = w.p;
+    const int ew = int(std::min<long long>((long long)D * p / kQmThreads + 1, (long long)num_sms() * 8));
+    const dim3 ggrid(D / kGemmBM, (p + kGemmBN - 1) / kGemmBN);
+    const size_t chol_smem = size_t(p) * p * 8;
+    const size_t eig_smem = size_t(2) * p * p * 8 + size_t(p + 2) * 16 + size_t(2 * p + 4) * 4;
+    const size_t pol_smem = size_t(5) * r * r * 8 + size_t(r + 2) * 16 + size_t(2 * r + 4) * 4;
+    static bool configured[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        e = cudaFuncSetAttribute(k_qm_chol_inv, cudaFuncAttributeMaxDynamicSharedMemorySize, int(96 * 96 * 8));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_qm_top_eig, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(2 * 96 * 96 * 8 + 98 * 16 + 196 * 4));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_qm_polar, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(5 * 64 * 64 * 8 + 66 * 16 + 132 * 4));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    // X <- orthonormal basis of the columns of X (CholeskyQR, twice)
+    auto orth = [&](double *X, double *tmp) -> cudaError_t {
+        for (int rep = 0; rep < 2; ++rep) {
+            k_qm_gram<<<w.nblk, kQmThreads, 0, s>>>(X, X, w.P, D, p, p, p);
+            k_qm_gram_reduce<<<(p * p + 255) / 256, 256, 0, s>>>(w.P, w.G, w.nblk, p * p);
+            k_qm_chol_inv<<<1, kQmThreads, chol_smem, s>>>(w.G, w.Wt, p, status);
+            k_qm_apply<<<ew, kQmThreads, 0, s>>>(X, w.Wt, tmp, D, p, p, p, p, 1);
+            const cudaError_t e2 = qm_check(4);
+            if (e2 != cudaSuccess) return e2;
+            cudaMemcpyAsync(X, tmp, size_t(D) * p * 8, cudaMemcpyDeviceToDevice, s);
+        }
+        return cudaGetLastError();
+    };
+    // Y <- dT^T X = R_in (R_out^T X) - X, using Z as scratch
+    auto dtT = [&](const double *X, double *Y, double *Zs) {
+        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_out, X, Zs, nullptr, D, p, p);
+        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_in, Zs, Y, X, D, p, p);
+        return qm_check(2);
+    };
+    // Y <- dT X = R_out (R_in^T X) - X
+    auto dt = [&](const double *X, double *Y, double *Zs) {
+        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_in, X, Zs, nullptr, D, p, p);
+        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_out, Zs, Y, X, D, p, p);
+        return qm_check(2);
+    };
+    k_qm_init<<<ew, kQmThreads, 0, s>>>(w.X, D, p, p);
+    if ((e = qm_check(1)) != cudaSuccess) return e;
+    if ((e = orth(w.X, w.Y)) != cudaSuccess) return e;
+    for (int it = 0; it < iters; ++it) {
+        if ((e = dtT(w.X, w.Y, w.Z)) != cudaSuccess) return e;
+        if ((e = dt(w.Y, w.X, w.Z)) != cudaSuccess) return e;
+        if ((e = orth(w.X, w.Y)) != cudaSuccess) return e;
+    }
+    // Rayleigh-Ritz: S = (dT^T X)^T (dT^T X), top-r eigenvectors W, Q = X W (into Z)
+    if ((e = dtT(w.X, w.Y, w.Z)) != cudaSuccess) return e;
+    k_qm_gram<<<w.nblk, kQmThreads, 0, s>>>(w.Y, w.Y, w.P, D, p, p, p);
+    k_qm_gram_reduce<<<(p * p + 255) / 256, 256, 0, s>>>(w.P, w.G, w.nblk, p * p);
+    k_qm_top_eig<<<1, kQmThreads, eig_smem, s>>>(w.G, w.Wt, p, r);
+    k_qm_apply<<<ew, kQmThreads, 0, s>>>(w.X, w.Wt, w.Z, D, p, r, p, p, 0);  // Q in Z (row stride p)
+    if ((e = qm_check(4)) != cudaSuccess) return e;
+    // T_sub = (R_out^T Q)^T (R_in^T Q)
+    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_out, w.Z, w.X, nullptr, D, r, p);
+    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_in, w.Z, w.Y, nullptr, D, r, p);
+    k_qm_gram<<<w.nblk, kQmThreads, 0, s>>>(w.X, w.Y, w.P, D, r, r, p);
+    k_qm_gram_reduce<<<(r * r + 255) / 256, 256, 0, s>>>(w.P, w.G, w.nblk, r * r);
+    k_qm_polar<<<1, kQmThreads, pol_smem, s>>>(w.G, M, r, status);
+    k_qm_out<<<ew, kQmThreads, 0, s>>>(w.Z, Q, D, r, p);
+    return qm_check(6);
+}
+
+}  // namespace rsq

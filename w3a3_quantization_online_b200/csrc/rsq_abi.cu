@@ -352,6 +352,31 @@ int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *code
                                         static_cast<cudaStream_t>(stream)));
 }
 
+uint64_t rsq_qm_workspace_bytes(int D, int r) {
+    if (!rsq::qm_supports(D, r)) return 0;
+    return uint64_t(rsq::qm_workspace_bytes(D, r));
+}
+
+int rsq_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M, void *workspace,
+                 uint64_t workspace_bytes, void *stream) {
+    if (!rsq::qm_supports(D, r)) return RSQ_ERR_SHAPE;
+    if (iters < 1 || iters > 1000) return RSQ_ERR_VALUE;
+    if (!R_in || !R_out || !Q || !M || !workspace) return RSQ_ERR_NULL;
+    if (!aligned16(R_in) || !aligned16(R_out) || !aligned16(Q) || !aligned16(M) || !aligned16(workspace))
+        return RSQ_ERR_ALIGN;
+    const uint64_t need = uint64_t(rsq::qm_workspace_bytes(D, r));
+    if (workspace_bytes < need) return RSQ_ERR_VALUE;
+    const Span rin = span(R_in, uint64_t(D) * D * 4), rout = span(R_out, uint64_t(D) * D * 4);
+    const Span sq = span(Q, uint64_t(D) * r * 4), sm = span(M, uint64_t(r) * r * 4), sw = span(workspace, need);
+    const Span outs[3] = {sq, sm, sw};
+    for (int i = 0; i < 3; ++i) {
+        if (overlap(outs[i], rin) || overlap(outs[i], rout)) return RSQ_ERR_ALIAS;
+        for (int j = i + 1; j < 3; ++j)
+            if (overlap(outs[i], outs[j])) return RSQ_ERR_ALIAS;
+    }
+    return finish(rsq::launch_qm_build(R_in, R_out, D, r, iters, Q, M, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 const char *rsq_status_string(int status) {
     switch (status) {
         case RSQ_OK: return "RSQ_OK";
@@ -363,7 +388,7 @@ const char *rsq_status_string(int status) {
         case RSQ_ERR_ALIAS: return "RSQ_ERR_ALIAS: buffers overlap (only x_out == x is allowed)";
         case RSQ_ERR_UNSUPPORTED: return "RSQ_ERR_UNSUPPORTED: configuration not built";
         case RSQ_ERR_CUDA: return "RSQ_ERR_CUDA: a CUDA call failed (see rsq_last_cuda_error)";
-        case RSQ_ERR_VALUE: return "RSQ_ERR_VALUE: eps must be finite and >= 0";
+        case RSQ_ERR_VALUE: return "RSQ_ERR_VALUE: a scalar argument is out of range";
         default: return "unknown rsq status";
     }
 }

@@ -40,6 +40,10 @@ _lib.rht_head_mix_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, 
 _lib.rht_head_mix_quant.restype = _i32
 _lib.w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.w4a4_gemm.restype = _i32
+_lib.rsq_qm_build.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_uint64, _vp]
+_lib.rsq_qm_build.restype = _i32
+_lib.rsq_qm_workspace_bytes.argtypes = [_i32, _i32]
+_lib.rsq_qm_workspace_bytes.restype = ctypes.c_uint64
 _lib.rsq_status_string.argtypes = [_i32]
 _lib.rsq_status_string.restype = ctypes.c_char_p
 _lib.rsq_last_cuda_error.argtypes = []
@@ -56,7 +60,8 @@ _lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
 _lib.rsq_selftest_wait_timeout.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rht_heads",
-            "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "rsq_status_string",
+            "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "rsq_qm_build", "rsq_qm_workspace_bytes",
+            "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
 
@@ -297,3 +302,28 @@ def w4a4_gemm(codes_a: torch.Tensor, scales_a: torch.Tensor, codes_w: torch.Tens
     _check(_lib.w4a4_gemm(_ptr(codes_a), _ptr(scales_a), _ptr(codes_w), _ptr(scales_w), _ptr(y), _ptr(acc), T, N,
                           2 * kb, code, _stream(stream)))
     return y
+
+
+def qm_workspace_bytes(D: int, r: int) -> int:
+    return int(_lib.rsq_qm_workspace_bytes(D, r))
+
+
+def qm_build(R_in: torch.Tensor, R_out: torch.Tensor, r: int, iters: int = 16,
+             workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Offline (Q, M) of the alignment from the rotations on both sides of a residual connection.
+
+    Returns (Q D x r float32, M r x r float32).  workspace: a uint8 CUDA tensor of at
+    least qm_workspace_bytes(D, r) bytes (allocated here when None)."""
+    _need(R_in, "R_in", torch.float32); _need(R_out, "R_out", torch.float32)
+    D = R_in.shape[0]
+    need = qm_workspace_bytes(D, r)
+    if need == 0:
+        raise RsqError(2)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=R_in.device)
+    _need(workspace, "workspace", torch.uint8)
+    Q = torch.empty((D, r), dtype=torch.float32, device=R_in.device)
+    M = torch.empty((r, r), dtype=torch.float32, device=R_in.device)
+    _check(_lib.rsq_qm_build(_ptr(R_in), _ptr(R_out), D, r, iters, _ptr(Q), _ptr(M), _ptr(workspace),
+                             workspace.numel(), _stream(stream)))
+    return Q, M

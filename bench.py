@@ -101,8 +101,9 @@ def peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d.get("bf16_tflops", 1590.0)),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 def kernel_source_sha(files) -> str:
@@ -603,6 +604,97 @@ def kernel_metrics(dev, stream, workload: str, steps: int, warmup: int, pk: dict
     return kern
 
 
+def _time_loop(stream, fn, steps: int, warmup: int) -> float:
+    """Mean microseconds per call over `steps` back-to-back calls (CUDA events)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / steps
+
+
+def _hbm(byts: int, us: float, pk: dict, T: int, shape: str) -> dict:
+    gbs = byts / (us * 1e-6) / 1e9
+    return {"shape": shape, "avg_us": us, "bound": "hbm", "algorithmic_bytes_per_launch": byts, "achieved_gbs": gbs,
+            "frac": gbs / pk["hbm_gbs"], "tokens_per_s": T / (us * 1e-6)}
+
+
+def next_rows_metrics(dev, stream, pk: dict) -> dict:
+    """The rows beyond the online path's core (each bounded to well under a
+    second of GPU time): the SiLU-gated down_proj RHT, the attention-side
+    Hadamards, the W4A4 GEMM and the offline (Q, M) construction."""
+    import torch
+    from w3a3_quantization_online_b200 import inputs, rsq
+    out = {}
+    # gated down_proj input, T = 4096, d = 12288: fused gate vs rht_quant of a stored product
+    g = inputs.down_proj_gate_case(T=4096)
+    a, b = (torch.from_numpy(v).to(dev).to(torch.bfloat16) for v in (g.a, g.b))
+    sg = torch.from_numpy(g.signs).to(dev)
+    ch = torch.empty((g.T, g.d // 2), dtype=torch.uint8, device=dev)
+    sh = torch.empty((g.T,), dtype=torch.float32, device=dev)
+    us = _time_loop(stream, lambda: rsq.rht_quant_silu_gate(a, b, sg, 12, ch, sh, bits=4, stream=stream), 50, 3)
+    out["silu_gate_rht_quant"] = _hbm(g.T * (2 * g.d * 2 + g.d // 2 + 4) + g.d, us, pk, g.T,
+                                      "T=4096, d=12288 = 1024*12, a and b bf16 in, INT4 out")
+    del a, b, ch, sh
+    # attention: 16384 tokens x 32 heads x 128
+    c = inputs.attention_case(T=16384)
+    x = torch.from_numpy(c.x).to(dev).to(torch.bfloat16)
+    s = torch.from_numpy(c.signs).to(dev)
+    xo = torch.empty_like(x)
+    cq = torch.empty((c.T, c.d // 2), dtype=torch.uint8, device=dev)
+    sq = torch.empty((c.T, 32), dtype=torch.float32, device=dev)
+    st = torch.empty((c.T,), dtype=torch.float32, device=dev)
+    us = _time_loop(stream, lambda: rsq.rht_heads(x, s, 32, xo, stream=stream), 50, 3)
+    out["rht_heads"] = _hbm(c.T * c.d * 2 * 2 + c.d, us, pk, c.T, "T=16384, 32 heads x 128, bf16 in and out")
+    us = _time_loop(stream, lambda: rsq.rht_heads_quant(x, s, 32, cq, sq, bits=4, stream=stream), 50, 3)
+    out["rht_heads_quant"] = _hbm(c.T * (c.d * 2 + c.d // 2 + 32 * 4) + c.d, us, pk, c.T,
+                                  "T=16384, 32 heads x 128, INT4 per (token, head)")
+    us = _time_loop(stream, lambda: rsq.rht_head_mix_quant(x, s, 32, cq, st, bits=4, stream=stream), 50, 3)
+    out["rht_head_mix_quant"] = _hbm(c.T * (c.d * 2 + c.d // 2 + 4) + c.d, us, pk, c.T,
+                                     "T=16384, 32 heads x 128, INT4 per token")
+    del x, xo, cq, sq, st
+    # W4A4 GEMM: the hidden stream through a 4096 x 4096 INT4 projection
+    gm = inputs.gemm_case(16384, 4096, 4096, 21)
+    ca, cw = torch.from_numpy(gm.codes_a).to(dev), torch.from_numpy(gm.codes_w).to(dev)
+    sa, sw = torch.from_numpy(gm.scales_a).to(dev), torch.from_numpy(gm.scales_w).to(dev)
+    y = torch.empty((gm.T, gm.N), dtype=torch.float16, device=dev)
+    us = _time_loop(stream, lambda: rsq.w4a4_gemm(ca, sa, cw, sw, y=y, stream=stream), 20, 3)
+    ops = 2.0 * gm.T * gm.N * gm.K
+    peak_i8 = pk.get("bf16_tflops", 1590.0) * 2.0
+    out["w4a4_gemm"] = {"shape": "T=16384, N=4096, K=4096, INT4 x INT4 -> fp16", "avg_us": us, "bound": "tensor",
+                        "algorithmic_ops_per_launch": ops, "achieved_tops": ops / (us * 1e-6) / 1e12,
+                        "peak_tops": peak_i8, "frac": ops / (us * 1e-6) / 1e12 / peak_i8,
+                        "peak_source": "measured cuBLAS bf16 TFLOP/s (burst) x 2, the nominal int8 / bf16 dense ratio "
+                                       "(4.5 / 2.25 PFLOP/s)"}
+    del ca, cw, y
+    # offline (Q, M) construction, D = 4096, r = 32
+    R_in, R_out = inputs.near_hadamard_pair(4096, 77)
+    Ri = torch.from_numpy(R_in.astype(np.float32)).to(dev)
+    Ro = torch.from_numpy(R_out.astype(np.float32)).to(dev)
+    ws = torch.empty(rsq.qm_workspace_bytes(4096, 32), dtype=torch.uint8, device=dev)
+    iters = 16
+    us = _time_loop(stream, lambda: rsq.qm_build(Ri, Ro, 32, iters=iters, workspace=ws, stream=stream), 3, 1)
+    # float64 FMAs of the skinny products: per iteration and in the Ritz step 2 products with
+    # each rotation (D^2 p each), plus the T_sub products (2 D^2 r)
+    D, p_ = 4096, 64
+    flops = 2.0 * (4 * iters + 2) * D * D * p_ + 2.0 * 2 * D * D * 32
+    peak64 = 148 * 64 * 2 * 1.965e9 / 1e12
+    out["qm_build"] = {"shape": "D=4096, r=32, 16 iterations", "avg_ms": us / 1e3, "bound": "alu",
+                       "algorithmic_fp64_flops": flops, "achieved_tflops_fp64": flops / (us * 1e-6) / 1e12,
+                       "peak_tflops_fp64": peak64, "frac": flops / (us * 1e-6) / 1e12 / peak64,
+                       "peak_source": "148 SMs x 64 FP64 FMA/clock x 2 x 1.965 GHz (unit counts and max clock)"}
+    torch.cuda.empty_cache()
+    return out
+
+
 def secondary_metrics(dev, stream, pk: dict) -> dict:
     """The other configurations, bounded to a few seconds of GPU time: W3A3
     (T=8192, D=8192, INT3: alignment and RHT 2^13), the down_proj RHT
@@ -615,6 +707,7 @@ def secondary_metrics(dev, stream, pk: dict) -> dict:
     out["chain16"] = chain_metrics(dev, stream, 16, 50, 5, pk)
     out["chain16384"] = chain_metrics(dev, stream, 16384, 10, 3, pk)
     torch.cuda.empty_cache()
+    out.update(next_rows_metrics(dev, stream, pk))
     return out
 
 

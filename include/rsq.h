@@ -200,8 +200,10 @@ int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *code
  * row-major, orthogonal up to rounding.  T - I is never formed: its products
  * with D x p blocks come from the two inputs.  The subspace comes from `iters`
  * steps (1..1000, RSQ_ERR_VALUE otherwise) of subspace iteration on
- * (T - I)(T - I)^T with p = 64 (r <= 32) or 96 (r <= 64) columns and a
- * Rayleigh-Ritz step; 8 to 20 steps suffice when the r-th and (r+1)-th
+ * (T - I)(T - I)^T + mu I (mu a thousandth of the block's mean eigenvalue: it
+ * keeps the block at full rank when T - I has rank below p and leaves the
+ * leading subspace unchanged) with p = 64 (r <= 32) or 96 (r <= 64) columns and
+ * a Rayleigh-Ritz step; 8 to 20 steps suffice when the r-th and (r+1)-th
  * singular values differ by 10 % or more.  Q is unique only up to rotations
  * within equal singular values: the singular values of the deviation of a
  * rotation come in pairs, so use an even r.  Float64 accumulation throughout.
@@ -211,8 +213,8 @@ int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *code
  * caller, 16-byte aligned; its contents on entry do not matter.  Outputs and
  * workspace may not overlap the inputs or each other (RSQ_ERR_ALIAS).  Device
  * status bits (rsq_device_status): 2 = a Gram matrix of the iteration was not
- * positive definite (R_in or R_out not orthogonal, or T - I of rank below p),
- * 4 = T_sub singular; the outputs are then invalid. */
+ * positive definite (R_in or R_out far from orthogonal), 4 = T_sub singular;
+ * the outputs are then invalid. */
 int rsq_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
                  void *workspace, uint64_t workspace_bytes, void *stream);
 

@@ -64,11 +64,13 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&v)[8]) {
 
 // ---------------------------------------------------------------------------
 // Gated FFN product SiLU(a) * b = a * sigmoid(a) * b in fp32 (the down_proj
-// input), sigmoid(a) = 1 / (1 + e^-a).  For a below about -88, e^-a overflows
-// to +inf and the reciprocal gives 0, the limit of the product.
+// input), sigmoid(a) = 1 / (1 + e^-a), with CUDA's accurate expf (the fast
+// exponential's relative error grows with |a|, and a row of equal gates would
+// carry it straight into the scale).  For a below about -88, e^-a overflows to
+// +inf and the reciprocal gives 0, the limit of the product.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float silu_gate(float a, float b) {
-    return (a * __frcp_rn(1.0f + __expf(-a))) * b;
+    return (a * __frcp_rn(1.0f + expf(-a))) * b;
 }
 
 // ---------------------------------------------------------------------------

@@ -10,8 +10,11 @@
 // dT^T X = R_in (R_out^T X) - X are skinny products with the two input
 // rotations (D x D float32, read as stored), so the workspace is a few D x p
 // blocks.  The top-r left singular subspace comes from subspace iteration on
-// dT dT^T with a block of p = 64 (r <= 32) or 96 (r <= 64) columns, each
-// iteration re-orthonormalised by CholeskyQR2, then a Rayleigh-Ritz step
+// dT dT^T + mu I with a block of p = 64 (r <= 32) or 96 (r <= 64) columns
+// (mu = 1e-3 of the mean eigenvalue in the current block keeps the block at
+// full rank when dT has rank below p; it moves every eigenvalue alike, so the
+// leading subspace is the same), each iteration re-orthonormalised by
+// CholeskyQR2, then a Rayleigh-Ritz step
 // (eigenvectors of (dT^T X)^T (dT^T X)) picks the r leading directions.
 // T_sub = (R_out^T Q)^T (R_in^T Q); its polar factor comes from the symmetric
 // eigen-decomposition T_sub^T T_sub = V S^2 V^T (well conditioned: T_sub is
@@ -35,12 +38,14 @@ constexpr int kQmThreads = 256;
 constexpr int kGemmBM = 32, kGemmBN = 64, kGemmBK = 32;
 constexpr int kGramRows = 128;  // rows of X per partial Gram block
 
-// C[i][c] = sum_j op(A)[i][j] B[j][c] (- S[i][c]), A D x D float32 row-major
-// (op(A) = A or A^T), B, C, S D x ncols float64 with row stride ld.
+// C[i][c] = sum_j op(A)[i][j] B[j][c] (- S[i][c]) (+ mu P[i][c]), A D x D
+// float32 row-major (op(A) = A or A^T), B, C, S, P D x ncols float64 with row
+// stride ld, mu a device scalar.  C may be P (each element is read, then
+// written, by the same thread).
 template <bool TRANS>
 __global__ void __launch_bounds__(kQmThreads)
-k_qm_gemm(const float *__restrict__ A, const double *__restrict__ B, double *__restrict__ C,
-          const double *__restrict__ S, int D, int ncols, int ld) {
+k_qm_gemm(const float *__restrict__ A, const double *__restrict__ B, double *C, const double *__restrict__ S,
+          const double *P, const double *__restrict__ mu, int D, int ncols, int ld) {
     __shared__ double sa[kGemmBK][kGemmBM + 1];  // sa[j][i] = op(A)[i0 + i][j0 + j]
     __shared__ double sb[kGemmBK][kGemmBN];
     const int tid = threadIdx.x;
@@ -79,7 +84,11 @@ k_qm_gemm(const float *__restrict__ A, const double *__restrict__ B, double *__r
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int i = i0 + ty + 16 * h, c = c0 + tx + 16 * k;
-            if (c < ncols) C[(size_t)i * ld + c] = S ? acc[h][k] - S[(size_t)i * ld + c] : acc[h][k];
+            if (c < ncols) {
+                double v = S ? acc[h][k] - S[(size_t)i * ld + c] : acc[h][k];
+                if (P) v = fma(*mu, P[(size_t)i * ld + c], v);
+                C[(size_t)i * ld + c] = v;
+            }
         }
 }
 
@@ -95,6 +104,33 @@ k_qm_gram(const double *__restrict__ X, const double *__restrict__ Y, double *__
         for (int i = r0; i < r1; ++i) s = fma(X[(size_t)i * ld + a], Y[(size_t)i * ld + b], s);
         P[(size_t)blk * p * q + e] = s;
     }
+}
+
+// Partial sums of squares of a block of kGramRows rows of Y (D x p, row stride ld).
+__global__ void __launch_bounds__(kQmThreads)
+k_qm_sumsq(const double *__restrict__ Y, double *__restrict__ part, int D, int p, int ld) {
+    __shared__ double red[kQmThreads];
+    const int r0 = blockIdx.x * kGramRows, r1 = min(D, r0 + kGramRows);
+    double s = 0.0;
+    for (int e = threadIdx.x; e < (r1 - r0) * p; e += kQmThreads) {
+        const double v = Y[(size_t)(r0 + e / p) * ld + e % p];
+        s = fma(v, v, s);
+    }
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int h = kQmThreads / 2; h > 0; h >>= 1) {  // fixed tree
+        if (threadIdx.x < h) red[threadIdx.x] += red[threadIdx.x + h];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) part[blockIdx.x] = red[0];
+}
+
+// The shift of the iteration operator, mu = 1e-3 * ||Y||_F^2 / p (a thousandth
+// of the mean eigenvalue of X^T dT dT^T X), or 1 when Y = 0 (T = I).
+__global__ void k_qm_mu(const double *__restrict__ part, int nblk, int p, double *__restrict__ mu) {
+    double s = 0.0;
+    for (int b = 0; b < nblk; ++b) s += part[b];
+    *mu = s > 0.0 ? 1e-3 * s / double(p) : 1.0;
 }
 
 // G = sum over blocks of P (fixed order).
@@ -362,7 +398,7 @@ __global__ void k_qm_out(const double *__restrict__ Qd, float *__restrict__ Q, i
 }
 
 struct QmWork {
-    double *X, *Y, *Z, *P, *G, *Wt;
+    double *X, *Y, *Z, *P, *G, *Wt, *mu;
     int p, nblk;
 };
 
@@ -377,6 +413,7 @@ size_t qm_layout(int D, int r, QmWork *w, void *base) {
     };
     const size_t oX = take(size_t(D) * p * 8), oY = take(size_t(D) * p * 8), oZ = take(size_t(D) * p * 8);
     const size_t oP = take(size_t(nblk) * p * p * 8), oG = take(size_t(p) * p * 8), oW = take(size_t(p) * p * 8);
+    const size_t oM = take(8);
     if (w) {
         char *b = static_cast<char *>(base);
         w->X = reinterpret_cast<double *>(b + oX);
@@ -385,6 +422,7 @@ size_t qm_layout(int D, int r, QmWork *w, void *base) {
         w->P = reinterpret_cast<double *>(b + oP);
         w->G = reinterpret_cast<double *>(b + oG);
         w->Wt = reinterpret_cast<double *>(b + oW);
+        w->mu = reinterpret_cast<double *>(b + oM);
         w->p = p;
         w->nblk = nblk;
     }
@@ -444,22 +482,26 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     };
     // Y <- dT^T X = R_in (R_out^T X) - X, using Z as scratch
     auto dtT = [&](const double *X, double *Y, double *Zs) {
-        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_out, X, Zs, nullptr, D, p, p);
-        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_in, Zs, Y, X, D, p, p);
+        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_out, X, Zs, nullptr, nullptr, nullptr, D, p, p);
+        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_in, Zs, Y, X, nullptr, nullptr, D, p, p);
         return qm_check(2);
     };
-    // Y <- dT X = R_out (R_in^T X) - X
-    auto dt = [&](const double *X, double *Y, double *Zs) {
-        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_in, X, Zs, nullptr, D, p, p);
-        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_out, Zs, Y, X, D, p, p);
-        return qm_check(2);
+    // X <- dT Y + mu X = R_out (R_in^T Y) - Y + mu X: the shift mu > 0 keeps the
+    // block at full rank when dT has rank below p (the leading subspace does
+    // not change: the spectrum only moves by mu)
+    auto dt_shift = [&](const double *Y, double *X, double *Zs) {
+        k_qm_sumsq<<<w.nblk, kQmThreads, 0, s>>>(Y, w.P, D, p, p);
+        k_qm_mu<<<1, 1, 0, s>>>(w.P, w.nblk, p, w.mu);
+        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_in, Y, Zs, nullptr, nullptr, nullptr, D, p, p);
+        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_out, Zs, X, Y, X, w.mu, D, p, p);
+        return qm_check(4);
     };
     k_qm_init<<<ew, kQmThreads, 0, s>>>(w.X, D, p, p);
     if ((e = qm_check(1)) != cudaSuccess) return e;
     if ((e = orth(w.X, w.Y)) != cudaSuccess) return e;
     for (int it = 0; it < iters; ++it) {
         if ((e = dtT(w.X, w.Y, w.Z)) != cudaSuccess) return e;
-        if ((e = dt(w.Y, w.X, w.Z)) != cudaSuccess) return e;
+        if ((e = dt_shift(w.Y, w.X, w.Z)) != cudaSuccess) return e;
         if ((e = orth(w.X, w.Y)) != cudaSuccess) return e;
     }
     // Rayleigh-Ritz: S = (dT^T X)^T (dT^T X), top-r eigenvectors W, Q = X W (into Z)
@@ -470,8 +512,8 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     k_qm_apply<<<ew, kQmThreads, 0, s>>>(w.X, w.Wt, w.Z, D, p, r, p, p, 0);  // Q in Z (row stride p)
     if ((e = qm_check(4)) != cudaSuccess) return e;
     // T_sub = (R_out^T Q)^T (R_in^T Q)
-    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_out, w.Z, w.X, nullptr, D, r, p);
-    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_in, w.Z, w.Y, nullptr, D, r, p);
+    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_out, w.Z, w.X, nullptr, nullptr, nullptr, D, r, p);
+    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_in, w.Z, w.Y, nullptr, nullptr, nullptr, D, r, p);
     k_qm_gram<<<w.nblk, kQmThreads, 0, s>>>(w.X, w.Y, w.P, D, r, r, p);
     k_qm_gram_reduce<<<(r * r + 255) / 256, 256, 0, s>>>(w.P, w.G, w.nblk, r * r);
     k_qm_polar<<<1, kQmThreads, pol_smem, s>>>(w.G, M, r, status);

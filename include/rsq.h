@@ -221,6 +221,28 @@ int rsq_qm_build(const float *R_in, const float *R_out, int D, int r, int iters,
 /* Workspace bytes rsq_qm_build needs for (D, r); 0 for an unsupported shape. */
 uint64_t rsq_qm_workspace_bytes(int D, int r);
 
+/* rsq_qm_build for callers that cannot allocate device memory.  Some callers
+ * cannot call cudaMalloc or take a workspace from anywhere: a plugin running
+ * inside a host application whose memory pool already owns the device memory,
+ * or code on a latency-critical path where cudaMalloc's implicit device-wide
+ * synchronisation is not acceptable.  This entry point uses a scratch array
+ * that is part of the library itself: 8 MiB of device memory that every GPU on
+ * which the library is loaded holds until the process exits.  It allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library call).  Shapes whose
+ * workspace (rsq_qm_workspace_bytes) exceeds 8 MiB are rejected with
+ * RSQ_ERR_SHAPE: r <= 32 fits up to D = 4608, r > 32 up to D = 2816.  The
+ * first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call on a device shares the one array, and the
+ * array keeps the last call's contents (the kernels write every scratch byte
+ * before they read it, so no clearing is needed): calls whose work overlaps on
+ * the GPU (two streams, or two host threads) race and give wrong results;
+ * serialise them.  Arguments, outputs and errors otherwise as rsq_qm_build.
+ * The pages have no counterpart: this is a deployment variant, not a step of
+ * the method. */
+int rsq_qm_build_fixed_scratch(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
+                               void *stream);
+
 /* Human-readable name of an rsq_status value (static storage; never NULL). */
 const char *rsq_status_string(int status);
 

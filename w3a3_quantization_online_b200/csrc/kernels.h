@@ -84,6 +84,10 @@ bool qm_supports(int D, int r);
 size_t qm_workspace_bytes(int D, int r);
 cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
                             void *workspace, cudaStream_t s);
+// The library's own fixed scratch array for the construction (size, and its
+// device address on the current device: obtained once per device).
+size_t qm_static_scratch_bytes();
+cudaError_t qm_static_scratch(void **ptr);
 
 // Randomised Hadamard of order 4096 or 8192 with the first stage on tcgen05
 // (m = 1, bf16, INT4/INT3).

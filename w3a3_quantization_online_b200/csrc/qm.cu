@@ -438,6 +438,34 @@ cudaError_t qm_check(int n) {
 
 size_t qm_workspace_bytes(int D, int r) { return qm_layout(D, r, nullptr, nullptr); }
 
+// ---- the variant that allocates nothing: a fixed scratch array in the
+// library's device image (every GPU that loads the library holds it until the
+// process exits).  Host code only ever sees the array's host-side stand-in; the
+// device address comes from cudaGetSymbolAddress, once per device, with that
+// device current.
+namespace {
+constexpr size_t kQmStaticBytes = size_t(8) << 20;  // 8 MiB: D <= 4608 at r <= 32, D <= 2816 above
+static __device__ __align__(256) unsigned char g_qm_scratch[kQmStaticBytes];
+}  // namespace
+
+size_t qm_static_scratch_bytes() { return kQmStaticBytes; }
+
+cudaError_t qm_static_scratch(void **ptr) {
+    static void *addr[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_qm_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
+
 bool qm_supports(int D, int r) { return D >= 64 && D <= 16384 && D % 64 == 0 && r >= 1 && r <= 64 && r <= D / 2; }
 
 cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,

@@ -377,6 +377,23 @@ int rsq_qm_build(const float *R_in, const float *R_out, int D, int r, int iters,
     return finish(rsq::launch_qm_build(R_in, R_out, D, r, iters, Q, M, workspace, static_cast<cudaStream_t>(stream)));
 }
 
+int rsq_qm_build_fixed_scratch(const float *R_in, const float *R_out, int D, int r, int iters, float *Q, float *M,
+                               void *stream) {
+    if (!rsq::qm_supports(D, r)) return RSQ_ERR_SHAPE;
+    if (rsq::qm_workspace_bytes(D, r) > rsq::qm_static_scratch_bytes()) return RSQ_ERR_SHAPE;
+    if (iters < 1 || iters > 1000) return RSQ_ERR_VALUE;
+    if (!R_in || !R_out || !Q || !M) return RSQ_ERR_NULL;
+    if (!aligned16(R_in) || !aligned16(R_out) || !aligned16(Q) || !aligned16(M)) return RSQ_ERR_ALIGN;
+    const Span rin = span(R_in, uint64_t(D) * D * 4), rout = span(R_out, uint64_t(D) * D * 4);
+    const Span sq = span(Q, uint64_t(D) * r * 4), sm = span(M, uint64_t(r) * r * 4);
+    if (overlap(sq, rin) || overlap(sq, rout) || overlap(sm, rin) || overlap(sm, rout) || overlap(sq, sm))
+        return RSQ_ERR_ALIAS;
+    void *scratch = nullptr;
+    const cudaError_t e = rsq::qm_static_scratch(&scratch);
+    if (e != cudaSuccess) return finish(e);
+    return finish(rsq::launch_qm_build(R_in, R_out, D, r, iters, Q, M, scratch, static_cast<cudaStream_t>(stream)));
+}
+
 const char *rsq_status_string(int status) {
     switch (status) {
         case RSQ_OK: return "RSQ_OK";

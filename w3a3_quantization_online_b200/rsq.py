@@ -43,6 +43,8 @@ _lib.w4a4_gemm.restype = _i32
 _lib.rsq_qm_build.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_uint64, _vp]
 _lib.rsq_qm_build.restype = _i32
 _lib.rsq_qm_workspace_bytes.argtypes = [_i32, _i32]
+_lib.rsq_qm_build_fixed_scratch.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.rsq_qm_build_fixed_scratch.restype = _i32
 _lib.rsq_qm_workspace_bytes.restype = ctypes.c_uint64
 _lib.rsq_status_string.argtypes = [_i32]
 _lib.rsq_status_string.restype = ctypes.c_char_p
@@ -61,6 +63,7 @@ _lib.rsq_selftest_wait_timeout.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rht_heads",
             "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "rsq_qm_build", "rsq_qm_workspace_bytes",
+            "rsq_qm_build_fixed_scratch",
             "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
@@ -326,4 +329,18 @@ def qm_build(R_in: torch.Tensor, R_out: torch.Tensor, r: int, iters: int = 16,
     M = torch.empty((r, r), dtype=torch.float32, device=R_in.device)
     _check(_lib.rsq_qm_build(_ptr(R_in), _ptr(R_out), D, r, iters, _ptr(Q), _ptr(M), _ptr(workspace),
                              workspace.numel(), _stream(stream)))
+    return Q, M
+
+
+def qm_build_fixed_scratch(R_in: torch.Tensor, R_out: torch.Tensor, r: int, iters: int = 16,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """qm_build on the library's own fixed scratch array (no workspace argument).
+
+    Shapes whose workspace exceeds the array are rejected; calls whose work
+    overlaps on the GPU share the array and must be serialised."""
+    _need(R_in, "R_in", torch.float32); _need(R_out, "R_out", torch.float32)
+    D = R_in.shape[0]
+    Q = torch.empty((D, r), dtype=torch.float32, device=R_in.device)
+    M = torch.empty((r, r), dtype=torch.float32, device=R_in.device)
+    _check(_lib.rsq_qm_build_fixed_scratch(_ptr(R_in), _ptr(R_out), D, r, iters, _ptr(Q), _ptr(M), _stream(stream)))
     return Q, M

@@ -258,7 +258,8 @@ uint64_t rsq_launch_count(void);
  * bf16, D in {4096, 8192} and r <= 32, the tensor-core cluster kernel; the
  * CUDA-core kernel for everything else), 1 = always the CUDA-core kernel,
  * 2 = only the tensor-core cluster kernel, 4 = only the decode kernel (2 and 4
- * return RSQ_ERR_UNSUPPORTED for calls they cannot serve).  Process-wide;
+ * return RSQ_ERR_UNSUPPORTED for calls they cannot serve; 3 is not a valid
+ * choice).  Process-wide;
  * returns the previous setting, or -1 for an invalid value.  All compute the
  * same function; this exists for testing and measurement. */
 int rsq_select_align_kernel(int which);

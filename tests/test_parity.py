@@ -362,7 +362,7 @@ def test_generic_kernel_at_the_tensor_core_shapes(generic_align, T):
     check_align(a, label=f"generic w3a3 T={T}")
 
 
-@pytest.mark.parametrize("which", [2, 3])
+@pytest.mark.parametrize("which", [2])
 def test_tensor_core_kernel_serves_the_hot_shapes(which):
     rsq = _rsq()
     prev = rsq.select_align_kernel(which)
@@ -792,7 +792,7 @@ def test_residual_align_only_matches_oracle():
         H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, dtype, f"align {dtype}")
 
 
-@pytest.mark.parametrize("which", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("which", [0, 1, 2, 4])
 def test_residual_align_kernels(which):
     """rsq_residual_align through the decode kernel (small T), the tensor-core
     kernel (bf16, D = 4096 / 8192) and the CUDA-core kernel, each without the
@@ -804,7 +804,6 @@ def test_residual_align_kernels(which):
         shapes = {0: [(1, 4096), (16, 4096), (17, 4096), (1000, 4096), (300, 8192)],
                   1: [(16, 4096), (300, 4096)],
                   2: [(1, 4096), (200, 4096), (3001, 4096), (129, 8192)],
-                  3: [(1, 4096), (65, 4096), (200, 4096), (3001, 4096), (129, 8192)],
                   4: [(1, 4096), (16, 4096), (32, 2048), (31, 8192)]}[which]
         for T, D in shapes:
             a = inputs.align_case(T, D, 32, T + D, dtype="bf16", n_outliers=8, outlier_scale=100.0)

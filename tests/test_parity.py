@@ -621,6 +621,44 @@ def test_head_mix_quant(n_heads, d_head, dtype, bits):
     check_head_mix(c, n_heads, False, label=f"head mix {n_heads}x{d_head} no signs")
 
 
+@pytest.mark.parametrize("which", [3, 1])
+@pytest.mark.parametrize("n_heads,d_head,T", [(32, 128, 600), (16, 64, 600), (32, 128, 1), (3, 128, 1000)])
+def test_heads_tensor_core_and_cuda_core_kernels(which, n_heads, d_head, T):
+    """rht_heads / rht_heads_quant through the tensor-core per-head kernel
+    (which = 3; 128-token tiles, a ragged last tile, CTA ranges that cross a
+    head boundary) and through the CUDA-core kernel (which = 1), bf16, each
+    against the oracle."""
+    rsq = _rsq()
+    prev = rsq.select_rht_kernel(which)
+    try:
+        for bits in (4, 3):
+            c = inputs.rht_case(T, n_heads * d_head, 1, T + n_heads + bits, dtype="bf16", bits=bits, n_outliers=3,
+                                outlier_scale=20.0)
+            if T > 7:
+                c.x[7, d_head:2 * d_head] = 0.0  # a zero head
+            x = _to_dev(c.x, "bf16")
+            s = torch.from_numpy(c.signs).to(DEV)
+            out = rsq.rht_heads(x, s, n_heads)
+            torch.cuda.synchronize()
+            H.check_aligned(_host(out), oracle.head_rht(c.x, c.signs, n_heads), c.x, "bf16",
+                            f"heads kernel {which} {n_heads}x{d_head} T={T}")
+            check_heads_quant(c, n_heads, True, label=f"heads quant kernel {which} {n_heads}x{d_head} T={T} b={bits}")
+        assert rsq.device_status() == 0
+    finally:
+        rsq.select_rht_kernel(prev)
+
+
+def test_heads_tensor_core_kernel_rejects_other_shapes():
+    rsq = _rsq()
+    prev = rsq.select_rht_kernel(3)
+    try:
+        x = torch.zeros((4, 3 * 256), dtype=torch.bfloat16, device=DEV)
+        with pytest.raises(rsq.RsqError):
+            rsq.rht_heads(x, None, 3)
+    finally:
+        rsq.select_rht_kernel(prev)
+
+
 def test_attention_transforms_full_size_sampled():
     """T = 16384 tokens of 32 x 128 attention activations: per-head rotation,
     per-head key quantisation and head mixing with per-token quantisation, in

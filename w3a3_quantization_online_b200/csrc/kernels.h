@@ -67,6 +67,10 @@ cudaError_t launch_head_rht(const void *x, const int8_t *signs, void *x_out, uin
                             long long T, int d, int n_heads, int bits, bool quant, int dtype, cudaStream_t s);
 cudaError_t launch_head_mix(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
                             int n_heads, int bits, int dtype, cudaStream_t s);
+// The same per-head rotation / quantisation on the tensor cores (bf16, d_h in {64, 128}).
+bool head_tc_supports(int d, int n_heads, int dtype, long long T);
+cudaError_t launch_head_tc(const void *x, const int8_t *signs, void *x_out, uint8_t *codes, float *scales,
+                           long long T, int d, int n_heads, int bits, bool quant, cudaStream_t s);
 
 // INT4 consumer GEMM: y = round16(float(codes_a codes_w^T) * sa[t] * sw[n]),
 // fp16 (out_f16) or bf16 out, optional raw int32 accumulators.

@@ -271,6 +271,11 @@ int rht_heads(const void *x, const int8_t *signs, int n_heads, void *x_out, int6
     const Span sx = span(x, bytes), so = span(x_out, bytes);
     if (x != x_out && overlap(sx, so)) return RSQ_ERR_ALIAS;
     if (signs && overlap(so, span(signs, uint64_t(d)))) return RSQ_ERR_ALIAS;
+    const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
+    if (which != 1 && rsq::head_tc_supports(d, n_heads, dtype, T))
+        return finish(rsq::launch_head_tc(x, signs, x_out, nullptr, nullptr, T, d, n_heads, 4, false,
+                                          static_cast<cudaStream_t>(stream)));
+    if (which == 3) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_head_rht(x, signs, x_out, nullptr, nullptr, T, d, n_heads, 4, false, dtype,
                                        static_cast<cudaStream_t>(stream)));
 }
@@ -291,6 +296,11 @@ int rht_heads_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *co
         const Span sg = span(signs, uint64_t(d));
         if (overlap(sc, sg) || overlap(ss, sg)) return RSQ_ERR_ALIAS;
     }
+    const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
+    if (which != 1 && rsq::head_tc_supports(d, n_heads, dtype, T))
+        return finish(rsq::launch_head_tc(x, signs, nullptr, codes, scales, T, d, n_heads, bits, true,
+                                          static_cast<cudaStream_t>(stream)));
+    if (which == 3) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_head_rht(x, signs, nullptr, codes, scales, T, d, n_heads, bits, true, dtype,
                                        static_cast<cudaStream_t>(stream)));
 }

@@ -168,7 +168,7 @@ int rht_heads_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *co
  * symmetric absmax quantisation and packing as for rht_quant
  * (scales[t] = max_i |v_ti| / qmax).  n_heads a power of two in [2, 64];
  * d % 16 == 0; d_h = d / n_heads (any, it is the stride) with
- * d_h <= 512 (n_heads <= 16) or d_h <= 256 (n_heads >= 32). */
+ * d_h <= 512 (n_heads <= 32) or d_h <= 256 (n_heads = 64). */
 int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales,
                        int64_t T, int d, int bits, int dtype, void *stream);
 

@@ -20,11 +20,12 @@
 // positive row factor).
 //
 // k_head_mix: one CTA per token row at a time; thread t owns JP consecutive
-// columns j of every head (JP = 2, or 1 from 32 heads), i.e. JP * n_h values,
+// columns j of every head (JP = 2, or 1 for 64 heads), i.e. JP * n_h values,
 // and runs the n_h-point transform in registers.  Loads of one head are 4 or 2
 // bytes per thread, contiguous over the warp.  The row absmax is a block
 // reduction; the int8 codes are staged in shared memory and packed 8 at a time
-// (INT4 words or INT3 24-bit groups).
+// (INT4 words or INT3 24-bit groups).  The signs are read once per thread into a
+// bit mask per column.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -131,6 +132,16 @@ k_head_mix(const typename IO::T *__restrict__ x, const int8_t *__restrict__ sign
     const int qmax = (1 << (bits - 1)) - 1;
     const long long row_bytes = (long long)d * bits / 8;
     const float inv_sqrt = rsqrtf(float(NH));
+    // this thread's signs (the same for every row) as bit masks, one per column
+    uint64_t neg[JP];
+#pragma unroll
+    for (int q = 0; q < JP; ++q) {
+        neg[q] = 0;
+        if (own && signs)
+#pragma unroll
+            for (int h = 0; h < NH; ++h)
+                if (signs[h * dh + j0 + q] < 0) neg[q] |= uint64_t(1) << h;
+    }
 
     for (long long t = blockIdx.x; t < T; t += gridDim.x) {
         float v[NH][JP];
@@ -140,9 +151,8 @@ k_head_mix(const typename IO::T *__restrict__ x, const int8_t *__restrict__ sign
             for (int h = 0; h < NH; ++h)
 #pragma unroll
                 for (int q = 0; q < JP; ++q) {
-                    float f = IO::to_f(xr[h * dh + q]);
-                    if (signs && signs[h * dh + j0 + q] < 0) f = -f;
-                    v[h][q] = f;
+                    const float f = IO::to_f(xr[h * dh + q]);
+                    v[h][q] = (neg[q] >> h) & 1 ? -f : f;
                 }
         } else {
 #pragma unroll
@@ -213,7 +223,7 @@ cudaError_t launch_head_rht_typed(const void *x, const int8_t *signs, void *x_ou
 template <class IO, int NH>
 cudaError_t launch_head_mix_nh(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
                                int dh, int bits, cudaStream_t s) {
-    constexpr int JP = NH >= 32 ? 1 : 2;
+    constexpr int JP = NH >= 64 ? 1 : 2;
     const int threads = ((dh / JP + 31) / 32) * 32;
     const size_t smem = size_t(NH) * dh;
     auto kern = k_head_mix<IO, NH, JP>;
@@ -254,7 +264,7 @@ bool head_rht_supports(int d, int n_heads) {
 bool head_mix_supports(int d, int n_heads) {
     if (n_heads < 2 || n_heads > 64 || (n_heads & (n_heads - 1)) || d % n_heads) return false;
     const int dh = d / n_heads;
-    const int jp = n_heads >= 32 ? 1 : 2;
+    const int jp = n_heads >= 64 ? 1 : 2;
     return dh % jp == 0 && dh / jp <= kHeadThreads && d % 8 == 0;
 }
 

@@ -305,8 +305,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         if (tid == 0 && has_tile(0)) {
 #pragma unroll 1
             for (int s = 0; s < kSlabs; ++s) {
+                if (err) break;  // no arming without the load that completes it
                 mbar_expect_tx(bar(kBarLd + s), slab_tx);
-                if (!err) tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(0)),
+                tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, int(tile_t0(0)),
                             bar(kBarLd + s));
             }
         }
@@ -429,7 +430,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (lane < CS && lane != int(crank))
                     if (!err) bulk_copy_to_cluster(mapa(row_addr, uint32_t(lane)), row_addr, 128u,
                                          mapa(bar(kBarZ), uint32_t(lane)));
-                if (lane == 0) mbar_arrive(bar(kBarZ));
+                if (lane == 0 && !err) mbar_arrive(bar(kBarZ));
             }
 
             // ---- c = z Q^T (hi/lo split): quarter q into TMEM columns [128 q, 128 q + 128),
@@ -437,7 +438,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
             // last anyway), so that parts 0-2 start pass 1 as soon as theirs is done
             if (warp == kMma2Warp && lane == 0) {
                 if (!mbar_wait(bar(kBarZ), ph, err != 0)) err |= kErrMbarTimeout;
-                if (next) mbar_expect_tx(bar(kBarZ), uint32_t(kZTx));
+                if (next && !err) mbar_expect_tx(bar(kBarZ), uint32_t(kZTx));
                 tc_fence_after();
                 fence_proxy_async();
                 const uint64_t ad0 = opaque(smem_desc_sw128(smem_u32(sz), 1024));
@@ -515,8 +516,9 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 #pragma unroll 1
                         for (int s = 0; s < kSlabs; ++s) {
                             bulk_wait_read_n(kSlabs - 1 - s);
+                            if (err) break;  // no arming without the load that completes it
                             mbar_expect_tx(bar(kBarLd + s), slab_tx);
-                            if (!err) tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, tn,
+                            tma_load_2d(smem_u32(sx + s * kSlabBytes), &tm_x, col0 + s * kSlabCols, tn,
                                         bar(kBarLd + s));
                         }
                     }
@@ -557,10 +559,10 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                 if (dst_cta == 0 && mo < nrows) p.scales[t0 + mo] = am_t > 0.f ? (am_t * rs) / float(qmax) : 0.f;
                 if (!err) st_async_v2(mapa(smem_u32(sprm + mo * 8), uint32_t(dst_cta)), __float_as_uint(q.inv),
                             __float_as_uint(q.pre), mapa(bar(kBarPrm), uint32_t(dst_cta)));
-                if (tid == 0 && next) mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
+                if (tid == 0 && next && !err) mbar_expect_tx(bar(kBarSt), uint32_t(CS * TPO * 16));
             }
             if (!mbar_wait(bar(kBarPrm), ph, err != 0)) err |= kErrMbarTimeout;
-            if (tid == 0 && next) mbar_expect_tx(bar(kBarPrm), uint32_t(kTileM * 8));
+            if (tid == 0 && next && !err) mbar_expect_tx(bar(kBarPrm), uint32_t(kTileM * 8));
             RowQuant rq;
             rq.inv = reinterpret_cast<const float *>(sprm + m * 8)[0];
             rq.pre = reinterpret_cast<const float *>(sprm + m * 8)[1];

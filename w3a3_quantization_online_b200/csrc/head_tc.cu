@@ -161,11 +161,12 @@ k_head_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
             for (int k = 0; k < nk; ++k) {
                 const int st = k % kStages;
                 if (k >= kStages) wait(kBarEmpty + st, uint32_t(k / kStages - 1) & 1u);
+                if (err) break;  // no arming without the loads that complete it
                 mbar_expect_tx(bar(kBarFull + st), kTx);
                 const int c0 = head_of(k) * DH, r0 = tok0_of(k);
 #pragma unroll
                 for (int s = 0; s < kSlabs; ++s)
-                    if (!err) tma_load_2d(smem_u32(xs(st) + s * kTok * 128), &tm_x, c0 + 64 * s, r0, bar(kBarFull + st));
+                    tma_load_2d(smem_u32(xs(st) + s * kTok * 128), &tm_x, c0 + 64 * s, r0, bar(kBarFull + st));
             }
         }
         __syncwarp();

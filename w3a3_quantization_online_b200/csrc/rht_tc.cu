@@ -212,9 +212,9 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     // others by the epilogue of the group that last used the stage
     auto load_group = [&](int it) {
         const int s = it % kStages;
+        if (err) return;  // no arming without the load that completes it
         mbar_expect_tx(bar_full + 8 * s, kStageBytes);
-        if (!err) tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok),
-                              bar_full + 8 * s);
+        tma_load_3d(smem_u32(sstage + s * kStageBytes), &tm_x, 0, 0, int((g0 + it * gstep) * kTok), bar_full + 8 * s);
     };
     if (tid == 0)
         for (int it = 0; it < kStages && it < nmine; ++it) load_group(it);

@@ -170,11 +170,10 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
             for (int ks = 0; ks < KS; ++ks) {
                 const int s = ks % kP;
                 if (!mbar_wait(bar(kPEmpty + s), uint32_t((ks / kP) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
+                if (err) break;  // no arming without the loads that complete it
                 mbar_expect_tx(bar(kPFull + s), uint32_t(kPA + kPB));
-                if (!err) {
-                    tma_load_2d(smem_u32(pk_a(s)), &tm_a, ks * (kBK / 2), int(m0), bar(kPFull + s));
-                    tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
-                }
+                tma_load_2d(smem_u32(pk_a(s)), &tm_a, ks * (kBK / 2), int(m0), bar(kPFull + s));
+                tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
             }
         }
         __syncwarp();

@@ -257,11 +257,9 @@ uint64_t rsq_launch_count(void);
  * 16 CTAs on FP32 FMAs, which takes up to 32 rows on request; otherwise, for
  * bf16, D in {4096, 8192} and r <= 32, the tensor-core cluster kernel; the
  * CUDA-core kernel for everything else), 1 = always the CUDA-core kernel,
- * 2 = only the tensor-core cluster kernel, 3 = only the streamed tensor-core
- * kernel (bf16, D in {4096, 8192}, r <= 32: clusters of D / 1024 CTAs, each
- * token tile read three times through a small shared-memory ring), 4 = only
- * the decode kernel (2, 3 and 4 return RSQ_ERR_UNSUPPORTED for calls they
- * cannot serve).  Process-wide;
+ * 2 = only the tensor-core cluster kernel, 4 = only the decode kernel (2 and 4
+ * return RSQ_ERR_UNSUPPORTED for calls they cannot serve; 3 is not a valid
+ * choice).  Process-wide;
  * returns the previous setting, or -1 for an invalid value.  All compute the
  * same function; this exists for testing and measurement. */
 int rsq_select_align_kernel(int which);

@@ -132,23 +132,13 @@ def test_chain_32_layers_teacher_forced(T):
     np.testing.assert_allclose(n1, np.linalg.norm(xr, axis=1), rtol=2e-3)
 
 
-@pytest.mark.parametrize("which", [0, 3])
-def test_chain_32_layers_prefill_16384_sampled(which):
+def test_chain_32_layers_prefill_16384_sampled():
     """The 32-layer chain at prefill size (T = 16384, in place, bench launch
     configuration): every layer runs on the whole stream on the GPU; before
     each layer the sampled rows of the GPU's bf16 stream are taken as that
     layer's oracle input (teacher forcing), and after it that layer's x_out,
-    codes and scales of those rows are checked against the oracle.  Through
-    the default kernel choice (0) and the streamed tensor-core kernel (3)."""
+    codes and scales of those rows are checked against the oracle."""
     rsq = _rsq()
-    prev = rsq.select_align_kernel(which)
-    try:
-        _chain_prefill(rsq)
-    finally:
-        rsq.select_align_kernel(prev)
-
-
-def _chain_prefill(rsq):
     T = 16384
     x0, qs, ms, _, _ = inputs.chain_case(T=T)
     rows = _sample(T, 40, seed=4)
@@ -372,7 +362,7 @@ def test_generic_kernel_at_the_tensor_core_shapes(generic_align, T):
     check_align(a, label=f"generic w3a3 T={T}")
 
 
-@pytest.mark.parametrize("which", [2, 3])
+@pytest.mark.parametrize("which", [2])
 def test_tensor_core_kernel_serves_the_hot_shapes(which):
     rsq = _rsq()
     prev = rsq.select_align_kernel(which)
@@ -405,43 +395,6 @@ def test_tensor_core_kernel_serves_the_hot_shapes(which):
         ref = oracle.align_norm_quant(a.x, a.Q, a.M, 4, a.eps)
         H.check_codes(codes16.cpu().numpy(), ref["q"], ref["pre"], 4, "tc 16B-aligned codes")
         H.check_scales(sc.cpu().numpy(), ref["scales"], "tc 16B-aligned codes")
-    finally:
-        rsq.select_align_kernel(prev)
-
-
-@pytest.mark.parametrize("T,D", [(4352, 4096), (16384, 4096), (8192, 8192)])
-def test_streamed_kernel_several_tiles_per_cluster(T, D):
-    """The streamed tensor-core kernel (selection 3) with several token tiles
-    per cluster, so that every ring stage, TMEM buffer and exchange barrier runs
-    through many phases: sampled rows (first and last tile included) against
-    the oracle, INT4 at D = 4096 and INT3 at D = 8192; in place equals out of
-    place; the residual-only x_out equals that of the norm + quantiser call;
-    and 200 launches back to back (each may start before the previous one ends)
-    reproduce the first outputs bit for bit with a clean status word."""
-    rsq = _rsq()
-    prev = rsq.select_align_kernel(rsq.ALIGN_STREAM)
-    try:
-        a = inputs.llama7b_case(T=T)[0] if D == 4096 else inputs.w3a3_case(T=T)[0]
-        rows = _sample(T, 40, seed=T)
-        check_align(a, rows, f"stream T={T} D={D}")
-        x = _to_dev(a.x, "bf16")
-        Q = torch.from_numpy(a.Q).to(DEV)
-        M = torch.from_numpy(a.M).to(DEV)
-        xo, c0, s0 = rsq.rsq_align_norm_quant(x, Q, M, bits=a.bits)
-        ref = [xo.view(torch.int16).clone(), c0.clone(), s0.clone()]
-        xr = rsq.rsq_residual_align(x, Q, M)
-        torch.cuda.synchronize()
-        assert torch.equal(xr.view(torch.int16), ref[0]), "residual-only x_out"
-        for i in range(200):
-            rsq.rsq_align_norm_quant(x, Q, M, x_out=xo, codes=c0, scales=s0, bits=a.bits)
-        torch.cuda.synchronize()
-        for u, v in zip((xo.view(torch.int16), c0, s0), ref):
-            assert torch.equal(u, v), "back-to-back launches"
-        xi = x.clone()
-        _, ci, si = rsq.rsq_align_norm_quant(xi, Q, M, x_out=xi, bits=a.bits)
-        torch.cuda.synchronize()
-        assert torch.equal(xi.view(torch.int16), ref[0]) and torch.equal(ci, ref[1]) and torch.equal(si, ref[2])
-        assert rsq.device_status() == 0
     finally:
         rsq.select_align_kernel(prev)
 
@@ -877,7 +830,7 @@ def test_residual_align_only_matches_oracle():
         H.check_aligned(_host(xo), oracle.residual_align(a.x, a.Q, a.M), a.x, dtype, f"align {dtype}")
 
 
-@pytest.mark.parametrize("which", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("which", [0, 1, 2, 4])
 def test_residual_align_kernels(which):
     """rsq_residual_align through the decode kernel (small T), the tensor-core
     kernel (bf16, D = 4096 / 8192) and the CUDA-core kernel, each without the
@@ -889,7 +842,6 @@ def test_residual_align_kernels(which):
         shapes = {0: [(1, 4096), (16, 4096), (17, 4096), (1000, 4096), (300, 8192)],
                   1: [(16, 4096), (300, 4096)],
                   2: [(1, 4096), (200, 4096), (3001, 4096), (129, 8192)],
-                  3: [(1, 4096), (200, 4096), (3001, 4096), (129, 8192)],
                   4: [(1, 4096), (16, 4096), (32, 2048), (31, 8192)]}[which]
         for T, D in shapes:
             a = inputs.align_case(T, D, 32, T + D, dtype="bf16", n_outliers=8, outlier_scale=100.0)

@@ -38,14 +38,8 @@ cudaError_t launch_align_tc(const void *x, const float *Q, const float *M, void 
                             float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
                             bool *launched);
 
-// Tensor-core alignment + RMSNorm + quantiser with each token tile streamed
-// three times through a 4-stage shared-memory ring (clusters of D / 1024 CTAs;
-// bf16, D in {4096, 8192}, r <= 32); same contract as launch_align_tc.
-bool align_stream_supports(int D, int r, int dtype, long long T);
-cudaError_t launch_align_stream(const void *x, const float *Q, const float *M, void *x_out, uint8_t *codes,
-                                float *scales, long long T, int D, int r, int bits, float eps, cudaStream_t s,
-                                bool *launched);
-
+// Tensor-core alignment + RMSNorm + quantiser with two 64-row tiles in flight
+// per CTA (bf16, D in {4096, 8192}, r <= 32); same contract as launch_align_tc.
 // Decode-size alignment + RMSNorm + quantiser: one cluster of 16 CTAs, FP32 FMAs
 // (T <= 32, 2048 <= D <= 8192, D % 128 == 0, r <= 32, bf16 or fp32 I/O).
 // Returns cudaErrorNotSupported if the cluster cannot be co-scheduled.

@@ -22,7 +22,7 @@ __device__ int g_status_taken;
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
-std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 3 streamed tensor core, 4 decode
+std::atomic<int> g_align_kernel{0};  // 0 auto, 1 generic, 2 cluster tensor core, 4 decode
 std::atomic<int> g_rht_kernel{0};    // 0 auto, 1 generic, 3 tensor core, 4 Kronecker 12288
 thread_local int g_last_cuda_error = 0;
 
@@ -162,12 +162,6 @@ int rsq_residual_align(const void *x, const float *Q, const float *M, void *x_ou
         const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, dtype, cs);
         if (e != cudaErrorNotSupported) return finish(e);
     }
-    if (which == 3 && rsq::align_stream_supports(D, r, dtype, T)) {
-        bool launched = false;
-        const cudaError_t e = rsq::launch_align_stream(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, cs, &launched);
-        if (e != cudaSuccess) return finish(e);
-        if (launched) return RSQ_OK;
-    }
     if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
         bool launched = false;
         const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, nullptr, nullptr, T, D, r, 0, 0.f, cs, &launched);
@@ -203,19 +197,13 @@ int rsq_align_norm_quant(const void *x, const float *Q, const float *M, void *x_
         const cudaError_t e = rsq::launch_align_decode(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype, cs);
         if (e != cudaErrorNotSupported) return finish(e);  // not co-schedulable: another kernel serves it
     }
-    if (which == 3 && rsq::align_stream_supports(D, r, dtype, T)) {
-        bool launched = false;
-        const cudaError_t e = rsq::launch_align_stream(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, cs, &launched);
-        if (e != cudaSuccess) return finish(e);
-        if (launched) return RSQ_OK;
-    }
     if ((which == 0 || which == 2) && rsq::align_tc_supports(D, r, dtype, T)) {
         bool launched = false;
         const cudaError_t e = rsq::launch_align_tc(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, cs, &launched);
         if (e != cudaSuccess) return finish(e);
         if (launched) return RSQ_OK;
     }
-    if (which >= 2) return RSQ_ERR_UNSUPPORTED;
+    if (which == 2 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_align_generic(x, Q, M, x_out, codes, scales, T, D, r, bits, eps, dtype,
                                             true, static_cast<cudaStream_t>(stream)));
 }
@@ -423,7 +411,7 @@ const char *rsq_status_string(int status) {
 int rsq_last_cuda_error(void) { return g_last_cuda_error; }
 
 int rsq_select_align_kernel(int which) {
-    if (which < 0 || which > 4) return -1;
+    if (which < 0 || which > 4 || which == 3) return -1;
     return rsq::g_align_kernel.exchange(which);
 }
 

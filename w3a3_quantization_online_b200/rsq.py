@@ -68,7 +68,7 @@ EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quan
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
             "rsq_selftest_wait_timeout")
 
-ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_STREAM, ALIGN_DECODE = 0, 1, 2, 3, 4
+ALIGN_AUTO, ALIGN_GENERIC, ALIGN_TENSOR_CORE, ALIGN_DECODE = 0, 1, 2, 4
 RHT_AUTO, RHT_GENERIC, RHT_TENSOR_CORE, RHT_KRONECKER = 0, 1, 3, 4
 
 

@@ -269,10 +269,11 @@ int rsq_select_align_kernel(int which);
  * INT4; shared-memory radix-16 kernel otherwise), 1 = always the radix-16
  * kernel, 3 = only the tensor-core kernel, 4 = only the Kronecker kernel (3 and
  * 4 return RSQ_ERR_UNSUPPORTED for other shapes).  The same setting chooses
- * the kernel of rht_heads and rht_heads_quant: the tensor-core per-head kernel
- * (bf16, d_h in {64, 128}) unless it is 1, which selects the CUDA-core
- * per-head kernel; 3 returns RSQ_ERR_UNSUPPORTED for the shapes the
- * tensor-core kernel does not serve.  Process-wide; returns the previous
+ * the kernel of rht_heads and rht_heads_quant (the tensor-core per-head kernel
+ * for bf16, d_h in {64, 128}) and of rht_head_mix_quant (the tensor-core
+ * kernel for bf16, 32 heads of 128) unless it is 1, which selects the
+ * CUDA-core kernels; 3 returns RSQ_ERR_UNSUPPORTED for the shapes the
+ * tensor-core kernels do not serve.  Process-wide; returns the previous
  * setting, -1 if invalid.  All compute the same function; this exists for
  * testing and measurement. */
 int rsq_select_rht_kernel(int which);

@@ -648,6 +648,31 @@ def test_heads_tensor_core_and_cuda_core_kernels(which, n_heads, d_head, T):
         rsq.select_rht_kernel(prev)
 
 
+@pytest.mark.parametrize("which", [3, 1])
+@pytest.mark.parametrize("T", [1, 3, 5, 600, 1001])
+def test_head_mix_tensor_core_and_cuda_core_kernels(which, T):
+    """rht_head_mix_quant at 32 heads x 128 through the tensor-core kernel
+    (which = 3; groups of four tokens, a ragged last group when T % 4 != 0)
+    and through the CUDA-core kernel (which = 1), bf16, INT4 and INT3, with
+    and without signs, with a zero row and a row whose absmax is below 2^-64,
+    each against the oracle."""
+    rsq = _rsq()
+    prev = rsq.select_rht_kernel(which)
+    try:
+        for bits in (4, 3):
+            c = inputs.rht_case(T, 4096, 1, T + 11 * bits, dtype="bf16", bits=bits, n_outliers=3,
+                                outlier_scale=20.0)
+            if T > 2:
+                c.x[1] = 0.0
+                c.x[2] *= np.float32(2.0 ** -120)
+                c.x = inputs.round_to_bf16(c.x)
+            check_head_mix(c, 32, True, label=f"head mix kernel {which} T={T} b={bits}")
+            check_head_mix(c, 32, False, label=f"head mix kernel {which} T={T} b={bits} no signs")
+        assert rsq.device_status() == 0
+    finally:
+        rsq.select_rht_kernel(prev)
+
+
 def test_heads_tensor_core_kernel_rejects_other_shapes():
     rsq = _rsq()
     prev = rsq.select_rht_kernel(3)

@@ -67,6 +67,10 @@ cudaError_t launch_head_rht(const void *x, const int8_t *signs, void *x_out, uin
                             long long T, int d, int n_heads, int bits, bool quant, int dtype, cudaStream_t s);
 cudaError_t launch_head_mix(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
                             int n_heads, int bits, int dtype, cudaStream_t s);
+// Head mixing + per-token quantiser on the tensor cores (bf16, 32 heads of 128).
+bool head_mix_tc_supports(int d, int n_heads, int dtype, long long T);
+cudaError_t launch_head_mix_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
+                               int bits, cudaStream_t s);
 // The same per-head rotation / quantisation on the tensor cores (bf16, d_h in {64, 128}).
 bool head_tc_supports(int d, int n_heads, int dtype, long long T);
 cudaError_t launch_head_tc(const void *x, const int8_t *signs, void *x_out, uint8_t *codes, float *scales,

@@ -321,6 +321,10 @@ int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t 
         const Span sg = span(signs, uint64_t(d));
         if (overlap(sc, sg) || overlap(ss, sg)) return RSQ_ERR_ALIAS;
     }
+    const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
+    if (which != 1 && rsq::head_mix_tc_supports(d, n_heads, dtype, T))
+        return finish(rsq::launch_head_mix_tc(x, signs, codes, scales, T, bits, static_cast<cudaStream_t>(stream)));
+    if (which == 3) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_head_mix(x, signs, codes, scales, T, d, n_heads, bits, dtype,
                                        static_cast<cudaStream_t>(stream)));
 }

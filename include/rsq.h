@@ -190,6 +190,22 @@ int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t 
 int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *codes_w, const float *scales_w,
               void *y, int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream);
 
+/* The weight codes of w4a4_gemm unpacked once (the weights of a layer do not
+ * change between calls): w_s8[n * K + k] = the 4-bit two's complement value
+ * qw[n][k] sign-extended to int8 (N x K bytes, row-major).  Same N, K limits
+ * as w4a4_gemm; codes_w and w_s8 16-byte aligned and not overlapping
+ * (RSQ_ERR_ALIGN, RSQ_ERR_ALIAS).  Asynchronous on `stream`.  No counterpart
+ * in the pages: a storage form of the same weights for the GEMM below. */
+int w4a4_prepare_weights(const uint8_t *codes_w, int N, int K, int8_t *w_s8, void *stream);
+
+/* w4a4_gemm with the weights as written by w4a4_prepare_weights: the same
+ * acc and y bit for bit (acc is exact for any int8 weights).  The int8 weights
+ * go to the tensor cores without an unpack step: every 128-row block of
+ * activations would otherwise unpack the whole weight again.  Checks as for
+ * w4a4_gemm, with w_s8 N x K bytes. */
+int w4a4_gemm_s8w(const uint8_t *codes_a, const float *scales_a, const int8_t *w_s8, const float *scales_w,
+                  void *y, int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream);
+
 /* Offline construction of the alignment's (Q, M) from the rotations on both
  * sides of a residual connection.  ReSpinQuant paper notes, key design 2:
  * T = R_out R_in^T; Q = the top-r left singular vectors of T - I (D x r,

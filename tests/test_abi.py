@@ -205,6 +205,39 @@ def test_w4a4_gemm_rejects(kw, want):
     assert rsq.launch_count() == before
 
 
+def _gemm_s8w(ca=X, sa=S, w=Q, sw=M, y=XO, acc=C, T=4, N=256, K=4096, dt=2):
+    return L.w4a4_gemm_s8w(ca, sa, w, sw, y, acc, T, N, K, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(ca=None), NULL), (dict(w=None), NULL), (dict(y=None), NULL), (dict(dt=0), DTYPE), (dict(N=4), SHAPE),
+    (dict(K=64), SHAPE), (dict(w=Q + 8), ALIGN), (dict(y=Q + 512 * 1024), ALIAS), (dict(acc=Q + 1024 * 1024 - 16), ALIAS),
+])
+def test_w4a4_gemm_s8w_rejects(kw, want):
+    """The prepared-weight GEMM checks the int8 weights as N x K bytes (a span
+    twice that of the packed codes)."""
+    before = rsq.launch_count()
+    assert _gemm_s8w(**kw) == want
+    assert rsq.launch_count() == before
+
+
+@pytest.mark.parametrize("args,want", [
+    ((Q, 256, 4096, XO), None), ((None, 256, 4096, XO), NULL), ((Q, 256, 4096, None), NULL),
+    ((Q, 4, 4096, XO), SHAPE), ((Q, 256, 100, XO), SHAPE), ((Q + 4, 256, 4096, XO), ALIGN),
+    ((Q, 256, 4096, Q + 256 * 2048 - 16), ALIAS), ((Q, 256, 4096, Q - 256 * 4096 + 16), ALIAS),
+])
+def test_w4a4_prepare_weights_rejects(args, want):
+    import torch
+    if want is None:
+        if torch.cuda.is_available():
+            pytest.skip("would launch on fake pointers")
+        assert L.w4a4_prepare_weights(*args, None) == CUDA  # valid arguments reach the launch (no GPU here)
+        return
+    before = rsq.launch_count()
+    assert L.w4a4_prepare_weights(*args, None) == want
+    assert rsq.launch_count() == before
+
+
 def _qm(ri=X, ro=XB, D=4096, r=32, it=16, q=Q, m=M, ws=C, wsb=1 << 30):
     return L.rsq_qm_build(ri, ro, D, r, it, q, m, ws, wsb, None)
 

@@ -700,14 +700,30 @@ def test_attention_transforms_full_size_sampled():
     check_head_mix(c, 32, True, rows, "head mix T=16384")
 
 
-def run_gemm(case, out="f16", with_acc=True, rows=None):
+def unpack_int4_rows(codes: np.ndarray) -> np.ndarray:
+    """Packed 4-bit two's complement codes (element 2i in the low nibble of
+    byte i) -> int8 values, written out from the packing rule."""
+    c = codes.astype(np.int16)
+    lo, hi = c & 15, c >> 4
+    out = np.empty((codes.shape[0], 2 * codes.shape[1]), dtype=np.int16)
+    out[:, 0::2], out[:, 1::2] = lo, hi
+    return np.where(out >= 8, out - 16, out).astype(np.int8)
+
+
+def run_gemm(case, out="f16", with_acc=True, rows=None, prepared=False):
     rsq = _rsq()
     ca = torch.from_numpy(case.codes_a).to(DEV)
     cw = torch.from_numpy(case.codes_w).to(DEV)
     sa = torch.from_numpy(case.scales_a).to(DEV)
     sw = torch.from_numpy(case.scales_w).to(DEV)
     acc = torch.empty((case.T, case.N), dtype=torch.int32, device=DEV) if with_acc else None
-    y = rsq.w4a4_gemm(ca, sa, cw, sw, acc=acc, out_dtype=torch.float16 if out == "f16" else torch.bfloat16)
+    od = torch.float16 if out == "f16" else torch.bfloat16
+    if prepared:
+        w8 = rsq.w4a4_prepare_weights(cw)
+        np.testing.assert_array_equal(w8.cpu().numpy(), unpack_int4_rows(case.codes_w))
+        y = rsq.w4a4_gemm_s8w(ca, sa, w8, sw, acc=acc, out_dtype=od)
+    else:
+        y = rsq.w4a4_gemm(ca, sa, cw, sw, acc=acc, out_dtype=od)
     assert rsq.device_status() == 0
     sel = slice(None) if rows is None else rows
     ref = oracle.w4a4_gemm(case.codes_a[sel], case.scales_a[sel], case.codes_w, case.scales_w)
@@ -720,11 +736,14 @@ def run_gemm(case, out="f16", with_acc=True, rows=None):
 @pytest.mark.parametrize("T,N,K", [(1, 8, 128), (128, 256, 128), (127, 264, 256), (300, 512, 1024),
                                    (129, 4096, 4096), (515, 1000, 384)])
 @pytest.mark.parametrize("out", ["f16", "bf16"])
-def test_w4a4_gemm(T, N, K, out):
+@pytest.mark.parametrize("prepared", [False, True])
+def test_w4a4_gemm(T, N, K, out, prepared):
     """The INT4 GEMM on tcgen05 (kind::i8): exact int32 products over the full
     4-bit range, then the scale epilogue, against the oracle; several tiles and
-    ragged edges in both output dimensions."""
-    run_gemm(inputs.gemm_case(T, N, K, T + N + K), out)
+    ragged edges in both output dimensions.  With prepared = True the weights
+    go through w4a4_prepare_weights (checked against the packing rule) and
+    w4a4_gemm_s8w."""
+    run_gemm(inputs.gemm_case(T, N, K, T + N + K), out, prepared=prepared)
 
 
 def test_w4a4_gemm_without_accumulator_copy_matches():
@@ -762,11 +781,16 @@ def test_w4a4_gemm_consumes_the_quantiser_codes():
     assert np.all(np.abs(yg - ref["y"][same]) <= bound)
 
 
-def test_w4a4_gemm_full_size_sampled():
+@pytest.mark.parametrize("prepared", [False, True])
+def test_w4a4_gemm_full_size_sampled(prepared):
     """T = 16384, N = K = 4096 (the hidden stream through a 4096 x 4096 INT4
-    projection), sampled rows against the oracle."""
+    projection), sampled rows against the oracle; packed and prepared weights
+    give the same outputs bit for bit."""
     c = inputs.gemm_case(16384, 4096, 4096, 21)
-    run_gemm(c, "f16", with_acc=True, rows=_sample(16384, 24, seed=3))
+    y = run_gemm(c, "f16", with_acc=True, rows=_sample(16384, 24, seed=3), prepared=prepared)
+    if prepared:
+        y0 = run_gemm(c, "f16", with_acc=False, rows=np.array([0]), prepared=False)
+        assert torch.equal(y.view(torch.int16), y0.view(torch.int16))
 
 
 def run_qm(D, r, seed, iters=16, **kw):

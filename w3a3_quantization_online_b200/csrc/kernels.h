@@ -79,8 +79,11 @@ cudaError_t launch_head_tc(const void *x, const int8_t *signs, void *x_out, uint
 // INT4 consumer GEMM: y = round16(float(codes_a codes_w^T) * sa[t] * sw[n]),
 // fp16 (out_f16) or bf16 out, optional raw int32 accumulators.
 bool w4a4_gemm_supports(long long T, int N, int K);
-cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const uint8_t *codes_w, const float *sw,
+// w: packed weight codes (N x K/2), or with w_prepared the int8 weights (N x K)
+// written by launch_w4a4_unpack_weights.
+cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const void *w, bool w_prepared, const float *sw,
                              void *y, int32_t *acc, long long T, int N, int K, int out_f16, cudaStream_t s);
+cudaError_t launch_w4a4_unpack_weights(const uint8_t *codes_w, int8_t *w_s8, int N, int K, cudaStream_t s);
 
 // Offline (Q, M) construction from two rotations; workspace from the caller.
 bool qm_supports(int D, int r);

@@ -329,18 +329,22 @@ int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t 
                                        static_cast<cudaStream_t>(stream)));
 }
 
-int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *codes_w, const float *scales_w, void *y,
-              int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream) {
+// Shared checks and launch of the two GEMM entry points: w is the packed weight
+// codes (N x K/2 bytes) or, with w_prepared, the int8 weights (N x K bytes).
+static int w4a4_gemm_common(const uint8_t *codes_a, const float *scales_a, const void *w, bool w_prepared,
+                            const float *scales_w, void *y, int32_t *acc, int64_t T, int N, int K, int out_dtype,
+                            void *stream) {
     if (out_dtype != RSQ_BF16 && out_dtype != RSQ_F16) return RSQ_ERR_DTYPE;
     if (T < 0 || N < 8 || N % 8 != 0 || N > 65536 || K < 128 || K % 128 != 0 || K > 65536) return RSQ_ERR_SHAPE;
     if (T == 0) return RSQ_OK;
     if (!rsq::w4a4_gemm_supports(T, N, K)) return RSQ_ERR_SHAPE;
-    if (!codes_a || !scales_a || !codes_w || !scales_w || !y) return RSQ_ERR_NULL;
-    if (!aligned16(codes_a) || !aligned16(scales_a) || !aligned16(codes_w) || !aligned16(scales_w) || !aligned16(y) ||
+    if (!codes_a || !scales_a || !w || !scales_w || !y) return RSQ_ERR_NULL;
+    if (!aligned16(codes_a) || !aligned16(scales_a) || !aligned16(w) || !aligned16(scales_w) || !aligned16(y) ||
         (acc && !aligned16(acc)))
         return RSQ_ERR_ALIGN;
-    const Span in[4] = {span(codes_a, uint64_t(T) * (K / 2)), span(scales_a, uint64_t(T) * 4),
-                        span(codes_w, uint64_t(N) * (K / 2)), span(scales_w, uint64_t(N) * 4)};
+    const uint64_t w_bytes = uint64_t(N) * (w_prepared ? K : K / 2);
+    const Span in[4] = {span(codes_a, uint64_t(T) * (K / 2)), span(scales_a, uint64_t(T) * 4), span(w, w_bytes),
+                        span(scales_w, uint64_t(N) * 4)};
     const Span sy = span(y, uint64_t(T) * N * 2);
     for (const Span &i : in)
         if (overlap(sy, i)) return RSQ_ERR_ALIAS;
@@ -350,8 +354,26 @@ int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *code
         for (const Span &i : in)
             if (overlap(sacc, i)) return RSQ_ERR_ALIAS;
     }
-    return finish(rsq::launch_w4a4_gemm(codes_a, scales_a, codes_w, scales_w, y, acc, T, N, K, out_dtype == RSQ_F16,
-                                        static_cast<cudaStream_t>(stream)));
+    return finish(rsq::launch_w4a4_gemm(codes_a, scales_a, w, w_prepared, scales_w, y, acc, T, N, K,
+                                        out_dtype == RSQ_F16, static_cast<cudaStream_t>(stream)));
+}
+
+int w4a4_gemm(const uint8_t *codes_a, const float *scales_a, const uint8_t *codes_w, const float *scales_w, void *y,
+              int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream) {
+    return w4a4_gemm_common(codes_a, scales_a, codes_w, false, scales_w, y, acc, T, N, K, out_dtype, stream);
+}
+
+int w4a4_prepare_weights(const uint8_t *codes_w, int N, int K, int8_t *w_s8, void *stream) {
+    if (N < 8 || N % 8 != 0 || N > 65536 || K < 128 || K % 128 != 0 || K > 65536) return RSQ_ERR_SHAPE;
+    if (!codes_w || !w_s8) return RSQ_ERR_NULL;
+    if (!aligned16(codes_w) || !aligned16(w_s8)) return RSQ_ERR_ALIGN;
+    if (overlap(span(codes_w, uint64_t(N) * (K / 2)), span(w_s8, uint64_t(N) * K))) return RSQ_ERR_ALIAS;
+    return finish(rsq::launch_w4a4_unpack_weights(codes_w, w_s8, N, K, static_cast<cudaStream_t>(stream)));
+}
+
+int w4a4_gemm_s8w(const uint8_t *codes_a, const float *scales_a, const int8_t *w_s8, const float *scales_w, void *y,
+                  int32_t *acc, int64_t T, int N, int K, int out_dtype, void *stream) {
+    return w4a4_gemm_common(codes_a, scales_a, w_s8, true, scales_w, y, acc, T, N, K, out_dtype, stream);
 }
 
 uint64_t rsq_qm_workspace_bytes(int D, int r) {

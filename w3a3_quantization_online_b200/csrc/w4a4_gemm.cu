@@ -23,6 +23,12 @@
 //  * Epilogue, warps 2-9: TMEM -> registers, float(acc) * sa * sw, rounded to
 //    fp16 or bf16 into a swizzled staging tile, written by TMA (4 slabs of 64
 //    columns); optionally the raw int32 accumulators as well.
+//  * Prepared weights (w4a4_gemm_s8w): the weight codes, unpacked once to
+//    int8 by w4a4_prepare_weights, are TMA-loaded straight into the SWIZZLE_128B
+//    K-major operand layout; only the activation codes are unpacked, and the
+//    ring of operand stages is four deep (the packed ring holds A alone).
+//    Without it every 128-row M tile unpacks the whole weight again: two thirds
+//    of the unpack work and of its shared-memory traffic.
 // Every mbarrier wait is bounded; a timeout sets a bit in the device status
 // word, no further asynchronous work is issued, and the CTA drains what is in
 // flight before freeing TMEM.
@@ -44,21 +50,29 @@ constexpr int kPA = kBM * kBK / 2;  // packed A bytes per stage (8 KB)
 constexpr int kPB = kBN * kBK / 2;  // packed B bytes per stage (16 KB)
 constexpr int kUA = kBM * kBK;      // unpacked A bytes per stage (16 KB)
 constexpr int kUB = kBN * kBK;      // unpacked B bytes per stage (32 KB)
-constexpr int kP = 3, kU = 2;       // ring depths
 constexpr int kUnpackWarps = 8;
 constexpr int kGThreads = (2 + kUnpackWarps) * 32;
 constexpr int kGTmemCols = 256;
 
-constexpr int kOffPk = 0;                           // packed ring
-constexpr int kOffUn = kOffPk + kP * (kPA + kPB);   // unpacked ring (1024-aligned: 73728)
-constexpr int kOffSw = kOffUn + kU * (kUA + kUB);   // 256 column scales
-constexpr int kOffBar = kOffSw + kBN * 4;
-enum : int { kPFull = 0, kPEmpty = kPFull + kP, kUFull = kPEmpty + kP, kUEmpty = kUFull + kU, kAcc = kUEmpty + kU,
-             kGBars = kAcc + 1 };
-constexpr int kOffTm = kOffBar + kGBars * 8;
-constexpr int kGSmem = kOffTm + 16 + 1024;
-static_assert(kOffUn % 1024 == 0 && (kUA + kUB) % 1024 == 0, "swizzle atoms");
-static_assert(kU * (kUA + kUB) >= kBM * kBN * 2, "epilogue staging fits in the unpacked ring");
+// PREP = false: packed A and B ring of 3, unpacked ring of 2.  PREP = true: the
+// int8 weights go by TMA into the operand ring, whose stages hold both
+// operands: packed A ring of 4, operand ring of 4.
+template <bool PREP>
+struct GemmCfg {
+    static constexpr int kP = PREP ? 4 : 3, kU = PREP ? 4 : 2;  // ring depths
+    static constexpr int kPStage = PREP ? kPA : kPA + kPB;
+    static constexpr int kOffPk = 0;                                    // packed ring
+    static constexpr int kOffUn = (kOffPk + kP * kPStage + 1023) / 1024 * 1024;  // operand ring
+    static constexpr int kOffSw = kOffUn + kU * (kUA + kUB);            // 256 column scales
+    static constexpr int kOffBar = kOffSw + kBN * 4;
+    static constexpr int kPFull = 0, kPEmpty = kPFull + kP, kUFull = kPEmpty + kP, kUEmpty = kUFull + kU;
+    static constexpr int kAcc = kUEmpty + kU, kGBars = kAcc + 1;
+    static constexpr int kOffTm = kOffBar + kGBars * 8;
+    static constexpr int kGSmem = kOffTm + 16 + 1024;
+    static_assert(kOffUn % 1024 == 0 && (kUA + kUB) % 1024 == 0, "swizzle atoms");
+    static_assert(kU * (kUA + kUB) >= kBM * kBN * 2, "epilogue staging fits in the operand ring");
+    static_assert(kGSmem <= 232448, "shared memory per CTA");
+};
 
 struct GemmArgs {
     const float *sa;
@@ -125,18 +139,23 @@ __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
     return pack_bf16x2(a, b);
 }
 
-template <class OUT>
+template <class OUT, bool PREP>
 __global__ void __launch_bounds__(kGThreads, 1)
 k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
             const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
+    using C = GemmCfg<PREP>;
+    constexpr int kP = C::kP, kU = C::kU, kPStage = C::kPStage, kOffPk = C::kOffPk, kOffUn = C::kOffUn;
+    constexpr int kOffSw = C::kOffSw, kOffBar = C::kOffBar, kOffTm = C::kOffTm;
+    constexpr int kPFull = C::kPFull, kPEmpty = C::kPEmpty, kUFull = C::kUFull, kUEmpty = C::kUEmpty;
+    constexpr int kAcc = C::kAcc, kGBars = C::kGBars;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
     float *ssw = reinterpret_cast<float *>(base + kOffSw);
     const uint32_t bars = smem_u32(base + kOffBar);
     auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTm);
-    auto pk_a = [&](int s) { return base + kOffPk + s * (kPA + kPB); };
-    auto pk_b = [&](int s) { return base + kOffPk + s * (kPA + kPB) + kPA; };
+    auto pk_a = [&](int s) { return base + kOffPk + s * kPStage; };
+    auto pk_b = [&](int s) { return base + kOffPk + s * kPStage + kPA; };  // packed weights only
     auto un_a = [&](int s) { return base + kOffUn + s * (kUA + kUB); };
     auto un_b = [&](int s) { return base + kOffUn + s * (kUA + kUB) + kUA; };
 
@@ -148,7 +167,9 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
 
     if (tid == 0) {
         for (int i = 0; i < kGBars; ++i)
-            mbar_init(bar(i), (i >= kPEmpty && i < kPEmpty + kP) || (i >= kUFull && i < kUFull + kU) ? kUnpackWarps : 1);
+            mbar_init(bar(i), (i >= kPEmpty && i < kPEmpty + kP) ? kUnpackWarps
+                              : (i >= kUFull && i < kUFull + kU) ? kUnpackWarps + (PREP ? 1 : 0)  // + the weight load
+                              : 1);
         fence_mbar_init();
         prefetch_tmap(&tm_a);
         prefetch_tmap(&tm_b);
@@ -171,9 +192,18 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
                 const int s = ks % kP;
                 if (!mbar_wait(bar(kPEmpty + s), uint32_t((ks / kP) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
                 if (err) break;  // no arming without the loads that complete it
-                mbar_expect_tx(bar(kPFull + s), uint32_t(kPA + kPB));
+                mbar_expect_tx(bar(kPFull + s), uint32_t(kPStage));
                 tma_load_2d(smem_u32(pk_a(s)), &tm_a, ks * (kBK / 2), int(m0), bar(kPFull + s));
-                tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
+                if (PREP) {
+                    // int8 weights straight into the operand stage, once the product has freed it
+                    const int u = ks % kU;
+                    if (!mbar_wait(bar(kUEmpty + u), uint32_t((ks / kU) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
+                    if (err) break;
+                    mbar_expect_tx(bar(kUFull + u), uint32_t(kUB));
+                    tma_load_2d(smem_u32(un_b(u)), &tm_b, ks * kBK, n0, bar(kUFull + u));
+                } else {
+                    tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
+                }
             }
         }
         __syncwarp();
@@ -203,17 +233,19 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
             const int s = ks % kP, u = ks % kU;
             if (!mbar_wait(bar(kPFull + s), uint32_t((ks / kP) & 1), err != 0)) err |= kErrMbarTimeout;
             if (!mbar_wait(bar(kUEmpty + u), uint32_t((ks / kU) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
-            const uint8_t *pa = pk_a(s), *pb = pk_b(s);
+            const uint8_t *pa = pk_a(s), *pb = PREP ? nullptr : pk_b(s);
             uint8_t *ua = un_a(u), *ub = un_b(u);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {  // A: 512 chunks
                 const int i = u_tid + 256 * j;
                 unpack_chunk(pa, ua, i >> 2, i & 3);
             }
+            if (!PREP) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {  // B: 1024 chunks
-                const int i = u_tid + 256 * j;
-                unpack_chunk(pb, ub, i >> 2, i & 3);
+                for (int j = 0; j < 4; ++j) {  // B: 1024 chunks
+                    const int i = u_tid + 256 * j;
+                    unpack_chunk(pb, ub, i >> 2, i & 3);
+                }
             }
             fence_proxy_async_cta();  // unpacked operands (generic writes) -> tensor core (async proxy)
             __syncwarp();
@@ -313,23 +345,31 @@ bool w4a4_gemm_supports(long long T, int N, int K) {
     return T >= 1 && T <= 65535LL * kBM && N >= 8 && N % 8 == 0 && K >= kBK && K % kBK == 0 && K <= 65536;
 }
 
-cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const uint8_t *codes_w, const float *sw,
+cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const void *w, bool w_prepared, const float *sw,
                              void *y, int32_t *acc, long long T, int N, int K, int out_f16, cudaStream_t s) {
-    static bool configured[2][64];
+    static bool configured[4][64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int *status = device_status_word();
     if (!status) return cudaErrorInvalidDevice;
-    auto kern = out_f16 ? k_w4a4_gemm<__half> : k_w4a4_gemm<__nv_bfloat16>;
-    if (dev >= 0 && dev < 64 && !configured[out_f16 ? 1 : 0][dev]) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem);
+    using KernFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
+    const KernFn kern = w_prepared ? (out_f16 ? k_w4a4_gemm<__half, true> : k_w4a4_gemm<__nv_bfloat16, true>)
+                                   : (out_f16 ? k_w4a4_gemm<__half, false> : k_w4a4_gemm<__nv_bfloat16, false>);
+    const int smem = w_prepared ? GemmCfg<true>::kGSmem : GemmCfg<false>::kGSmem;
+    const int variant = (w_prepared ? 2 : 0) + (out_f16 ? 1 : 0);
+    if (dev >= 0 && dev < 64 && !configured[variant][dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        configured[out_f16 ? 1 : 0][dev] = true;
+        configured[variant][dev] = true;
     }
     CUtensorMap ma, mb, my;
+    const bool ok_b = w_prepared
+        // int8 weights: 128-byte rows of K values, swizzled as the operand
+        ? make_map_2d(&mb, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B)
+        : make_map_2d(&mb, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, kBK / 2, kBN, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!make_map_2d(&ma, codes_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K / 2, kBK / 2, kBM, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map_2d(&mb, codes_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, kBK / 2, kBN, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !ok_b ||
         !make_map_2d(&my, y, out_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, T, N, 64,
                      kBM, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
@@ -342,8 +382,36 @@ cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const uint
     a.N = N;
     a.K = K;
     const dim3 grid(unsigned((N + kBN - 1) / kBN), unsigned((T + kBM - 1) / kBM));
-    kern<<<grid, kGThreads, kGSmem, s>>>(ma, mb, my, a);
+    kern<<<grid, kGThreads, smem, s>>>(ma, mb, my, a);
     e = cudaGetLastError();
+    if (e == cudaSuccess) count_launch();
+    return e;
+}
+
+// The weight codes unpacked once to int8 (sign-extended 4-bit values, element
+// order kept): 16 packed bytes -> 32 int8 per thread, grid-stride.
+__global__ void __launch_bounds__(256)
+k_w4a4_unpack_weights(const uint4 *__restrict__ codes, uint4 *__restrict__ w, long long n16) {
+    for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n16; i += (long long)gridDim.x * 256) {
+        const uint4 pk = codes[i];
+        uint32_t o[8];
+        unpack8(pk.x, o[0], o[1]);
+        unpack8(pk.y, o[2], o[3]);
+        unpack8(pk.z, o[4], o[5]);
+        unpack8(pk.w, o[6], o[7]);
+        w[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+        w[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+cudaError_t launch_w4a4_unpack_weights(const uint8_t *codes_w, int8_t *w_s8, int N, int K, cudaStream_t s) {
+    const long long n16 = (long long)N * (K / 2) / 16;  // K % 128 == 0: whole 16-byte chunks
+    long long grid = (n16 + 255) / 256;
+    const long long cap = 8LL * num_sms();
+    if (grid > cap) grid = cap;
+    k_w4a4_unpack_weights<<<unsigned(grid), 256, 0, s>>>(reinterpret_cast<const uint4 *>(codes_w),
+                                                         reinterpret_cast<uint4 *>(w_s8), n16);
+    const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;
 }

@@ -40,6 +40,10 @@ _lib.rht_head_mix_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, 
 _lib.rht_head_mix_quant.restype = _i32
 _lib.w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.w4a4_gemm.restype = _i32
+_lib.w4a4_prepare_weights.argtypes = [_vp, _i32, _i32, _vp, _vp]
+_lib.w4a4_prepare_weights.restype = _i32
+_lib.w4a4_gemm_s8w.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
+_lib.w4a4_gemm_s8w.restype = _i32
 _lib.rsq_qm_build.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_uint64, _vp]
 _lib.rsq_qm_build.restype = _i32
 _lib.rsq_qm_workspace_bytes.argtypes = [_i32, _i32]
@@ -62,7 +66,8 @@ _lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
 _lib.rsq_selftest_wait_timeout.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rht_heads",
-            "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "rsq_qm_build", "rsq_qm_workspace_bytes",
+            "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "w4a4_prepare_weights", "w4a4_gemm_s8w",
+            "rsq_qm_build", "rsq_qm_workspace_bytes",
             "rsq_qm_build_fixed_scratch",
             "rsq_status_string",
             "rsq_last_cuda_error", "rsq_launch_count", "rsq_select_align_kernel", "rsq_select_rht_kernel", "rsq_device_status",
@@ -304,6 +309,42 @@ def w4a4_gemm(codes_a: torch.Tensor, scales_a: torch.Tensor, codes_w: torch.Tens
     code = RSQ_F16 if out_dtype == torch.float16 else RSQ_BF16
     _check(_lib.w4a4_gemm(_ptr(codes_a), _ptr(scales_a), _ptr(codes_w), _ptr(scales_w), _ptr(y), _ptr(acc), T, N,
                           2 * kb, code, _stream(stream)))
+    return y
+
+
+def w4a4_prepare_weights(codes_w: torch.Tensor, w_s8: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The packed INT4 weight codes (N x K/2 uint8) unpacked once to int8 (N x K) for w4a4_gemm_s8w."""
+    _need(codes_w, "codes_w", torch.uint8)
+    N, kb = codes_w.shape
+    if w_s8 is None:
+        w_s8 = torch.empty((N, 2 * kb), dtype=torch.int8, device=codes_w.device)
+    _need(w_s8, "w_s8", torch.int8)
+    if tuple(w_s8.shape) != (N, 2 * kb):
+        raise ValueError("w_s8 must be N x K")
+    _check(_lib.w4a4_prepare_weights(_ptr(codes_w), N, 2 * kb, _ptr(w_s8), _stream(stream)))
+    return w_s8
+
+
+def w4a4_gemm_s8w(codes_a: torch.Tensor, scales_a: torch.Tensor, w_s8: torch.Tensor, scales_w: torch.Tensor,
+                  y: Optional[torch.Tensor] = None, acc: Optional[torch.Tensor] = None, out_dtype=torch.float16,
+                  stream=None) -> torch.Tensor:
+    """w4a4_gemm with the weights prepared by w4a4_prepare_weights (N x K int8)."""
+    _need(codes_a, "codes_a", torch.uint8); _need(w_s8, "w_s8", torch.int8)
+    _need(scales_a, "scales_a", torch.float32); _need(scales_w, "scales_w", torch.float32)
+    T, kb = codes_a.shape
+    N = w_s8.shape[0]
+    if w_s8.shape[1] != 2 * kb:
+        raise ValueError("codes_a and w_s8 disagree on K")
+    if out_dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("out_dtype must be float16 or bfloat16")
+    if y is None:
+        y = torch.empty((T, N), dtype=out_dtype, device=codes_a.device)
+    _need(y, "y", out_dtype)
+    if acc is not None:
+        _need(acc, "acc", torch.int32)
+    code = RSQ_F16 if out_dtype == torch.float16 else RSQ_BF16
+    _check(_lib.w4a4_gemm_s8w(_ptr(codes_a), _ptr(scales_a), _ptr(w_s8), _ptr(scales_w), _ptr(y), _ptr(acc), T, N,
+                              2 * kb, code, _stream(stream)))
     return y
 
 

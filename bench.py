@@ -705,7 +705,17 @@ def next_rows_metrics(dev, stream, pk: dict) -> dict:
                         "peak_tops": peak_i8, "frac": ops / (us * 1e-6) / 1e12 / peak_i8,
                         "peak_source": "measured cuBLAS bf16 TFLOP/s (burst) x 2, the nominal int8 / bf16 dense ratio "
                                        "(4.5 / 2.25 PFLOP/s)"}
-    del ca, cw, y
+    # the same GEMM with the weights prepared once (int8), and the preparation itself
+    w8 = torch.empty((gm.N, gm.K), dtype=torch.int8, device=dev)
+    us_p = _time_loop(stream, lambda: rsq.w4a4_prepare_weights(cw, w8, stream=stream), 20, 3)
+    us = _time_loop(stream, lambda: rsq.w4a4_gemm_s8w(ca, sa, w8, sw, y=y, stream=stream), 20, 3)
+    out["w4a4_gemm_s8w"] = {"shape": "T=16384, N=4096, K=4096, INT4 activations x prepared int8 weights -> fp16",
+                            "avg_us": us, "bound": "tensor", "algorithmic_ops_per_launch": ops,
+                            "achieved_tops": ops / (us * 1e-6) / 1e12, "peak_tops": peak_i8,
+                            "frac": ops / (us * 1e-6) / 1e12 / peak_i8,
+                            "prepare_weights_us": us_p,
+                            "note": "w4a4_prepare_weights runs once per weight matrix, not per call"}
+    del ca, cw, y, w8
     # offline (Q, M) construction, D = 4096, r = 32
     R_in, R_out = inputs.near_hadamard_pair(4096, 77)
     Ri = torch.from_numpy(R_in.astype(np.float32)).to(dev)

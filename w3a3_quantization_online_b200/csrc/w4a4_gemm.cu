@@ -51,26 +51,29 @@ constexpr int kPB = kBN * kBK / 2;  // packed B bytes per stage (16 KB)
 constexpr int kUA = kBM * kBK;      // unpacked A bytes per stage (16 KB)
 constexpr int kUB = kBN * kBK;      // unpacked B bytes per stage (32 KB)
 constexpr int kUnpackWarps = 8;
-constexpr int kGThreads = (2 + kUnpackWarps) * 32;
-constexpr int kGTmemCols = 256;
+constexpr int kEpiWarps = 4;                   // one per TMEM lane quadrant
+constexpr int kFirstEpiWarp = 2 + kUnpackWarps;
+constexpr int kGThreads = (2 + kUnpackWarps + kEpiWarps) * 32;
+constexpr int kGTmemCols = 512;                // two 256-column int32 accumulators
+constexpr int kSlabOut = kBM * 128;            // one 64-column output slab of 16-bit values (16 KB)
 
-// PREP = false: packed A and B ring of 3, unpacked ring of 2.  PREP = true: the
+// PREP = false: packed A and B ring of 3, operand ring of 2.  PREP = true: the
 // int8 weights go by TMA into the operand ring, whose stages hold both
-// operands: packed A ring of 4, operand ring of 4.
+// operands: packed A ring of 4, operand ring of 3.  Two 16 KB output staging
+// slabs for the epilogue.
 template <bool PREP>
 struct GemmCfg {
-    static constexpr int kP = PREP ? 4 : 3, kU = PREP ? 4 : 2;  // ring depths
+    static constexpr int kP = PREP ? 4 : 3, kU = PREP ? 3 : 2;  // ring depths
     static constexpr int kPStage = PREP ? kPA : kPA + kPB;
     static constexpr int kOffPk = 0;                                    // packed ring
     static constexpr int kOffUn = (kOffPk + kP * kPStage + 1023) / 1024 * 1024;  // operand ring
-    static constexpr int kOffSw = kOffUn + kU * (kUA + kUB);            // 256 column scales
-    static constexpr int kOffBar = kOffSw + kBN * 4;
+    static constexpr int kOffOut = kOffUn + kU * (kUA + kUB);           // 2 output staging slabs
+    static constexpr int kOffBar = kOffOut + 2 * kSlabOut;
     static constexpr int kPFull = 0, kPEmpty = kPFull + kP, kUFull = kPEmpty + kP, kUEmpty = kUFull + kU;
-    static constexpr int kAcc = kUEmpty + kU, kGBars = kAcc + 1;
+    static constexpr int kAccFull = kUEmpty + kU, kAccEmpty = kAccFull + 2, kGBars = kAccEmpty + 2;
     static constexpr int kOffTm = kOffBar + kGBars * 8;
     static constexpr int kGSmem = kOffTm + 16 + 1024;
-    static_assert(kOffUn % 1024 == 0 && (kUA + kUB) % 1024 == 0, "swizzle atoms");
-    static_assert(kU * (kUA + kUB) >= kBM * kBN * 2, "epilogue staging fits in the operand ring");
+    static_assert(kOffUn % 1024 == 0 && (kUA + kUB) % 1024 == 0 && kOffOut % 1024 == 0, "swizzle atoms");
     static_assert(kGSmem <= 232448, "shared memory per CTA");
 };
 
@@ -145,12 +148,11 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
     using C = GemmCfg<PREP>;
     constexpr int kP = C::kP, kU = C::kU, kPStage = C::kPStage, kOffPk = C::kOffPk, kOffUn = C::kOffUn;
-    constexpr int kOffSw = C::kOffSw, kOffBar = C::kOffBar, kOffTm = C::kOffTm;
+    constexpr int kOffOut = C::kOffOut, kOffBar = C::kOffBar, kOffTm = C::kOffTm;
     constexpr int kPFull = C::kPFull, kPEmpty = C::kPEmpty, kUFull = C::kUFull, kUEmpty = C::kUEmpty;
-    constexpr int kAcc = C::kAcc, kGBars = C::kGBars;
+    constexpr int kAccFull = C::kAccFull, kAccEmpty = C::kAccEmpty, kGBars = C::kGBars;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
-    float *ssw = reinterpret_cast<float *>(base + kOffSw);
     const uint32_t bars = smem_u32(base + kOffBar);
     auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTm);
@@ -160,15 +162,27 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
     auto un_b = [&](int s) { return base + kOffUn + s * (kUA + kUB) + kUA; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n0 = blockIdx.x * kBN;
-    const long long m0 = (long long)blockIdx.y * kBM;
     const int KS = p.K / kBK;
+    const int ntn = (p.N + kBN - 1) / kBN;
+    const long long ntiles = (long long)((p.T + kBM - 1) / kBM) * ntn;
+    // this CTA's output tiles: blockIdx.x, + gridDim.x, ... (n fastest: consecutive
+    // CTAs share the activation block in L2)
+    const int nmine = blockIdx.x < ntiles ? int((ntiles - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+    auto tile_mn = [&](int i, long long &m0, int &n0) {
+        const long long tile = blockIdx.x + (long long)i * gridDim.x;
+        m0 = (tile / ntn) * kBM;
+        n0 = int(tile % ntn) * kBN;
+    };
     int err = 0;
+    auto wait = [&](int b, uint32_t ph) {
+        if (!mbar_wait(bar(b), ph, err != 0)) err |= kErrMbarTimeout;
+    };
 
     if (tid == 0) {
         for (int i = 0; i < kGBars; ++i)
             mbar_init(bar(i), (i >= kPEmpty && i < kPEmpty + kP) ? kUnpackWarps
                               : (i >= kUFull && i < kUFull + kU) ? kUnpackWarps + (PREP ? 1 : 0)  // + the weight load
+                              : (i >= kAccEmpty && i < kAccEmpty + 2) ? kEpiWarps
                               : 1);
         fence_mbar_init();
         prefetch_tmap(&tm_a);
@@ -179,127 +193,167 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
         tmem_alloc(smem_u32(tmem_slot), kGTmemCols);
         tmem_relinquish();
     }
-    for (int i = tid; i < kBN; i += kGThreads) ssw[i] = n0 + i < p.N ? p.sw[n0 + i] : 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // The rings run on one K-step counter g across all of this CTA's tiles.
     if (warp == 0) {
         // ---- TMA producer
         if (lane == 0) {
-            for (int ks = 0; ks < KS; ++ks) {
-                const int s = ks % kP;
-                if (!mbar_wait(bar(kPEmpty + s), uint32_t((ks / kP) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
-                if (err) break;  // no arming without the loads that complete it
-                mbar_expect_tx(bar(kPFull + s), uint32_t(kPStage));
-                tma_load_2d(smem_u32(pk_a(s)), &tm_a, ks * (kBK / 2), int(m0), bar(kPFull + s));
-                if (PREP) {
-                    // int8 weights straight into the operand stage, once the product has freed it
-                    const int u = ks % kU;
-                    if (!mbar_wait(bar(kUEmpty + u), uint32_t((ks / kU) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
-                    if (err) break;
-                    mbar_expect_tx(bar(kUFull + u), uint32_t(kUB));
-                    tma_load_2d(smem_u32(un_b(u)), &tm_b, ks * kBK, n0, bar(kUFull + u));
-                } else {
-                    tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
+            int g = 0;
+            for (int i = 0; i < nmine && !err; ++i) {
+                long long m0;
+                int n0;
+                tile_mn(i, m0, n0);
+                for (int ks = 0; ks < KS; ++ks, ++g) {
+                    const int s = g % kP;
+                    wait(kPEmpty + s, uint32_t((g / kP) & 1) ^ 1u);
+                    if (err) break;  // no arming without the loads that complete it
+                    mbar_expect_tx(bar(kPFull + s), uint32_t(kPStage));
+                    tma_load_2d(smem_u32(pk_a(s)), &tm_a, ks * (kBK / 2), int(m0), bar(kPFull + s));
+                    if (PREP) {
+                        // int8 weights straight into the operand stage, once the product has freed it
+                        const int u = g % kU;
+                        wait(kUEmpty + u, uint32_t((g / kU) & 1) ^ 1u);
+                        if (err) break;
+                        mbar_expect_tx(bar(kUFull + u), uint32_t(kUB));
+                        tma_load_2d(smem_u32(un_b(u)), &tm_b, ks * kBK, n0, bar(kUFull + u));
+                    } else {
+                        tma_load_2d(smem_u32(pk_b(s)), &tm_b, ks * (kBK / 2), n0, bar(kPFull + s));
+                    }
                 }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---- tensor-core issue
+        // ---- tensor-core issue: tile i accumulates in TMEM columns [256 (i & 1), +256)
         if (lane == 0) {
             const uint32_t idesc = idesc_s8_s32(kBM, kBN);
-            for (int ks = 0; ks < KS; ++ks) {
-                const int u = ks % kU;
-                if (!mbar_wait(bar(kUFull + u), uint32_t((ks / kU) & 1), err != 0)) err |= kErrMbarTimeout;
+            int g = 0;
+            for (int i = 0; i < nmine; ++i) {
+                const int ab = i & 1;
+                wait(kAccEmpty + ab, uint32_t((i >> 1) & 1) ^ 1u);  // its previous tile has been read out
                 tc_fence_after();
-                const uint64_t ad = smem_desc_sw128(smem_u32(un_a(u)), 1024);
-                const uint64_t bd = smem_desc_sw128(smem_u32(un_b(u)), 1024);
+                for (int ks = 0; ks < KS; ++ks, ++g) {
+                    const int u = g % kU;
+                    wait(kUFull + u, uint32_t((g / kU) & 1));
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc_sw128(smem_u32(un_a(u)), 1024);
+                    const uint64_t bd = smem_desc_sw128(smem_u32(un_b(u)), 1024);
 #pragma unroll
-                for (int k = 0; k < kBK / 32; ++k)  // K steps of 32 int8 = 32 bytes
-                    if (!err) umma_i8(tmem, ad + uint64_t((k * 32) >> 4), bd + uint64_t((k * 32) >> 4), idesc,
-                                      (ks | k) != 0);
-                if (!err) umma_commit(bar(kUEmpty + u));
+                    for (int k = 0; k < kBK / 32; ++k)  // K steps of 32 int8 = 32 bytes
+                        if (!err) umma_i8(tmem + uint32_t(256 * ab), ad + uint64_t((k * 32) >> 4),
+                                          bd + uint64_t((k * 32) >> 4), idesc, (ks | k) != 0);
+                    if (!err) umma_commit(bar(kUEmpty + u));
+                }
+                if (!err) umma_commit(bar(kAccFull + ab));
             }
-            if (!err) umma_commit(bar(kAcc));
         }
         __syncwarp();
-    } else {
+    } else if (warp < kFirstEpiWarp) {
         // ---- unpack
         const int u_tid = tid - 64;  // 0..255
-        for (int ks = 0; ks < KS; ++ks) {
-            const int s = ks % kP, u = ks % kU;
-            if (!mbar_wait(bar(kPFull + s), uint32_t((ks / kP) & 1), err != 0)) err |= kErrMbarTimeout;
-            if (!mbar_wait(bar(kUEmpty + u), uint32_t((ks / kU) & 1) ^ 1u, err != 0)) err |= kErrMbarTimeout;
-            const uint8_t *pa = pk_a(s), *pb = PREP ? nullptr : pk_b(s);
-            uint8_t *ua = un_a(u), *ub = un_b(u);
+        int g = 0;
+        for (int i = 0; i < nmine; ++i) {
+            for (int ks = 0; ks < KS; ++ks, ++g) {
+                const int s = g % kP, u = g % kU;
+                wait(kPFull + s, uint32_t((g / kP) & 1));
+                wait(kUEmpty + u, uint32_t((g / kU) & 1) ^ 1u);
+                const uint8_t *pa = pk_a(s), *pb = PREP ? nullptr : pk_b(s);
+                uint8_t *ua = un_a(u), *ub = un_b(u);
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {  // A: 512 chunks
-                const int i = u_tid + 256 * j;
-                unpack_chunk(pa, ua, i >> 2, i & 3);
-            }
-            if (!PREP) {
+                for (int j = 0; j < 2; ++j) {  // A: 512 chunks
+                    const int c = u_tid + 256 * j;
+                    unpack_chunk(pa, ua, c >> 2, c & 3);
+                }
+                if (!PREP) {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {  // B: 1024 chunks
-                    const int i = u_tid + 256 * j;
-                    unpack_chunk(pb, ub, i >> 2, i & 3);
+                    for (int j = 0; j < 4; ++j) {  // B: 1024 chunks
+                        const int c = u_tid + 256 * j;
+                        unpack_chunk(pb, ub, c >> 2, c & 3);
+                    }
+                }
+                fence_proxy_async_cta();  // unpacked operands (generic writes) -> tensor core (async proxy)
+                __syncwarp();
+                if (lane == 0 && !err) {
+                    mbar_arrive(bar(kPEmpty + s));
+                    mbar_arrive(bar(kUFull + u));
                 }
             }
-            fence_proxy_async_cta();  // unpacked operands (generic writes) -> tensor core (async proxy)
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar(kPEmpty + s));
-                mbar_arrive(bar(kUFull + u));
-            }
         }
-
-        // ---- epilogue: quadrant of TMEM lanes, half of the 256 columns
-        if (!mbar_wait(bar(kAcc), 0u, err != 0)) err |= kErrMbarTimeout;
-        tc_fence_after();
-        const int q = warp & 3, ch = (warp - 2) >> 2;
+    } else {
+        // ---- epilogue: TMEM lane quadrant q (one output row per thread), 64-column
+        // slabs through two staging buffers, each written back by one TMA store
+        const int q = warp & 3;
         const int r = 32 * q + lane;
-        const long long row = m0 + r;
-        const float sa = row < p.T ? p.sa[row] : 0.f;
-        uint8_t *stage = base + kOffUn;  // 4 slabs of 128 rows x 64 columns (128 B per row, SWIZZLE_128B)
+        const bool leader = warp == kFirstEpiWarp && lane == 0;
+        int slabs_done = 0;
+        for (int i = 0; i < nmine; ++i) {
+            const int ab = i & 1;
+            long long m0;
+            int n0;
+            tile_mn(i, m0, n0);
+            const long long row = m0 + r;
+            const float sa = row < p.T ? p.sa[row] : 0.f;
+            wait(kAccFull + ab, uint32_t((i >> 1) & 1));
+            __syncwarp();
+            tc_fence_after();
 #pragma unroll 1
-        for (int b = 0; b < 4; ++b) {  // 32-column blocks of this thread's 128 columns
-            uint32_t v[32];
-            tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(128 * ch + 32 * b), v);
-            tmem_wait_ld();
-            const int c0 = 128 * ch + 32 * b;  // first column of the block within the tile
-            if (p.acc && row < p.T) {
-                int32_t *dst = p.acc + row * p.N + n0 + c0;
-                if (n0 + c0 + 32 <= p.N) {
+            for (int sl = 0; sl < kBN / 64; ++sl, ++slabs_done) {
+                const int sb = slabs_done & 1;
+                uint8_t *slab = base + kOffOut + sb * kSlabOut;
+                // staging buffer sb is free once the store issued from it two slabs ago has read it
+                if (leader) bulk_wait_read<1>();
+                named_sync(1, kEpiWarps * 32);
+                if (n0 + 64 * sl < p.N) {
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<int4 *>(dst + e) = make_int4(int(v[e]), int(v[e + 1]), int(v[e + 2]), int(v[e + 3]));
-                } else {
-                    for (int e = 0; e < 32; ++e)
-                        if (n0 + c0 + e < p.N) dst[e] = int(v[e]);
+                    for (int h = 0; h < 2; ++h) {  // 32-column blocks
+                        uint32_t v[32];
+                        tmem_ld32(tmem + (uint32_t(32 * q) << 16) + uint32_t(256 * ab + 64 * sl + 32 * h), v);
+                        tmem_wait_ld();
+                        const int c0 = 64 * sl + 32 * h;  // first column of the block within the tile
+                        if (p.acc && row < p.T) {
+                            int32_t *dst = p.acc + row * p.N + n0 + c0;
+                            if (n0 + c0 + 32 <= p.N) {
+#pragma unroll
+                                for (int e = 0; e < 32; e += 4)
+                                    *reinterpret_cast<int4 *>(dst + e) =
+                                        make_int4(int(v[e]), int(v[e + 1]), int(v[e + 2]), int(v[e + 3]));
+                            } else {
+                                for (int e = 0; e < 32; ++e)
+                                    if (n0 + c0 + e < p.N) dst[e] = int(v[e]);
+                            }
+                        }
+                        uint32_t o[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int c = n0 + c0 + 2 * e;
+                            const float w0 = c < p.N ? __ldg(p.sw + c) : 0.f;
+                            const float w1 = c + 1 < p.N ? __ldg(p.sw + c + 1) : 0.f;
+                            o[e] = pack2<OUT>(float(int(v[2 * e])) * sa * w0, float(int(v[2 * e + 1])) * sa * w1);
+                        }
+                        uint8_t *srow = slab + r * 128;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            *reinterpret_cast<uint4 *>(srow + swz(r, 4 * h + c)) =
+                                make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                    }
+                }
+                fence_proxy_async_cta();  // staged outputs (generic writes) -> TMA store (async proxy)
+                named_sync(1, kEpiWarps * 32);
+                if (leader) {
+                    if (!err && n0 + 64 * sl < p.N) tma_store_2d(&tm_y, smem_u32(slab), n0 + 64 * sl, int(m0));
+                    bulk_commit();
                 }
             }
-            uint32_t o[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                o[e] = pack2<OUT>(float(int(v[2 * e])) * sa * ssw[c0 + 2 * e],
-                                  float(int(v[2 * e + 1])) * sa * ssw[c0 + 2 * e + 1]);
-            uint8_t *slab = stage + (c0 >> 6) * (kBM * 128) + r * 128;
-            const int ck0 = (c0 & 63) >> 3;  // first 16-byte chunk (8 outputs) within the slab row
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<uint4 *>(slab + swz(r, ck0 + c)) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+            // every TMEM load of this tile is complete: the accumulator may take tile i + 2
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0 && !err) mbar_arrive(bar(kAccEmpty + ab));
         }
-        fence_proxy_async_cta();
-        named_sync(1, kUnpackWarps * 32);
-        if (u_tid == 0) {
-            if (!err)
-                for (int s = 0; s < 4; ++s)
-                    if (n0 + 64 * s < p.N) tma_store_2d(&tm_y, smem_u32(stage + s * (kBM * 128)), n0 + 64 * s, int(m0));
-            bulk_commit();
-            bulk_wait0();
-        }
+        if (leader) bulk_wait0();
     }
 
     tc_fence_before();
@@ -381,8 +435,11 @@ cudaError_t launch_w4a4_gemm(const uint8_t *codes_a, const float *sa, const void
     a.T = T;
     a.N = N;
     a.K = K;
-    const dim3 grid(unsigned((N + kBN - 1) / kBN), unsigned((T + kBM - 1) / kBM));
-    kern<<<grid, kGThreads, smem, s>>>(ma, mb, my, a);
+    // persistent: one CTA per SM (at most one per output tile)
+    const long long ntiles = ((T + kBM - 1) / kBM) * ((N + kBN - 1) / kBN);
+    long long grid = num_sms();
+    if (grid > ntiles) grid = ntiles;
+    kern<<<unsigned(grid), kGThreads, smem, s>>>(ma, mb, my, a);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();
     return e;

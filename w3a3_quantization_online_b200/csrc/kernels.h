@@ -52,11 +52,15 @@ cudaError_t launch_align_decode(const void *x, const float *Q, const float *M, v
 cudaError_t launch_rht_gate_generic(const void *a, const void *b, const int8_t *signs, int m, uint8_t *codes,
                                     float *scales, int64_t T, int d, int bits, int dtype, cudaStream_t s);
 
-// Randomised Hadamard H_1024 (x) H_12 of order 12288 (Paley H_12), bf16, INT4.
-// With b != nullptr the input is SiLU(x) * b (the gated down_proj input).
-bool rht_kron_supports(int d, int m, int dtype, int bits, long long T);
-cudaError_t launch_rht_kron(const void *x, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
-                            long long T, cudaStream_t s);
+// Randomised Hadamard H_1024 (x) H_12 of order 12288 (Paley H_12), bf16, INT4, with
+// the H_128 stage of H_1024 on the tensor cores.
+bool rht_kron_tc_supports(int d, int m, int dtype, int bits, long long T);
+cudaError_t launch_rht_kron_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T,
+                               cudaStream_t s);
+// The gated down_proj input SiLU(a) * b (fp32) through the same transform on the CUDA cores.
+bool rht_kron_gate_supports(int d, int m, int dtype, int bits, long long T);
+cudaError_t launch_rht_kron_gate(const void *a, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
+                                 long long T, cudaStream_t s);
 
 // Attention: per-head randomised Hadamard (I (x) H_dh), rotation only (x_out)
 // or with per-(token, head) quantisation (quant), and head mixing (H_nh (x) I)

@@ -1,31 +1,29 @@
-// rht_kron.cu -- randomised Hadamard transform of order d = 12288 = 1024 x 12
-// (H_1024 (x) H_12, H_12 the Paley type-I matrix, q = 11) + per-token INT4
-// quantiser, bf16 input: the down_proj input of a 12288-wide FFN.
+// rht_kron.cu -- the gated down_proj input of a 12288-wide FFN, g = SiLU(a) * b
+// in fp32, through the randomised Hadamard transform of order d = 12288 =
+// 1024 x 12 (H_1024 (x) H_12, H_12 the Paley type-I matrix, q = 11) and the
+// per-token INT4 quantiser, bf16 inputs.  (Without the gate the tensor-core
+// kernel of rht_kron_tc.cu serves this transform.)
 //
 // Infra Quant II, QuaRot / Method: for d = 2^n m the online Hadamard is
 // H_{2^n} (x) H_m, applied as a fast Walsh-Hadamard transform along the stride-m
-// index and a dense H_m on each contiguous group of m; the random signs first.
-// QuaRot / Method: per-token symmetric absmax quantisation; 1/sqrt(d) goes to
-// the scale.
+// index and a dense H_m on each contiguous group of m; the random signs first;
+// the online Hadamard sits on the down_proj input.  QuaRot / Method:
+// per-token symmetric absmax quantisation; 1/sqrt(d) goes to the scale.
 //
-// One CTA per token row at a time (two CTAs per SM), 256 threads; the next row
-// is staged in shared memory by a bulk copy while the current one is
-// transformed (bounded wait, device status word).  With i =
-// 12 a + b (a < 1024, b < 12), thread t first owns the four groups a = 4t..4t+3
-// (48 contiguous values):
-//   1. load, signs (XOR of the bf16 sign bits), dense H_12 on each group in
-//      registers (packed f32x2 over pairs of groups);
+// One CTA per token row at a time (two CTAs per SM), 256 threads; the next rows
+// of a and b are staged in shared memory by bulk copies while the current one
+// is transformed (bounded wait, device status word).  With i = 12 a + b
+// (a < 1024, b < 12), thread t first owns the four groups a = 4t..4t+3 (48
+// contiguous values):
+//   1. load a and b, the gate SiLU(a) * b in fp32 (never rounded to bf16), the
+//      signs on the fp32 sign bit (48 sign bits per thread), dense H_12 on each
+//      group in registers (packed f32x2 over pairs of groups);
 //   2. FWHT along a: bits 0-1 in the thread, bits 2-6 (the lane) by warp
 //      shuffles;
 //   3. one transpose through shared memory (blocks padded to 52 floats against
 //      bank conflicts) so that thread (a0, h) owns a = a0 + 128 k (k < 8) and
 //      b = 6h..6h+5; FWHT bits 7-9 in the thread;
 //   4. block absmax, codes of 6 consecutive columns per (thread, k) = 3 bytes.
-// With GATE the input row is the gated FFN product SiLU(a) * b (QuaRot /
-// Method: the online Hadamard sits on the down_proj input), formed in fp32
-// from the two staged projection rows in step 1 and never rounded to bf16; the
-// signs are then applied to the fp32 sign bit (one bit per element, 48 per
-// thread).
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -87,19 +85,17 @@ __device__ __forceinline__ void h12_pair(const float2 (&u)[12], float2 (&out)[12
     }
 }
 
-template <int BITS, bool GATE>
+template <int BITS>
 __global__ void __launch_bounds__(kKThreads, 2)
-k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ xb,
+k_rht_kron_gate(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ xb,
            const int8_t *__restrict__ signs, uint8_t *__restrict__ codes,
            float *__restrict__ scales, long long T, int *status) {
     static_assert(BITS == 4, "6 codes of 4 bits make 3 whole bytes");
     extern __shared__ float4 km4[];
     float *buf = reinterpret_cast<float *>(km4);                    // 256 x 52 floats
-    // without GATE: bf16 sign masks, 8 per uint4; with GATE: 48 sign bits per thread
-    uint4 *smask = reinterpret_cast<uint4 *>(buf + kKThreads * kKBlk);
-    uint64_t *sbits = reinterpret_cast<uint64_t *>(smask);
-    uint4 *srow = GATE ? smask + kKThreads / 2 : smask + kKd / 8;  // the row being processed (bf16)
-    uint4 *srow_b = srow + kKd / 8;                                 // GATE: the second projection row
+    uint64_t *sbits = reinterpret_cast<uint64_t *>(buf + kKThreads * kKBlk);  // 48 sign bits per thread
+    uint4 *srow = reinterpret_cast<uint4 *>(sbits + kKThreads);     // the row of a being processed (bf16)
+    uint4 *srow_b = srow + kKd / 8;                                 // the row of b
     __shared__ float red[kKThreads / 32];
     __shared__ __align__(8) uint64_t bar_row;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -108,26 +104,18 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict_
     constexpr int qmax = 7;
     constexpr int row_bytes = kKd / 2;
 
-    if (GATE) {
+    {
         uint64_t w = 0;  // bit e: sign of element 48 tid + e
         for (int e = 0; e < 48; ++e) w |= uint64_t(signs[48 * tid + e] < 0) << e;
         sbits[tid] = w;
-    } else {
-        for (int i = tid; i < kKd / 8; i += kKThreads) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                w[e] = (signs[8 * i + 2 * e] < 0 ? 0x8000u : 0u) | (signs[8 * i + 2 * e + 1] < 0 ? 0x80000000u : 0u);
-            smask[i] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
     }
     if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
         if (blockIdx.x < T) {  // the first row (the next ones are staged while the previous is transformed)
-            mbar_expect_tx(bar, GATE ? 2 * kKd * 2 : kKd * 2);
-            if (!err) bulk_load_1d(smem_u32(srow), x + (long long)blockIdx.x * kKd, kKd * 2, bar);
-            if (GATE && !err) bulk_load_1d(smem_u32(srow_b), xb + (long long)blockIdx.x * kKd, kKd * 2, bar);
+            mbar_expect_tx(bar, 2 * kKd * 2);
+            bulk_load_1d(smem_u32(srow), x + (long long)blockIdx.x * kKd, kKd * 2, bar);
+            bulk_load_1d(smem_u32(srow_b), xb + (long long)blockIdx.x * kKd, kKd * 2, bar);
         }
     }
     __syncthreads();
@@ -140,7 +128,7 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict_
         // ---- 1. 48 values (groups a = 4 tid + g) from the staged row, signs, H_12
         if (!mbar_wait(bar, uint32_t(it) & 1u, err != 0)) err |= kErrMbarTimeout;
         float2 p[2][12];  // p[h][k] = (group 2h, group 2h+1) entry k
-        if (GATE) {
+        {
             const uint4 *src = srow + 6 * tid, *srcb = srow_b + 6 * tid;
             const uint64_t sb = sbits[tid];
 #pragma unroll
@@ -159,22 +147,6 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict_
                 }
             }
             fence_proxy_async_cta();  // these reads before the next row's bulk copies
-        } else {
-            const uint4 *src = srow + 6 * tid;
-#pragma unroll
-            for (int c = 0; c < 6; ++c) {
-                uint4 u = src[c];
-                const uint4 mk = smask[6 * tid + c];
-                const uint32_t w[4] = {u.x ^ mk.x, u.y ^ mk.y, u.z ^ mk.z, u.w ^ mk.w};
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int e = 8 * c + q, g = e / 12, k = e % 12;
-                    const float f = __uint_as_float(q & 1 ? (w[q >> 1] & 0xFFFF0000u) : (w[q >> 1] << 16));
-                    if (g & 1) p[g >> 1][k].y = f;
-                    else p[g >> 1][k].x = f;
-                }
-            }
-            fence_proxy_async_cta();  // these reads before the next row's bulk copy
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -225,10 +197,10 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict_
             }
         }
         __syncthreads();  // the staged row is consumed: bring in the next one
-        if (tid == 0 && t + gridDim.x < T) {
-            mbar_expect_tx(bar, GATE ? 2 * kKd * 2 : kKd * 2);
-            if (!err) bulk_load_1d(smem_u32(srow), x + (t + gridDim.x) * kKd, kKd * 2, bar);
-            if (GATE && !err) bulk_load_1d(smem_u32(srow_b), xb + (t + gridDim.x) * kKd, kKd * 2, bar);
+        if (tid == 0 && t + gridDim.x < T && !err) {  // no arming without the loads that complete it
+            mbar_expect_tx(bar, 2 * kKd * 2);
+            bulk_load_1d(smem_u32(srow), x + (t + gridDim.x) * kKd, kKd * 2, bar);
+            bulk_load_1d(smem_u32(srow_b), xb + (t + gridDim.x) * kKd, kKd * 2, bar);
         }
         // thread (a0, hb) now takes a = a0 + 128 k (k < 8), b = 6 hb .. 6 hb + 5
         float2 r[8][3];
@@ -295,31 +267,29 @@ k_rht_kron(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict_
 
 }  // namespace
 
-bool rht_kron_supports(int d, int m, int dtype, int bits, long long T) {
+bool rht_kron_gate_supports(int d, int m, int dtype, int bits, long long T) {
     return d == kKd && m == 12 && dtype == 1 && bits == 4 && T >= 1 && T <= 0x7FFFFFFFLL;
 }
 
-cudaError_t launch_rht_kron(const void *x, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
-                            long long T, cudaStream_t s) {
-    static bool configured[2][64];
-    const bool gate = b != nullptr;
+cudaError_t launch_rht_kron_gate(const void *a, const void *b, const int8_t *signs, uint8_t *codes, float *scales,
+                                 long long T, cudaStream_t s) {
+    static bool configured[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    // transpose buffer; sign masks (bf16 masks, or 48 sign bits per thread); the staged row(s)
-    const size_t smem = size_t(kKThreads) * kKBlk * 4 + (gate ? size_t(kKThreads) * 8 : size_t(kKd / 8) * 16) +
-                        size_t(kKd) * 2 * (gate ? 2 : 1);
+    // transpose buffer; 48 sign bits per thread; the staged rows of a and b
+    const size_t smem = size_t(kKThreads) * kKBlk * 4 + size_t(kKThreads) * 8 + size_t(kKd) * 2 * 2;
     int *status = device_status_word();
     if (!status) return cudaErrorInvalidValue;
-    auto kern = gate ? k_rht_kron<4, true> : k_rht_kron<4, false>;
-    if (dev >= 0 && dev < 64 && !configured[gate][dev]) {
+    auto kern = k_rht_kron_gate<4>;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return e;
-        configured[gate][dev] = true;
+        configured[dev] = true;
     }
     const long long cap = (long long)num_sms() * 2;
     const int grid = int(T < cap ? T : cap);
-    kern<<<grid, kKThreads, smem, s>>>(static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(b),
+    kern<<<grid, kKThreads, smem, s>>>(static_cast<const __nv_bfloat16 *>(a), static_cast<const __nv_bfloat16 *>(b),
                                        signs, codes, scales, T, status);
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launch();

@@ -226,8 +226,8 @@ int rht_quant(const void *x, const int8_t *signs, int m, uint8_t *codes, float *
     const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
     if ((which == 0 || which == 3) && rsq::rht_tc_supports(d, m, dtype, bits, T))
         return finish(rsq::launch_rht_tc(x, signs, codes, scales, T, d, bits, static_cast<cudaStream_t>(stream)));
-    if ((which == 0 || which == 4) && rsq::rht_kron_supports(d, m, dtype, bits, T))
-        return finish(rsq::launch_rht_kron(x, nullptr, signs, codes, scales, T, static_cast<cudaStream_t>(stream)));
+    if ((which == 0 || which == 4) && rsq::rht_kron_tc_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_kron_tc(x, signs, codes, scales, T, static_cast<cudaStream_t>(stream)));
     if (which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_generic(x, signs, m, codes, scales, T, d, bits, dtype,
                                           static_cast<cudaStream_t>(stream)));
@@ -254,8 +254,8 @@ int rht_quant_silu_gate(const void *a, const void *b, const int8_t *signs, int m
         return RSQ_ERR_ALIAS;
     const int which = rsq::g_rht_kernel.load(std::memory_order_relaxed);
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if ((which == 0 || which == 4) && rsq::rht_kron_supports(d, m, dtype, bits, T))
-        return finish(rsq::launch_rht_kron(a, b, signs, codes, scales, T, cs));
+    if ((which == 0 || which == 4) && rsq::rht_kron_gate_supports(d, m, dtype, bits, T))
+        return finish(rsq::launch_rht_kron_gate(a, b, signs, codes, scales, T, cs));
     if (which == 3 || which == 4) return RSQ_ERR_UNSUPPORTED;
     return finish(rsq::launch_rht_gate_generic(a, b, signs, m, codes, scales, T, d, bits, dtype, cs));
 }

@@ -110,14 +110,36 @@ __device__ __forceinline__ void h12_pair(const float2 (&u)[12], float2 (&out)[12
     }
 }
 
+// Low nibbles of 8 codes (the low bits of the rounded floats r[k]) -> one word,
+// code k in nibble k.
+__device__ __forceinline__ uint32_t nibbles8(const uint32_t (&r)[8]) {
+    const uint32_t ev = prmt(prmt(r[0], r[2], 0x0040u), prmt(r[4], r[6], 0x0040u), 0x5410u);
+    const uint32_t od = prmt(prmt(r[1], r[3], 0x0040u), prmt(r[5], r[7], 0x0040u), 0x5410u);
+    return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
+}
+
+// Codes of the 96 values w[p][b] = (v[12 (2p) + b], v[12 (2p + 1) + b]) in output
+// order n = 12 a0 + b: 12 words, words 3p .. 3p + 2 holding groups 2p and 2p + 1.
 template <bool SCALED>
-__device__ __forceinline__ void quant96(const float (&v)[96], const RowQuant &rq, uint32_t (&w)[12]) {
+__device__ __forceinline__ void quant_pairs(const float2 (&w)[4][12], const RowQuant &rq, uint32_t (&out)[12]) {
+    const float2 inv2 = make_float2(rq.inv, rq.inv), mag2 = make_float2(kRoundMagic, kRoundMagic);
 #pragma unroll
-    for (int k = 0; k < 12; ++k) {
-        float f[8];
+    for (int p = 0; p < 4; ++p) {
+        uint32_t e[12], o[12];  // rounded codes of group 2p (even) and 2p + 1 (odd)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = v[8 * k + e];
-        w[k] = pack8_fast<4>(f, rq.inv, rq.pre, SCALED);
+        for (int b = 0; b < 12; ++b) {
+            float2 t = w[p][b];
+            if (SCALED) t = mul2(t, make_float2(rq.pre, rq.pre));
+            const float2 q = fma2(t, inv2, mag2);  // |v| <= amax: no clamp needed
+            e[b] = __float_as_uint(q.x);
+            o[b] = __float_as_uint(q.y);
+        }
+        const uint32_t r0[8] = {e[0], e[1], e[2], e[3], e[4], e[5], e[6], e[7]};
+        const uint32_t r1[8] = {e[8], e[9], e[10], e[11], o[0], o[1], o[2], o[3]};
+        const uint32_t r2[8] = {o[4], o[5], o[6], o[7], o[8], o[9], o[10], o[11]};
+        out[3 * p] = nibbles8(r0);
+        out[3 * p + 1] = nibbles8(r1);
+        out[3 * p + 2] = nibbles8(r2);
     }
 }
 
@@ -219,7 +241,9 @@ k_rht_kron_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict
             if (gtid == 0 && it + kStages < nmine) load_row(it + kStages);
             __syncwarp();
             tc_fence_after();
-            float v[96];  // v[12 a0 + b] = D[a1][(a0, b)]
+            // w[p][b] = (D[a1][12 (2p) + b], D[a1][12 (2p + 1) + b]): one pairing of the
+            // values for every step, so that the packed operations need no moves
+            float2 w[4][12];
             {
                 uint32_t r[32];
                 const uint32_t taddr = tmem + (uint32_t(gw * 32) << 16) + uint32_t(slot * 128);
@@ -228,55 +252,56 @@ k_rht_kron_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict
                     tmem_ld32(taddr + 32 * h, r);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) v[32 * h + k] = __uint_as_float(r[k]);
+                    for (int k = 0; k < 32; ++k) {
+                        const int n = 32 * h + k, a0 = n / 12, b = n % 12;
+                        if (a0 & 1) w[a0 >> 1][b].y = __uint_as_float(r[k]);
+                        else w[a0 >> 1][b].x = __uint_as_float(r[k]);
+                    }
                 }
             }
-            // H_8 along a0 (element stride 12), packed over pairs of b
+            // H_8 along a0: bit 0 inside each pair, bits 1 and 2 between pairs
 #pragma unroll
-            for (int s = 1; s < 8; s <<= 1)
+            for (int p = 0; p < 4; ++p)
 #pragma unroll
-                for (int a0 = 0; a0 < 8; ++a0)
-                    if (!(a0 & s))
+                for (int b = 0; b < 12; ++b) w[p][b] = make_float2(w[p][b].x + w[p][b].y, w[p][b].x - w[p][b].y);
 #pragma unroll
-                        for (int c = 0; c < 6; ++c) {
-                            const int i0 = 12 * a0 + 2 * c, i1 = 12 * (a0 | s) + 2 * c;
-                            const float2 u = make_float2(v[i0], v[i0 + 1]), w = make_float2(v[i1], v[i1 + 1]);
-                            const float2 sm = add2(u, w), df = sub2(u, w);
-                            v[i0] = sm.x;
-                            v[i0 + 1] = sm.y;
-                            v[i1] = df.x;
-                            v[i1 + 1] = df.y;
+            for (int s = 1; s < 4; s <<= 1)
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    if (!(p & s))
+#pragma unroll
+                        for (int b = 0; b < 12; ++b) {
+                            const float2 u = w[p][b], x = w[p | s][b];
+                            w[p][b] = add2(u, x);
+                            w[p | s][b] = sub2(u, x);
                         }
-            // dense H_12 along b on each group a0, packed over pairs of groups
+            // dense H_12 along b on groups 2p and 2p + 1 at once
 #pragma unroll
-            for (int g = 0; g < 8; g += 2) {
-                float2 u[12], o[12];
+            for (int p = 0; p < 4; ++p) {
+                float2 o[12];
+                h12_pair(w[p], o);
 #pragma unroll
-                for (int k = 0; k < 12; ++k) u[k] = make_float2(v[12 * g + k], v[12 * (g + 1) + k]);
-                h12_pair(u, o);
-#pragma unroll
-                for (int k = 0; k < 12; ++k) {
-                    v[12 * g + k] = o[k].x;
-                    v[12 * (g + 1) + k] = o[k].y;
-                }
+                for (int k = 0; k < 12; ++k) w[p][k] = o[k];
             }
             float mx[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 96; k += 2) mx[(k >> 1) & 3] = max3(mx[(k >> 1) & 3], fabsf(v[k]), fabsf(v[k + 1]));
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int b = 0; b < 12; ++b) mx[b & 3] = max3(mx[b & 3], fabsf(w[p][b].x), fabsf(w[p][b].y));
             const float wm = warp_max_nonneg(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
             if (lane == 0) sred[gw] = wm;
             named_sync(named, kGroupThreads);  // the four warps of this row
             const float amax = fmaxf(fmaxf(sred[0], sred[1]), fmaxf(sred[2], sred[3]));
             const long long t = r0 + (long long)it * rstep;
             const RowQuant rq = row_quant(amax, qmax);
-            uint32_t w[12];
+            uint32_t wd[12];
             if (rq.pre == 1.0f)  // the same for the whole row
-                quant96<false>(v, rq, w);
+                quant_pairs<false>(w, rq, wd);
             else
-                quant96<true>(v, rq, w);
+                quant_pairs<true>(w, rq, wd);
             uint4 *dst = reinterpret_cast<uint4 *>(codes + t * row_bytes + 48 * a1);
 #pragma unroll
-            for (int k = 0; k < 3; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            for (int k = 0; k < 3; ++k) dst[k] = make_uint4(wd[4 * k], wd[4 * k + 1], wd[4 * k + 2], wd[4 * k + 3]);
             if (gtid == 0) scales[t] = amax > 0.f ? amax / (float(qmax) * sqrtf(float(kKD))) : 0.f;
             // no barrier here: the group's next epilogue follows its next pre-product
             // barrier, which orders these sred reads and TMEM loads before any later write

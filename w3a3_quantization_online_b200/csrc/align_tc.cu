@@ -208,7 +208,7 @@ k_align_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     constexpr int kZTx = (CS - 1) * TPO * 128;  // z rows arriving from the other CTAs
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = smem_align1024(smem_raw);
     uint8_t *sx = base + L::kOffX;
     uint8_t *sq = base + L::kOffQ;
     uint8_t *sz = base + L::kOffZ;

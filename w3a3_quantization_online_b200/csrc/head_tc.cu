@@ -112,7 +112,7 @@ k_head_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUte
     constexpr int kSlabs = L::kSlabs;
     constexpr uint32_t kTx = uint32_t(L::kTileBytes);
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = smem_align1024(smem_raw);
     uint8_t *sb = base + L::kOffB;
     auto xs = [&](int st) { return base + L::kOffX + st * L::kTileBytes; };
     auto os = [&](int b) { return base + L::kOffOut + b * L::kTileBytes; };

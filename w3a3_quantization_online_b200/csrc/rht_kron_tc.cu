@@ -149,7 +149,7 @@ k_rht_kron_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict
     constexpr int qmax = 7;
     constexpr int row_bytes = kKD / 2;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = smem_align1024(smem_raw);
     uint8_t *sa = base + kOffA;
     uint8_t *smask = base + kOffMask;
     uint8_t *sstage = base + kOffStage;

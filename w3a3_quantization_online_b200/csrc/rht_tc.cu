@@ -144,7 +144,7 @@ k_rht_tc(const __grid_constant__ CUtensorMap tm_x, const int8_t *__restrict__ si
     constexpr int qmax = (1 << (BITS - 1)) - 1;
     constexpr int row_bytes = S::kD * BITS / 8;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = smem_align1024(smem_raw);
     uint8_t *sa = base + kOffA;
     uint8_t *smask = base + kOffMask;
     uint8_t *sstage = base + kOffStage;

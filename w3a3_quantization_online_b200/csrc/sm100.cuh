@@ -21,6 +21,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory window advanced to the next 1024-byte boundary
+// (SWIZZLE_128B tiles need it).  The offset is added to the shared array
+// itself, so the compiler still knows every pointer derived from the result
+// to be in shared memory and emits shared-space loads and stores; rounding
+// the address through an integer would make every such access generic.
+__device__ __forceinline__ uint8_t *smem_align1024(uint8_t *raw) {
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

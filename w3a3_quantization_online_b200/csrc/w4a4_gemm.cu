@@ -152,7 +152,7 @@ k_w4a4_gemm(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CU
     constexpr int kPFull = C::kPFull, kPEmpty = C::kPEmpty, kUFull = C::kUFull, kUEmpty = C::kUEmpty;
     constexpr int kAccFull = C::kAccFull, kAccEmpty = C::kAccEmpty, kGBars = C::kGBars;
     extern __shared__ uint8_t gsm_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = smem_align1024(gsm_raw);
     const uint32_t bars = smem_u32(base + kOffBar);
     auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + kOffTm);

@@ -237,7 +237,7 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // Shared-memory matrix descriptor, SWIZZLE_128B canonical layout: 8-row groups
 // of 128-byte rows, groups `sbo` bytes apart.  LBO is ignored by the K-major
 // swizzled layout and only matters for MN-major operands wider than one
-// 64-element atom (never the case here).
+// 64-element atom (those use smem_desc_sw128_lbo below).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t sbo_bytes) {
     uint64_t d = 0;
     d |= uint64_t((saddr >> 4) & 0x3FFF);          // start address

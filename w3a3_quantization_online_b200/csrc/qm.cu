@@ -35,75 +35,165 @@ namespace rsq {
 namespace {
 
 constexpr int kQmThreads = 256;
-constexpr int kGemmBM = 32, kGemmBN = 64, kGemmBK = 32;
 constexpr int kGramRows = 128;  // rows of X per partial Gram block
+
+// Skinny product tiles: a CTA computes 16 rows x 64 columns of C; its two halves
+// of 128 threads take the two halves of the K range (D / 2 each) and add their
+// partial sums at the end in a fixed order (no atomics).  A half stages K steps
+// of 32 through two shared buffers (the next step's tiles are loaded into
+// registers while the current one is multiplied); a thread holds 2 x 4 outputs.
+constexpr int kGemmBM = 16, kGemmBN = 64, kGemmBK = 32;
+constexpr int kGemmThreads = 256;
+constexpr int kGemmLdA = kGemmBM + 2;                          // row stride of the A tile (doubles)
+constexpr int kGemmTileA = kGemmBK * kGemmLdA, kGemmTileB = kGemmBK * kGemmBN;
+constexpr int kGemmHalf = 2 * (kGemmTileA + kGemmTileB);       // doubles per half (two buffers)
+constexpr size_t kGemmSmem = size_t(2) * kGemmHalf * 8;
 
 // C[i][c] = sum_j op(A)[i][j] B[j][c] (- S[i][c]) (+ mu P[i][c]), A D x D
 // float32 row-major (op(A) = A or A^T), B, C, S, P D x ncols float64 with row
-// stride ld, mu a device scalar.  C may be P (each element is read, then
-// written, by the same thread).
+// stride ld (even, ncols <= ld), mu a device scalar.  C may be P (each element
+// is read, then written, by the same thread).  D a multiple of 64.
 template <bool TRANS>
-__global__ void __launch_bounds__(kQmThreads)
+__global__ void __launch_bounds__(kGemmThreads)
 k_qm_gemm(const float *__restrict__ A, const double *__restrict__ B, double *C, const double *__restrict__ S,
           const double *P, const double *__restrict__ mu, int D, int ncols, int ld) {
-    __shared__ double sa[kGemmBK][kGemmBM + 1];  // sa[j][i] = op(A)[i0 + i][j0 + j]
-    __shared__ double sb[kGemmBK][kGemmBN];
-    const int tid = threadIdx.x;
+    extern __shared__ double gsm[];
+    const int tid = threadIdx.x, half = tid >> 7, t = tid & 127;
+    double *sa = gsm + half * kGemmHalf;  // [buffer][k][i], row stride kGemmLdA
+    double *sb = sa + 2 * kGemmTileA;     // [buffer][k][c]
     const int i0 = blockIdx.x * kGemmBM, c0 = blockIdx.y * kGemmBN;
-    const int ty = tid >> 4, tx = tid & 15;  // rows ty, ty + 16; columns tx + 16 k
-    double acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-    for (int j0 = 0; j0 < D; j0 += kGemmBK) {
-        for (int e = tid; e < kGemmBM * kGemmBK; e += kQmThreads) {
-            if (TRANS) {  // op(A)[i][j] = A[j][i]: rows j of A, contiguous in i
-                const int jj = e / kGemmBM, ii = e % kGemmBM;
-                sa[jj][ii] = double(A[(size_t)(j0 + jj) * D + i0 + ii]);
-            } else {      // A[i][j], contiguous in j
-                const int ii = e / kGemmBK, jj = e % kGemmBK;
-                sa[jj][ii] = double(A[(size_t)(i0 + ii) * D + j0 + jj]);
-            }
+    const int ty = t >> 4, tx = t & 15;   // rows 2 ty, 2 ty + 1; columns 2 tx + {0, 1} and 32 + 2 tx + {0, 1}
+    const int steps = D / kGemmBK / 2, k_first = half * steps * kGemmBK;
+    float4 ra;                            // the next step's A values (one float4 per thread)
+    double2 rb[8];                        // and B values (eight pairs per thread)
+    auto load = [&](int k0) {
+        if (TRANS) {  // op(A)[i][k] = A[k][i]: 32 rows k of 16 contiguous i
+            ra = *reinterpret_cast<const float4 *>(A + (size_t)(k0 + (t >> 2)) * D + i0 + 4 * (t & 3));
+        } else {      // A[i][k]: 16 rows i of 32 contiguous k
+            ra = *reinterpret_cast<const float4 *>(A + (size_t)(i0 + (t >> 3)) * D + k0 + 4 * (t & 7));
         }
-        for (int e = tid; e < kGemmBK * kGemmBN; e += kQmThreads) {
-            const int jj = e / kGemmBN, cc = e % kGemmBN;
-            sb[jj][cc] = c0 + cc < ncols ? B[(size_t)(j0 + jj) * ld + c0 + cc] : 0.0;
-        }
-        __syncthreads();
-#pragma unroll 4
-        for (int jj = 0; jj < kGemmBK; ++jj) {
-            const double a0 = sa[jj][ty], a1 = sa[jj][ty + 16];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const double b = sb[jj][tx + 16 * k];
-                acc[0][k] = fma(a0, b, acc[0][k]);
-                acc[1][k] = fma(a1, b, acc[1][k]);
+        for (int j = 0; j < 8; ++j) {  // 32 rows k of 32 column pairs: a warp reads one row
+            const int idx = t + 128 * j, kk = idx >> 5, cc = 2 * (idx & 31);
+            double2 v = make_double2(0.0, 0.0);
+            if (c0 + cc < ncols) {
+                v = *reinterpret_cast<const double2 *>(B + (size_t)(k0 + kk) * ld + c0 + cc);
+                if (c0 + cc + 1 >= ncols) v.y = 0.0;
+            }
+            rb[j] = v;
+        }
+    };
+    auto store = [&](int buf) {
+        double *a = sa + buf * kGemmTileA;
+        double *b = sb + buf * kGemmTileB;
+        if (TRANS) {
+            const int kk = t >> 2, ii = 4 * (t & 3);
+            a[kk * kGemmLdA + ii] = double(ra.x);
+            a[kk * kGemmLdA + ii + 1] = double(ra.y);
+            a[kk * kGemmLdA + ii + 2] = double(ra.z);
+            a[kk * kGemmLdA + ii + 3] = double(ra.w);
+        } else {
+            const int ii = t >> 3, kk = 4 * (t & 7);
+            a[kk * kGemmLdA + ii] = double(ra.x);
+            a[(kk + 1) * kGemmLdA + ii] = double(ra.y);
+            a[(kk + 2) * kGemmLdA + ii] = double(ra.z);
+            a[(kk + 3) * kGemmLdA + ii] = double(ra.w);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int idx = t + 128 * j;
+            *reinterpret_cast<double2 *>(b + (idx >> 5) * kGemmBN + 2 * (idx & 31)) = rb[j];
+        }
+    };
+    double acc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+    load(k_first);
+    store(0);
+    __syncthreads();
+    for (int st = 0; st < steps; ++st) {
+        const int cur = st & 1;
+        if (st + 1 < steps) load(k_first + (st + 1) * kGemmBK);
+        const double *a = sa + cur * kGemmTileA;
+        const double *b = sb + cur * kGemmTileB;
+#pragma unroll 8
+        for (int kk = 0; kk < kGemmBK; ++kk) {
+            const double2 av = *reinterpret_cast<const double2 *>(a + kk * kGemmLdA + 2 * ty);
+            const double2 b0 = *reinterpret_cast<const double2 *>(b + kk * kGemmBN + 2 * tx);
+            const double2 b1 = *reinterpret_cast<const double2 *>(b + kk * kGemmBN + 32 + 2 * tx);
+            const double bv[4] = {b0.x, b0.y, b1.x, b1.y};
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                acc[0][n] = fma(av.x, bv[n], acc[0][n]);
+                acc[1][n] = fma(av.y, bv[n], acc[1][n]);
             }
         }
+        if (st + 1 < steps) store(cur ^ 1);
         __syncthreads();
     }
+    // the second half's partial sums through shared memory, then first + second
+    double *red = gsm;  // [8][128]
+    if (half == 1) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = i0 + ty + 16 * h, c = c0 + tx + 16 * k;
-            if (c < ncols) {
-                double v = S ? acc[h][k] - S[(size_t)i * ld + c] : acc[h][k];
-                if (P) v = fma(*mu, P[(size_t)i * ld + c], v);
-                C[(size_t)i * ld + c] = v;
+            for (int n = 0; n < 4; ++n) red[(4 * m + n) * 128 + t] = acc[m][n];
+    }
+    __syncthreads();
+    if (half == 0) {
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int i = i0 + 2 * ty + m, c = c0 + (n < 2 ? 2 * tx + n : 32 + 2 * tx + n - 2);
+                if (c < ncols) {
+                    double v = acc[m][n] + red[(4 * m + n) * 128 + t];
+                    if (S) v -= S[(size_t)i * ld + c];
+                    if (P) v = fma(*mu, P[(size_t)i * ld + c], v);
+                    C[(size_t)i * ld + c] = v;
+                }
             }
-        }
+    }
 }
 
-// Partial cross-Gram of a block of kGramRows rows: P[blk][a][b] = sum_i X[i][a] Y[i][b].
+// Partial cross-Gram of a block of kGramRows rows: P[blk][a][b] = sum_i X[i][a] Y[i][b]
+// (p, q <= 96), the rows in order.  Rows pass through shared memory 16 at a
+// time; thread (ta, tb) of a 16 x 16 grid holds the outputs a = ta + 16 m,
+// b = tb + 16 n.
+constexpr int kGramChunk = 16, kGramMax = 96, kGramPer = kGramMax / 16;
 __global__ void __launch_bounds__(kQmThreads)
 k_qm_gram(const double *__restrict__ X, const double *__restrict__ Y, double *__restrict__ P, int D, int p, int q,
           int ld) {
-    const int blk = blockIdx.x;
+    __shared__ double sx[kGramChunk][kGramMax], sy[kGramChunk][kGramMax];
+    const int blk = blockIdx.x, tid = threadIdx.x, ta = tid & 15, tb = tid >> 4;
     const int r0 = blk * kGramRows, r1 = min(D, r0 + kGramRows);
-    for (int e = threadIdx.x; e < p * q; e += kQmThreads) {
-        const int a = e / q, b = e % q;
-        double s = 0.0;
-        for (int i = r0; i < r1; ++i) s = fma(X[(size_t)i * ld + a], Y[(size_t)i * ld + b], s);
-        P[(size_t)blk * p * q + e] = s;
+    double acc[kGramPer][kGramPer];
+#pragma unroll
+    for (int m = 0; m < kGramPer; ++m)
+#pragma unroll
+        for (int n = 0; n < kGramPer; ++n) acc[m][n] = 0.0;
+    for (int c0 = r0; c0 < r1; c0 += kGramChunk) {
+        const int rows = min(kGramChunk, r1 - c0);
+        for (int e = tid; e < rows * p; e += kQmThreads) sx[e / p][e % p] = X[(size_t)(c0 + e / p) * ld + e % p];
+        for (int e = tid; e < rows * q; e += kQmThreads) sy[e / q][e % q] = Y[(size_t)(c0 + e / q) * ld + e % q];
+        __syncthreads();
+        for (int rr = 0; rr < rows; ++rr) {
+#pragma unroll
+            for (int m = 0; m < kGramPer; ++m) {
+                if (ta + 16 * m >= p) continue;
+                const double xv = sx[rr][ta + 16 * m];
+#pragma unroll
+                for (int n = 0; n < kGramPer; ++n)
+                    if (tb + 16 * n < q) acc[m][n] = fma(xv, sy[rr][tb + 16 * n], acc[m][n]);
+            }
+        }
+        __syncthreads();
     }
+#pragma unroll
+    for (int m = 0; m < kGramPer; ++m)
+#pragma unroll
+        for (int n = 0; n < kGramPer; ++n) {
+            const int a = ta + 16 * m, b = tb + 16 * n;
+            if (a < p && b < q) P[(size_t)blk * p * q + (size_t)a * q + b] = acc[m][n];
+        }
 }
 
 // Partial sums of squares of a block of kGramRows rows of Y (D x p, row stride ld).
@@ -203,8 +293,10 @@ __device__ void qm_jacobi(double *a, double *v, int n, double *cs, int *pr) {
             }
             __syncthreads();
             // columns: a <- a J, v <- v J (J rotates columns p, q of each pair)
+            // (consecutive threads take different pairs of one row: the column
+            // stride n would put a warp's accesses in one bank)
             for (int e = tid; e < (m / 2) * n; e += blockDim.x) {
-                const int k = e / n, row = e % n;
+                const int row = e / (m / 2), k = e % (m / 2);
                 const int p = pr[2 * k], q = pr[2 * k + 1];
                 if (q >= n) continue;
                 const double c = cs[2 * k], s = cs[2 * k + 1];
@@ -246,15 +338,20 @@ __device__ void qm_order_desc(const double *a, int n, int *order) {
 }
 
 // CHOL: G (p x p) = Rc^T Rc; out = Rc^-1 (upper triangular).  status bit 2 if G
-// is not positive definite.  One p x p shared array: the Cholesky factor L
-// (Rc = L^T) fills the lower triangle, then L^-1 is written transposed into the
-// strict upper triangle (entry (i, c), i > c, of L^-1 at (c, i)).
+// is not positive definite.  Two p x p shared arrays: the Cholesky factor L
+// (Rc = L^T) in the lower triangle of the first, X = L^-1 in the second; a
+// copy of the current column of L keeps the trailing update free of
+// shared-memory bank conflicts.
 __global__ void __launch_bounds__(kQmThreads) k_qm_chol_inv(const double *__restrict__ G, double *__restrict__ out,
                                                             int p, int *status) {
     extern __shared__ double sm[];
-    double *L = sm;
+    double *L = sm, *X = sm + p * p;
+    __shared__ double colj[kGramMax];
     const int tid = threadIdx.x;
-    for (int e = tid; e < p * p; e += blockDim.x) L[e] = G[e];
+    for (int e = tid; e < p * p; e += blockDim.x) {
+        L[e] = G[e];
+        X[e] = (e / p == e % p) ? 1.0 : 0.0;
+    }
     __shared__ int bad;
     if (tid == 0) bad = 0;
     __syncthreads();
@@ -266,28 +363,36 @@ __global__ void __launch_bounds__(kQmThreads) k_qm_chol_inv(const double *__rest
         }
         __syncthreads();
         const double djj = L[j * p + j];
-        for (int i = j + 1 + tid; i < p; i += blockDim.x) L[i * p + j] /= djj;
+        for (int i = j + 1 + tid; i < p; i += blockDim.x) {
+            const double lij = L[i * p + j] / djj;
+            L[i * p + j] = lij;
+            colj[i] = lij;
+        }
         __syncthreads();
         const int w = p - j - 1;
         for (int e = tid; e < w * w; e += blockDim.x) {
             const int i = j + 1 + e / w, k = j + 1 + e % w;
-            if (k <= i) L[i * p + k] -= L[i * p + j] * L[k * p + j];
+            if (k <= i) L[i * p + k] -= colj[i] * colj[k];
         }
         __syncthreads();
     }
-    // column c of L^-1 by forward substitution (one column per thread); its
-    // entries below the diagonal go to row c of the strict upper triangle
-    for (int c = tid; c < p; c += blockDim.x) {
-        for (int i = c + 1; i < p; ++i) {
-            double s = -L[i * p + c] / L[c * p + c];
-            for (int k = c + 1; k < i; ++k) s -= L[i * p + k] * L[c * p + k];
-            L[c * p + i] = s / L[i * p + i];
+    // X = L^-1 by forward elimination on the rows of [L | I]: row k of X is
+    // final once divided by L[k][k]; it is then taken from the rows below
+    // (only its columns c <= k are nonzero)
+    for (int k = 0; k < p; ++k) {
+        const double dkk = L[k * p + k];
+        for (int c = tid; c <= k; c += blockDim.x) X[k * p + c] /= dkk;
+        __syncthreads();
+        const int w = k + 1;
+        for (int e = tid; e < (p - k - 1) * w; e += blockDim.x) {
+            const int i = k + 1 + e / w, c = e % w;
+            X[i * p + c] -= L[i * p + k] * X[k * p + c];
         }
+        __syncthreads();
     }
-    __syncthreads();
-    for (int e = tid; e < p * p; e += blockDim.x) {  // Rc^-1 = (L^-1)^T: entry (i, c) = L^-1 (c, i)
+    for (int e = tid; e < p * p; e += blockDim.x) {  // Rc^-1 = (L^-1)^T: entry (i, c) = X[c][i]
         const int i = e / p, c = e % p;
-        out[e] = i < c ? L[i * p + c] : (i == c ? 1.0 / L[c * p + c] : 0.0);
+        out[e] = i <= c ? X[c * p + i] : 0.0;
     }
     if (tid == 0 && bad) atomicOr(status, 2);
 }
@@ -476,8 +581,8 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     qm_layout(D, r, &w, workspace);
     const int p = w.p;
     const int ew = int(std::min<long long>((long long)D * p / kQmThreads + 1, (long long)num_sms() * 8));
-    const dim3 ggrid(D / kGemmBM, (p + kGemmBN - 1) / kGemmBN);
-    const size_t chol_smem = size_t(p) * p * 8;
+    const dim3 ggrid(D / kGemmBM, (p + kGemmBN - 1) / kGemmBN), rgrid(D / kGemmBM, (r + kGemmBN - 1) / kGemmBN);
+    const size_t chol_smem = size_t(2) * p * p * 8;
     const size_t eig_smem = size_t(2) * p * p * 8 + size_t(p + 2) * 16 + size_t(2 * p + 4) * 4;
     const size_t pol_smem = size_t(5) * r * r * 8 + size_t(r + 2) * 16 + size_t(2 * r + 4) * 4;
     static bool configured[64];
@@ -485,7 +590,11 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && !configured[dev]) {
-        e = cudaFuncSetAttribute(k_qm_chol_inv, cudaFuncAttributeMaxDynamicSharedMemorySize, int(96 * 96 * 8));
+        e = cudaFuncSetAttribute(k_qm_chol_inv, cudaFuncAttributeMaxDynamicSharedMemorySize, int(2 * 96 * 96 * 8));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_qm_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_qm_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGemmSmem));
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_qm_top_eig, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      int(2 * 96 * 96 * 8 + 98 * 16 + 196 * 4));
@@ -510,8 +619,8 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     };
     // Y <- dT^T X = R_in (R_out^T X) - X, using Z as scratch
     auto dtT = [&](const double *X, double *Y, double *Zs) {
-        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_out, X, Zs, nullptr, nullptr, nullptr, D, p, p);
-        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_in, Zs, Y, X, nullptr, nullptr, D, p, p);
+        k_qm_gemm<true><<<ggrid, kGemmThreads, kGemmSmem, s>>>(R_out, X, Zs, nullptr, nullptr, nullptr, D, p, p);
+        k_qm_gemm<false><<<ggrid, kGemmThreads, kGemmSmem, s>>>(R_in, Zs, Y, X, nullptr, nullptr, D, p, p);
         return qm_check(2);
     };
     // X <- dT Y + mu X = R_out (R_in^T Y) - Y + mu X: the shift mu > 0 keeps the
@@ -520,8 +629,8 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     auto dt_shift = [&](const double *Y, double *X, double *Zs) {
         k_qm_sumsq<<<w.nblk, kQmThreads, 0, s>>>(Y, w.P, D, p, p);
         k_qm_mu<<<1, 1, 0, s>>>(w.P, w.nblk, p, w.mu);
-        k_qm_gemm<true><<<ggrid, kQmThreads, 0, s>>>(R_in, Y, Zs, nullptr, nullptr, nullptr, D, p, p);
-        k_qm_gemm<false><<<ggrid, kQmThreads, 0, s>>>(R_out, Zs, X, Y, X, w.mu, D, p, p);
+        k_qm_gemm<true><<<ggrid, kGemmThreads, kGemmSmem, s>>>(R_in, Y, Zs, nullptr, nullptr, nullptr, D, p, p);
+        k_qm_gemm<false><<<ggrid, kGemmThreads, kGemmSmem, s>>>(R_out, Zs, X, Y, X, w.mu, D, p, p);
         return qm_check(4);
     };
     k_qm_init<<<ew, kQmThreads, 0, s>>>(w.X, D, p, p);
@@ -540,8 +649,8 @@ cudaError_t launch_qm_build(const float *R_in, const float *R_out, int D, int r,
     k_qm_apply<<<ew, kQmThreads, 0, s>>>(w.X, w.Wt, w.Z, D, p, r, p, p, 0);  // Q in Z (row stride p)
     if ((e = qm_check(4)) != cudaSuccess) return e;
     // T_sub = (R_out^T Q)^T (R_in^T Q)
-    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_out, w.Z, w.X, nullptr, nullptr, nullptr, D, r, p);
-    k_qm_gemm<true><<<dim3(D / kGemmBM, 1), kQmThreads, 0, s>>>(R_in, w.Z, w.Y, nullptr, nullptr, nullptr, D, r, p);
+    k_qm_gemm<true><<<rgrid, kGemmThreads, kGemmSmem, s>>>(R_out, w.Z, w.X, nullptr, nullptr, nullptr, D, r, p);
+    k_qm_gemm<true><<<rgrid, kGemmThreads, kGemmSmem, s>>>(R_in, w.Z, w.Y, nullptr, nullptr, nullptr, D, r, p);
     k_qm_gram<<<w.nblk, kQmThreads, 0, s>>>(w.X, w.Y, w.P, D, r, r, p);
     k_qm_gram_reduce<<<(r * r + 255) / 256, 256, 0, s>>>(w.P, w.G, w.nblk, r * r);
     k_qm_polar<<<1, kQmThreads, pol_smem, s>>>(w.G, M, r, status);

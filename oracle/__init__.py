@@ -53,6 +53,8 @@ def lib():
             L.ora_head_mix_quant.argtypes = [i64, i32, i32, i32, _D, _I8, _I8, _U8, _D, _D]
             L.ora_w4a4_gemm.argtypes = [i64, i32, i32, _U8, _D, _U8, _D, ctypes.POINTER(ctypes.c_int32), _D]
             L.ora_rht_quant_gate.argtypes = [i64, i32, i32, i32, _D, _D, _D, _I8, _I8, _U8, _D, _D]
+            L.ora_kron_affine.argtypes = [i64, i32, i32, _D, _D, _D, _D]
+            L.ora_kron_affine_quant.argtypes = [i64, i32, i32, i32, _D, _D, _D, _I8, _U8, _D, _D]
             _lib = L
     return _lib
 
@@ -272,6 +274,38 @@ def head_mix_quant(x, signs, n_heads: int, bits: int, want_pre: bool = True) -> 
                                   _p(scales, _D), _p(pre, _D))
     if rc:
         raise ValueError(f"oracle rejected d={d}, n_heads={n_heads}, bits={bits} (rc={rc})")
+    return {"q": q, "codes": codes, "scales": scales, "pre": pre}
+
+
+def kron_affine(x, P1, P2) -> np.ndarray:
+    """FlatQuant's Kronecker affine transform of each row: x P with P = P1 (x) P2,
+    computed as vec(P1^T X P2) with X the n1 x n2 row-major reshape of the row."""
+    x, P1, P2 = _f64(x), _f64(P1), _f64(P2)
+    T, n = x.shape
+    n1, n2 = P1.shape[0], P2.shape[0]
+    if n1 * n2 != n:
+        raise ValueError(f"n1 * n2 = {n1 * n2} != row length {n}")
+    v = np.empty_like(x)
+    if lib().ora_kron_affine(T, n1, n2, _p(P1, _D), _p(P2, _D), _p(x, _D), _p(v, _D)):
+        raise ValueError(f"n1={n1}, n2={n2}")
+    return v
+
+
+def kron_affine_quant(x, P1, P2, bits: int, want_pre: bool = True) -> dict:
+    """Kronecker affine transform -> symmetric per-token quantisation -> pack."""
+    x, P1, P2 = _f64(x), _f64(P1), _f64(P2)
+    T, n = x.shape
+    n1, n2 = P1.shape[0], P2.shape[0]
+    if n1 * n2 != n:
+        raise ValueError(f"n1 * n2 = {n1 * n2} != row length {n}")
+    q = np.empty((T, n), dtype=np.int8)
+    codes = np.empty((T, n * bits // 8), dtype=np.uint8)
+    scales = np.empty(T, dtype=np.float64)
+    pre = np.empty_like(x) if want_pre else None
+    rc = lib().ora_kron_affine_quant(T, n1, n2, bits, _p(P1, _D), _p(P2, _D), _p(x, _D), _p(q, _I8),
+                                     _p(codes, _U8), _p(scales, _D), _p(pre, _D))
+    if rc:
+        raise ValueError(f"oracle rejected n1={n1}, n2={n2}, bits={bits} (rc={rc})")
     return {"q": q, "codes": codes, "scales": scales, "pre": pre}
 
 

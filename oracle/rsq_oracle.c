@@ -47,7 +47,17 @@
  *   - RMSNorm is n = x / sqrt(mean(x^2) + eps), with no weight;
  *   - INT4 packing: element 2i in the low nibble of byte i, 2i+1 in the high
  *     nibble, two's complement; INT3 packing: 8 codes per 3 bytes, code k of a
- *     group in bits [3k, 3k+3) of the little-endian 24-bit word.
+ *     group in bits [3k, 3k+3) of the little-endian 24-bit word;
+ *   - FlatQuant's Kronecker affine transform: a token row x of length
+ *     n = n1 n2 is the row vector vec(X) of the n1 x n2 matrix
+ *     X[a][b] = x[a n2 + b] (row-major vec), and x P with P = P1 (x) P2 is
+ *     vec(P1^T X P2); the quantiser that follows is the symmetric one above
+ *     (not FlatQuant's asymmetric grid, which the rest of the pages do not
+ *     use), with no clipping factor.
+ *
+ *   [IQ2] also: FlatQuant (the Kronecker-product affine transform
+ *         P = P1 (x) P2 with vec(V)(P1 (x) P2) = vec(P1^T V P2), fused with
+ *         the activation quantiser in one kernel).
  */
 #include <math.h>
 #include <stdint.h>
@@ -606,5 +616,84 @@ int ora_w4a4_gemm(int64_t T, int N, int K, const uint8_t *ca, const double *sa, 
         free(qa);
     }
     free(qw);
+    return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FlatQuant's Kronecker affine transform                                   */
+/* ------------------------------------------------------------------------ */
+
+/* [IQ2] FlatQuant: x P = vec(P1^T X P2) for P = P1 (x) P2, X the n1 x n2
+ * row-major reshape of the row x.  P1 is n1 x n1, P2 is n2 x n2, row-major.
+ * First Z = P1^T X (Z[i][b] = sum_a P1[a][i] X[a][b]), then V = Z P2
+ * (V[i][j] = sum_b Z[i][b] P2[b][j]), v[i n2 + j] = V[i][j]. */
+static void kron_affine_row(int n1, int n2, const double *P1, const double *P2, const double *x, double *z,
+                            double *v)
+{
+    for (int i = 0; i < n1; ++i)
+        for (int b = 0; b < n2; ++b) {
+            double acc = 0.0;
+            for (int a = 0; a < n1; ++a) acc += P1[a * n1 + i] * x[a * n2 + b];
+            z[i * n2 + b] = acc;
+        }
+    for (int i = 0; i < n1; ++i)
+        for (int j = 0; j < n2; ++j) {
+            double acc = 0.0;
+            for (int b = 0; b < n2; ++b) acc += z[i * n2 + b] * P2[b * n2 + j];
+            v[i * n2 + j] = acc;
+        }
+}
+
+/* The transform alone (tests of the index convention). */
+int ora_kron_affine(int64_t T, int n1, int n2, const double *P1, const double *P2, const double *x, double *v)
+{
+    if (n1 < 1 || n2 < 1) return -1;
+    int64_t n = (int64_t)n1 * n2;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)n);
+        if (!z) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) kron_affine_row(n1, n2, P1, P2, x + t * n, z, v + t * n);
+        }
+        free(z);
+    }
+    return err;
+}
+
+/* [IQ2] FlatQuant: the affine transform fused with the activation quantiser,
+ * Q(P1^T X P2) per token row; the per-token symmetric quantiser and packing
+ * as for the other paths. */
+int ora_kron_affine_quant(int64_t T, int n1, int n2, int bits, const double *P1, const double *P2,
+                          const double *x, int8_t *q, uint8_t *codes, double *scales, double *pre)
+{
+    if (n1 < 1 || n2 < 1) return -1;
+    int n = n1 * n2;
+    if ((bits != 3 && bits != 4) || (n * bits) % 8 || (bits == 3 && n % 8)) return -1;
+    int row_bytes = n * bits / 8;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)n);
+        double *v = (double *)malloc(sizeof(double) * (size_t)n);
+        if (!z || !v) {
+#pragma omp atomic write
+            err = -2;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                kron_affine_row(n1, n2, P1, P2, x + t * n, z, v);
+                scales[t] = quant_row(n, bits, v, q + t * n, pre ? pre + t * n : NULL);
+                if (bits == 4) pack_int4_row(n, q + t * n, codes + t * row_bytes);
+                else pack_int3_row(n, q + t * n, codes + t * row_bytes);
+            }
+        }
+        free(z);
+        free(v);
+    }
     return err;
 }

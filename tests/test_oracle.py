@@ -580,3 +580,61 @@ def test_qm_feeds_the_online_path():
     x = np.random.default_rng(2).normal(size=(7, 256))
     np.testing.assert_allclose(oracle.residual_align(x, c["Q"], c["M"]), x @ oracle.t_hat(c["Q"], c["M"]).T,
                                rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# FlatQuant's Kronecker affine transform (Infra Quant II, FlatQuant):
+# x P with P = P1 (x) P2 is vec(P1^T X P2), X the row-major n1 x n2 reshape
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("n1,n2", [(4, 8), (8, 4), (3, 5), (12, 16)])
+def test_kron_affine_equals_the_explicit_kronecker_product(n1, n2):
+    # numpy's kron gives P[a n2 + b][i n2 + j] = P1[a][i] P2[b][j]; the factors are
+    # not symmetric and the shapes not square, so a transposed factor, swapped
+    # roles of n1 and n2 or a column-major reshape all fail
+    rng = np.random.default_rng(100 * n1 + n2)
+    P1, P2 = rng.standard_normal((n1, n1)), rng.standard_normal((n2, n2))
+    x = rng.standard_normal((5, n1 * n2))
+    ref = x @ np.kron(P1, P2)
+    np.testing.assert_allclose(oracle.kron_affine(x, P1, P2), ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+
+
+def test_kron_affine_is_undone_by_the_inverse_factors():
+    # (P1 (x) P2)^-1 = P1^-1 (x) P2^-1
+    c = inputs.kron_affine_case(6, 8, 16, 2, dtype="f32")
+    v = oracle.kron_affine(c.x, c.P1, c.P2)
+    back = oracle.kron_affine(v, np.linalg.inv(c.P1.astype(np.float64)), np.linalg.inv(c.P2.astype(np.float64)))
+    np.testing.assert_allclose(back, c.x, rtol=0, atol=1e-9 * np.abs(c.x).max())
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_kron_affine_quant_with_identity_factors_is_the_plain_quantiser(bits):
+    c = inputs.kron_affine_case(7, 8, 16, 4, dtype="f32", bits=bits)
+    r = oracle.kron_affine_quant(c.x, np.eye(8), np.eye(16), bits)
+    q, a, _ = oracle.quant_sym(c.x, bits)
+    np.testing.assert_array_equal(r["q"], q)
+    np.testing.assert_array_equal(r["scales"], a)
+    np.testing.assert_array_equal(r["codes"], oracle.pack(q, bits))
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_kron_affine_quant_with_sylvester_factors_is_the_hadamard_path(bits):
+    # H_n1 (x) H_n2 = H_{n1 n2} (Sylvester, index a n2 + b): the codes are those of
+    # the unrandomised Hadamard path, whose values carry the extra 1/sqrt(d)
+    n1, n2 = 16, 32
+    c = inputs.kron_affine_case(9, n1, n2, 5, dtype="f32", bits=bits)
+    r = oracle.kron_affine_quant(c.x, oracle.sylvester(n1), oracle.sylvester(n2), bits)
+    h = oracle.rht_quant(c.x, np.ones(n1 * n2, dtype=np.int8), 1, bits)
+    np.testing.assert_array_equal(r["q"], h["q"])
+    np.testing.assert_allclose(r["scales"], h["scales"] * math.sqrt(n1 * n2), rtol=1e-12)
+
+
+def test_kron_affine_quant_zero_rows_and_step_bound():
+    c = inputs.kron_affine_case(6, 8, 8, 6, dtype="f32", bits=4)
+    x = c.x.copy()
+    x[2] = 0.0
+    r = oracle.kron_affine_quant(x, c.P1, c.P2, 4)
+    assert r["scales"][2] == 0.0 and not r["q"][2].any()
+    v = oracle.kron_affine(x, c.P1, c.P2)
+    deq = r["q"].astype(np.float64) * r["scales"][:, None]
+    assert np.all(np.abs(deq - v) <= 0.5 * r["scales"][:, None] * (1 + 1e-12))

@@ -21,7 +21,12 @@ Recipe (numpy ``Generator(PCG64)``, one independent stream per array, keyed by
   for the polar-decomposed rotation that calibration would produce
   (ReSpinQuant page, "key design 2" and "key design 3");
 * ``signs``: int8 +-1 drawn uniformly (Infra Quant II page, QuaRot background:
-  the randomised Hadamard H diag(s) with s drawn from {+1, -1}).
+  the randomised Hadamard H diag(s) with s drawn from {+1, -1});
+* ``P1``, ``P2`` of FlatQuant's Kronecker affine transform (Infra Quant II page,
+  FlatQuant: two small invertible matrices, learned by calibration): each is
+  the orthonormal QR factor of a Gaussian matrix times a diagonal of
+  exp(N(0, 0.25^2)) column scales, an invertible, well-conditioned, not
+  orthogonal stand-in for a learned factor; handed over as float32.
 
 Q and M are handed to the kernels as float32; the float64 originals are kept
 for the pins that need exact orthogonality.
@@ -34,7 +39,7 @@ from typing import Optional
 import numpy as np
 
 # stream ids of SeedSequence([seed, stream])
-_S_X, _S_OUTLIER, _S_Q, _S_A, _S_SIGNS, _S_GATE = 0, 1, 2, 3, 4, 5
+_S_X, _S_OUTLIER, _S_Q, _S_A, _S_SIGNS, _S_GATE, _S_P1, _S_P2 = 0, 1, 2, 3, 4, 5, 6, 7
 
 _CHUNK_ROWS = 2048
 
@@ -181,6 +186,52 @@ class RhtCase:
         return self.x.shape[1]
 
 
+def affine_factor(n: int, seed: int, stream: int) -> np.ndarray:
+    """n x n invertible float32 matrix: orthonormal QR factor of a Gaussian matrix
+    (columns sign-fixed) times exp(N(0, 0.25^2)) column scales."""
+    rng = _rng(seed, stream)
+    q, rr = np.linalg.qr(rng.standard_normal((n, n)))
+    sgn = np.sign(np.diag(rr))
+    sgn[sgn == 0] = 1.0
+    c = np.exp(0.25 * rng.standard_normal(n))
+    return (q * (sgn * c)[None, :]).astype(np.float32)
+
+
+@dataclasses.dataclass
+class KronAffineCase:
+    """Inputs of one Kronecker affine transform + quantiser problem."""
+    name: str
+    x: np.ndarray          # T x (n1 n2) float32 holding the exact I/O values
+    P1: np.ndarray         # n1 x n1 float32
+    P2: np.ndarray         # n2 x n2 float32
+    dtype: str
+    bits: int
+
+    @property
+    def T(self) -> int:
+        return self.x.shape[0]
+
+    @property
+    def d(self) -> int:
+        return self.x.shape[1]
+
+    @property
+    def n1(self) -> int:
+        return self.P1.shape[0]
+
+    @property
+    def n2(self) -> int:
+        return self.P2.shape[0]
+
+
+def kron_affine_case(T: int, n1: int, n2: int, seed: int, *, dtype: str = "bf16", bits: int = 4,
+                     n_outliers: int = 8, outlier_scale: float = 20.0, name: str = "") -> KronAffineCase:
+    d = n1 * n2
+    x = activations(T, d, seed, "normal", min(n_outliers, d), outlier_scale, dtype)
+    return KronAffineCase(name or f"affine_T{T}_{n1}x{n2}", x, affine_factor(n1, seed, _S_P1),
+                          affine_factor(n2, seed, _S_P2), dtype, bits)
+
+
 def align_case(T: int, D: int, r: int, seed: int, *, dtype: str = "bf16", bits: int = 4,
                dist: str = "normal", n_outliers: int = 0, outlier_scale: float = 1.0,
                qm_seed: Optional[int] = None, eps: float = 1e-5, name: str = "") -> AlignCase:
@@ -322,6 +373,13 @@ def down_proj_gate_case(T: int = 4096) -> GateCase:
 def down_proj_case(T: int = 4096):
     """FFN down_proj input SiLU(a)*b, d=12288=1024*12, bf16, H_1024 (x) H_12, INT4."""
     return rht_case(T, 12288, 12, 2, dtype="bf16", bits=4, dist="silu_gate", name=f"downproj_T{T}_d12288")
+
+
+def flatquant_case(T: int = 16384) -> KronAffineCase:
+    """FlatQuant's Kronecker affine transform on the hidden stream: d = 4096 =
+    64 x 64 (n1 = n2 = 64, the split that minimises n1 + n2), bf16, 8 outlier
+    channels x20, INT4."""
+    return kron_affine_case(T, 64, 64, 11, dtype="bf16", bits=4, name=f"flatquant_T{T}_64x64")
 
 
 def w3a3_case(T: int = 8192):

@@ -692,6 +692,23 @@ def next_rows_metrics(dev, stream, pk: dict) -> dict:
     out["rht_head_mix_quant"] = _hbm(c.T * (c.d * 2 + c.d // 2 + 4) + c.d, us, pk, c.T,
                                      "T=16384, 32 heads x 128, INT4 per token")
     del x, xo, cq, sq, st
+    # FlatQuant's Kronecker affine transform on the hidden stream: d = 4096 = 64 x 64, bf16, INT4
+    f = inputs.flatquant_case()
+    xf = torch.from_numpy(f.x).to(dev).to(torch.bfloat16)
+    P1, P2 = torch.from_numpy(f.P1).to(dev), torch.from_numpy(f.P2).to(dev)
+    cf = torch.empty((f.T, f.d // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty((f.T,), dtype=torch.float32, device=dev)
+    us = _time_loop(stream, lambda: rsq.kron_affine_quant(xf, P1, P2, cf, sf, bits=4, stream=stream), 20, 3)
+    flops = 2.0 * f.T * f.d * (f.n1 + f.n2)
+    peak64 = 148 * 64 * 2 * 1.965e9 / 1e12
+    byts = f.T * (2 * f.d + f.d // 2 + 4) + 4 * (f.n1 * f.n1 + f.n2 * f.n2)
+    out["kron_affine_quant"] = {"shape": "T=16384, d=4096 = 64 x 64, bf16 in, INT4 out, float64 products",
+                                "avg_us": us, "bound": "alu", "algorithmic_fp64_flops": flops,
+                                "achieved_tflops_fp64": flops / (us * 1e-6) / 1e12, "peak_tflops_fp64": peak64,
+                                "frac": flops / (us * 1e-6) / 1e12 / peak64,
+                                "achieved_gbs": byts / (us * 1e-6) / 1e9, "tokens_per_s": f.T / (us * 1e-6),
+                                "peak_source": "148 SMs x 64 FP64 FMA/clock x 2 x 1.965 GHz (unit counts and max clock)"}
+    del xf, cf, sf
     # W4A4 GEMM: the hidden stream through a 4096 x 4096 INT4 projection
     gm = inputs.gemm_case(16384, 4096, 4096, 21)
     ca, cw = torch.from_numpy(gm.codes_a).to(dev), torch.from_numpy(gm.codes_w).to(dev)

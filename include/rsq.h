@@ -172,6 +172,24 @@ int rht_heads_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *co
 int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t *codes, float *scales,
                        int64_t T, int d, int bits, int dtype, void *stream);
 
+/* FlatQuant's Kronecker affine transform fused with the quantiser.  Infra
+ * Quant II, FlatQuant: a linear layer's input row x of length d = n1 * n2 is
+ * transformed by P = P1 (x) P2 (two small invertible matrices found by
+ * calibration) as x P = vec(P1^T X P2), X the n1 x n2 row-major reshape of the
+ * row (X[a][b] = x[a*n2 + b]); the one kernel keeps P1 and P2 on chip and
+ * quantises each transformed row before writing it:
+ *     v_t = vec(P1^T X_t P2),  scales[t] = max_i |v_ti| / qmax,
+ * codes and packing as for rht_quant (the symmetric quantiser, no clipping
+ * factor).  x: T x d elements of `dtype`.  P1: n1 x n1 float32, P2: n2 x n2
+ * float32, row-major, any values.  The two products accumulate in float64
+ * (the factors are dense, and float32 sums over n1 + n2 terms would miss the
+ * scales' 1e-6 relative bound).  Shapes: n1 and n2 multiples of 4 in
+ * [4, 128] with d <= 4096 (RSQ_ERR_SHAPE otherwise).  The outputs
+ * may not overlap any input or each other (RSQ_ERR_ALIAS).  Streams, errors,
+ * alignment as above. */
+int kron_affine_quant(const void *x, const float *P1, const float *P2, int n1, int n2, uint8_t *codes,
+                      float *scales, int64_t T, int bits, int dtype, void *stream);
+
 /* The INT4 consumer GEMM of the quantised activations (W4A4).  Infra Quant II,
  * QuaRot / Method: the INT4 GEMM's INT32 output becomes 16-bit float and is
  * multiplied by the activation's per-row scale and the weight's per-column

@@ -188,6 +188,30 @@ def test_head_transforms_accept_null_signs():
     assert _heads(sg=None) == CUDA and _heads_q(sg=None) == CUDA and _mix_q(sg=None) == CUDA
 
 
+def _aff(x=X, p1=Q, p2=M, n1=64, n2=64, c=C, s=S, T=4, bits=4, dt=BF16):
+    return L.kron_affine_quant(x, p1, p2, n1, n2, c, s, T, bits, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(x=None), NULL), (dict(p1=None), NULL), (dict(p2=None), NULL), (dict(c=None), NULL), (dict(s=None), NULL),
+    (dict(bits=2), BITS), (dict(dt=2), DTYPE), (dict(T=-1), SHAPE),
+    (dict(n1=2, n2=8), SHAPE),                        # below 4
+    (dict(n1=6, n2=8), SHAPE),                        # not a multiple of 4
+    (dict(n1=4, n2=256), SHAPE),                      # n2 > 128
+    (dict(n1=128, n2=64), SHAPE),                     # d = 8192 > 4096
+    (dict(x=X + 8), ALIGN), (dict(p1=Q + 4), ALIGN), (dict(p2=M + 2), ALIGN), (dict(c=C + 4), ALIGN),
+    (dict(s=S + 8), ALIGN),
+    (dict(c=X + 4096), ALIAS),                        # codes inside x
+    (dict(s=Q + 256), ALIAS),                         # scales inside P1
+    (dict(c=M), ALIAS),                               # codes over P2
+    (dict(s=C + 16), ALIAS),                          # scales inside codes
+])
+def test_kron_affine_quant_rejects(kw, want):
+    before = rsq.launch_count()
+    assert _aff(**kw) == want
+    assert rsq.launch_count() == before
+
+
 def _gemm(ca=X, sa=S, cw=Q, sw=M, y=XO, acc=C, T=4, N=256, K=4096, dt=2):
     return L.w4a4_gemm(ca, sa, cw, sw, y, acc, T, N, K, dt, None)
 
@@ -271,6 +295,7 @@ def test_empty_batch_is_a_no_op():
     assert _heads(x=None, xo=None, T=0) == OK
     assert _heads_q(x=None, c=None, s=None, T=0) == OK
     assert _mix_q(x=None, c=None, s=None, T=0) == OK
+    assert _aff(x=None, p1=None, p2=None, c=None, s=None, T=0) == OK
     assert _gemm(ca=None, sa=None, y=None, acc=None, T=0) == OK
     assert rsq.launch_count() == before
 

@@ -952,3 +952,47 @@ def test_deterministic_repeat():
     c2 = run_rht(h)
     for u, v in zip(c1, c2):
         np.testing.assert_array_equal(u, v)
+
+
+# --------------------------------------------------------------------------
+# FlatQuant's Kronecker affine transform vec(P1^T X P2) + quantiser
+# --------------------------------------------------------------------------
+
+def run_affine(case):
+    rsq = _rsq()
+    x = _to_dev(case.x, case.dtype)
+    P1, P2 = torch.from_numpy(case.P1).to(DEV), torch.from_numpy(case.P2).to(DEV)
+    codes, scales = rsq.kron_affine_quant(x, P1, P2, bits=case.bits)
+    assert rsq.device_status() == 0
+    return codes.cpu().numpy(), scales.cpu().numpy()
+
+
+def check_affine(case, rows=None, label=""):
+    codes, scales = run_affine(case)
+    sel = slice(None) if rows is None else rows
+    ref = oracle.kron_affine_quant(case.x[sel], case.P1, case.P2, case.bits)
+    H.check_scales(scales[sel], ref["scales"], label)
+    return H.check_codes(codes[sel], ref["q"], ref["pre"], case.bits, label)
+
+
+@pytest.mark.parametrize("n1,n2,dtype,bits,T", [(64, 64, "bf16", 4, 300), (64, 64, "f32", 3, 149),
+                                                 (32, 128, "bf16", 4, 97), (128, 32, "f32", 4, 5),
+                                                 (4, 4, "bf16", 4, 1), (8, 16, "bf16", 3, 333),
+                                                 (12, 20, "f32", 4, 37)])
+def test_kron_affine_quant(n1, n2, dtype, bits, T):
+    """Whole outputs of every token row: square and non-square factors (so a
+    transposed factor or swapped roles of n1 and n2 would fail), fp32 and bf16
+    input, INT4 and INT3, an all-zero row, more rows than SMs (each CTA walks
+    several) and a single row."""
+    c = inputs.kron_affine_case(T, n1, n2, 7 + n1, dtype=dtype, bits=bits)
+    if T > 3:
+        c.x[2] = 0.0
+    check_affine(c, label=f"affine {n1}x{n2} {dtype} INT{bits} T={T}")
+
+
+def test_kron_affine_quant_full_size_sampled():
+    """The bench's workload (T = 16384, d = 4096 = 64 x 64, bf16, INT4) in its
+    launch configuration, compared on sampled rows."""
+    c = inputs.flatquant_case()
+    rows = np.r_[0:64, 8000:8064, c.T - 64:c.T]
+    check_affine(c, rows=rows, label="flatquant T=16384 sampled")

@@ -105,4 +105,12 @@ bool rht_tc_supports(int d, int m, int dtype, int bits, long long T);
 cudaError_t launch_rht_tc(const void *x, const int8_t *signs, uint8_t *codes, float *scales, long long T, int d,
                           int bits, cudaStream_t s);
 
+// FlatQuant's Kronecker affine transform vec(P1^T X P2) + per-token quantiser,
+// float64 products on the CUDA cores: n1, n2 multiples of 4 in [4, 128],
+// n1 n2 <= 4096.
+bool kron_affine_supports(int n1, int n2);
+cudaError_t launch_kron_affine_quant(const void *x, const float *P1, const float *P2, int n1, int n2,
+                                     uint8_t *codes, float *scales, long long T, int bits, int dtype,
+                                     cudaStream_t s);
+
 }  // namespace rsq

@@ -329,6 +329,27 @@ int rht_head_mix_quant(const void *x, const int8_t *signs, int n_heads, uint8_t 
                                        static_cast<cudaStream_t>(stream)));
 }
 
+int kron_affine_quant(const void *x, const float *P1, const float *P2, int n1, int n2, uint8_t *codes,
+                      float *scales, int64_t T, int bits, int dtype, void *stream) {
+    if (bits != 3 && bits != 4) return RSQ_ERR_BITS;
+    if (dtype != RSQ_F32 && dtype != RSQ_BF16) return RSQ_ERR_DTYPE;
+    if (T < 0 || !rsq::kron_affine_supports(n1, n2)) return RSQ_ERR_SHAPE;
+    if (T == 0) return RSQ_OK;
+    if (!x || !P1 || !P2 || !codes || !scales) return RSQ_ERR_NULL;
+    if (!aligned16(x) || !aligned16(P1) || !aligned16(P2) || !aligned16(codes) || !aligned16(scales))
+        return RSQ_ERR_ALIGN;
+    const int64_t d = int64_t(n1) * n2;
+    const Span sx = span(x, uint64_t(T) * d * elem_bytes(dtype));
+    const Span s1 = span(P1, uint64_t(n1) * n1 * 4), s2 = span(P2, uint64_t(n2) * n2 * 4);
+    const Span sc = span(codes, uint64_t(T) * d * bits / 8), ss = span(scales, uint64_t(T) * 4);
+    const Span ins[3] = {sx, s1, s2};
+    for (int i = 0; i < 3; ++i)
+        if (overlap(sc, ins[i]) || overlap(ss, ins[i])) return RSQ_ERR_ALIAS;
+    if (overlap(sc, ss)) return RSQ_ERR_ALIAS;
+    return finish(rsq::launch_kron_affine_quant(x, P1, P2, n1, n2, codes, scales, T, bits, dtype,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
 // Shared checks and launch of the two GEMM entry points: w is the packed weight
 // codes (N x K/2 bytes) or, with w_prepared, the int8 weights (N x K bytes).
 static int w4a4_gemm_common(const uint8_t *codes_a, const float *scales_a, const void *w, bool w_prepared,

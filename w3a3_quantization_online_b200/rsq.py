@@ -38,6 +38,8 @@ _lib.rht_heads_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i3
 _lib.rht_heads_quant.restype = _i32
 _lib.rht_head_mix_quant.argtypes = [_vp, _vp, _i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.rht_head_mix_quant.restype = _i32
+_lib.kron_affine_quant.argtypes = [_vp, _vp, _vp, _i32, _i32, _vp, _vp, _i64, _i32, _i32, _vp]
+_lib.kron_affine_quant.restype = _i32
 _lib.w4a4_gemm.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp]
 _lib.w4a4_gemm.restype = _i32
 _lib.w4a4_prepare_weights.argtypes = [_vp, _i32, _i32, _vp, _vp]
@@ -66,7 +68,7 @@ _lib.rsq_selftest_wait_timeout.argtypes = [_i32, _vp]
 _lib.rsq_selftest_wait_timeout.restype = _i32
 
 EXPORTED = ("rsq_residual_align", "rsq_align_norm_quant", "rht_quant", "rht_quant_silu_gate", "rht_heads",
-            "rht_heads_quant", "rht_head_mix_quant", "w4a4_gemm", "w4a4_prepare_weights", "w4a4_gemm_s8w",
+            "rht_heads_quant", "rht_head_mix_quant", "kron_affine_quant", "w4a4_gemm", "w4a4_prepare_weights", "w4a4_gemm_s8w",
             "rsq_qm_build", "rsq_qm_workspace_bytes",
             "rsq_qm_build_fixed_scratch",
             "rsq_status_string",
@@ -284,6 +286,26 @@ def rht_head_mix_quant(x: torch.Tensor, signs: Optional[torch.Tensor], n_heads: 
     _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
     _check(_lib.rht_head_mix_quant(_ptr(x), _signs_ptr(signs), n_heads, _ptr(codes), _ptr(scales), T, d, bits,
                                    _dtype_code(x), _stream(stream)))
+    return codes, scales
+
+
+def kron_affine_quant(x: torch.Tensor, P1: torch.Tensor, P2: torch.Tensor,
+                      codes: Optional[torch.Tensor] = None, scales: Optional[torch.Tensor] = None, bits: int = 4,
+                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """FlatQuant's Kronecker affine transform vec(P1^T X P2) of each row, then per-token INT{bits} codes."""
+    _need(x, "x")
+    _need(P1, "P1", torch.float32); _need(P2, "P2", torch.float32)
+    T, d = x.shape
+    n1, n2 = P1.shape[0], P2.shape[0]
+    if P1.shape != (n1, n1) or P2.shape != (n2, n2) or n1 * n2 != d:
+        raise ValueError(f"P1 {tuple(P1.shape)} and P2 {tuple(P2.shape)} do not factor a row of {d}")
+    if codes is None:
+        codes = torch.empty((T, d * bits // 8), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _need(codes, "codes", torch.uint8); _need(scales, "scales", torch.float32)
+    _check(_lib.kron_affine_quant(_ptr(x), _ptr(P1), _ptr(P2), n1, n2, _ptr(codes), _ptr(scales), T, bits,
+                                  _dtype_code(x), _stream(stream)))
     return codes, scales
 
 
